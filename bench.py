@@ -1,0 +1,466 @@
+#!/usr/bin/env python
+"""Benchmark: SPAttention band-sparse attention, forward + backward, on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl spa|reference]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+spa_attn_fwd (1 kernel) then the three backward steps (row sums D, the dK/dV
+pass, the dQ pass).  Inputs are resident in HBM when the timed region starts;
+each of q, k, v, dout is larger than the 126 MB L2, so no flush is needed
+between steps.  The metric is useful TFLOP/s: 14 * d * (permitted pairs) per
+step (forward 4 d, backward 10 d per pair -- the two GEMMs of the forward and
+the five of the backward, over the band's pairs only, never the tile padding),
+over the device time of the K timed steps, max over ranks.
+
+N > 1 (torchrun, one process per GPU): every rank runs its own independent
+batch of the same workload (weak scaling); the only collectives are the
+barrier and the max of the timings.
+
+--impl reference times the fp64 CPU oracle (the slow, plain implementation the
+tests check against) on a bounded sample of the same workload and prints the
+same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import datetime as _dt
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from head_partitioned_distance_b200 import synth  # noqa: E402
+
+METRIC = "band-sparse attn fwd+bwd useful TFLOP/s and % of B200 bf16 tensor peak"
+UNIT = "TFLOP/s"
+DEFAULT_WORKLOAD = "b1_h32_n32768_d128"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS = ("spa_fwd_kernel", "spa_bwd_delta_kernel", "spa_bwd_dkdv_kernel", "spa_bwd_dq_kernel")
+
+
+# --------------------------------------------------------------------- counting
+def band_pairs_prefix(P: int, lo: int, hi: int) -> int:
+    """Permitted pairs among query rows [0, P) of a head with band [lo, hi):
+    distance delta occurs in max(0, P - delta) rows."""
+    return sum(max(0, P - dd) for dd in range(lo, hi))
+
+
+def workload_pairs(N: int, bands) -> int:
+    return sum(band_pairs_prefix(N, lo, hi) for lo, hi in zip(*bands))
+
+
+def kernel_work(w, pairs: int):
+    """Algorithmic work per launch of each kernel (FLOPs over permitted pairs,
+    or bytes for the row-sum kernel)."""
+    d = w.d
+    rows = w.B * w.H * w.N
+    return {
+        "spa_fwd_kernel": ("tensor", 4 * d * pairs),            # S = QK^T, O += PV
+        "spa_bwd_delta_kernel": ("hbm", 2 * rows * d * 2 + rows * 4),  # read O, dO; write D
+        "spa_bwd_dkdv_kernel": ("tensor", 8 * d * pairs),       # S^T, dP^T, dV, dK
+        "spa_bwd_dq_kernel": ("tensor", 6 * d * pairs),         # S, dP, dQ
+    }
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            p = json.load(f)
+        return {k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def kernel_src_sha() -> str:
+    csrc = os.path.join(ROOT, "head_partitioned_distance_b200", "csrc")
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(csrc)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(csrc, name), "rb") as f:
+                h.update(name.encode() + b"\0" + f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch of `kernel` from a committed ncu summary under
+    profiles/, when the summary was taken on the current kernel sources."""
+    prof = os.path.join(ROOT, "profiles")
+    if not os.path.isdir(prof):
+        return None
+    sha = kernel_src_sha()
+    for name in sorted(os.listdir(prof)):
+        if not name.endswith((".md", ".txt")):
+            continue
+        fields = {}
+        with open(os.path.join(prof, name)) as f:
+            for line in f:
+                if line.startswith("traffic:"):
+                    for kv in line[len("traffic:"):].split():
+                        if "=" in kv:
+                            a, b = kv.split("=", 1)
+                            fields[a] = b
+                    if (fields.get("kernel") == kernel and fields.get("workload") == workload
+                            and fields.get("src_sha") == sha):
+                        return float(fields["dram_bytes_per_launch"])
+    return None
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.t0 = self.t1 = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.gpu_index)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def mark_start(self):
+        self.t0 = _dt.datetime.now()
+
+    def mark_end(self):
+        self.t1 = _dt.datetime.now()
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+                    "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = []
+        for line in out.splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 10:
+                continue
+            try:
+                ts = _dt.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
+            except ValueError:
+                continue
+            rows.append((ts, parts))
+        inside = [p for ts, p in rows if self.t0 and self.t1 and self.t0 <= ts <= self.t1]
+        sample = inside if inside else [p for _, p in rows]
+        sm = [float(p[2]) for p in sample if p[2].replace(".", "").isdigit()]
+        smax = [float(p[3]) for p in sample if p[3].replace(".", "").isdigit()]
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for p in sample:
+            for n, val in zip(names, p[6:10]):
+                if val.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sample),
+                "window": "timed region" if inside else "whole run (no sample fell inside the timed region)",
+                "power_w_max": max((float(p[4]) for p in sample
+                                    if p[4].replace(".", "").isdigit()), default=None)}
+
+
+# --------------------------------------------------------------------- distributed
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, local, world
+
+
+def dist_init(backend: str, local: int):
+    import torch.distributed as dist
+    if backend == "nccl":
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend=backend, timeout=_dt.timedelta(seconds=120))
+    return dist
+
+
+def reduce_max(value: float, device) -> float:
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()):
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def aggregate(useful_flops_per_rank_step: float, steps: int, world: int, max_ms: float) -> float:
+    """Whole-job throughput: the work of every rank over the slowest rank's time."""
+    return world * useful_flops_per_rank_step * steps / (max_ms * 1e-3) / 1e12
+
+
+# --------------------------------------------------------------------- CPU oracle timing
+def oracle_sample(w, bands, prefix_rows: int):
+    """Time the fp64 oracle's forward + backward on a causal prefix of head 0
+    of batch 0: query rows [0, prefix_rows) with that head's band.  Those rows'
+    outputs equal the full-sequence ones (causal rows only look back).
+    Returns (useful flops, seconds, threads, description)."""
+    import oracle
+    q, k, v, do = synth.make_inputs(1, 1, prefix_rows, w.d, seed=w.seed)
+    f = lambda t: t.to(torch.float64).numpy()
+    lo, hi = [bands[0][0]], [bands[1][0]]
+    t0 = time.perf_counter()
+    oracle.spa_fwd(f(q), f(k), f(v), w.scale, lo, hi)
+    oracle.spa_bwd(f(q), f(k), f(v), f(do), w.scale, lo, hi)
+    secs = time.perf_counter() - t0
+    pairs = band_pairs_prefix(prefix_rows, lo[0], hi[0])
+    desc = (f"oracle spa_fwd + spa_bwd (fp64, OpenMP) on head 0, query rows [0, {prefix_rows}) "
+            f"of the {w.name} workload (band [{lo[0]}, {hi[0]}), d={w.d}); {pairs} pairs")
+    return 14 * w.d * pairs, secs, oracle.num_threads(), desc
+
+
+def calibrate_prefix(w, bands, target_s: float, start: int = 256):
+    """Double the prefix until one oracle run takes at least target_s / 2 (or
+    the prefix covers the sequence).  Returns the last run:
+    (prefix, flops, seconds, threads, description)."""
+    P = min(start, w.N)
+    while True:
+        fl, secs, cores, desc = oracle_sample(w, bands, P)
+        if secs >= target_s / 2 or P >= w.N:
+            return P, fl, secs, cores, desc
+        P = min(2 * P, w.N)
+
+
+def run_reference(args):
+    rank, local, world = dist_setup()
+    if rank != 0:
+        return 0
+    w = synth.WORKLOADS[args.workload]
+    import oracle
+    lo, hi = oracle.bands(w.N, w.H)
+    bands = ([int(x) for x in lo], [int(x) for x in hi])
+    budget = 150.0  # seconds for the whole --steps/--warmup run
+    per_step = budget / max(args.steps + args.warmup, 1)
+    P = calibrate_prefix(w, bands, min(per_step, 20.0), start=128)[0]
+    for _ in range(args.warmup):
+        oracle_sample(w, bands, P)
+    total_flops, total_s = 0.0, 0.0
+    for _ in range(args.steps):
+        fl, s, cores, desc = oracle_sample(w, bands, P)
+        total_flops += fl
+        total_s += s
+    value = total_flops / total_s / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": desc + " per step"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# --------------------------------------------------------------------- GPU arm
+def run_spa(args):
+    from head_partitioned_distance_b200 import spa
+
+    rank, local, world = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200); there is no CPU path")
+    dist = dist_init("nccl", local) if world > 1 else None
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = synth.WORKLOADS[args.workload]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    bands = spa.spa_band_bounds(N, H)
+    pairs = B * workload_pairs(N, bands)
+    useful = 14 * d * pairs
+
+    # independent batch per rank (weak scaling)
+    q, k, v, do = synth.make_inputs(B, H, N, d, w.seed + 7919 * rank, w.qkv_mult, w.rms_qk, w.do_mult)
+    host = {"q": q, "k": k, "v": v, "do": do}
+    qd, kd, vd, dod = (t.to(device) for t in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd)
+    ws = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    scale = w.scale
+
+    def step(ev=None):
+        spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, stream=stream)
+        if ev is not None:
+            ev[0].record(stream)
+        spa.spa_attn_bwd_preprocess(o, dod, ws, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, ws, dk, dv, scale, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+        spa.spa_attn_bwd_dq(qd, kd, vd, dod, lse, ws, dq, scale, stream=stream)
+        if ev is not None:
+            ev[3].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after warm-up")
+
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(visible.split(",")[local] if visible else local)
+    sampler.start()
+    K = args.steps
+    t_start = torch.cuda.Event(enable_timing=True)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    sampler.mark_start()
+    t_start.record(stream)
+    for s in range(K):
+        step(evs[s])
+    torch.cuda.synchronize(device)
+    sampler.mark_end()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after the timed region")
+    elapsed_ms = t_start.elapsed_time(evs[-1][3])
+    per_kernel_ms = {name: 0.0 for name in KERNELS}
+    prev = t_start
+    for s in range(K):
+        e = evs[s]
+        per_kernel_ms["spa_fwd_kernel"] += prev.elapsed_time(e[0])
+        per_kernel_ms["spa_bwd_delta_kernel"] += e[0].elapsed_time(e[1])
+        per_kernel_ms["spa_bwd_dkdv_kernel"] += e[1].elapsed_time(e[2])
+        per_kernel_ms["spa_bwd_dq_kernel"] += e[2].elapsed_time(e[3])
+        prev = e[3]
+    max_ms = reduce_max(elapsed_ms, device)
+    value = aggregate(useful, K, world, max_ms)
+
+    # ------------------------------------------------ end to end, host buffers
+    E = max(2, min(5, K))
+    pin = {n: t.pin_memory() for n, t in host.items()}
+    out_h = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in
+             (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_h.values())
+
+    def e2e_step():
+        qd.copy_(pin["q"], non_blocking=True)
+        kd.copy_(pin["k"], non_blocking=True)
+        vd.copy_(pin["v"], non_blocking=True)
+        dod.copy_(pin["do"], non_blocking=True)
+        spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, stream=stream)
+        spa.spa_attn_bwd(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, scale, stream=stream)
+        for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv)):
+            out_h[n].copy_(t, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+    e2e_value = aggregate(useful, E, world, e2e_ms)
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after the end-to-end region")
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        work = kernel_work(w, pairs)
+        kern = {}
+        for name in KERNELS:
+            bound, units = work[name]
+            avg_ms = per_kernel_ms[name] / K
+            if bound == "tensor":
+                achieved = units / (avg_ms * 1e-3) / 1e12
+                peak = peaks["bf16_tflops"]
+                unit = "TFLOP/s"
+            else:
+                achieved = units / (avg_ms * 1e-3) / 1e9
+                peak = peaks["hbm_gbs"]
+                unit = "GB/s"
+            kern[name] = {"bound": bound, "avg_ms": avg_ms, "share": per_kernel_ms[name] / elapsed_ms,
+                          "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                          "algorithmic_per_launch": units}
+        dom = max(KERNELS, key=lambda n: per_kernel_ms[n])
+        dk_ = kern[dom]
+        roofline = {"bound": dk_["bound"], "achieved": dk_["achieved"], "peak": dk_["peak"],
+                    "unit": dk_["unit"], "frac": dk_["frac"],
+                    "traffic": ncu_traffic(dom, w.name), "kernel": dom,
+                    "peak_source": f"{peak_src} ({'bf16_tflops burst' if dk_['bound'] == 'tensor' else 'hbm_gbs'})"}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            P, fl, secs, cores, desc = calibrate_prefix(w, bands, args.cpu_seconds, start=512)
+            cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+                   "sample": desc, "seconds": secs}
+        per_gpu = value / world
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": max_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "pct_of_bf16_peak": 100.0 * per_gpu / peaks["bf16_tflops"],
+            "pct_of_bf16_peak_sustained": 100.0 * per_gpu / peaks["bf16_tflops_sustained"],
+            "peaks": {**peaks, "source": peak_src},
+            "tokens_per_s": world * B * N * K / (max_ms * 1e-3),
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d,
+                       "bands": "balanced distance partitioning", "pairs_per_rank": pairs,
+                       "useful_flops_per_rank_step": useful,
+                       "l2": "no flush: q, k, v, dout are each larger than L2 "
+                             f"({B * H * N * d * 2 / 2**20:.0f} MiB bf16)",
+                       "parallelism": f"{world} independent replicas (one batch each)"},
+            "roofline": roofline,
+            "kernels": kern,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": e2e_ms / E},
+            "gpu_launches": 4 * K,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["spa", "reference"], default="spa")
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_spa(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

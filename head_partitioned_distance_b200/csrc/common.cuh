@@ -1,0 +1,93 @@
+// common.cuh -- pieces shared by the kernels: launch parameters, the device
+// error word, and bounded mbarrier waits.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "ptx.cuh"
+#include "sched.cuh"
+
+namespace spa {
+
+constexpr int kMaxHeads = 256;
+
+// Status codes mirrored from spa.h (kept numerically identical).
+constexpr int kStatusOk = 0;
+constexpr int kStatusTimeout = 4;
+
+// Longest a thread waits on one mbarrier phase before the kernel gives up.
+constexpr uint64_t kWaitLimitNs = 2000000000ull;
+// Longest the exit path waits for its own copies and MMAs in flight.
+constexpr uint64_t kDrainLimitNs = 200000000ull;
+
+struct AttnParams {
+  int B;
+  int H;
+  int64_t N;
+  float scale;        // multiplies q.k
+  float scale_log2;   // scale * log2(e): scores in base-2 units
+  // forward: lse is written; backward: lse (read) and delta (workspace)
+  float* lse;
+  float* delta;
+  // raw pointers, for the rows that empty units write directly
+  void* o;
+  void* dq;
+  void* dk;
+  void* dv;
+  const void* o_in;
+  const void* dout;
+  int32_t lo[kMaxHeads];
+  int32_t hi[kMaxHeads];
+};
+
+// The library's device error word: a kernel that times out on a wait stores
+// kStatusTimeout here; spa_device_status() reads and clears it.
+__device__ int g_spa_status;
+
+// Bounded wait on one mbarrier phase.  Returns false when the CTA aborted:
+// either this wait ran past kWaitLimitNs (it then raises the CTA's abort flag
+// and the device error word) or another thread already raised the flag.
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  const uint32_t a = ptx::smem_u32(bar);
+  if (ptx::mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (true) {
+#pragma unroll 1
+    for (int n = 0; n < 32; ++n)
+      if (ptx::mbar_try_wait(a, parity)) return true;
+    if (*abort_flag) return false;
+    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+      *abort_flag = 1;
+      atomicExch(&g_spa_status, kStatusTimeout);
+      return false;
+    }
+  }
+}
+
+// Wait used on the exit path only: gives up silently after kDrainLimitNs.
+__device__ __forceinline__ bool bar_drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t a = ptx::smem_u32(bar);
+  const uint64_t t0 = ptx::globaltimer_ns();
+  while (!ptx::mbar_try_wait(a, parity)) {
+    if (ptx::globaltimer_ns() - t0 > kDrainLimitNs) {
+      atomicExch(&g_spa_status, kStatusTimeout);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
+  return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// Zero `rows` rows of a [.., d] bf16 matrix starting at `base` (16-byte
+// stores, all threads of the CTA cooperating).
+__device__ __forceinline__ void zero_rows_bf16(void* base, int64_t rows, int d) {
+  uint4* p = reinterpret_cast<uint4*>(base);
+  const int64_t n16 = rows * d / 8;
+  for (int64_t e = threadIdx.x; e < n16; e += blockDim.x) p[e] = make_uint4(0, 0, 0, 0);
+}
+
+}  // namespace spa

@@ -1,0 +1,368 @@
+// spa.cu -- the C ABI of libspa.so (declared in include/spa.h): argument
+// checks, TMA tensor maps, and kernel launches.  One translation unit so the
+// device error word is shared by every kernel without relocatable code.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstring>
+#include <mutex>
+
+#include "spa.h"
+
+#include "bwd.cuh"
+#include "common.cuh"
+#include "fwd.cuh"
+#include "sched.cuh"
+
+namespace {
+
+using spa::AttnParams;
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// [B*H][N][d] bf16 tensor viewed as 3-D (d, N, B*H); box = 64 columns x rows x 1,
+// 128-byte swizzle (matches the kernels' shared-memory layout), zero fill
+// outside the tensor.
+int make_map(CUtensorMap* m, const void* ptr, int64_t N, int64_t BH, int d, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return SPA_ERR_CUDA;
+  cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
+  cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
+  cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? SPA_OK : SPA_ERR_CUDA;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(int B, int H, int64_t N, int d) {
+  if (B < 1 || H < 1 || N < 1) return SPA_ERR_INVAL;
+  if (N > 2147483647LL) return SPA_ERR_INVAL;
+  if (B > 65535 || H > spa::kMaxHeads) return SPA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128) return SPA_ERR_UNSUPPORTED;
+  return SPA_OK;
+}
+
+// Fill p.lo/p.hi from explicit bands (lo/hi non-null) or from Balanced
+// Distance Partitioning.
+int fill_bands(AttnParams& p, int H, int64_t N, const int32_t* lo, const int32_t* hi) {
+  if ((lo == nullptr) != (hi == nullptr)) return SPA_ERR_INVAL;
+  if (lo == nullptr) {
+    if (H > N) return SPA_ERR_INVAL;
+    for (int h = 0; h < H; ++h) spa::band_of_head(N, H, h, &p.lo[h], &p.hi[h]);
+    return SPA_OK;
+  }
+  for (int h = 0; h < H; ++h) {
+    if (lo[h] < 0 || lo[h] >= hi[h] || (int64_t)hi[h] > N) return SPA_ERR_INVAL;
+    p.lo[h] = lo[h];
+    p.hi[h] = hi[h];
+  }
+  return SPA_OK;
+}
+
+// Opt a kernel into its dynamic shared memory once per device.
+template <typename K>
+int prepare_kernel(K kernel, uint32_t smem_bytes, std::atomic<uint64_t>& done_mask) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPA_ERR_CUDA;
+  const uint64_t bit = 1ull << (dev & 63);
+  if (done_mask.load(std::memory_order_acquire) & bit) return SPA_OK;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_bytes) !=
+      cudaSuccess)
+    return SPA_ERR_CUDA;
+  done_mask.fetch_or(bit, std::memory_order_acq_rel);
+  return SPA_OK;
+}
+
+int launch_status() { return cudaGetLastError() == cudaSuccess ? SPA_OK : SPA_ERR_CUDA; }
+
+template <int D>
+int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, AttnParams& p,
+             cudaStream_t stream) {
+  using C = spa::FwdCfg<D>;
+  static std::atomic<uint64_t> prepared{0};
+  const int64_t BH = (int64_t)p.B * p.H;
+  CUtensorMap mq, mk, mv, mo;
+  int st;
+  if ((st = make_map(&mq, q, p.N, BH, D, C::BQ)) || (st = make_map(&mk, k, p.N, BH, D, C::BK)) ||
+      (st = make_map(&mv, v, p.N, BH, D, C::BK)) || (st = make_map(&mo, o, p.N, BH, D, C::BQ)))
+    return st;
+  if ((st = prepare_kernel(spa::spa_fwd_kernel<D>, C::SMEM_BYTES, prepared))) return st;
+  p.lse = lse;
+  p.o = o;
+  dim3 grid((unsigned)((p.N + C::BQ - 1) / C::BQ), (unsigned)p.H, (unsigned)p.B);
+  spa::spa_fwd_kernel<D><<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  return launch_status();
+}
+
+enum BwdStep { kStepDelta = 1, kStepDkDv = 2, kStepDq = 4, kStepAll = 7 };
+
+template <int D>
+int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
+             const float* lse, void* dq, void* dk, void* dv, float* delta, AttnParams& p,
+             cudaStream_t stream, int steps) {
+  using KC = spa::DkvCfg<D>;
+  using QC = spa::DqCfg<D>;
+  static std::atomic<uint64_t> prepared_kv{0}, prepared_q{0};
+  const int64_t BH = (int64_t)p.B * p.H;
+  int st;
+  p.lse = const_cast<float*>(lse);
+  p.delta = delta;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  if (steps & kStepDelta) {
+    const int64_t rows = BH * p.N;
+    const int64_t threads = rows * (D / 8);
+    const int64_t blocks = (threads + 255) / 256;
+    if (blocks > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+    spa::spa_bwd_delta_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(
+        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), delta, rows);
+    if ((st = launch_status())) return st;
+  }
+  if (steps & kStepDkDv) {
+    // key tiles of 128 rows, query tiles of 64 rows
+    CUtensorMap kq, kk, kv, kdo, kdk, kdv;
+    if ((st = make_map(&kq, q, p.N, BH, D, KC::BQ)) || (st = make_map(&kk, k, p.N, BH, D, KC::BK)) ||
+        (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)) ||
+        (st = make_map(&kdk, dk, p.N, BH, D, KC::BK)) || (st = make_map(&kdv, dv, p.N, BH, D, KC::BK)))
+      return st;
+    if ((st = prepare_kernel(spa::spa_bwd_dkdv_kernel<D>, KC::SMEM_BYTES, prepared_kv))) return st;
+    dim3 gkv((unsigned)((p.N + KC::BK - 1) / KC::BK), (unsigned)p.H, (unsigned)p.B);
+    spa::spa_bwd_dkdv_kernel<D><<<gkv, 192, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
+    if ((st = launch_status())) return st;
+  }
+  if (steps & kStepDq) {
+    // query tiles of 128 rows, key tiles of 64 rows
+    CUtensorMap qq, qk, qv, qdo, qdq;
+    if ((st = make_map(&qq, q, p.N, BH, D, QC::BQ)) || (st = make_map(&qk, k, p.N, BH, D, QC::BK)) ||
+        (st = make_map(&qv, v, p.N, BH, D, QC::BK)) || (st = make_map(&qdo, dout, p.N, BH, D, QC::BQ)) ||
+        (st = make_map(&qdq, dq, p.N, BH, D, QC::BQ)))
+      return st;
+    if ((st = prepare_kernel(spa::spa_bwd_dq_kernel<D>, QC::SMEM_BYTES, prepared_q))) return st;
+    dim3 gq((unsigned)((p.N + QC::BQ - 1) / QC::BQ), (unsigned)p.H, (unsigned)p.B);
+    spa::spa_bwd_dq_kernel<D><<<gq, 192, QC::SMEM_BYTES, stream>>>(qq, qk, qv, qdo, qdq, p);
+    if ((st = launch_status())) return st;
+  }
+  return SPA_OK;
+}
+
+int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+              int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  if (!q || !k || !v || !o || !lse) return SPA_ERR_INVAL;
+  if (!std::isfinite(scale)) return SPA_ERR_INVAL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+    return SPA_ERR_UNSUPPORTED;
+  static AttnParams zero{};
+  AttnParams p = zero;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.scale = scale;
+  p.scale_log2 = scale * spa::kLog2e;
+  if ((st = fill_bands(p, H, N, lo, hi))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? fwd_impl<64>(q, k, v, o, lse, p, s) : fwd_impl<128>(q, k, v, o, lse, p, s);
+}
+
+int bwd_entry(const void* q, const void* k, const void* v, const void* o, const void* dout,
+              const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int H, int64_t N,
+              int d, float scale, const int32_t* lo, const int32_t* hi, void* stream, int steps) {
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  // every step reads the workspace (D); each checks the tensors it touches
+  if (!workspace) return SPA_ERR_INVAL;
+  if ((steps & kStepDelta) && (!o || !dout)) return SPA_ERR_INVAL;
+  if ((steps & (kStepDkDv | kStepDq)) && (!q || !k || !v || !dout || !lse)) return SPA_ERR_INVAL;
+  if ((steps & kStepDkDv) && (!dk || !dv)) return SPA_ERR_INVAL;
+  if ((steps & kStepDq) && !dq) return SPA_ERR_INVAL;
+  if (!std::isfinite(scale)) return SPA_ERR_INVAL;
+  for (const void* t : {q, k, v, o, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (t && !aligned(t, 16)) return SPA_ERR_UNSUPPORTED;
+  if ((lse && !aligned(lse, 4)) || !aligned(workspace, 4)) return SPA_ERR_UNSUPPORTED;
+  static AttnParams zero{};
+  AttnParams p = zero;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.scale = scale;
+  p.scale_log2 = scale * spa::kLog2e;
+  if ((st = fill_bands(p, H, N, lo, hi))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* delta = static_cast<float*>(workspace);
+  return d == 64 ? bwd_impl<64>(q, k, v, o, dout, lse, dq, dk, dv, delta, p, s, steps)
+                 : bwd_impl<128>(q, k, v, o, dout, lse, dq, dk, dv, delta, p, s, steps);
+}
+
+struct BandArgs {
+  int32_t lo[spa::kMaxHeads];
+  int32_t hi[spa::kMaxHeads];
+};
+
+__global__ void tile_class_kernel(int64_t N, int H, int Bq, int Bk, int nqt, int nkt,
+                                  const __grid_constant__ BandArgs bands, uint8_t* out) {
+  const int64_t total = (int64_t)H * nqt * nkt;
+  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < total;
+       e += (int64_t)gridDim.x * blockDim.x) {
+    const int u = (int)(e % nkt);
+    const int t = (int)((e / nkt) % nqt);
+    const int h = (int)(e / ((int64_t)nkt * nqt));
+    out[e] = spa::tile_class(N, bands.lo[h], bands.hi[h], t, Bq, u, Bk);
+  }
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* spa_status_string(int status) {
+  switch (status) {
+    case SPA_OK: return "SPA_OK";
+    case SPA_ERR_INVAL: return "SPA_ERR_INVAL: invalid argument";
+    case SPA_ERR_UNSUPPORTED: return "SPA_ERR_UNSUPPORTED: shape or alignment not supported";
+    case SPA_ERR_CUDA: return "SPA_ERR_CUDA: CUDA call or kernel launch failed";
+    case SPA_ERR_TIMEOUT: return "SPA_ERR_TIMEOUT: a device-side wait ran out of time";
+    default: return "unknown spa status";
+  }
+}
+
+int spa_version(void) { return 100; }
+
+int spa_band_bounds(int64_t N, int H, int32_t* lo, int32_t* hi) {
+  if (!lo || !hi || H < 1 || N < 1 || (int64_t)H > N || N > 2147483647LL) return SPA_ERR_INVAL;
+  for (int h = 0; h < H; ++h) spa::band_of_head(N, H, h, &lo[h], &hi[h]);
+  return SPA_OK;
+}
+
+int spa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                 int64_t N, int d, float scale, void* stream) {
+  return fwd_entry(q, k, v, o, lse, B, H, N, d, scale, nullptr, nullptr, stream);
+}
+
+int spa_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                    int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+  if (!lo || !hi) return SPA_ERR_INVAL;
+  return fwd_entry(q, k, v, o, lse, B, H, N, d, scale, lo, hi, stream);
+}
+
+size_t spa_attn_bwd_workspace_bytes(int B, int H, int64_t N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  return (size_t)B * (size_t)H * (size_t)N * sizeof(float);
+}
+
+int spa_attn_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                 const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int H,
+                 int64_t N, int d, float scale, void* stream) {
+  return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, d, scale, nullptr, nullptr,
+                   stream, kStepAll);
+}
+
+int spa_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                    const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int H,
+                    int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi,
+                    void* stream) {
+  if (!lo || !hi) return SPA_ERR_INVAL;
+  return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, d, scale, lo, hi, stream,
+                   kStepAll);
+}
+
+int spa_attn_bwd_preprocess(const void* o, const void* dout, void* workspace, int B, int H, int64_t N,
+                            int d, void* stream) {
+  return bwd_entry(nullptr, nullptr, nullptr, o, dout, nullptr, nullptr, nullptr, nullptr, workspace, B,
+                   H, N, d, 1.0f, nullptr, nullptr, stream, kStepDelta);
+}
+
+int spa_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                      const void* workspace, void* dk, void* dv, int B, int H, int64_t N, int d,
+                      float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+  return bwd_entry(q, k, v, nullptr, dout, lse, nullptr, dk, dv, const_cast<void*>(workspace), B, H, N,
+                   d, scale, lo, hi, stream, kStepDkDv);
+}
+
+int spa_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                    const void* workspace, void* dq, int B, int H, int64_t N, int d, float scale,
+                    const int32_t* lo, const int32_t* hi, void* stream) {
+  return bwd_entry(q, k, v, nullptr, dout, lse, dq, nullptr, nullptr, const_cast<void*>(workspace), B, H,
+                   N, d, scale, lo, hi, stream, kStepDq);
+}
+
+int spa_tile_schedule(int64_t N, int H, const int32_t* lo, const int32_t* hi, int Bq, int Bk,
+                      int32_t* kt_begin, int32_t* kt_end, uint8_t* tile_class, int32_t* qt_begin,
+                      int32_t* qt_end) {
+  if (N < 1 || N > 2147483647LL || H < 1 || H > spa::kMaxHeads || Bq < 1 || Bk < 1 || Bq > 4096 ||
+      Bk > 4096)
+    return SPA_ERR_INVAL;
+  AttnParams p{};
+  int st = fill_bands(p, H, N, lo, hi);
+  if (st) return st;
+  const int nqt = (int)((N + Bq - 1) / Bq), nkt = (int)((N + Bk - 1) / Bk);
+  for (int h = 0; h < H; ++h) {
+    for (int t = 0; t < nqt; ++t) {
+      const spa::Strip s = spa::key_strip(N, p.lo[h], p.hi[h], (int64_t)t * Bq, Bq, Bk);
+      if (kt_begin) kt_begin[(int64_t)h * nqt + t] = s.end < s.begin ? 0 : s.begin;
+      if (kt_end) kt_end[(int64_t)h * nqt + t] = s.end < s.begin ? -1 : s.end;
+      if (tile_class)
+        for (int u = 0; u < nkt; ++u)
+          tile_class[((int64_t)h * nqt + t) * nkt + u] = spa::tile_class(N, p.lo[h], p.hi[h], t, Bq, u, Bk);
+    }
+    for (int u = 0; u < nkt; ++u) {
+      const spa::Strip s = spa::query_strip(N, p.lo[h], p.hi[h], (int64_t)u * Bk, Bk, Bq);
+      if (qt_begin) qt_begin[(int64_t)h * nkt + u] = s.end < s.begin ? 0 : s.begin;
+      if (qt_end) qt_end[(int64_t)h * nkt + u] = s.end < s.begin ? -1 : s.end;
+    }
+  }
+  return SPA_OK;
+}
+
+int spa_tile_classes_device(int64_t N, int H, const int32_t* lo, const int32_t* hi, int Bq, int Bk,
+                            uint8_t* tile_class_dev, void* stream) {
+  if (N < 1 || N > 2147483647LL || H < 1 || H > spa::kMaxHeads || Bq < 1 || Bk < 1 || Bq > 4096 ||
+      Bk > 4096 || !tile_class_dev)
+    return SPA_ERR_INVAL;
+  AttnParams p{};
+  int st = fill_bands(p, H, N, lo, hi);
+  if (st) return st;
+  BandArgs bands{};
+  std::memcpy(bands.lo, p.lo, sizeof(bands.lo));
+  std::memcpy(bands.hi, p.hi, sizeof(bands.hi));
+  const int nqt = (int)((N + Bq - 1) / Bq), nkt = (int)((N + Bk - 1) / Bk);
+  tile_class_kernel<<<148 * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(N, H, Bq, Bk, nqt, nkt, bands,
+                                                                            tile_class_dev);
+  return launch_status();
+}
+
+int spa_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return SPA_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, spa::g_spa_status, sizeof(int)) != cudaSuccess) return SPA_ERR_CUDA;
+  if (v != 0) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(spa::g_spa_status, &z, sizeof(int)) != cudaSuccess) return SPA_ERR_CUDA;
+  }
+  return v == 0 ? SPA_OK : SPA_ERR_TIMEOUT;
+}
+
+}  // extern "C"

@@ -1,0 +1,183 @@
+/*
+ * spa.h -- C ABI of libspa.so: SPAttention band-sparse causal attention on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The method ("Making Every Head Count: Sparse Attention Without the
+ * Speed-Performance Trade-off", arXiv 2511.09596, abstract and Figure 1
+ * caption): the causal distance range [0, N) is split by Balanced Distance
+ * Partitioning into H contiguous, non-overlapping bands of width floor(N/H)
+ * or ceil(N/H), head 0 nearest; head h attends only to keys whose causal
+ * distance i - j lies in its band [lo_h, hi_h).  Softmax is unchanged and only
+ * runs over that permitted set ("Story of Attention -- Part 4", section 1,
+ * Sparse-Attention equation).  The H heads together cover every causal pair
+ * once, so a layer costs one causal O(N^2) attention.
+ *
+ * Conventions shared by every entry point:
+ *  - Tensors q, k, v, o, dout, dq, dk, dv are bf16, layout [B][H][N][d]
+ *    row-major contiguous, in DEVICE memory, 16-byte aligned.  lse and the
+ *    backward workspace are fp32 [B][H][N], device memory, 4-byte aligned.
+ *  - The caller owns every buffer; the library allocates no device memory.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream) and never synchronise the host, except
+ *    spa_device_status.
+ *  - scale multiplies q.k before the softmax (1/sqrt(d) for standard
+ *    attention).  Softmax statistics and accumulation are fp32.
+ *  - A query row whose permitted set is empty (i < lo_h) gets o = 0 and
+ *    lse = -inf; it passes no gradient.  Keys that no query reaches get
+ *    dk = dv = 0.  Every element of every output is written.
+ *  - Supported: d in {64, 128}; 1 <= H <= 256; 1 <= N <= 2^31 - 1;
+ *    1 <= B <= 65535.
+ *  - Return value: SPA_OK (0) or one of the spa_status_t codes below.  An
+ *    argument error is reported before anything is launched.
+ *  - Thread safety: every entry point may be called from several host
+ *    threads at once.
+ */
+#ifndef SPA_H
+#define SPA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define SPA_API __attribute__((visibility("default")))
+#else
+#define SPA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum spa_status {
+  SPA_OK = 0,
+  SPA_ERR_INVAL = 1,       /* null pointer, bad size, bad band */
+  SPA_ERR_UNSUPPORTED = 2, /* d, H or alignment outside what the kernels take */
+  SPA_ERR_CUDA = 3,        /* a CUDA runtime/driver call or launch failed */
+  SPA_ERR_TIMEOUT = 4      /* a device-side wait hit its time limit (see spa_device_status) */
+} spa_status_t;
+
+/* Human-readable name of a status code (static string, never NULL). */
+SPA_API const char* spa_status_string(int status);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+SPA_API int spa_version(void);
+
+/*
+ * Balanced Distance Partitioning ("Making Every Head Count", Figure 1
+ * caption): lo[h] = floor(h*N/H), hi[h] = floor((h+1)*N/H), in 64-bit
+ * integer arithmetic.  lo, hi: HOST arrays of H int32 entries, caller-owned.
+ * Requires 1 <= H <= N <= 2^31 - 1, else SPA_ERR_INVAL.
+ */
+SPA_API int spa_band_bounds(int64_t N, int H, int32_t* lo, int32_t* hi);
+
+/*
+ * Forward pass.  For every (b, h, i):
+ *   S_i = { j : 0 <= j <= i, lo_h <= i - j < hi_h },
+ *   lse_i = log(sum_{j in S_i} exp(scale * q_i.k_j))  (natural log),
+ *   o_i   = sum_{j in S_i} exp(scale * q_i.k_j - lse_i) v_j.
+ * q, k, v: inputs [B][H][N][d]; o: output [B][H][N][d]; lse: output [B][H][N].
+ * Bands are the Balanced Distance Partitioning ones (requires H <= N).
+ */
+SPA_API int spa_attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int H, int64_t N, int d, float scale, void* stream);
+
+/*
+ * Same as spa_attn_fwd with explicit per-head bands: lo, hi are HOST arrays of
+ * H int32 entries with 0 <= lo[h] < hi[h] <= N (bands may overlap or leave
+ * gaps; lo = 0, hi = N on every head is dense causal attention per head).
+ */
+SPA_API int spa_attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                    int B, int H, int64_t N, int d, float scale,
+                    const int32_t* lo, const int32_t* hi, void* stream);
+
+/* Bytes of device workspace that spa_attn_bwd needs: 4 * B * H * N (the fp32
+ * row sums D_i = sum_c dout_ic * o_ic).  Returns 0 on bad sizes. */
+SPA_API size_t spa_attn_bwd_workspace_bytes(int B, int H, int64_t N);
+
+/*
+ * Backward pass: gradients of L = sum(o * dout) with respect to q, k, v.
+ * The pages give no backward; it is the derivative of the forward above:
+ *   P_ij  = exp(scale * q_i.k_j - lse_i)   (j in S_i),
+ *   D_i   = sum_c dout_ic o_ic,
+ *   dS_ij = P_ij (dout_i.v_j - D_i),
+ *   dq_i  = scale sum_j dS_ij k_j,  dk_j = scale sum_i dS_ij q_i,
+ *   dv_j  = sum_i P_ij dout_i.
+ * Inputs q, k, v, o (forward output), dout, lse (forward output); outputs dq,
+ * dk, dv [B][H][N][d].  workspace: device buffer of at least
+ * spa_attn_bwd_workspace_bytes(B, H, N) bytes, caller-owned, contents
+ * overwritten.  dq, dk, dv must not alias any input.
+ */
+SPA_API int spa_attn_bwd(const void* q, const void* k, const void* v, const void* o,
+                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                 void* workspace, int B, int H, int64_t N, int d, float scale,
+                 void* stream);
+
+/* Backward with explicit per-head bands (same rules as spa_attn_fwd_ex). */
+SPA_API int spa_attn_bwd_ex(const void* q, const void* k, const void* v, const void* o,
+                    const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                    void* workspace, int B, int H, int64_t N, int d, float scale,
+                    const int32_t* lo, const int32_t* hi, void* stream);
+
+/*
+ * The three steps spa_attn_bwd runs, callable one by one (for example to run
+ * the dk/dv and dq passes on two streams once the first step is done).  Same
+ * tensors and rules as spa_attn_bwd; lo/hi are HOST band arrays or both NULL
+ * for the Balanced Distance Partitioning bands.
+ *  1. spa_attn_bwd_preprocess: workspace[b,h,i] = D_i = sum_c dout_ic o_ic.
+ *  2. spa_attn_bwd_dkdv: dk, dv from q, k, v, dout, lse and D (one CTA per key
+ *     tile, walking the query tiles its band reaches).
+ *  3. spa_attn_bwd_dq:   dq from q, k, v, dout, lse and D (one CTA per query
+ *     tile, walking the same key strip as the forward).
+ * Steps 2 and 3 only read the workspace and may run concurrently.
+ */
+SPA_API int spa_attn_bwd_preprocess(const void* o, const void* dout, void* workspace, int B, int H,
+                                    int64_t N, int d, void* stream);
+SPA_API int spa_attn_bwd_dkdv(const void* q, const void* k, const void* v, const void* dout,
+                              const float* lse, const void* workspace, void* dk, void* dv, int B,
+                              int H, int64_t N, int d, float scale, const int32_t* lo,
+                              const int32_t* hi, void* stream);
+SPA_API int spa_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dout,
+                            const float* lse, const void* workspace, void* dq, int B, int H,
+                            int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi,
+                            void* stream);
+
+/*
+ * Band tile schedule, as the kernels walk it (host evaluation of the same
+ * code the device runs).  Query tile t covers rows [t*Bq, t*Bq + Bq), key
+ * tile u keys [u*Bk, u*Bk + Bk); positions >= N are not permitted.
+ * For each head h and query tile t (index h*nqt + t, nqt = ceil(N/Bq)):
+ *   kt_begin, kt_end: first and last key tile of the diagonal strip, or
+ *   kt_begin = 0, kt_end = -1 when no row of the tile has a permitted key.
+ * tile_class [H][nqt][nkt] (nkt = ceil(N/Bk)): 0 = outside the strip,
+ *   1 = edge (needs the per-element distance predicate), 2 = interior (every
+ *   element permitted, no mask).
+ * For each head h and key tile u (index h*nkt + u):
+ *   qt_begin, qt_end: the query tiles the backward dk/dv pass walks for that
+ *   key tile (qt_end = -1 when none).
+ * All arrays are HOST memory, caller-owned; any of them may be NULL.
+ * 1 <= Bq, Bk <= 4096; bands as in spa_attn_fwd_ex.
+ */
+SPA_API int spa_tile_schedule(int64_t N, int H, const int32_t* lo, const int32_t* hi, int Bq, int Bk,
+                      int32_t* kt_begin, int32_t* kt_end, uint8_t* tile_class,
+                      int32_t* qt_begin, int32_t* qt_end);
+
+/*
+ * The tile_class matrix of spa_tile_schedule computed ON THE DEVICE by the
+ * classification code the kernels inline.  tile_class_dev: DEVICE buffer of
+ * H * nqt * nkt bytes; asynchronous on `stream`.
+ */
+SPA_API int spa_tile_classes_device(int64_t N, int H, const int32_t* lo, const int32_t* hi, int Bq,
+                            int Bk, uint8_t* tile_class_dev, void* stream);
+
+/*
+ * Synchronises `stream` and returns the library's device error word, then
+ * clears it: SPA_OK, or SPA_ERR_TIMEOUT when a kernel gave up on a wait (the
+ * kernel then wrote incomplete outputs and released its tensor memory).
+ */
+SPA_API int spa_device_status(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SPA_H */

@@ -1,0 +1,151 @@
+"""CPU-side checks of the C-ABI library: it loads, exports every symbol that
+include/spa.h declares, and its host code (bands, tile schedule, argument
+checks) is right.  No compute call reaches a GPU here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle
+from head_partitioned_distance_b200 import spa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    src = open(os.path.join(ROOT, "include", "spa.h")).read()
+    return set(re.findall(r"SPA_API\s+[\w\s\*]+?\b(spa_\w+)\s*\(", src))
+
+
+def test_header_declares_the_abi():
+    names = _declared_symbols()
+    for must in ("spa_band_bounds", "spa_attn_fwd", "spa_attn_bwd", "spa_attn_fwd_ex",
+                 "spa_attn_bwd_ex", "spa_attn_bwd_workspace_bytes", "spa_tile_schedule",
+                 "spa_device_status", "spa_status_string"):
+        assert must in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = ctypes.CDLL(spa.LIB_PATH)
+    for name in _declared_symbols():
+        assert hasattr(lib, name), name
+    # and the binding marshals exactly those
+    assert set(spa.EXPORTS) == _declared_symbols()
+
+
+def test_status_strings_and_version():
+    for s in range(5):
+        assert spa.spa_status_string(s).startswith("SPA_")
+    assert spa.spa_version() >= 100
+
+
+def test_band_bounds_bit_exact_against_oracle():
+    for N in range(1, 130):
+        for H in range(1, N + 1):
+            lo, hi = spa.spa_band_bounds(N, H)
+            olo, ohi = oracle.bands(N, H)
+            assert lo == olo.tolist() and hi == ohi.tolist()
+    for N, H in [(4096, 16), (8192, 32), (32768, 32), (30001, 32), (1001, 8), (1000, 8),
+                 (2 ** 31 - 1, 256), (2 ** 31 - 1, 7)]:
+        lo, hi = spa.spa_band_bounds(N, H)
+        olo, ohi = oracle.bands(N, H)
+        assert lo == olo.tolist() and hi == ohi.tolist()
+
+
+def test_band_bounds_rejects_bad_requests():
+    for N, H in [(0, 1), (3, 4), (5, 0), (2 ** 31, 2)]:
+        with pytest.raises(spa.SpaError) as e:
+            spa.spa_band_bounds(N, H)
+        assert e.value.status == spa.SPA_ERR_INVAL
+
+
+# Tile sizes the kernels use: forward (128, 128), dK/dV pass (64 queries x
+# 128 keys), dQ pass (128 queries x 64 keys); plus odd sizes.
+TILE_CASES = [
+    (256, 4, 128, 128), (256, 4, 64, 128), (256, 4, 128, 64),
+    (1024, 8, 128, 128), (1000, 8, 128, 128), (1001, 8, 64, 128), (1001, 8, 128, 64),
+    (777, 5, 128, 128), (256, 256, 128, 128), (255, 200, 64, 128), (130, 2, 128, 128), (1, 1, 128, 128),
+    (129, 3, 128, 128), (97, 7, 16, 8), (4096, 16, 128, 128), (4096, 16, 64, 128),
+]
+
+
+@pytest.mark.parametrize("N,H,Bq,Bk", TILE_CASES)
+def test_tile_schedule_bit_exact_against_brute_force(N, H, Bq, Bk):
+    sch = spa.spa_tile_schedule(N, H, Bq, Bk)
+    lo, hi = oracle.bands(N, H)
+    want = oracle.tile_classes(N, lo, hi, Bq, Bk)
+    np.testing.assert_array_equal(sch["tile_class"], want)
+    nqt, nkt = want.shape[1:]
+    for h in range(H):
+        for t in range(nqt):
+            us = np.nonzero(want[h, t])[0]
+            if len(us) == 0:
+                assert sch["kt_end"][h, t] < sch["kt_begin"][h, t]
+            else:
+                # the strip is exactly the contiguous run of non-empty tiles
+                assert (sch["kt_begin"][h, t], sch["kt_end"][h, t]) == (us[0], us[-1])
+                assert len(us) == us[-1] - us[0] + 1
+        for u in range(nkt):
+            ts = np.nonzero(want[h, :, u])[0]
+            if len(ts) == 0:
+                assert sch["qt_end"][h, u] < sch["qt_begin"][h, u]
+            else:
+                assert (sch["qt_begin"][h, u], sch["qt_end"][h, u]) == (ts[0], ts[-1])
+                assert len(ts) == ts[-1] - ts[0] + 1
+
+
+@pytest.mark.parametrize("N,H,h_list", [(8192, 32, [0, 1, 15, 31]), (30001, 32, [0, 7, 31]),
+                                        (32768, 32, [0, 31])])
+def test_tile_schedule_large_heads_against_brute_force(N, H, h_list):
+    # brute force over whole tiles is quadratic in N; check selected heads
+    lo, hi = oracle.bands(N, H)
+    sch = spa.spa_tile_schedule(N, H, 128, 128)
+    for h in h_list:
+        want = oracle.tile_classes(N, lo[h:h + 1], hi[h:h + 1], 128, 128)
+        np.testing.assert_array_equal(sch["tile_class"][h], want[0])
+
+
+def test_tile_schedule_explicit_bands():
+    N = 500
+    lo = [0, 0, 37, 100, 499]
+    hi = [500, 1, 250, 101, 500]
+    sch = spa.spa_tile_schedule(N, 5, 128, 64, lo, hi)
+    want = oracle.tile_classes(N, lo, hi, 128, 64)
+    np.testing.assert_array_equal(sch["tile_class"], want)
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_entry_points_reject_bad_arguments_before_any_launch():
+    L = spa._lib
+    p = _fake(1 << 20)  # never dereferenced: every call below fails its checks first
+    f = lambda *a: L.spa_attn_fwd(p, p, p, p, p, *a, None)
+    assert f(1, 4, 256, 96, 0.1) == spa.SPA_ERR_UNSUPPORTED      # d
+    assert f(1, 300, 400, 64, 0.1) == spa.SPA_ERR_UNSUPPORTED    # H > 256
+    assert f(1, 8, 4, 64, 0.1) == spa.SPA_ERR_INVAL              # H > N
+    assert f(0, 4, 256, 64, 0.1) == spa.SPA_ERR_INVAL            # B
+    assert f(1, 4, 0, 64, 0.1) == spa.SPA_ERR_INVAL              # N
+    assert f(1, 4, 2 ** 31, 64, 0.1) == spa.SPA_ERR_INVAL        # N too large
+    assert f(1, 4, 256, 64, float("nan")) == spa.SPA_ERR_INVAL   # scale
+    assert L.spa_attn_fwd(p, None, p, p, p, 1, 4, 256, 64, 0.1, None) == spa.SPA_ERR_INVAL
+    odd = _fake((1 << 20) + 8)
+    assert L.spa_attn_fwd(p, p, odd, p, p, 1, 4, 256, 64, 0.1, None) == spa.SPA_ERR_UNSUPPORTED
+    # explicit bands: empty, reversed, out of range
+    for lo, hi in (([0, 5], [0, 6]), ([3, 1], [2, 9]), ([0, 0], [8, 300])):
+        a = (ctypes.c_int32 * 2)(*lo)
+        b = (ctypes.c_int32 * 2)(*hi)
+        assert L.spa_attn_fwd_ex(p, p, p, p, p, 1, 2, 256, 64, 0.1, a, b, None) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_fwd_ex(p, p, p, p, p, 1, 2, 256, 64, 0.1, None, None, None) == spa.SPA_ERR_INVAL
+    g = lambda *a: L.spa_attn_bwd(p, p, p, p, p, p, p, p, p, p, *a, None)
+    assert g(1, 4, 256, 80, 0.1) == spa.SPA_ERR_UNSUPPORTED
+    assert g(1, 8, 4, 64, 0.1) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_bwd(p, p, p, p, p, p, p, p, p, None, 1, 4, 256, 64, 0.1, None) == spa.SPA_ERR_INVAL
+
+
+def test_workspace_size():
+    assert spa.spa_attn_bwd_workspace_bytes(4, 32, 8192) == 4 * 32 * 8192 * 4
+    assert spa.spa_attn_bwd_workspace_bytes(0, 1, 1) == 0

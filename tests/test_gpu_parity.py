@@ -1,0 +1,227 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 CPU oracle
+on the same seeded bf16 inputs.
+
+Tolerances (fp64 oracle as the truth):
+  O                      max |o - o_ref|                      <= 2e-2
+  lse (finite rows)      max |lse - lse_ref|                  <= 1e-3
+  lse (empty rows)       exactly -inf where the oracle has -inf
+  dq, dk, dv (each)      max |g - g_ref| / max |g_ref|        <= 5e-2
+  NaN anywhere           failure
+  tile classes           bit-exact
+Small shapes compare every element; the full-size workloads compare sampled
+rows that the oracle computes one by one (every head's first/last rows and
+band edges, plus random rows)."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_partitioned_distance_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL, GRAD_TOL = 2e-2, 1e-3, 5e-2
+
+
+@pytest.fixture(scope="module")
+def spa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from head_partitioned_distance_b200 import spa as mod
+    return mod
+
+
+def _f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def _gpu_run(spa, q, k, v, do, scale, lo=None, hi=None, backward=True):
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = spa.attention_forward(qd, kd, vd, scale, lo, hi)
+    out = {"o": o, "lse": lse}
+    if backward:
+        dq, dk, dv = spa.attention_backward(qd, kd, vd, o, dod, lse, scale, lo, hi)
+        out.update(dq=dq, dk=dk, dv=dv)
+    torch.cuda.synchronize()
+    assert spa.spa_device_status() == spa.SPA_OK
+    return {k_: _f64(v_) for k_, v_ in out.items()}
+
+
+def _check_lse(lse, ref):
+    neg = np.isneginf(ref)
+    assert np.array_equal(np.isneginf(lse), neg), "empty-band rows must be exactly -inf"
+    if (~neg).any():
+        assert np.abs(lse[~neg] - ref[~neg]).max() <= LSE_TOL
+
+
+def _check_grad(g, ref, name):
+    assert not np.isnan(g).any(), name
+    denom = np.abs(ref).max()
+    err = np.abs(g - ref).max()
+    if denom == 0:
+        assert err == 0, name
+    else:
+        assert err / denom <= GRAD_TOL, (name, err, denom)
+
+
+def _full_check(spa, q, k, v, do, scale, lo=None, hi=None):
+    got = _gpu_run(spa, q, k, v, do, scale, lo, hi)
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    lo_o = None if lo is None else np.array(lo)
+    hi_o = None if hi is None else np.array(hi)
+    o_ref, lse_ref = oracle.spa_fwd(qf, kf, vf, scale, lo_o, hi_o)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert not np.isnan(got[name]).any(), name
+    assert np.abs(got["o"] - o_ref).max() <= O_TOL
+    _check_lse(got["lse"], lse_ref)
+    dq, dk, dv = oracle.spa_bwd(qf, kf, vf, dof, scale, lo_o, hi_o)
+    _check_grad(got["dq"], dq, "dq")
+    _check_grad(got["dk"], dk, "dk")
+    _check_grad(got["dv"], dv, "dv")
+    return got
+
+
+SMALL_WORKLOADS = ["b1_h4_n256_d64", "b1_h8_n1024_d64", "b1_h8_n1000_d64", "b1_h8_n1001_d64"]
+
+
+@pytest.mark.parametrize("name", SMALL_WORKLOADS)
+def test_small_workloads_every_element(spa, name):
+    w = synth.WORKLOADS[name]
+    q, k, v, do = synth.workload_inputs(w)
+    _full_check(spa, q, k, v, do, w.scale)
+
+
+# shapes that span several tiles, ragged tails, width-1 bands, one head,
+# both head dims, batches > 1
+EDGE_SHAPES = [
+    (1, 1, 1, 64), (1, 1, 1, 128), (1, 1, 200, 64), (2, 1, 384, 128), (1, 3, 129, 128),
+    (1, 4, 127, 64), (2, 5, 777, 128), (1, 64, 64, 64), (1, 256, 256, 64), (1, 2, 130, 128),
+    (3, 7, 500, 64), (1, 8, 2048, 128),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d", EDGE_SHAPES)
+def test_edge_shapes_every_element(spa, B, H, N, d):
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=7 + N + H)
+    _full_check(spa, q, k, v, do, 1 / math.sqrt(d))
+
+
+@pytest.mark.parametrize("kind", ["full", "first_half", "shared_window", "odd"])
+def test_explicit_bands(spa, kind):
+    B, H, N, d = 1, 4, 600, 64
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=99)
+    lo, hi = oracle.bands(N, H)
+    if kind == "full":           # dense causal attention on every head
+        lo, hi = [0] * H, [N] * H
+    elif kind == "first_half":   # first half of each band
+        hi = [int(a + max((b - a) // 2, 1)) for a, b in zip(lo, hi)]
+        lo = [int(a) for a in lo]
+    elif kind == "shared_window":  # every head the same local window
+        lo, hi = [0] * H, [96] * H
+    else:
+        lo, hi = [0, 3, 257, 599], [1, 400, 300, 600]
+    _full_check(spa, q, k, v, do, 0.125, [int(x) for x in lo], [int(x) for x in hi])
+
+
+def test_dense_causal_equals_torch_sdpa_in_fp32(spa):
+    # an independent library path: full bands on every head is causal attention
+    B, H, N, d = 2, 4, 512, 128
+    q, k, v, _ = synth.make_inputs(B, H, N, d, seed=5)
+    got = _gpu_run(spa, q, k, v, q, 1 / math.sqrt(d), [0] * H, [N] * H, backward=False)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        q.float(), k.float(), v.float(), is_causal=True).double().numpy()
+    assert np.abs(got["o"] - ref).max() <= O_TOL
+
+
+def test_deterministic(spa):
+    w = synth.WORKLOADS["b1_h8_n1001_d64"]
+    q, k, v, do = synth.workload_inputs(w)
+    a = _gpu_run(spa, q, k, v, do, w.scale)
+    b = _gpu_run(spa, q, k, v, do, w.scale)
+    for name in a:
+        assert np.array_equal(a[name], b[name], equal_nan=True), name
+
+
+def test_autograd_function(spa):
+    B, H, N, d = 1, 4, 300, 64
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=3)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (t.to(dev).requires_grad_() for t in (q, k, v))
+    o = spa.spattention(qd, kd, vd)
+    o.backward(do.to(dev))
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    o_ref, _ = oracle.spa_fwd(qf, kf, vf, d ** -0.5)
+    assert np.abs(_f64(o) - o_ref).max() <= O_TOL
+    for g, ref, n in zip((qd.grad, kd.grad, vd.grad), oracle.spa_bwd(qf, kf, vf, dof, d ** -0.5),
+                         "qkv"):
+        _check_grad(_f64(g), ref, n)
+
+
+@pytest.mark.parametrize("N,H,Bq,Bk", [(1024, 8, 128, 128), (1001, 8, 64, 128), (1001, 8, 128, 64),
+                                       (4096, 16, 128, 128), (97, 7, 16, 8)])
+def test_tile_classes_on_device_bit_exact(spa, N, H, Bq, Bk):
+    nqt, nkt = -(-N // Bq), -(-N // Bk)
+    out = torch.full((H, nqt, nkt), 255, dtype=torch.uint8, device="cuda:0")
+    spa.spa_tile_classes_device(N, H, Bq, Bk, out)
+    lo, hi = oracle.bands(N, H)
+    np.testing.assert_array_equal(out.cpu().numpy(), oracle.tile_classes(N, lo, hi, Bq, Bk))
+
+
+# ---------------------------------------------------------------------------
+# full-size workloads, in the launch configuration the benchmark times:
+# sampled rows against the oracle's one-row entry points
+# ---------------------------------------------------------------------------
+LARGE = ["b8_h16_n4096_d128", "b4_h32_n8192_d128", "b1_h32_n32768_d128", "b1_h32_n30001_d128"]
+
+
+def _sampled_check(spa, w, n_random, n_key_rows):
+    q, k, v, do = synth.workload_inputs(w)
+    got = _gpu_run(spa, q, k, v, do, w.scale)
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert not np.isnan(got[name]).any(), name
+    B, H, N, d = w.B, w.H, w.N, w.d
+    lo, hi = oracle.bands(N, H)
+    per_head = [[int(lo[h]) - 1, int(lo[h]), int(lo[h]) + 1, int(lo[h]) + 127, int(lo[h]) + 128]
+                for h in range(H)]
+    rows = synth.sample_rows(B, H, N, n_random, seed=w.seed, per_head=per_head)
+    g = torch.Generator().manual_seed(w.seed + 1)
+    key_rows = sorted(set(torch.randint(0, B * H * N, (n_key_rows,), generator=g).tolist()
+                          + [N - 1, (H - 1) * N + N - 1 - int(lo[H - 1])]))
+    flat = lambda x: x.reshape(B * H * N, -1)
+    ok = {"o": [], "dq": [], "dk": [], "dv": []}
+    refs = {"o": [], "dq": [], "dk": [], "dv": []}
+    lse_got, lse_ref = [], []
+    # group rows by (b, h) and hand the oracle one head at a time
+    for bh in sorted(set(r // N for r in rows) | set(r // N for r in key_rows)):
+        h = bh % H
+        sl = lambda t: _f64(t.reshape(B * H, N, d)[bh])[None, None]
+        qh, kh, vh, doh = sl(q), sl(k), sl(v), sl(do)
+        blo, bhi = lo[h:h + 1], hi[h:h + 1]
+        rs = [r % N for r in rows if r // N == bh]
+        if rs:
+            o_r, l_r = oracle.spa_fwd_rows(qh, kh, vh, w.scale, rs, blo, bhi)
+            dq_r = oracle.spa_bwd_dq_rows(qh, kh, vh, doh, w.scale, rs, blo, bhi)
+            idx = [bh * N + i for i in rs]
+            ok["o"].append(flat(got["o"])[idx]); refs["o"].append(o_r)
+            ok["dq"].append(flat(got["dq"])[idx]); refs["dq"].append(dq_r)
+            lse_got.append(got["lse"].reshape(-1)[idx]); lse_ref.append(l_r)
+        ks = [r % N for r in key_rows if r // N == bh]
+        if ks:
+            dk_r, dv_r = oracle.spa_bwd_dkdv_rows(qh, kh, vh, doh, w.scale, ks, blo, bhi)
+            idx = [bh * N + j for j in ks]
+            ok["dk"].append(flat(got["dk"])[idx]); refs["dk"].append(dk_r)
+            ok["dv"].append(flat(got["dv"])[idx]); refs["dv"].append(dv_r)
+    cat = lambda xs: np.concatenate(xs, axis=0)
+    assert np.abs(cat(ok["o"]) - cat(refs["o"])).max() <= O_TOL
+    _check_lse(np.concatenate(lse_got), np.concatenate(lse_ref))
+    for name in ("dq", "dk", "dv"):
+        _check_grad(cat(ok[name]), cat(refs[name]), name)
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_full_size_workloads_sampled_rows(spa, name):
+    w = synth.WORKLOADS[name]
+    _sampled_check(spa, w, n_random=48, n_key_rows=12)
