@@ -57,12 +57,18 @@ def _check_lse(lse, ref):
         assert np.abs(lse[~neg] - ref[~neg]).max() <= LSE_TOL
 
 
+# When the exact gradient is identically zero (a softmax over one key: dS =
+# P (dO.v - D) = 0), the relative error is undefined; the bf16 rounding of o
+# inside D leaves a residue of order 1e-7 * |dO| |v|, checked absolutely.
+ZERO_GRAD_ABS_TOL = 1e-4
+
+
 def _check_grad(g, ref, name):
     assert not np.isnan(g).any(), name
     denom = np.abs(ref).max()
     err = np.abs(g - ref).max()
     if denom == 0:
-        assert err == 0, name
+        assert err <= ZERO_GRAD_ABS_TOL, (name, err)
     else:
         assert err / denom <= GRAD_TOL, (name, err, denom)
 
