@@ -236,6 +236,41 @@ __global__ void tile_class_kernel(int64_t N, int H, int Bq, int Bk, int nqt, int
 
 }  // namespace
 
+// ---------------------------------------------------------------------------
+// Scratch for spa_attn_bwd_noalloc: the fp32 row sums D_i of the backward, in
+// a file-scope device array so that the call allocates nothing.  Every GPU
+// that loads this library holds these SPA_NOALLOC_MAX_ROWS * 4 bytes (4 MiB)
+// until the process exits.  Host code cannot use the array's name as a device
+// address; noalloc_scratch() looks the address up once per device.
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) float g_spa_noalloc_delta[SPA_NOALLOC_MAX_ROWS];
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of g_spa_noalloc_delta on the current device.  The first
+// call on a device resolves it with cudaGetSymbolAddress (that device being
+// current) and caches it; later calls only read the cache.
+int noalloc_scratch(void** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPA_ERR_CUDA;
+  if (dev < 0 || dev >= kMaxDevices) return SPA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_ptr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_spa_noalloc_delta) != cudaSuccess || p == nullptr)
+      return SPA_ERR_CUDA;
+    g_noalloc_ptr[dev] = p;
+  }
+  *out = g_noalloc_ptr[dev];
+  return SPA_OK;
+}
+
+}  // namespace
+
 extern "C" {
 
 const char* spa_status_string(int status) {
@@ -352,6 +387,20 @@ int spa_tile_classes_device(int64_t N, int H, const int32_t* lo, const int32_t* 
   tile_class_kernel<<<148 * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(N, H, Bq, Bk, nqt, nkt, bands,
                                                                             tile_class_dev);
   return launch_status();
+}
+
+int spa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                         const void* dout, const float* lse, void* dq, void* dk, void* dv, int B,
+                         int H, int64_t N, int d, float scale, void* stream) {
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  if ((int64_t)B * H * N > (int64_t)SPA_NOALLOC_MAX_ROWS) return SPA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  if ((st = noalloc_scratch(&scratch))) return st;
+  // The preprocess step overwrites D for every row before the two passes read
+  // it, so the scratch needs no clearing between calls.
+  return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, scratch, B, H, N, d, scale, nullptr, nullptr,
+                   stream, kStepAll);
 }
 
 int spa_device_status(void* stream) {

@@ -44,6 +44,7 @@ EXPORTS = {
     "spa_attn_bwd_preprocess": ([_vp, _vp, _vp, _int, _int, _i64, _int, _vp], _int),
     "spa_attn_bwd_dkdv": ([_vp] * 8 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_dq": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
+    "spa_attn_bwd_noalloc": ([_vp] * 9 + [_int, _int, _i64, _int, _f32, _vp], _int),
     "spa_tile_schedule": ([_i64, _int, _i32p, _i32p, _int, _int, _i32p, _i32p, _u8p, _i32p, _i32p],
                           _int),
     "spa_tile_classes_device": ([_i64, _int, _i32p, _i32p, _int, _int, _vp, _vp], _int),
@@ -150,6 +151,26 @@ def spa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, scale: float, lo=
     else:
         _check(_lib.spa_attn_bwd_ex(*ptrs, B, H, N, d, scale, _i32(lo), _i32(hi), s),
                "spa_attn_bwd_ex")
+    return dq, dk, dv
+
+
+SPA_NOALLOC_MAX_ROWS = 1 << 20
+
+
+def spa_attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, scale: float, stream=None):
+    """Backward without a workspace argument and without any allocation, for
+    callers that cannot call cudaMalloc (see spa_attn_bwd_noalloc in spa.h):
+    the row sums D go to a library-owned device array of
+    SPA_NOALLOC_MAX_ROWS floats, shared by every call -- calls that overlap on
+    the GPU race on it.  B * H * N must not exceed SPA_NOALLOC_MAX_ROWS."""
+    B, H, N, d = _dims(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    _need(lse, (B, H, N), torch.float32, "lse")
+    ptrs = [t.data_ptr() for t in (q, k, v, o, dout, lse, dq, dk, dv)]
+    _check(_lib.spa_attn_bwd_noalloc(*ptrs, B, H, N, d, scale, _stream_ptr(stream)),
+           "spa_attn_bwd_noalloc")
     return dq, dk, dv
 
 

@@ -16,7 +16,9 @@
  *  - Tensors q, k, v, o, dout, dq, dk, dv are bf16, layout [B][H][N][d]
  *    row-major contiguous, in DEVICE memory, 16-byte aligned.  lse and the
  *    backward workspace are fp32 [B][H][N], device memory, 4-byte aligned.
- *  - The caller owns every buffer; the library allocates no device memory.
+ *  - The caller owns every buffer; no call allocates device memory (the
+ *    one library-owned buffer is the static scratch array of
+ *    spa_attn_bwd_noalloc, below).
  *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
  *    NULL = the legacy default stream) and never synchronise the host, except
  *    spa_device_status.
@@ -140,6 +142,32 @@ SPA_API int spa_attn_bwd_dq(const void* q, const void* k, const void* v, const v
                             const float* lse, const void* workspace, void* dq, int B, int H,
                             int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi,
                             void* stream);
+
+/*
+ * Backward pass that allocates nothing and takes no workspace argument.
+ * The paper has no counterpart: this entry point exists for callers that
+ * cannot call cudaMalloc -- for example a plugin running inside a host
+ * framework that owns all device memory through its own pool allocator (a
+ * raw cudaMalloc behind its back would escape its budget), or a caller that
+ * must not risk the device-wide synchronisation cudaMalloc/cudaFree may
+ * cause.  Same inputs, outputs and results as spa_attn_bwd with the Balanced
+ * Distance Partitioning bands.
+ *  - Scratch: the row sums D live in a library-owned, file-scope device array
+ *    of SPA_NOALLOC_MAX_ROWS floats (4 MiB), held by every GPU that loads the
+ *    library until the process exits.  B * H * N above SPA_NOALLOC_MAX_ROWS is
+ *    rejected with SPA_ERR_UNSUPPORTED before anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current) and caches it; make that
+ *    first call before any stream capture.
+ *  - All calls share the one array and it keeps the last call's contents
+ *    (nothing in it needs to start at zero: each call rewrites the rows it
+ *    uses before reading them).  Calls whose work overlaps on the GPU -- two
+ *    streams, or two host threads -- race on it; serialise them.
+ */
+#define SPA_NOALLOC_MAX_ROWS (1 << 20)
+SPA_API int spa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void* o,
+                                 const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                 int B, int H, int64_t N, int d, float scale, void* stream);
 
 /*
  * Band tile schedule, as the kernels walk it (host evaluation of the same
