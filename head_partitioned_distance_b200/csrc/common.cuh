@@ -27,6 +27,9 @@ struct AttnParams {
   int64_t N;
   float scale;        // multiplies q.k
   float scale_log2;   // scale * log2(e): scores in base-2 units
+  // persistent forward: units (non-empty 256-row blocks) and all-empty blocks per batch
+  int units_per_batch;
+  int fills_per_batch;
   // forward: lse is written; backward: lse (read) and delta (workspace)
   float* lse;
   float* delta;

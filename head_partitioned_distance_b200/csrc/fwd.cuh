@@ -1,16 +1,24 @@
 // fwd.cuh -- band-sparse attention forward for sm_100a.
 //
-// One CTA per unit (b, h, query tile of 128 rows).  The unit walks the
-// diagonal strip of 128-key tiles its band needs (sched.cuh), flash style:
-//   S = Q K^T         tcgen05.mma, bf16 x bf16 -> fp32 in TMEM (double-buffered)
-//   P = exp(S - m)    softmax warps, one thread per row, fp32 online softmax,
-//                     per-element distance predicate on edge tiles only
-//   O += P V          tcgen05.mma, P as bf16 from 128B-swizzled shared memory
-// then O / l -> bf16 through shared memory and a TMA store; lse = m + ln l.
+// Persistent grid (one CTA per SM).  A unit is (b, h, 256 query rows), split
+// into two 128-row Q tiles that two softmax warpgroups process in ping-pong:
+// while one warpgroup turns its scores into probabilities, the tensor core
+// works on the other tile.  Each tile walks the diagonal strip of 128-key
+// tiles its band needs (sched.cuh); the unit streams the union of the two
+// strips through a 2-stage K/V ring:
+//   S_t = Q_t K^T   tcgen05.mma, both operands from 128B-swizzled smem, fp32 in TMEM
+//   P_t = exp2(S_t - m)   softmax warpgroup t, one thread per row; the
+//                   distance predicate only on edge tiles; P_t written back
+//                   as bf16 over the first half of S_t in TMEM
+//   O_t += P_t V    tcgen05.mma with A = P_t read from TMEM, B = V from smem
+// The running max is only moved (and O_t rescaled) when it grows by more than
+// 2^8, so probabilities stay <= 256 and most tiles skip the rescale.  O and
+// lse are written straight from registers; rows that precede their band get
+// o = 0 and lse = -inf.
 //
-// Warp roles (192 threads): warps 0-3 softmax + epilogue (thread r owns row
-// r, which is TMEM lane r), warp 4 TMA producer, warp 5 MMA issuer and TMEM
-// owner.  K/V tiles stream through a 2-stage ring; every wait is bounded.
+// Warp roles (320 threads): warps 0-3 tile 0, warps 4-7 tile 1 (thread r of a
+// warpgroup owns row r = TMEM lane r), warp 8 TMA producer, warp 9 MMA issuer
+// and TMEM owner.  Every wait is bounded (common.cuh).
 //
 // Softmax restricted to a permitted set: "Story of Attention -- Part 4",
 // section 1 (Sparse-Attention equation); bands: "Making Every Head Count",
@@ -23,93 +31,124 @@ namespace spa {
 
 template <int D>
 struct FwdCfg {
-  static constexpr int BQ = 128;
-  static constexpr int BK = 128;
-  static constexpr int NS = 2;         // K/V ring stages
-  static constexpr int DB = D / 64;    // 64-column (128-byte) blocks per row
+  static constexpr int BQ = 128;        // rows per Q tile (one warpgroup)
+  static constexpr int TILES = 2;       // Q tiles per unit
+  static constexpr int BU = BQ * TILES; // rows per unit
+  static constexpr int BK = 128;        // keys per K/V tile
+  static constexpr int NS = 2;          // K/V ring stages
+  static constexpr int DB = D / 64;     // 64-column (128-byte) blocks per row
   static constexpr uint32_t Q_BYTES = BQ * D * 2;
   static constexpr uint32_t KV_BYTES = BK * D * 2;
-  static constexpr uint32_t P_BYTES = BQ * BK * 2;
   static constexpr uint32_t OFF_Q = 0;
-  static constexpr uint32_t OFF_K = OFF_Q + Q_BYTES;
+  static constexpr uint32_t OFF_K = OFF_Q + TILES * Q_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + NS * KV_BYTES;
-  static constexpr uint32_t OFF_P = OFF_V + NS * KV_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_P + P_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_V + NS * KV_BYTES;
   // + alignment slack; at least 116 KB so that one CTA (and its 512 TMEM
   // columns) owns an SM even for d = 64
   static constexpr uint32_t SMEM_BYTES =
       (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
-  static constexpr int NTHREADS = 192;
+  static constexpr int NTHREADS = 320;
   static constexpr uint32_t TMEM_COLS = 512;
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_O = 256;
+  // tile t: S_t (and P_t over its first 64 columns) at t*256, O_t at t*256 + 128
+  __host__ __device__ static constexpr uint32_t tm_s(int t) { return (uint32_t)t * 256u; }
+  __host__ __device__ static constexpr uint32_t tm_o(int t) { return (uint32_t)t * 256u + 128u; }
   static_assert(D == 64 || D == 128, "head dim");
 };
 
 struct FwdBars {
-  uint64_t q_full;
+  uint64_t q_full[2], q_empty[2];
   uint64_t k_full[2], v_full[2], kv_empty[2];
-  uint64_t s_full[2], s_free[2];
-  uint64_t p_full, o_done, drain;
+  uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
+  uint64_t drain;
   uint32_t tmem_base;
   int abort;
 };
 
+// One unit of the forward: rows [i0, i0 + 256) of head (b, h).
+struct FwdUnit {
+  int bh;
+  int32_t lo, hi;
+  int64_t i0;
+  int a[2], b[2];     // key-tile strip of each Q tile (b < a: tile inactive)
+  bool act[2];
+  int u0, u1;         // union of the active strips
+};
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__device__ __forceinline__ FwdUnit fwd_decode(int u, const AttnParams& p) {
+  using C = FwdCfg<D>;
+  FwdUnit U;
+  const int nblk = (int)((p.N + C::BU - 1) / C::BU);
+  const int b = u / p.units_per_batch;
+  int r = u % p.units_per_batch;
+  int h = 0;
+  for (; h < p.H; ++h) {
+    const int first = p.lo[h] / C::BU;
+    const int cnt = nblk - first;
+    if (r < cnt) break;
+    r -= cnt;
+  }
+  U.bh = b * p.H + h;
+  U.lo = p.lo[h];
+  U.hi = p.hi[h];
+  U.i0 = (int64_t)(p.lo[h] / C::BU + r) * C::BU;
+  U.u0 = 1 << 30;
+  U.u1 = -1;
+  for (int t = 0; t < 2; ++t) {
+    const int64_t it0 = U.i0 + (int64_t)t * C::BQ;
+    Strip s{0, -1};
+    if (it0 < p.N) s = key_strip(p.N, U.lo, U.hi, it0, C::BQ, C::BK);
+    U.a[t] = s.begin;
+    U.b[t] = s.end;
+    U.act[t] = s.end >= s.begin;
+    if (U.act[t]) {
+      U.u0 = min(U.u0, s.begin);
+      U.u1 = max(U.u1, s.end);
+    }
+  }
+  return U;
+}
+
+template <int D>
+__global__ void __launch_bounds__(320, 1)
     spa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_o,
-                   const __grid_constant__ AttnParams p) {
+                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
   using C = FwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   FwdBars* bars = reinterpret_cast<FwdBars*>(smem + C::OFF_BAR);
-
-  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int bh = b * p.H + h;
-  const int64_t N = p.N;
-  const int32_t lo = p.lo[h], hi = p.hi[h];
-  const int64_t i0 = (int64_t)t * C::BQ;
-  const Strip strip = key_strip(N, lo, hi, i0, C::BQ, C::BK);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t rows_here = min64(i0 + C::BQ, N) - i0;
-
-  if (strip.end < strip.begin) {
-    // No row of this tile reaches its band: o = 0, lse = -inf.
-    zero_rows_bf16(static_cast<uint16_t*>(p.o) + ((int64_t)bh * N + i0) * D, rows_here, D);
-    for (int r = threadIdx.x; r < rows_here; r += blockDim.x) p.lse[(int64_t)bh * N + i0 + r] = -INFINITY;
-    return;
-  }
-  const int nkt = strip.end - strip.begin + 1;
+  const int64_t N = p.N;
+  const int num_units = p.B * p.units_per_batch;
 
   const uint32_t sQ = ptx::smem_u32(smem + C::OFF_Q);
   const uint32_t sK = ptx::smem_u32(smem + C::OFF_K);
   const uint32_t sV = ptx::smem_u32(smem + C::OFF_V);
-  const uint32_t sP = ptx::smem_u32(smem + C::OFF_P);
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&bars->q_full, 1);
-    for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(&bars->k_full[s], 1);
-      ptx::mbar_init(&bars->v_full[s], 1);
-      ptx::mbar_init(&bars->kv_empty[s], 1);
-      ptx::mbar_init(&bars->s_full[s], 1);
-      ptx::mbar_init(&bars->s_free[s], 128);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&bars->q_full[i], 1);
+      ptx::mbar_init(&bars->q_empty[i], 1);
+      ptx::mbar_init(&bars->k_full[i], 1);
+      ptx::mbar_init(&bars->v_full[i], 1);
+      ptx::mbar_init(&bars->kv_empty[i], 1);
+      ptx::mbar_init(&bars->s_full[i], 1);
+      ptx::mbar_init(&bars->p_full[i], 128);
+      ptx::mbar_init(&bars->o_done[i], 1);
+      ptx::mbar_init(&bars->o_free[i], 128);
     }
-    ptx::mbar_init(&bars->p_full, 128);
-    ptx::mbar_init(&bars->o_done, 1);
     ptx::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
+  if (warp == 8 && lane == 0) {
     ptx::prefetch_tmap(&tm_q);
     ptx::prefetch_tmap(&tm_k);
     ptx::prefetch_tmap(&tm_v);
-    ptx::prefetch_tmap(&tm_o);
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -117,30 +156,43 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      ptx::mbar_arrive_expect_tx(&bars->q_full, C::Q_BYTES);
-      for (int c = 0; c < C::DB; ++c)
-        ptx::tma_load_3d(smem + C::OFF_Q + c * (C::BQ * 128), &tm_q, &bars->q_full, c * 64, (int)i0, bh);
-      int armed[2] = {0, 0};
-      for (int it = 0; it < nkt; ++it) {
-        const int s = it % C::NS;
-        const uint32_t n = it / C::NS;
-        if (!bar_wait(&bars->kv_empty[s], (n & 1) ^ 1, abort_flag)) break;
-        const int j0 = (strip.begin + it) * C::BK;
-        uint8_t* kdst = smem + C::OFF_K + s * C::KV_BYTES;
-        uint8_t* vdst = smem + C::OFF_V + s * C::KV_BYTES;
-        ptx::mbar_arrive_expect_tx(&bars->k_full[s], C::KV_BYTES);
-        for (int c = 0; c < C::DB; ++c)
-          ptx::tma_load_3d(kdst + c * (C::BK * 128), &tm_k, &bars->k_full[s], c * 64, j0, bh);
-        ptx::mbar_arrive_expect_tx(&bars->v_full[s], C::KV_BYTES);
-        for (int c = 0; c < C::DB; ++c)
-          ptx::tma_load_3d(vdst + c * (C::BK * 128), &tm_v, &bars->v_full[s], c * 64, j0, bh);
-        armed[s]++;
+      int nq[2] = {0, 0}, armed[2] = {0, 0};
+      int g = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const FwdUnit U = fwd_decode<D>(u, p);
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (!U.act[t]) continue;
+          ok = bar_wait(&bars->q_empty[t], (nq[t] & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          ++nq[t];
+          ptx::mbar_arrive_expect_tx(&bars->q_full[t], C::Q_BYTES);
+          for (int c = 0; c < C::DB; ++c)
+            ptx::tma_load_3d(smem + C::OFF_Q + t * C::Q_BYTES + c * (C::BQ * 128), &tm_q, &bars->q_full[t],
+                             c * 64, (int)(U.i0 + t * C::BQ), U.bh);
+        }
+        for (int it = U.u0; ok && it <= U.u1; ++it, ++g) {
+          const int s = g % C::NS;
+          ok = bar_wait(&bars->kv_empty[s], ((g / C::NS) & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          const int j0 = it * C::BK;
+          ptx::mbar_arrive_expect_tx(&bars->k_full[s], C::KV_BYTES);
+          for (int c = 0; c < C::DB; ++c)
+            ptx::tma_load_3d(smem + C::OFF_K + s * C::KV_BYTES + c * (C::BK * 128), &tm_k, &bars->k_full[s],
+                             c * 64, j0, U.bh);
+          ptx::mbar_arrive_expect_tx(&bars->v_full[s], C::KV_BYTES);
+          for (int c = 0; c < C::DB; ++c)
+            ptx::tma_load_3d(smem + C::OFF_V + s * C::KV_BYTES + c * (C::BK * 128), &tm_v, &bars->v_full[s],
+                             c * 64, j0, U.bh);
+          ++armed[s];
+        }
       }
       // Exit path: every load this thread issued has landed before the CTA ends.
-      bar_drain(&bars->q_full, 0);
+      for (int t = 0; t < 2; ++t)
+        if (nq[t] > 0) bar_drain(&bars->q_full[t], (nq[t] - 1) & 1);
       for (int s = 0; s < C::NS; ++s)
         if (armed[s] > 0) {
           bar_drain(&bars->k_full[s], (armed[s] - 1) & 1);
@@ -148,47 +200,96 @@ __global__ void __launch_bounds__(192, 1)
         }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BK, false, false);
       constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(128, D, false, true);
-      bool ok = bar_wait(&bars->q_full, 0, abort_flag);
-      for (int it = 0; ok && it <= nkt; ++it) {
-        if (it < nkt) {
-          const int s = it % C::NS, sb = it & 1;
-          ok = bar_wait(&bars->k_full[s], (it / C::NS) & 1, abort_flag) &&
-               bar_wait(&bars->s_free[sb], ((it >> 1) & 1) ^ 1, abort_flag);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint32_t dS = tmem + (sb ? C::TM_S1 : C::TM_S0);
-          const uint32_t kbase = sK + s * C::KV_BYTES;
+      int cq0 = 0, cq1 = 0, cp0 = 0, cp1 = 0, co0 = 0, co1 = 0;
+      int g = 0;
+      bool ok = true;
+      auto issue_s = [&](int t, int slot) {
+        const uint32_t kb = sK + slot * C::KV_BYTES;
+        const uint32_t qb = sQ + t * C::Q_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t a = sQ + (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-            const uint32_t bb = kbase + (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
-            ptx::mma_bf16(dS, ptx::sdesc_sw128(a, 0, 1024), ptx::sdesc_sw128(bb, 0, 1024), idesc_s,
-                          kk > 0);
-          }
-          ptx::mma_commit(&bars->s_full[sb]);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t a = qb + (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
+          const uint32_t bb = kb + (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
+          ptx::mma_bf16(tmem + C::tm_s(t), ptx::sdesc_sw128(a, 0, 1024), ptx::sdesc_sw128(bb, 0, 1024),
+                        idesc_s, kk > 0);
         }
-        if (it >= 1) {
-          const int pit = it - 1, s = pit % C::NS;
-          ok = bar_wait(&bars->p_full, pit & 1, abort_flag) &&
-               bar_wait(&bars->v_full[s], (pit / C::NS) & 1, abort_flag);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint32_t vbase = sV + s * C::KV_BYTES;
+        ptx::mma_commit(&bars->s_full[t]);
+      };
+      auto issue_pv = [&](int t, int slot, bool first) {
+        const uint32_t vb = sV + slot * C::KV_BYTES;
 #pragma unroll
-          for (int kk = 0; kk < C::BK / 16; ++kk) {
-            const uint32_t a = sP + (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-            const uint32_t bb = vbase + kk * (16 * 128);
-            ptx::mma_bf16(tmem + C::TM_O, ptx::sdesc_sw128(a, 0, 1024),
-                          ptx::sdesc_sw128(bb, C::BK * 128, 1024), idesc_o, (pit > 0 || kk > 0));
+        for (int kk = 0; kk < C::BK / 16; ++kk)
+          ptx::mma_bf16_ts(tmem + C::tm_o(t), tmem + C::tm_s(t) + kk * 8,
+                           ptx::sdesc_sw128(vb + kk * (16 * 128), C::BK * 128, 1024), idesc_o,
+                           (!first || kk > 0));
+      };
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const FwdUnit U = fwd_decode<D>(u, p);
+        if (U.u1 < U.u0) continue;
+        auto act = [&](int t, int it) { return U.act[t] && it >= U.a[t] && it <= U.b[t]; };
+        const int g0 = g;
+        auto slot = [&](int it) { return (g0 + it - U.u0) % C::NS; };
+        auto ring_par = [&](int it) { return (uint32_t)(((g0 + it - U.u0) / C::NS) & 1); };
+        if (U.act[0]) ok = bar_wait(&bars->q_full[0], (cq0++) & 1, abort_flag);
+        if (ok && U.act[1]) ok = bar_wait(&bars->q_full[1], (cq1++) & 1, abort_flag);
+        bool first0 = true, first1 = true;
+        ok = ok && bar_wait(&bars->k_full[slot(U.u0)], ring_par(U.u0), abort_flag);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (act(0, U.u0)) {
+          issue_s(0, slot(U.u0));
+          if (U.u0 == U.b[0]) ptx::mma_commit(&bars->q_empty[0]);
+        }
+        if (act(1, U.u0)) {
+          issue_s(1, slot(U.u0));
+          if (U.u0 == U.b[1]) ptx::mma_commit(&bars->q_empty[1]);
+        }
+        for (int it = U.u0; ok && it <= U.u1; ++it) {
+          const int s = slot(it);
+          const bool nxt = it + 1 <= U.u1;
+          ok = bar_wait(&bars->v_full[s], ring_par(it), abort_flag);
+          if (!ok) break;
+          // tile 0: O_0 += P_0 V, then S_0 for the next key tile
+          if (act(0, it)) {
+            ok = bar_wait(&bars->p_full[0], (cp0++) & 1, abort_flag);
+            if (ok && first0) ok = bar_wait(&bars->o_free[0], ((co0++) & 1) ^ 1, abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_pv(0, s, first0);
+            first0 = false;
+            if (it == U.b[0]) ptx::mma_commit(&bars->o_done[0]);
           }
-          ptx::mma_commit(&bars->o_done);
+          if (nxt) {
+            ok = bar_wait(&bars->k_full[slot(it + 1)], ring_par(it + 1), abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            if (act(0, it + 1)) {
+              issue_s(0, slot(it + 1));
+              if (it + 1 == U.b[0]) ptx::mma_commit(&bars->q_empty[0]);
+            }
+          }
+          // tile 1: O_1 += P_1 V, release the K/V stage, then S_1 for the next key tile
+          if (act(1, it)) {
+            ok = bar_wait(&bars->p_full[1], (cp1++) & 1, abort_flag);
+            if (ok && first1) ok = bar_wait(&bars->o_free[1], ((co1++) & 1) ^ 1, abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_pv(1, s, first1);
+            first1 = false;
+            if (it == U.b[1]) ptx::mma_commit(&bars->o_done[1]);
+          }
           ptx::mma_commit(&bars->kv_empty[s]);
+          if (nxt && act(1, it + 1)) {
+            issue_s(1, slot(it + 1));
+            if (it + 1 == U.b[1]) ptx::mma_commit(&bars->q_empty[1]);
+          }
         }
+        g = g0 + (U.u1 - U.u0 + 1);
       }
       // Exit path: every MMA this thread issued has completed.
       ptx::mma_commit(&bars->drain);
@@ -196,127 +297,195 @@ __global__ void __launch_bounds__(192, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int r = threadIdx.x;
-    const int64_t i = i0 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    float m = -INFINITY, l = 0.f;
+    // ------------------------------------------------------------ softmax warpgroups
+    const int t = warp / 4;                    // Q tile of this warpgroup
+    const int r = threadIdx.x - 128 * t;       // row within the tile = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::tm_s(t);
+    const uint32_t tO = tmem + lane_base + C::tm_o(t);
+    int cs = 0, cd = 0;
     bool ok = true;
-    for (int it = 0; it < nkt; ++it) {
-      const int sb = it & 1;
-      ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[sb], (it >> 1) & 1, abort_flag));
-      if (!ok) break;
-      ptx::tc_fence_after();
-      uint32_t sr[4][32];
-      const uint32_t taddr = tmem + lane_base + (sb ? C::TM_S1 : C::TM_S0);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) ptx::tmem_ld32(taddr + q * 32, sr[q]);
-      ptx::tmem_wait_ld();
-#pragma unroll
-      for (int q = 0; q < 4; ++q) ptx::reg_fence(sr[q]);
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->s_free[sb]);
-
-      const int64_t j0 = (int64_t)(strip.begin + it) * C::BK;
-      const bool interior = tile_is_interior(N, lo, hi, i0, C::BQ, j0, C::BK);
-      float x[128];
-      float tmax = -INFINITY;
-      const int64_t dist0 = i - j0;  // distance to the tile's first key
-#pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        float v = __uint_as_float(sr[c / 32][c % 32]) * p.scale_log2;
-        if (!interior) {
-          const int64_t dd = dist0 - c;
-          const bool allowed = (dd >= lo) && (dd < hi) && (j0 + c < N) && (i < N);
-          v = allowed ? v : -INFINITY;
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const FwdUnit U = fwd_decode<D>(u, p);
+      const int64_t it0 = U.i0 + (int64_t)t * C::BQ;
+      const int64_t i = it0 + r;
+      const bool act_t = t ? U.act[1] : U.act[0];
+      const int a_t = t ? U.a[1] : U.a[0];
+      const int b_t = t ? U.b[1] : U.b[0];
+      uint16_t* orow = static_cast<uint16_t*>(p.o) + ((int64_t)U.bh * N + i) * D;
+      if (!act_t) {
+        // rows of this tile precede their band (or lie past N)
+        if (i < N) {
+          for (int c = 0; c < D; c += 8) ptx::st_global_v4(orow + c, 0u, 0u, 0u, 0u);
+          p.lse[(int64_t)U.bh * N + i] = -INFINITY;
         }
-        x[c] = v;
-        tmax = fmaxf(tmax, v);
+        continue;
       }
-      const float m_new = fmaxf(m, tmax);
-      const float m_use = (m_new == -INFINITY) ? 0.f : m_new;
-      const float alpha = ptx::exp2_approx(m - m_use);  // 0 while the row has seen nothing
-
-      if (it > 0) {
-        // PV(it-1) must be complete before O is rescaled and P is overwritten.
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->o_done, (it - 1) & 1, abort_flag));
+      float m_ref = -INFINITY, l = 0.f;  // running max (base-2 units) and sum
+      for (int it = a_t; it <= b_t; ++it) {
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[t], (cs++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
-        const bool need = (m_new > m) && (m != -INFINITY);
-        if (__any_sync(0xffffffffu, need)) {
-          const float a = need ? alpha : 1.f;
+        const int64_t j0 = (int64_t)it * C::BK;
+        const bool interior = tile_is_interior(N, U.lo, U.hi, it0, C::BQ, j0, C::BK);
+        // Edge tile: the permitted keys of this row are the columns c with
+        // clo <= c <= clo + span (distance in [lo, hi), key and row inside N).
+        int clo = 0;
+        uint32_t span = 127;
+        if (!interior) {
+          const int64_t c_first = max64(i - U.hi + 1 - j0, 0);
+          const int64_t c_last = min64(min64(i - U.lo - j0, N - 1 - j0), 127);
+          if (i >= N || c_last < c_first) {
+            clo = 128;
+            span = 0;
+          } else {
+            clo = (int)c_first;
+            span = (uint32_t)(c_last - c_first);
+          }
+        }
+        // pass 1: row max of the raw scores (scale > 0 commutes with max)
+        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t sr[32];
+          ptx::tmem_ld32(tS + q * 32, sr);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(sr);
+          if (interior) {
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              mx0 = fmaxf(mx0, __uint_as_float(sr[e]));
+              mx1 = fmaxf(mx1, __uint_as_float(sr[e + 1]));
+              mx2 = fmaxf(mx2, __uint_as_float(sr[e + 2]));
+              mx3 = fmaxf(mx3, __uint_as_float(sr[e + 3]));
+            }
+          } else {
+            const int cb = q * 32 - clo;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              mx0 = fmaxf(mx0, (uint32_t)(cb + e) <= span ? __uint_as_float(sr[e]) : -INFINITY);
+              mx1 = fmaxf(mx1, (uint32_t)(cb + e + 1) <= span ? __uint_as_float(sr[e + 1]) : -INFINITY);
+              mx2 = fmaxf(mx2, (uint32_t)(cb + e + 2) <= span ? __uint_as_float(sr[e + 2]) : -INFINITY);
+              mx3 = fmaxf(mx3, (uint32_t)(cb + e + 3) <= span ? __uint_as_float(sr[e + 3]) : -INFINITY);
+            }
+          }
+        }
+        const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2);
+        const bool need = m_new > m_ref + 8.f;   // also true for a row's first finite max
+        const bool need_o = need && (m_ref != -INFINITY);
+        float alpha = 1.f;
+        if (need) {
+          alpha = ptx::exp2_approx(m_ref - m_new);  // 0 while the row had seen nothing
+          l *= alpha;
+          m_ref = m_new;
+        }
+        if (__any_sync(0xffffffffu, need_o)) {
+          // O_t is stable: the PV of the previous key tile completed before S_t did
+          const float a = need_o ? alpha : 1.f;
 #pragma unroll 1
           for (int c = 0; c < D; c += 32) {
             uint32_t o[32];
-            ptx::tmem_ld32(tmem + lane_base + C::TM_O + c, o);
+            ptx::tmem_ld32(tO + c, o);
             ptx::tmem_wait_ld();
             ptx::reg_fence(o);
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
-            ptx::tmem_st32(tmem + lane_base + C::TM_O + c, o);
+            ptx::tmem_st32(tO + c, o);
           }
-          ptx::tmem_wait_st();
         }
-      }
-      float rs = 0.f;
+        // pass 2: p = exp2(s * scale_log2 - m), bf16 pairs over the first half
+        // of S_t (chunk q of P covers columns [16q, 16q+16), already read)
+        const float c2 = p.scale_log2;
+        const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+        float sm0 = 0.f, sm1 = 0.f, sm2 = 0.f, sm3 = 0.f;
+#pragma unroll 1
+        for (int q = 0; q < 4; ++q) {
+          uint32_t sr[32];
+          ptx::tmem_ld32(tS + q * 32, sr);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(sr);
+          uint32_t pk[16];
+          const int cb = q * 32 - clo;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
-        x[c] = ptx::exp2_approx(x[c] - m_use);
-        rs += x[c];
+          for (int e = 0; e < 32; e += 4) {
+            float x0 = fmaf(__uint_as_float(sr[e]), c2, mneg);
+            float x1 = fmaf(__uint_as_float(sr[e + 1]), c2, mneg);
+            float x2 = fmaf(__uint_as_float(sr[e + 2]), c2, mneg);
+            float x3 = fmaf(__uint_as_float(sr[e + 3]), c2, mneg);
+            if (!interior) {
+              x0 = (uint32_t)(cb + e) <= span ? x0 : -INFINITY;
+              x1 = (uint32_t)(cb + e + 1) <= span ? x1 : -INFINITY;
+              x2 = (uint32_t)(cb + e + 2) <= span ? x2 : -INFINITY;
+              x3 = (uint32_t)(cb + e + 3) <= span ? x3 : -INFINITY;
+            }
+            const float p0 = ptx::exp2_approx(x0), p1 = ptx::exp2_approx(x1);
+            const float p2 = ptx::exp2_approx(x2), p3 = ptx::exp2_approx(x3);
+            sm0 += p0;
+            sm1 += p1;
+            sm2 += p2;
+            sm3 += p3;
+            pk[e / 2] = ptx::pack_bf16x2(p0, p1);
+            pk[e / 2 + 1] = ptx::pack_bf16x2(p2, p3);
+          }
+          ptx::tmem_st16(tS + q * 16, pk);
+        }
+        l += (sm0 + sm1) + (sm2 + sm3);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p_full[t]);
       }
-      l = l * alpha + rs;
-#pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const uint32_t addr = sP + (ch / 8) * (C::BQ * 128) + ptx::sw128_offset(r, ch % 8);
-        ptx::st_shared_v4(addr, ptx::pack_bf16x2(x[8 * ch + 0], x[8 * ch + 1]),
-                          ptx::pack_bf16x2(x[8 * ch + 2], x[8 * ch + 3]),
-                          ptx::pack_bf16x2(x[8 * ch + 4], x[8 * ch + 5]),
-                          ptx::pack_bf16x2(x[8 * ch + 6], x[8 * ch + 7]));
-      }
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->p_full);
-      m = m_new;
-    }
-    // ------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, bar_wait(&bars->o_done, (nkt - 1) & 1, abort_flag));
-    if (ok) {
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      ok = __all_sync(0xffffffffu, bar_wait(&bars->o_done[t], (cd++) & 1, abort_flag));
+      if (!ok) break;
       ptx::tc_fence_after();
       const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
       for (int c = 0; c < D; c += 32) {
         uint32_t o[32];
-        ptx::tmem_ld32(tmem + lane_base + C::TM_O + c, o);
+        ptx::tmem_ld32(tO + c, o);
         ptx::tmem_wait_ld();
         ptx::reg_fence(o);
+        if (i < N) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = c + q * 8;
-          const uint32_t addr = sQ + (col / 64) * (C::BQ * 128) + ptx::sw128_offset(r, (col % 64) / 8);
-          const float* f = reinterpret_cast<const float*>(&o[8 * q]);
-          ptx::st_shared_v4(addr, ptx::pack_bf16x2(f[0] * inv, f[1] * inv),
-                            ptx::pack_bf16x2(f[2] * inv, f[3] * inv),
-                            ptx::pack_bf16x2(f[4] * inv, f[5] * inv),
-                            ptx::pack_bf16x2(f[6] * inv, f[7] * inv));
+          for (int q = 0; q < 4; ++q) {
+            const float* f = reinterpret_cast<const float*>(&o[8 * q]);
+            ptx::st_global_v4(orow + c + 8 * q, ptx::pack_bf16x2(f[0] * inv, f[1] * inv),
+                              ptx::pack_bf16x2(f[2] * inv, f[3] * inv),
+                              ptx::pack_bf16x2(f[4] * inv, f[5] * inv),
+                              ptx::pack_bf16x2(f[6] * inv, f[7] * inv));
+          }
         }
       }
-      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars->o_free[t]);
+      if (i < N)
+        p.lse[(int64_t)U.bh * N + i] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
-    ptx::named_bar_sync(1, 128);
-    const bool all_ok = !*abort_flag;
-    if (all_ok && threadIdx.x == 0) {
-      for (int c = 0; c < C::DB; ++c)
-        ptx::tma_store_3d(&tm_o, smem + C::OFF_Q + c * (C::BQ * 128), c * 64, (int)i0, bh);
-      ptx::bulk_commit_group();
-      ptx::bulk_wait_group_all();
+  }
+
+  // ------------------------------------------------------------ empty blocks
+  // Whole 256-row blocks that precede their head's band: o = 0, lse = -inf.
+  {
+    const int num_fill = p.B * p.fills_per_batch;
+    for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
+      const int b = f / p.fills_per_batch;
+      int r = f % p.fills_per_batch;
+      int h = 0;
+      for (; h < p.H; ++h) {
+        const int cnt = p.lo[h] / C::BU;
+        if (r < cnt) break;
+        r -= cnt;
+      }
+      const int64_t row0 = (int64_t)(b * p.H + h) * N + (int64_t)r * C::BU;
+      zero_rows_bf16(static_cast<uint16_t*>(p.o) + row0 * D, C::BU, D);
+      for (int e = threadIdx.x; e < C::BU; e += blockDim.x) p.lse[row0 + e] = -INFINITY;
     }
-    if (all_ok && i < N)
-      p.lse[(int64_t)bh * N + i] = (l > 0.f) ? (m + log2f(l)) * 0.69314718055994531f : -INFINITY;
   }
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -97,22 +97,51 @@ int prepare_kernel(K kernel, uint32_t smem_bytes, std::atomic<uint64_t>& done_ma
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? SPA_OK : SPA_ERR_CUDA; }
 
+int sm_count(int* n) {
+  static std::atomic<int> cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SPA_ERR_CUDA;
+  const int slot = dev & 63;
+  int v = cache[slot].load(std::memory_order_relaxed);
+  if (v <= 0) {
+    if (cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || v <= 0)
+      return SPA_ERR_CUDA;
+    cache[slot].store(v, std::memory_order_relaxed);
+  }
+  *n = v;
+  return SPA_OK;
+}
+
 template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, AttnParams& p,
              cudaStream_t stream) {
   using C = spa::FwdCfg<D>;
   static std::atomic<uint64_t> prepared{0};
   const int64_t BH = (int64_t)p.B * p.H;
-  CUtensorMap mq, mk, mv, mo;
+  CUtensorMap mq, mk, mv;
   int st;
   if ((st = make_map(&mq, q, p.N, BH, D, C::BQ)) || (st = make_map(&mk, k, p.N, BH, D, C::BK)) ||
-      (st = make_map(&mv, v, p.N, BH, D, C::BK)) || (st = make_map(&mo, o, p.N, BH, D, C::BQ)))
+      (st = make_map(&mv, v, p.N, BH, D, C::BK)))
     return st;
   if ((st = prepare_kernel(spa::spa_fwd_kernel<D>, C::SMEM_BYTES, prepared))) return st;
+  // Work list of the persistent grid: per batch, every 256-row block of every
+  // head from the one holding lo_h on (units), and the blocks before it (fills).
+  const int64_t nblk = (p.N + C::BU - 1) / C::BU;
+  int64_t upb = 0, fpb = 0;
+  for (int h = 0; h < p.H; ++h) {
+    upb += nblk - p.lo[h] / C::BU;
+    fpb += p.lo[h] / C::BU;
+  }
+  if ((int64_t)p.B * upb > 2147483647LL || (int64_t)p.B * fpb > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+  p.units_per_batch = (int)upb;
+  p.fills_per_batch = (int)fpb;
   p.lse = lse;
   p.o = o;
-  dim3 grid((unsigned)((p.N + C::BQ - 1) / C::BQ), (unsigned)p.H, (unsigned)p.B);
-  spa::spa_fwd_kernel<D><<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, mo, p);
+  int sms = 0;
+  if ((st = sm_count(&sms))) return st;
+  const int64_t units = (int64_t)p.B * upb;
+  const unsigned grid = (unsigned)(units < sms ? units : sms);
+  spa::spa_fwd_kernel<D><<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -173,7 +202,7 @@ int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, 
   int st = check_shape(B, H, N, d);
   if (st) return st;
   if (!q || !k || !v || !o || !lse) return SPA_ERR_INVAL;
-  if (!std::isfinite(scale)) return SPA_ERR_INVAL;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return SPA_ERR_INVAL;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
     return SPA_ERR_UNSUPPORTED;
   static AttnParams zero{};
@@ -199,7 +228,7 @@ int bwd_entry(const void* q, const void* k, const void* v, const void* o, const 
   if ((steps & (kStepDkDv | kStepDq)) && (!q || !k || !v || !dout || !lse)) return SPA_ERR_INVAL;
   if ((steps & kStepDkDv) && (!dk || !dv)) return SPA_ERR_INVAL;
   if ((steps & kStepDq) && !dq) return SPA_ERR_INVAL;
-  if (!std::isfinite(scale)) return SPA_ERR_INVAL;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return SPA_ERR_INVAL;
   for (const void* t : {q, k, v, o, dout, (const void*)dq, (const void*)dk, (const void*)dv})
     if (t && !aligned(t, 16)) return SPA_ERR_UNSUPPORTED;
   if ((lse && !aligned(lse, 4)) || !aligned(workspace, 4)) return SPA_ERR_UNSUPPORTED;

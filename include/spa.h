@@ -23,7 +23,8 @@
  *    NULL = the legacy default stream) and never synchronise the host, except
  *    spa_device_status.
  *  - scale multiplies q.k before the softmax (1/sqrt(d) for standard
- *    attention).  Softmax statistics and accumulation are fp32.
+ *    attention); it must be finite and > 0, else SPA_ERR_INVAL.  Softmax
+ *    statistics and accumulation are fp32.
  *  - A query row whose permitted set is empty (i < lo_h) gets o = 0 and
  *    lse = -inf; it passes no gradient.  Keys that no query reaches get
  *    dk = dv = 0.  Every element of every output is written.

@@ -131,6 +131,8 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
     assert f(1, 4, 0, 64, 0.1) == spa.SPA_ERR_INVAL              # N
     assert f(1, 4, 2 ** 31, 64, 0.1) == spa.SPA_ERR_INVAL        # N too large
     assert f(1, 4, 256, 64, float("nan")) == spa.SPA_ERR_INVAL   # scale
+    assert f(1, 4, 256, 64, -0.125) == spa.SPA_ERR_INVAL         # scale must be > 0
+    assert f(1, 4, 256, 64, 0.0) == spa.SPA_ERR_INVAL
     assert L.spa_attn_fwd(p, None, p, p, p, 1, 4, 256, 64, 0.1, None) == spa.SPA_ERR_INVAL
     odd = _fake((1 << 20) + 8)
     assert L.spa_attn_fwd(p, p, odd, p, p, 1, 4, 256, 64, 0.1, None) == spa.SPA_ERR_UNSUPPORTED
