@@ -51,91 +51,121 @@ __global__ void __launch_bounds__(256) spa_bwd_delta_kernel(const uint16_t* __re
 }
 
 // ---------------------------------------------------------------------------
-// dK, dV: one CTA per (key tile of 128, h, b); query tiles of 64.
+// dK, dV: persistent grid; a unit is (b, h, key tile of 128 keys), walking
+// the 128-query tiles its band reaches.  Per query tile:
+//   S^T  = K Q^T      SS MMA -> TMEM [0,128)
+//   dP^T = V dO^T     SS MMA -> TMEM [128,256)
+//   P^T  = exp2(S^T c - lse2), masked on edge tiles; written as bf16 over S^T
+//   dS^T = P^T (dP^T - D);                          written as bf16 over dP^T
+//   dV  += P^T dO     TS MMA (A = P^T from TMEM) -> TMEM [256,384)
+//   dK  += dS^T Q     TS MMA (A = dS^T from TMEM) -> TMEM [384,512)
+// Two warpgroups share each tile: warpgroup w owns query columns
+// [64w, 64w+64) of every key row (thread r = key row r = TMEM lane r) and
+// writes its bf16 pairs to columns [64w, 64w+32) of the region it read, so
+// the two never touch each other's unread columns.  S^T of the next query
+// tile is issued right after dV (which read P^T) and dP^T right after dK, so
+// the tensor core runs while the warpgroups work.  Epilogue: warpgroup 0
+// writes dV, warpgroup 1 writes scale * dK, straight from TMEM to global.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DkvCfg {
-  static constexpr int BK = 128;  // keys per CTA (MMA M)
-  static constexpr int BQ = 64;   // queries per step (MMA N of S^T)
-  static constexpr int NS = 2;
+  static constexpr int BK = 128;  // keys per unit (MMA M)
+  static constexpr int BQ = 128;  // queries per step
+  static constexpr int NS = 2;    // Q/dO ring stages
   static constexpr int DB = D / 64;
   static constexpr uint32_t KT_BYTES = BK * D * 2;
   static constexpr uint32_t QT_BYTES = BQ * D * 2;
-  static constexpr uint32_t PT_BYTES = BK * BQ * 2;
   static constexpr uint32_t OFF_K = 0;
   static constexpr uint32_t OFF_V = OFF_K + KT_BYTES;
   static constexpr uint32_t OFF_Q = OFF_V + KT_BYTES;
   static constexpr uint32_t OFF_DO = OFF_Q + NS * QT_BYTES;
-  static constexpr uint32_t OFF_PT = OFF_DO + NS * QT_BYTES;
-  static constexpr uint32_t OFF_DST = OFF_PT + PT_BYTES;
-  static constexpr uint32_t OFF_VEC = OFF_DST + PT_BYTES;           // [NS][2][BQ] floats
+  static constexpr uint32_t OFF_VEC = OFF_DO + NS * QT_BYTES;  // [NS][2][BQ] floats: lse2, D
   static constexpr uint32_t OFF_BAR = OFF_VEC + NS * 2 * BQ * 4;
-  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t TM_ST = 0, TM_DPT = 64, TM_DV = 128, TM_DK = 128 + D;
-  static constexpr uint32_t TMEM_COLS = (128 + 2 * D <= 256) ? 256 : 512;
+  static constexpr uint32_t SMEM_BYTES =
+      (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
+  static constexpr int NTHREADS = 320;
+  static constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
 };
 
 struct DkvBars {
-  uint64_t kv_full;
+  uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full, s_free, p_full, ds_full, dv_done, dk_done, drain;
+  uint64_t s_full, dp_full, p_full, ds_full;
+  uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
   int abort;
 };
 
+// Key tiles of head h that some query reaches: u <= (N - 1 - lo) / 128.
+__device__ __forceinline__ int dkv_units_of_head(int64_t N, int32_t lo) {
+  return (int)((N - 1 - lo) / 128) + 1;
+}
+
+struct DkvUnit {
+  int bh;
+  int32_t lo, hi;
+  int64_t j0;
+  int qa, qb;  // query tiles walked
+};
+
+__device__ __forceinline__ DkvUnit dkv_decode(int u, const AttnParams& p) {
+  DkvUnit U;
+  const int b = u / p.units_per_batch;
+  int r = u % p.units_per_batch;
+  int h = 0;
+  for (; h < p.H; ++h) {
+    const int cnt = dkv_units_of_head(p.N, p.lo[h]);
+    if (r < cnt) break;
+    r -= cnt;
+  }
+  U.bh = b * p.H + h;
+  U.lo = p.lo[h];
+  U.hi = p.hi[h];
+  U.j0 = (int64_t)r * 128;
+  const Strip s = query_strip(p.N, U.lo, U.hi, U.j0, 128, 128);
+  U.qa = s.begin;
+  U.qb = s.end;
+  return U;
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     spa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                        const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                         const __grid_constant__ AttnParams p) {
   using C = DkvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   DkvBars* bars = reinterpret_cast<DkvBars*>(smem + C::OFF_BAR);
   float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC);
-
-  const int u = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int bh = b * p.H + h;
-  const int64_t N = p.N;
-  const int32_t lo = p.lo[h], hi = p.hi[h];
-  const int64_t j0 = (int64_t)u * C::BK;
-  const Strip strip = query_strip(N, lo, hi, j0, C::BK, C::BQ);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t rows_here = min64(j0 + C::BK, N) - j0;
-
-  if (strip.end < strip.begin) {
-    // No query reaches these keys: dk = dv = 0.
-    zero_rows_bf16(static_cast<uint16_t*>(p.dk) + ((int64_t)bh * N + j0) * D, rows_here, D);
-    zero_rows_bf16(static_cast<uint16_t*>(p.dv) + ((int64_t)bh * N + j0) * D, rows_here, D);
-    return;
-  }
-  const int nq = strip.end - strip.begin + 1;
+  const int64_t N = p.N;
+  const int num_units = p.B * p.units_per_batch;
 
   const uint32_t sK = ptx::smem_u32(smem + C::OFF_K);
   const uint32_t sV = ptx::smem_u32(smem + C::OFF_V);
   const uint32_t sQ = ptx::smem_u32(smem + C::OFF_Q);
   const uint32_t sDO = ptx::smem_u32(smem + C::OFF_DO);
-  const uint32_t sPT = ptx::smem_u32(smem + C::OFF_PT);
-  const uint32_t sDST = ptx::smem_u32(smem + C::OFF_DST);
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars->kv_full, 1);
+    ptx::mbar_init(&bars->kv_empty, 1);
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars->q_full[s], 1);
       ptx::mbar_init(&bars->q_empty[s], 1);
     }
     ptx::mbar_init(&bars->s_full, 1);
-    ptx::mbar_init(&bars->s_free, 128);
-    ptx::mbar_init(&bars->p_full, 128);
-    ptx::mbar_init(&bars->ds_full, 128);
-    ptx::mbar_init(&bars->dv_done, 1);
-    ptx::mbar_init(&bars->dk_done, 1);
+    ptx::mbar_init(&bars->dp_full, 1);
+    ptx::mbar_init(&bars->p_full, 256);
+    ptx::mbar_init(&bars->ds_full, 256);
+    ptx::mbar_init(&bars->acc_done, 1);
+    ptx::mbar_init(&bars->acc_free, 256);
     ptx::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
@@ -145,299 +175,382 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
 
-  if (warp == 4) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer warp
-    if (lane == 0) {
-      ptx::mbar_arrive_expect_tx(&bars->kv_full, 2 * C::KT_BYTES);
-      for (int c = 0; c < C::DB; ++c) {
-        ptx::tma_load_3d(smem + C::OFF_K + c * (C::BK * 128), &tm_k, &bars->kv_full, c * 64, (int)j0, bh);
-        ptx::tma_load_3d(smem + C::OFF_V + c * (C::BK * 128), &tm_v, &bars->kv_full, c * 64, (int)j0, bh);
-      }
-    }
-    int armed[2] = {0, 0};
-    for (int it = 0; it < nq; ++it) {
-      const int s = it % C::NS;
-      const bool ok =
-          __all_sync(0xffffffffu, bar_wait(&bars->q_empty[s], ((it / C::NS) & 1) ^ 1, abort_flag));
+    int nkv = 0, gq = 0, armed[2] = {0, 0};
+    bool ok = true;
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const DkvUnit U = dkv_decode(u, p);
+      ok = __all_sync(0xffffffffu, bar_wait(&bars->kv_empty, (nkv & 1) ^ 1, abort_flag));
       if (!ok) break;
-      const int64_t i0 = (int64_t)(strip.begin + it) * C::BQ;
-      // lse (in base-2 units) and D of this step's queries, for the softmax warps
-      float* vl = vec + s * 2 * C::BQ;
-      float* vd = vl + C::BQ;
-      for (int c = lane; c < C::BQ; c += 32) {
-        const int64_t i = i0 + c;
-        const bool in = i < N;
-        vl[c] = in ? p.lse[(int64_t)bh * N + i] * kLog2e : 0.f;
-        vd[c] = in ? p.delta[(int64_t)bh * N + i] : 0.f;
-      }
-      __syncwarp();
       if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::QT_BYTES);
+        ptx::mbar_arrive_expect_tx(&bars->kv_full, 2 * C::KT_BYTES);
         for (int c = 0; c < C::DB; ++c) {
-          ptx::tma_load_3d(smem + C::OFF_Q + s * C::QT_BYTES + c * (C::BQ * 128), &tm_q, &bars->q_full[s],
-                           c * 64, (int)i0, bh);
-          ptx::tma_load_3d(smem + C::OFF_DO + s * C::QT_BYTES + c * (C::BQ * 128), &tm_do,
-                           &bars->q_full[s], c * 64, (int)i0, bh);
+          ptx::tma_load_3d(smem + C::OFF_K + c * (C::BK * 128), &tm_k, &bars->kv_full, c * 64, (int)U.j0, U.bh);
+          ptx::tma_load_3d(smem + C::OFF_V + c * (C::BK * 128), &tm_v, &bars->kv_full, c * 64, (int)U.j0, U.bh);
         }
       }
-      armed[s]++;
+      ++nkv;
+      for (int qt = U.qa; qt <= U.qb; ++qt, ++gq) {
+        const int s = gq % C::NS;
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->q_empty[s], ((gq / C::NS) & 1) ^ 1, abort_flag));
+        if (!ok) break;
+        const int64_t i0 = (int64_t)qt * C::BQ;
+        // lse (base 2) and D of this step's queries, for the element-wise warps
+        float* vl = vec + s * 2 * C::BQ;
+        float* vd = vl + C::BQ;
+        for (int c = lane; c < C::BQ; c += 32) {
+          const int64_t i = i0 + c;
+          const bool in = i < N;
+          vl[c] = in ? p.lse[(int64_t)U.bh * N + i] * kLog2e : 0.f;
+          vd[c] = in ? p.delta[(int64_t)U.bh * N + i] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::QT_BYTES);
+          for (int c = 0; c < C::DB; ++c) {
+            ptx::tma_load_3d(smem + C::OFF_Q + s * C::QT_BYTES + c * (C::BQ * 128), &tm_q, &bars->q_full[s],
+                             c * 64, (int)i0, U.bh);
+            ptx::tma_load_3d(smem + C::OFF_DO + s * C::QT_BYTES + c * (C::BQ * 128), &tm_do,
+                             &bars->q_full[s], c * 64, (int)i0, U.bh);
+          }
+        }
+        ++armed[s];
+      }
     }
     if (lane == 0) {
-      bar_drain(&bars->kv_full, 0);
+      if (nkv > 0) bar_drain(&bars->kv_full, (nkv - 1) & 1);
       for (int s = 0; s < C::NS; ++s)
         if (armed[s] > 0) bar_drain(&bars->q_full[s], (armed[s] - 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idesc_g = ptx::idesc_bf16_f32(128, D, false, true);
-      bool ok = bar_wait(&bars->kv_full, 0, abort_flag);
-      for (int it = 0; ok && it < nq; ++it) {
-        const int s = it % C::NS;
-        ok = bar_wait(&bars->q_full[s], (it / C::NS) & 1, abort_flag) &&
-             bar_wait(&bars->s_free, (it & 1) ^ 1, abort_flag);
+      int nkv = 0, gq = 0, cp = 0, cds = 0, cacc = 0;
+      bool ok = true;
+      auto qstage = [&](int g) { return g % C::NS; };
+      auto issue_nt = [&](uint32_t dst, uint32_t a_base, int g) {  // dst = A (keys) x B^T (queries)
+        const uint32_t bb = (a_base == sK ? sQ : sDO) + qstage(g) * C::QT_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t a = a_base + (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
+          const uint32_t b = bb + (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
+          ptx::mma_bf16(tmem + dst, ptx::sdesc_sw128(a, 0, 1024), ptx::sdesc_sw128(b, 0, 1024), idesc_s, kk > 0);
+        }
+      };
+      auto issue_grad = [&](uint32_t dst, uint32_t a_col, uint32_t b_base, int g, bool first) {
+        const uint32_t bb = b_base + qstage(g) * C::QT_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk) {
+          const uint32_t acol = a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
+          ptx::mma_bf16_ts(tmem + dst, tmem + acol, ptx::sdesc_sw128(bb + kk * (16 * 128), C::BQ * 128, 1024),
+                           idesc_g, (!first || kk > 0));
+        }
+      };
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const DkvUnit U = dkv_decode(u, p);
+        const int nq = U.qb - U.qa + 1;
+        const int g0 = gq;
+        ok = bar_wait(&bars->kv_full, (nkv++) & 1, abort_flag) &&
+             bar_wait(&bars->q_full[qstage(g0)], (g0 / C::NS) & 1, abort_flag);
         if (!ok) break;
         ptx::tc_fence_after();
-        const uint32_t qb = sQ + s * C::QT_BYTES, dob = sDO + s * C::QT_BYTES;
-        // S^T = K Q^T and dP^T = V dO^T (both operands K-major along d)
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
-          const uint32_t qa = (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-          ptx::mma_bf16(tmem + C::TM_ST, ptx::sdesc_sw128(sK + ka, 0, 1024),
-                        ptx::sdesc_sw128(qb + qa, 0, 1024), idesc_s, kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t ka = (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
-          const uint32_t qa = (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-          ptx::mma_bf16(tmem + C::TM_DPT, ptx::sdesc_sw128(sV + ka, 0, 1024),
-                        ptx::sdesc_sw128(dob + qa, 0, 1024), idesc_s, kk > 0);
-        }
+        issue_nt(C::TM_ST, sK, g0);
         ptx::mma_commit(&bars->s_full);
-        // dV += P^T dO  (P^T K-major along queries; dO MN-major along d)
-        ok = bar_wait(&bars->p_full, it & 1, abort_flag);
+        issue_nt(C::TM_DPT, sV, g0);
+        ptx::mma_commit(&bars->dp_full);
+        for (int j = 0; j < nq; ++j) {
+          const int g = g0 + j;
+          ok = bar_wait(&bars->p_full, (cp++) & 1, abort_flag);
+          if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_grad(C::TM_DV, C::TM_ST, sDO, g, j == 0);          // dV += P^T dO
+          if (j + 1 < nq) {
+            ok = bar_wait(&bars->q_full[qstage(g + 1)], ((g + 1) / C::NS) & 1, abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_nt(C::TM_ST, sK, g + 1);                         // S^T of the next tile
+            ptx::mma_commit(&bars->s_full);
+          }
+          ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_grad(C::TM_DK, C::TM_DPT, sQ, g, j == 0);          // dK += dS^T Q
+          ptx::mma_commit(&bars->q_empty[qstage(g)]);
+          if (j + 1 < nq) {
+            issue_nt(C::TM_DPT, sV, g + 1);                        // dP^T of the next tile
+            ptx::mma_commit(&bars->dp_full);
+          }
+        }
         if (!ok) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          ptx::mma_bf16(tmem + C::TM_DV, ptx::sdesc_sw128(sPT + kk * 32, 0, 1024),
-                        ptx::sdesc_sw128(dob + kk * (16 * 128), C::BQ * 128, 1024), idesc_g,
-                        (it > 0 || kk > 0));
-        ptx::mma_commit(&bars->dv_done);
-        // dK += dS^T Q
-        ok = bar_wait(&bars->ds_full, it & 1, abort_flag);
-        if (!ok) break;
-        ptx::tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          ptx::mma_bf16(tmem + C::TM_DK, ptx::sdesc_sw128(sDST + kk * 32, 0, 1024),
-                        ptx::sdesc_sw128(qb + kk * (16 * 128), C::BQ * 128, 1024), idesc_g,
-                        (it > 0 || kk > 0));
-        ptx::mma_commit(&bars->dk_done);
-        ptx::mma_commit(&bars->q_empty[s]);
+        ++cacc;
+        ptx::mma_commit(&bars->acc_done);
+        ptx::mma_commit(&bars->kv_empty);
+        gq = g0 + nq;
       }
       ptx::mma_commit(&bars->drain);
       bar_drain(&bars->drain, 0);
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ softmax warps
-    const int r = threadIdx.x;  // key row within the tile
-    const int64_t j = j0 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------------------ element-wise warpgroups
+    const int w = warp / 4;                          // query columns [64w, 64w+64)
+    const int r = threadIdx.x - 128 * w;             // key row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::TM_ST + 64 * w;
+    const uint32_t tDP = tmem + lane_base + C::TM_DPT + 64 * w;
+    const float c2 = p.scale_log2;
+    int gq = 0, cs = 0, cdp = 0, cacc = 0;
     bool ok = true;
-    for (int it = 0; it < nq; ++it) {
-      const int s = it % C::NS;
-      ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, it & 1, abort_flag));
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const DkvUnit U = dkv_decode(u, p);
+      const int64_t j = U.j0 + r;
+      for (int qt = U.qa; qt <= U.qb; ++qt, ++gq) {
+        const int s = gq % C::NS;
+        const int64_t i0 = (int64_t)qt * C::BQ;
+        const bool interior = tile_is_interior(N, U.lo, U.hi, i0, C::BQ, U.j0, C::BK);
+        // Edge tile: query column q (0..127) is permitted for this key iff
+        // qlo <= q <= qlo + span.
+        int qlo = 0;
+        uint32_t span = 127;
+        if (!interior) {
+          const int64_t q_first = max64(j + U.lo - i0, 0);
+          const int64_t q_last = min64(min64(j + U.hi - 1 - i0, N - 1 - i0), 127);
+          if (j >= N || q_last < q_first) {
+            qlo = 128;
+            span = 0;
+          } else {
+            qlo = (int)q_first;
+            span = (uint32_t)(q_last - q_first);
+          }
+        }
+        const float* vl = vec + s * 2 * C::BQ + 64 * w;
+        const float* vd = vl + C::BQ;
+        const int cb = 64 * w - qlo;
+        // ---- P^T = exp2(S^T c - lse2)
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, (cs++) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        float pt[64];
+        {
+          uint32_t sr[2][32];
+          ptx::tmem_ld32(tS, sr[0]);
+          ptx::tmem_ld32(tS + 32, sr[1]);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(sr[0]);
+          ptx::reg_fence(sr[1]);
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            const float x = fmaf(__uint_as_float(sr[e / 32][e % 32]), c2, -vl[e]);
+            const float ev = ptx::exp2_approx(x);
+            pt[e] = (interior || (uint32_t)(cb + e) <= span) ? ev : 0.f;
+          }
+        }
+        {
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) pk[e] = ptx::pack_bf16x2(pt[2 * e], pt[2 * e + 1]);
+          ptx::tmem_st32(tS, pk);
+          ptx::tmem_wait_st();
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->p_full);
+        // ---- dS^T = P^T (dP^T - D)
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->dp_full, (cdp++) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        {
+          uint32_t dr[2][32];
+          ptx::tmem_ld32(tDP, dr[0]);
+          ptx::tmem_ld32(tDP + 32, dr[1]);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(dr[0]);
+          ptx::reg_fence(dr[1]);
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float d0 = pt[2 * e] * (__uint_as_float(dr[(2 * e) / 32][(2 * e) % 32]) - vd[2 * e]);
+            const float d1 =
+                pt[2 * e + 1] * (__uint_as_float(dr[(2 * e + 1) / 32][(2 * e + 1) % 32]) - vd[2 * e + 1]);
+            pk[e] = ptx::pack_bf16x2(d0, d1);
+          }
+          ptx::tmem_st32(tDP, pk);
+          ptx::tmem_wait_st();
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->ds_full);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t st[2][32], dpt[2][32];
-      ptx::tmem_ld32(tmem + lane_base + C::TM_ST, st[0]);
-      ptx::tmem_ld32(tmem + lane_base + C::TM_ST + 32, st[1]);
-      ptx::tmem_ld32(tmem + lane_base + C::TM_DPT, dpt[0]);
-      ptx::tmem_ld32(tmem + lane_base + C::TM_DPT + 32, dpt[1]);
-      ptx::tmem_wait_ld();
-      ptx::reg_fence(st[0]);
-      ptx::reg_fence(st[1]);
-      ptx::reg_fence(dpt[0]);
-      ptx::reg_fence(dpt[1]);
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->s_free);
-
-      const int64_t i0 = (int64_t)(strip.begin + it) * C::BQ;
-      const bool interior = tile_is_interior(N, lo, hi, i0, C::BQ, j0, C::BK);
-      const float* vl = vec + s * 2 * C::BQ;
-      const float* vd = vl + C::BQ;
-      float pt[64];
-      const int64_t dist0 = i0 - j;  // distance of the step's first query to this key
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float e = ptx::exp2_approx(__uint_as_float(st[c / 32][c % 32]) * p.scale_log2 - vl[c]);
-        bool allowed = true;
-        if (!interior) {
-          const int64_t dd = dist0 + c;
-          allowed = (dd >= lo) && (dd < hi) && (i0 + c < N) && (j < N);
-        }
-        pt[c] = allowed ? e : 0.f;
-      }
-      if (it > 0) {
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->dv_done, (it - 1) & 1, abort_flag));
-        if (!ok) break;
-      }
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        ptx::st_shared_v4(sPT + ptx::sw128_offset(r, ch), ptx::pack_bf16x2(pt[8 * ch], pt[8 * ch + 1]),
-                          ptx::pack_bf16x2(pt[8 * ch + 2], pt[8 * ch + 3]),
-                          ptx::pack_bf16x2(pt[8 * ch + 4], pt[8 * ch + 5]),
-                          ptx::pack_bf16x2(pt[8 * ch + 6], pt[8 * ch + 7]));
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->p_full);
-#pragma unroll
-      for (int c = 0; c < 64; ++c) pt[c] = pt[c] * (__uint_as_float(dpt[c / 32][c % 32]) - vd[c]);
-      if (it > 0) {
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->dk_done, (it - 1) & 1, abort_flag));
-        if (!ok) break;
-      }
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        ptx::st_shared_v4(sDST + ptx::sw128_offset(r, ch), ptx::pack_bf16x2(pt[8 * ch], pt[8 * ch + 1]),
-                          ptx::pack_bf16x2(pt[8 * ch + 2], pt[8 * ch + 3]),
-                          ptx::pack_bf16x2(pt[8 * ch + 4], pt[8 * ch + 5]),
-                          ptx::pack_bf16x2(pt[8 * ch + 6], pt[8 * ch + 7]));
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->ds_full);
-    }
-    // ------------------------------------------------------------ epilogue
-    if (ok) ok = __all_sync(0xffffffffu, bar_wait(&bars->dk_done, (nq - 1) & 1, abort_flag));
-    if (ok) {
-      ptx::tc_fence_after();
-      // dV -> the K tile's smem, scale * dK -> the V tile's smem (both free now)
+      const uint32_t src = tmem + lane_base + (w == 0 ? C::TM_DV : C::TM_DK);
+      const float mul = (w == 0) ? 1.f : p.scale;
+      uint16_t* grow = static_cast<uint16_t*>(w == 0 ? p.dv : p.dk) + ((int64_t)U.bh * N + j) * D;
 #pragma unroll 1
-      for (int which = 0; which < 2; ++which) {
-        const uint32_t src = tmem + lane_base + (which == 0 ? C::TM_DV : C::TM_DK);
-        const uint32_t dst = which == 0 ? sK : sV;
-        const float mul = which == 0 ? 1.f : p.scale;
-#pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
-          uint32_t g[32];
-          ptx::tmem_ld32(src + c, g);
-          ptx::tmem_wait_ld();
-          ptx::reg_fence(g);
+      for (int c = 0; c < D; c += 32) {
+        uint32_t g[32];
+        ptx::tmem_ld32(src + c, g);
+        ptx::tmem_wait_ld();
+        ptx::reg_fence(g);
+        if (j < N) {
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int col = c + q * 8;
-            const uint32_t addr = dst + (col / 64) * (C::BK * 128) + ptx::sw128_offset(r, (col % 64) / 8);
             const float* f = reinterpret_cast<const float*>(&g[8 * q]);
-            ptx::st_shared_v4(addr, ptx::pack_bf16x2(f[0] * mul, f[1] * mul),
+            ptx::st_global_v4(grow + c + 8 * q, ptx::pack_bf16x2(f[0] * mul, f[1] * mul),
                               ptx::pack_bf16x2(f[2] * mul, f[3] * mul),
                               ptx::pack_bf16x2(f[4] * mul, f[5] * mul),
                               ptx::pack_bf16x2(f[6] * mul, f[7] * mul));
           }
         }
       }
-      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars->acc_free);
     }
-    ptx::named_bar_sync(1, 128);
-    if (!*abort_flag && threadIdx.x == 0) {
-      for (int c = 0; c < C::DB; ++c) {
-        ptx::tma_store_3d(&tm_dv, smem + C::OFF_K + c * (C::BK * 128), c * 64, (int)j0, bh);
-        ptx::tma_store_3d(&tm_dk, smem + C::OFF_V + c * (C::BK * 128), c * 64, (int)j0, bh);
+  }
+
+  // ------------------------------------------------------------ keys no query reaches
+  {
+    const int num_fill = p.B * p.fills_per_batch;
+    const int nkt = (int)((N + 127) / 128);
+    for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
+      const int b = f / p.fills_per_batch;
+      int r = f % p.fills_per_batch;
+      int h = 0;
+      for (; h < p.H; ++h) {
+        const int cnt = nkt - dkv_units_of_head(N, p.lo[h]);
+        if (r < cnt) break;
+        r -= cnt;
       }
-      ptx::bulk_commit_group();
-      ptx::bulk_wait_group_all();
+      const int64_t kt = dkv_units_of_head(N, p.lo[h]) + r;
+      const int64_t row0 = (int64_t)(b * p.H + h) * N + kt * 128;
+      const int64_t rows = min64(kt * 128 + 128, N) - kt * 128;
+      zero_rows_bf16(static_cast<uint16_t*>(p.dk) + row0 * D, rows, D);
+      zero_rows_bf16(static_cast<uint16_t*>(p.dv) + row0 * D, rows, D);
     }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }
 }
 
 // ---------------------------------------------------------------------------
-// dQ: one CTA per (query tile of 128, h, b); key tiles of 64.
+// dQ: persistent grid; a unit is (b, h, query tile of 128 rows), walking the
+// same 128-key strip as the forward.  Per key tile j:
+//   S_j = Q K^T      SS MMA -> TMEM S buffer j % 2 ([0,128) or [128,256))
+//   dP  = dO V^T     SS MMA -> TMEM [256,384)
+//   dS  = P (dP - D), P = exp2(S c - lse2) masked on edge tiles; written as
+//                    bf16 over S buffer j % 2
+//   dQ += dS K       TS MMA (A = dS from TMEM, B = K MN-major) -> TMEM [384,512)
+// Two warpgroups share each tile: warpgroup w owns key columns [64w, 64w+64)
+// of every query row (thread r = row r = TMEM lane r).  S of the next key
+// tile goes to the other buffer before dQ of this one, so the tensor core
+// runs while the warpgroups work.  Epilogue: scale * dQ straight from TMEM to
+// global, warpgroup w writing head dims [D/2 w, D/2 (w+1)).
 // ---------------------------------------------------------------------------
 template <int D>
 struct DqCfg {
-  static constexpr int BQ = 128;  // queries per CTA (MMA M)
-  static constexpr int BK = 64;   // keys per step
-  static constexpr int NS = 2;
+  static constexpr int BQ = 128;  // queries per unit (MMA M)
+  static constexpr int BK = 128;  // keys per step
+  static constexpr int NS = 2;    // K/V ring stages
   static constexpr int DB = D / 64;
   static constexpr uint32_t QT_BYTES = BQ * D * 2;
   static constexpr uint32_t KT_BYTES = BK * D * 2;
-  static constexpr uint32_t DS_BYTES = BQ * BK * 2;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_DO = OFF_Q + QT_BYTES;
   static constexpr uint32_t OFF_K = OFF_DO + QT_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + NS * KT_BYTES;
-  static constexpr uint32_t OFF_DS = OFF_V + NS * KT_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_DS + DS_BYTES;
-  static constexpr uint32_t SMEM_BYTES = OFF_BAR + 256 + 1024;
-  static constexpr uint32_t TM_S = 0, TM_DP = 64, TM_DQ = 128;
-  static constexpr uint32_t TMEM_COLS = 256;
+  static constexpr uint32_t OFF_BAR = OFF_V + NS * KT_BYTES;
+  static constexpr uint32_t SMEM_BYTES =
+      (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
+  static constexpr int NTHREADS = 320;
+  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_DP = 256, TM_DQ = 384;
+  static constexpr uint32_t TMEM_COLS = 512;
 };
 
 struct DqBars {
-  uint64_t qdo_full;
-  uint64_t kv_full[2], kv_empty[2];
-  uint64_t s_full, s_free, ds_full, dq_done, drain;
+  uint64_t q_full, q_empty;
+  uint64_t k_full[2], v_full[2], kv_empty[2];
+  uint64_t s_full[2], dp_full, ds_full;  // s_full[b]: S buffer b written
+  uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
   int abort;
 };
 
+struct DqUnit {
+  int bh;
+  int32_t lo, hi;
+  int64_t i0;
+  int ka, kb;  // key tiles walked
+};
+
+__device__ __forceinline__ DqUnit dq_decode(int u, const AttnParams& p) {
+  DqUnit U;
+  const int nqt = (int)((p.N + 127) / 128);
+  const int b = u / p.units_per_batch;
+  int r = u % p.units_per_batch;
+  int h = 0;
+  for (; h < p.H; ++h) {
+    const int cnt = nqt - p.lo[h] / 128;
+    if (r < cnt) break;
+    r -= cnt;
+  }
+  U.bh = b * p.H + h;
+  U.lo = p.lo[h];
+  U.hi = p.hi[h];
+  U.i0 = (int64_t)(p.lo[h] / 128 + r) * 128;
+  const Strip s = key_strip(p.N, U.lo, U.hi, U.i0, 128, 128);
+  U.ka = s.begin;
+  U.kb = s.end;
+  return U;
+}
+
 template <int D>
-__global__ void __launch_bounds__(192, 1)
+__global__ void __launch_bounds__(320, 1)
     spa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                      const __grid_constant__ CUtensorMap tm_dq, const __grid_constant__ AttnParams p) {
+                      const __grid_constant__ AttnParams p) {
   using C = DqCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
   DqBars* bars = reinterpret_cast<DqBars*>(smem + C::OFF_BAR);
-
-  const int t = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
-  const int bh = b * p.H + h;
-  const int64_t N = p.N;
-  const int32_t lo = p.lo[h], hi = p.hi[h];
-  const int64_t i0 = (int64_t)t * C::BQ;
-  const Strip strip = key_strip(N, lo, hi, i0, C::BQ, C::BK);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
-  const int64_t rows_here = min64(i0 + C::BQ, N) - i0;
-
-  if (strip.end < strip.begin) {
-    zero_rows_bf16(static_cast<uint16_t*>(p.dq) + ((int64_t)bh * N + i0) * D, rows_here, D);
-    return;
-  }
-  const int nk = strip.end - strip.begin + 1;
+  const int64_t N = p.N;
+  const int num_units = p.B * p.units_per_batch;
 
   const uint32_t sQ = ptx::smem_u32(smem + C::OFF_Q);
   const uint32_t sDO = ptx::smem_u32(smem + C::OFF_DO);
   const uint32_t sK = ptx::smem_u32(smem + C::OFF_K);
   const uint32_t sV = ptx::smem_u32(smem + C::OFF_V);
-  const uint32_t sDS = ptx::smem_u32(smem + C::OFF_DS);
 
   if (threadIdx.x == 0) {
-    ptx::mbar_init(&bars->qdo_full, 1);
+    ptx::mbar_init(&bars->q_full, 1);
+    ptx::mbar_init(&bars->q_empty, 1);
     for (int s = 0; s < 2; ++s) {
-      ptx::mbar_init(&bars->kv_full[s], 1);
+      ptx::mbar_init(&bars->k_full[s], 1);
+      ptx::mbar_init(&bars->v_full[s], 1);
       ptx::mbar_init(&bars->kv_empty[s], 1);
     }
-    ptx::mbar_init(&bars->s_full, 1);
-    ptx::mbar_init(&bars->s_free, 128);
-    ptx::mbar_init(&bars->ds_full, 128);
-    ptx::mbar_init(&bars->dq_done, 1);
+    ptx::mbar_init(&bars->s_full[0], 1);
+    ptx::mbar_init(&bars->s_full[1], 1);
+    ptx::mbar_init(&bars->dp_full, 1);
+    ptx::mbar_init(&bars->ds_full, 256);
+    ptx::mbar_init(&bars->acc_done, 1);
+    ptx::mbar_init(&bars->acc_free, 256);
     ptx::mbar_init(&bars->drain, 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
@@ -447,164 +560,246 @@ __global__ void __launch_bounds__(192, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
 
-  if (warp == 4) {
+  if (warp == 8) {
+    // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
-      ptx::mbar_arrive_expect_tx(&bars->qdo_full, 2 * C::QT_BYTES);
-      for (int c = 0; c < C::DB; ++c) {
-        ptx::tma_load_3d(smem + C::OFF_Q + c * (C::BQ * 128), &tm_q, &bars->qdo_full, c * 64, (int)i0, bh);
-        ptx::tma_load_3d(smem + C::OFF_DO + c * (C::BQ * 128), &tm_do, &bars->qdo_full, c * 64, (int)i0, bh);
-      }
-      int armed[2] = {0, 0};
-      for (int it = 0; it < nk; ++it) {
-        const int s = it % C::NS;
-        if (!bar_wait(&bars->kv_empty[s], ((it / C::NS) & 1) ^ 1, abort_flag)) break;
-        const int jt = (strip.begin + it) * C::BK;
-        ptx::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * C::KT_BYTES);
+      int nq = 0, g = 0, armed[2] = {0, 0};
+      bool ok = true;
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const DqUnit U = dq_decode(u, p);
+        ok = bar_wait(&bars->q_empty, (nq & 1) ^ 1, abort_flag);
+        if (!ok) break;
+        ++nq;
+        ptx::mbar_arrive_expect_tx(&bars->q_full, 2 * C::QT_BYTES);
         for (int c = 0; c < C::DB; ++c) {
-          ptx::tma_load_3d(smem + C::OFF_K + s * C::KT_BYTES + c * (C::BK * 128), &tm_k, &bars->kv_full[s],
-                           c * 64, jt, bh);
-          ptx::tma_load_3d(smem + C::OFF_V + s * C::KT_BYTES + c * (C::BK * 128), &tm_v, &bars->kv_full[s],
-                           c * 64, jt, bh);
+          ptx::tma_load_3d(smem + C::OFF_Q + c * (C::BQ * 128), &tm_q, &bars->q_full, c * 64, (int)U.i0, U.bh);
+          ptx::tma_load_3d(smem + C::OFF_DO + c * (C::BQ * 128), &tm_do, &bars->q_full, c * 64, (int)U.i0, U.bh);
         }
-        armed[s]++;
+        for (int kt = U.ka; ok && kt <= U.kb; ++kt, ++g) {
+          const int s = g % C::NS;
+          ok = bar_wait(&bars->kv_empty[s], ((g / C::NS) & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          const int j0 = kt * C::BK;
+          ptx::mbar_arrive_expect_tx(&bars->k_full[s], C::KT_BYTES);
+          for (int c = 0; c < C::DB; ++c)
+            ptx::tma_load_3d(smem + C::OFF_K + s * C::KT_BYTES + c * (C::BK * 128), &tm_k, &bars->k_full[s],
+                             c * 64, j0, U.bh);
+          ptx::mbar_arrive_expect_tx(&bars->v_full[s], C::KT_BYTES);
+          for (int c = 0; c < C::DB; ++c)
+            ptx::tma_load_3d(smem + C::OFF_V + s * C::KT_BYTES + c * (C::BK * 128), &tm_v, &bars->v_full[s],
+                             c * 64, j0, U.bh);
+          ++armed[s];
+        }
       }
-      bar_drain(&bars->qdo_full, 0);
+      if (nq > 0) bar_drain(&bars->q_full, (nq - 1) & 1);
       for (int s = 0; s < C::NS; ++s)
-        if (armed[s] > 0) bar_drain(&bars->kv_full[s], (armed[s] - 1) & 1);
+        if (armed[s] > 0) {
+          bar_drain(&bars->k_full[s], (armed[s] - 1) & 1);
+          bar_drain(&bars->v_full[s], (armed[s] - 1) & 1);
+        }
     }
     __syncwarp();
-  } else if (warp == 5) {
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BK, false, false);
       constexpr uint32_t idesc_g = ptx::idesc_bf16_f32(128, D, false, true);
-      bool ok = bar_wait(&bars->qdo_full, 0, abort_flag);
-      for (int it = 0; ok && it < nk; ++it) {
-        const int s = it % C::NS;
-        ok = bar_wait(&bars->kv_full[s], (it / C::NS) & 1, abort_flag) &&
-             bar_wait(&bars->s_free, (it & 1) ^ 1, abort_flag);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        const uint32_t kb = sK + s * C::KT_BYTES, vb = sV + s * C::KT_BYTES;
-        // S = Q K^T and dP = dO V^T
+      int nq = 0, g = 0, gs = 0, cds = 0, cacc = 0;
+      bool ok = true;
+      auto issue_nt = [&](uint32_t dst, uint32_t a_base, uint32_t b_base) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qa = (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-          const uint32_t ka = (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
-          ptx::mma_bf16(tmem + C::TM_S, ptx::sdesc_sw128(sQ + qa, 0, 1024),
-                        ptx::sdesc_sw128(kb + ka, 0, 1024), idesc_s, kk > 0);
+          const uint32_t a = a_base + (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
+          const uint32_t b = b_base + (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
+          ptx::mma_bf16(tmem + dst, ptx::sdesc_sw128(a, 0, 1024), ptx::sdesc_sw128(b, 0, 1024), idesc_s, kk > 0);
         }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t qa = (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-          const uint32_t ka = (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
-          ptx::mma_bf16(tmem + C::TM_DP, ptx::sdesc_sw128(sDO + qa, 0, 1024),
-                        ptx::sdesc_sw128(vb + ka, 0, 1024), idesc_s, kk > 0);
-        }
-        ptx::mma_commit(&bars->s_full);
-        // dQ += dS K  (dS K-major along keys; K MN-major along d)
-        ok = bar_wait(&bars->ds_full, it & 1, abort_flag);
+      };
+      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+        const DqUnit U = dq_decode(u, p);
+        const int nk = U.kb - U.ka + 1;
+        const int g0 = g;
+        auto slot = [&](int jj) { return (g0 + jj) % C::NS; };
+        auto par = [&](int jj) { return (uint32_t)(((g0 + jj) / C::NS) & 1); };
+        auto sbuf = [&](int jj) { return ((gs + jj) & 1) ? C::TM_S1 : C::TM_S0; };
+        auto sbar = [&](int jj) { return &bars->s_full[(gs + jj) & 1]; };
+        ok = bar_wait(&bars->q_full, (nq++) & 1, abort_flag) && bar_wait(&bars->k_full[slot(0)], par(0), abort_flag);
         if (!ok) break;
         ptx::tc_fence_after();
+        issue_nt(sbuf(0), sQ, sK + slot(0) * C::KT_BYTES);
+        ptx::mma_commit(sbar(0));
+        ok = bar_wait(&bars->v_full[slot(0)], par(0), abort_flag);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_nt(C::TM_DP, sDO, sV + slot(0) * C::KT_BYTES);
+        ptx::mma_commit(&bars->dp_full);
+        for (int j = 0; j < nk; ++j) {
+          if (j + 1 < nk) {
+            ok = bar_wait(&bars->k_full[slot(j + 1)], par(j + 1), abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_nt(sbuf(j + 1), sQ, sK + slot(j + 1) * C::KT_BYTES);  // S of the next key tile
+            ptx::mma_commit(sbar(j + 1));
+          }
+          ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
+          if (ok && j == 0) ok = bar_wait(&bars->acc_free, (cacc & 1) ^ 1, abort_flag);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          {
+            // dQ += dS K: A = dS (bf16 pairs over S buffer j, key halves at +0 / +64),
+            // B = K tile MN-major along d
+            const uint32_t kb = sK + slot(j) * C::KT_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          ptx::mma_bf16(tmem + C::TM_DQ, ptx::sdesc_sw128(sDS + kk * 32, 0, 1024),
-                        ptx::sdesc_sw128(kb + kk * (16 * 128), C::BK * 128, 1024), idesc_g,
-                        (it > 0 || kk > 0));
-        ptx::mma_commit(&bars->dq_done);
-        ptx::mma_commit(&bars->kv_empty[s]);
+            for (int kk = 0; kk < C::BK / 16; ++kk) {
+              const uint32_t acol = sbuf(j) + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
+              ptx::mma_bf16_ts(tmem + C::TM_DQ, tmem + acol,
+                               ptx::sdesc_sw128(kb + kk * (16 * 128), C::BK * 128, 1024), idesc_g,
+                               (j > 0 || kk > 0));
+            }
+          }
+          ptx::mma_commit(&bars->kv_empty[slot(j)]);
+          if (j + 1 < nk) {
+            ok = bar_wait(&bars->v_full[slot(j + 1)], par(j + 1), abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_nt(C::TM_DP, sDO, sV + slot(j + 1) * C::KT_BYTES);  // dP of the next key tile
+            ptx::mma_commit(&bars->dp_full);
+          }
+        }
+        if (!ok) break;
+        ++cacc;
+        ptx::mma_commit(&bars->acc_done);
+        ptx::mma_commit(&bars->q_empty);
+        g = g0 + nk;
+        gs += nk;
       }
       ptx::mma_commit(&bars->drain);
       bar_drain(&bars->drain, 0);
     }
     __syncwarp();
   } else {
-    const int r = threadIdx.x;
-    const int64_t i = i0 + r;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const float lse2 = (i < N) ? p.lse[(int64_t)bh * N + i] * kLog2e : 0.f;
-    const float Di = (i < N) ? p.delta[(int64_t)bh * N + i] : 0.f;
+    // ------------------------------------------------------------ element-wise warpgroups
+    const int w = warp / 4;                      // key columns [64w, 64w+64)
+    const int r = threadIdx.x - 128 * w;         // query row = TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const float c2 = p.scale_log2;
+    int gs = 0, cdp = 0, cacc = 0;
     bool ok = true;
-    for (int it = 0; it < nk; ++it) {
-      ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, it & 1, abort_flag));
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+      const DqUnit U = dq_decode(u, p);
+      const int64_t i = U.i0 + r;
+      const bool in = i < N;
+      const float lse2 = in ? p.lse[(int64_t)U.bh * N + i] * kLog2e : 0.f;
+      const float Di = in ? p.delta[(int64_t)U.bh * N + i] : 0.f;
+      const float nlse2 = -lse2;
+      for (int kt = U.ka; kt <= U.kb; ++kt, ++gs) {
+        const uint32_t tS = tmem + lane_base + ((gs & 1) ? C::TM_S1 : C::TM_S0) + 64 * w;
+        const uint32_t tDP = tmem + lane_base + C::TM_DP + 64 * w;
+        const int64_t j0 = (int64_t)kt * C::BK;
+        const bool interior = tile_is_interior(N, U.lo, U.hi, U.i0, C::BQ, j0, C::BK);
+        int clo = 0;
+        uint32_t span = 127;
+        if (!interior) {
+          const int64_t c_first = max64(i - U.hi + 1 - j0, 0);
+          const int64_t c_last = min64(min64(i - U.lo - j0, N - 1 - j0), 127);
+          if (!in || c_last < c_first) {
+            clo = 128;
+            span = 0;
+          } else {
+            clo = (int)c_first;
+            span = (uint32_t)(c_last - c_first);
+          }
+        }
+        const int cb = 64 * w - clo;
+        // buffer gs & 1 is used for the (gs >> 1)-th time
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[gs & 1], (gs >> 1) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        float pv[64];
+        {
+          uint32_t sr[2][32];
+          ptx::tmem_ld32(tS, sr[0]);
+          ptx::tmem_ld32(tS + 32, sr[1]);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(sr[0]);
+          ptx::reg_fence(sr[1]);
+#pragma unroll
+          for (int e = 0; e < 64; ++e) {
+            const float ev = ptx::exp2_approx(fmaf(__uint_as_float(sr[e / 32][e % 32]), c2, nlse2));
+            pv[e] = (interior || (uint32_t)(cb + e) <= span) ? ev : 0.f;
+          }
+        }
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->dp_full, (cdp++) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        {
+          uint32_t dr[2][32];
+          ptx::tmem_ld32(tDP, dr[0]);
+          ptx::tmem_ld32(tDP + 32, dr[1]);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(dr[0]);
+          ptx::reg_fence(dr[1]);
+          uint32_t pk[32];
+#pragma unroll
+          for (int e = 0; e < 32; ++e) {
+            const float d0 = pv[2 * e] * (__uint_as_float(dr[(2 * e) / 32][(2 * e) % 32]) - Di);
+            const float d1 = pv[2 * e + 1] * (__uint_as_float(dr[(2 * e + 1) / 32][(2 * e + 1) % 32]) - Di);
+            pk[e] = ptx::pack_bf16x2(d0, d1);
+          }
+          ptx::tmem_st32(tS, pk);
+          ptx::tmem_wait_st();
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->ds_full);
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint32_t sv[2][32], dp[2][32];
-      ptx::tmem_ld32(tmem + lane_base + C::TM_S, sv[0]);
-      ptx::tmem_ld32(tmem + lane_base + C::TM_S + 32, sv[1]);
-      ptx::tmem_ld32(tmem + lane_base + C::TM_DP, dp[0]);
-      ptx::tmem_ld32(tmem + lane_base + C::TM_DP + 32, dp[1]);
-      ptx::tmem_wait_ld();
-      ptx::reg_fence(sv[0]);
-      ptx::reg_fence(sv[1]);
-      ptx::reg_fence(dp[0]);
-      ptx::reg_fence(dp[1]);
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->s_free);
-
-      const int64_t jt = (int64_t)(strip.begin + it) * C::BK;
-      const bool interior = tile_is_interior(N, lo, hi, i0, C::BQ, jt, C::BK);
-      const int64_t dist0 = i - jt;
-      float ds[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        const float e = ptx::exp2_approx(__uint_as_float(sv[c / 32][c % 32]) * p.scale_log2 - lse2);
-        bool allowed = true;
-        if (!interior) {
-          const int64_t dd = dist0 - c;
-          allowed = (dd >= lo) && (dd < hi) && (jt + c < N) && (i < N);
-        }
-        const float pv = allowed ? e : 0.f;
-        ds[c] = pv * (__uint_as_float(dp[c / 32][c % 32]) - Di);
-      }
-      if (it > 0) {
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->dq_done, (it - 1) & 1, abort_flag));
-        if (!ok) break;
-      }
-#pragma unroll
-      for (int ch = 0; ch < 8; ++ch)
-        ptx::st_shared_v4(sDS + ptx::sw128_offset(r, ch), ptx::pack_bf16x2(ds[8 * ch], ds[8 * ch + 1]),
-                          ptx::pack_bf16x2(ds[8 * ch + 2], ds[8 * ch + 3]),
-                          ptx::pack_bf16x2(ds[8 * ch + 4], ds[8 * ch + 5]),
-                          ptx::pack_bf16x2(ds[8 * ch + 6], ds[8 * ch + 7]));
-      ptx::fence_proxy_async_smem();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->ds_full);
-    }
-    if (ok) ok = __all_sync(0xffffffffu, bar_wait(&bars->dq_done, (nk - 1) & 1, abort_flag));
-    if (ok) {
-      ptx::tc_fence_after();
+      uint16_t* grow = static_cast<uint16_t*>(p.dq) + ((int64_t)U.bh * N + i) * D;
+      const float mul = p.scale;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
+      for (int c = w * (D / 2); c < (w + 1) * (D / 2); c += 32) {
         uint32_t g[32];
         ptx::tmem_ld32(tmem + lane_base + C::TM_DQ + c, g);
         ptx::tmem_wait_ld();
         ptx::reg_fence(g);
+        if (in) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int col = c + q * 8;
-          const uint32_t addr = sQ + (col / 64) * (C::BQ * 128) + ptx::sw128_offset(r, (col % 64) / 8);
-          const float* f = reinterpret_cast<const float*>(&g[8 * q]);
-          const float mul = p.scale;
-          ptx::st_shared_v4(addr, ptx::pack_bf16x2(f[0] * mul, f[1] * mul),
-                            ptx::pack_bf16x2(f[2] * mul, f[3] * mul),
-                            ptx::pack_bf16x2(f[4] * mul, f[5] * mul),
-                            ptx::pack_bf16x2(f[6] * mul, f[7] * mul));
+          for (int q = 0; q < 4; ++q) {
+            const float* f = reinterpret_cast<const float*>(&g[8 * q]);
+            ptx::st_global_v4(grow + c + 8 * q, ptx::pack_bf16x2(f[0] * mul, f[1] * mul),
+                              ptx::pack_bf16x2(f[2] * mul, f[3] * mul),
+                              ptx::pack_bf16x2(f[4] * mul, f[5] * mul),
+                              ptx::pack_bf16x2(f[6] * mul, f[7] * mul));
+          }
         }
       }
-      ptx::fence_proxy_async_smem();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars->acc_free);
     }
-    ptx::named_bar_sync(1, 128);
-    if (!*abort_flag && threadIdx.x == 0) {
-      for (int c = 0; c < C::DB; ++c)
-        ptx::tma_store_3d(&tm_dq, smem + C::OFF_Q + c * (C::BQ * 128), c * 64, (int)i0, bh);
-      ptx::bulk_commit_group();
-      ptx::bulk_wait_group_all();
+  }
+
+  // ------------------------------------------------------------ rows before their band
+  {
+    const int num_fill = p.B * p.fills_per_batch;
+    for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
+      const int b = f / p.fills_per_batch;
+      int r = f % p.fills_per_batch;
+      int h = 0;
+      for (; h < p.H; ++h) {
+        const int cnt = p.lo[h] / 128;
+        if (r < cnt) break;
+        r -= cnt;
+      }
+      const int64_t row0 = (int64_t)(b * p.H + h) * N + (int64_t)r * 128;
+      zero_rows_bf16(static_cast<uint16_t*>(p.dq) + row0 * D, 128, D);
     }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 5) {
+  if (warp == 9) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -171,27 +171,49 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if ((st = launch_status())) return st;
   }
   if (steps & kStepDkDv) {
-    // key tiles of 128 rows, query tiles of 64 rows
-    CUtensorMap kq, kk, kv, kdo, kdk, kdv;
+    // persistent grid over key tiles of 128 that some query reaches; the
+    // other key tiles only get zero rows
+    CUtensorMap kq, kk, kv, kdo;
     if ((st = make_map(&kq, q, p.N, BH, D, KC::BQ)) || (st = make_map(&kk, k, p.N, BH, D, KC::BK)) ||
-        (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)) ||
-        (st = make_map(&kdk, dk, p.N, BH, D, KC::BK)) || (st = make_map(&kdv, dv, p.N, BH, D, KC::BK)))
+        (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)))
       return st;
     if ((st = prepare_kernel(spa::spa_bwd_dkdv_kernel<D>, KC::SMEM_BYTES, prepared_kv))) return st;
-    dim3 gkv((unsigned)((p.N + KC::BK - 1) / KC::BK), (unsigned)p.H, (unsigned)p.B);
-    spa::spa_bwd_dkdv_kernel<D><<<gkv, 192, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
+    const int64_t nkt = (p.N + 127) / 128;
+    int64_t upb = 0;
+    for (int h = 0; h < p.H; ++h) upb += (p.N - 1 - p.lo[h]) / 128 + 1;
+    const int64_t fpb = (int64_t)p.H * nkt - upb;
+    if ((int64_t)p.B * p.H * nkt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+    p.units_per_batch = (int)upb;
+    p.fills_per_batch = (int)fpb;
+    int sms = 0;
+    if ((st = sm_count(&sms))) return st;
+    const int64_t units = (int64_t)p.B * upb;
+    const unsigned grid = (unsigned)(units < sms ? units : sms);
+    spa::spa_bwd_dkdv_kernel<D><<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, p);
     if ((st = launch_status())) return st;
   }
   if (steps & kStepDq) {
-    // query tiles of 128 rows, key tiles of 64 rows
-    CUtensorMap qq, qk, qv, qdo, qdq;
+    // persistent grid over query tiles of 128 with a row inside its band; the
+    // whole tiles before the band only get zero rows
+    CUtensorMap qq, qk, qv, qdo;
     if ((st = make_map(&qq, q, p.N, BH, D, QC::BQ)) || (st = make_map(&qk, k, p.N, BH, D, QC::BK)) ||
-        (st = make_map(&qv, v, p.N, BH, D, QC::BK)) || (st = make_map(&qdo, dout, p.N, BH, D, QC::BQ)) ||
-        (st = make_map(&qdq, dq, p.N, BH, D, QC::BQ)))
+        (st = make_map(&qv, v, p.N, BH, D, QC::BK)) || (st = make_map(&qdo, dout, p.N, BH, D, QC::BQ)))
       return st;
     if ((st = prepare_kernel(spa::spa_bwd_dq_kernel<D>, QC::SMEM_BYTES, prepared_q))) return st;
-    dim3 gq((unsigned)((p.N + QC::BQ - 1) / QC::BQ), (unsigned)p.H, (unsigned)p.B);
-    spa::spa_bwd_dq_kernel<D><<<gq, 192, QC::SMEM_BYTES, stream>>>(qq, qk, qv, qdo, qdq, p);
+    const int64_t nqt = (p.N + 127) / 128;
+    int64_t upb = 0, fpb = 0;
+    for (int h = 0; h < p.H; ++h) {
+      upb += nqt - p.lo[h] / 128;
+      fpb += p.lo[h] / 128;
+    }
+    if ((int64_t)p.B * p.H * nqt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+    p.units_per_batch = (int)upb;
+    p.fills_per_batch = (int)fpb;
+    int sms = 0;
+    if ((st = sm_count(&sms))) return st;
+    const int64_t units = (int64_t)p.B * upb;
+    const unsigned grid = (unsigned)(units < sms ? units : sms);
+    spa::spa_bwd_dq_kernel<D><<<grid, QC::NTHREADS, QC::SMEM_BYTES, stream>>>(qq, qk, qv, qdo, p);
     if ((st = launch_status())) return st;
   }
   return SPA_OK;
