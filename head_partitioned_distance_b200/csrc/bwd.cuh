@@ -90,7 +90,7 @@ struct DkvCfg {
 
 struct DkvBars {
   uint64_t kv_full, kv_empty;
-  uint64_t q_full[2], q_empty[2];
+  uint64_t q_full[2], q_empty[2], vec_full[2];
   uint64_t s_full, dp_full, p_full, ds_full;
   uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
@@ -154,6 +154,7 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars->q_full[s], 1);
       ptx::mbar_init(&bars->q_empty[s], 1);
+      ptx::mbar_init(&bars->vec_full[s], 1);
     }
     ptx::mbar_init(&bars->s_full, 1);
     ptx::mbar_init(&bars->dp_full, 1);
@@ -196,16 +197,6 @@ __global__ void __launch_bounds__(320, 1)
         ok = __all_sync(0xffffffffu, bar_wait(&bars->q_empty[s], ((gq / C::NS) & 1) ^ 1, abort_flag));
         if (!ok) break;
         const int64_t i0 = (int64_t)qt * C::BQ;
-        // lse (base 2) and D of this step's queries, for the element-wise warps
-        float* vl = vec + s * 2 * C::BQ;
-        float* vd = vl + C::BQ;
-        for (int c = lane; c < C::BQ; c += 32) {
-          const int64_t i = i0 + c;
-          const bool in = i < N;
-          vl[c] = in ? p.lse[(int64_t)U.bh * N + i] * kLog2e : 0.f;
-          vd[c] = in ? p.delta[(int64_t)U.bh * N + i] : 0.f;
-        }
-        __syncwarp();
         if (lane == 0) {
           ptx::mbar_arrive_expect_tx(&bars->q_full[s], 2 * C::QT_BYTES);
           for (int c = 0; c < C::DB; ++c) {
@@ -215,6 +206,18 @@ __global__ void __launch_bounds__(320, 1)
                              &bars->q_full[s], c * 64, (int)i0, U.bh);
           }
         }
+        // lse (base 2) and D of this step's queries, for the element-wise
+        // warps; behind their own barrier so the tile copies above go first
+        float* vl = vec + s * 2 * C::BQ;
+        float* vd = vl + C::BQ;
+        for (int c = lane; c < C::BQ; c += 32) {
+          const int64_t i = i0 + c;
+          const bool in = i < N;
+          vl[c] = in ? p.lse[(int64_t)U.bh * N + i] * kLog2e : 0.f;
+          vd[c] = in ? p.delta[(int64_t)U.bh * N + i] : 0.f;
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->vec_full[s]);
         ++armed[s];
       }
     }
@@ -331,56 +334,64 @@ __global__ void __launch_bounds__(320, 1)
         const float* vl = vec + s * 2 * C::BQ + 64 * w;
         const float* vd = vl + C::BQ;
         const int cb = 64 * w - qlo;
-        // ---- P^T = exp2(S^T c - lse2)
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, (cs++) & 1, abort_flag));
+        // ---- P^T = exp2(S^T c - lse2), two 32-column chunks; chunk h writes its
+        // bf16 pairs to columns [16h, 16h + 16), inside chunk 0 (already read)
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->vec_full[s], (gq / C::NS) & 1, abort_flag) &&
+                                         bar_wait(&bars->s_full, (cs++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
         float pt[64];
-        {
-          uint32_t sr[2][32];
-          ptx::tmem_ld32(tS, sr[0]);
-          ptx::tmem_ld32(tS + 32, sr[1]);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          uint32_t sr[32];
+          ptx::tmem_ld32(tS + 32 * h, sr);
           ptx::tmem_wait_ld();
-          ptx::reg_fence(sr[0]);
-          ptx::reg_fence(sr[1]);
+          ptx::reg_fence(sr);
+          uint32_t pk[16];
+          if (interior) {
+            // every query permitted; one exponential in four on the FMA pipe
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const float x = fmaf(__uint_as_float(sr[e / 32][e % 32]), c2, -vl[e]);
-            const float ev = ptx::exp2_approx(x);
-            pt[e] = (interior || (uint32_t)(cb + e) <= span) ? ev : 0.f;
+            for (int e = 0; e < 32; ++e) {
+              const int q = 32 * h + e;
+              const float x = fmaf(__uint_as_float(sr[e]), c2, -vl[q]);
+              pt[q] = ((e & 3) == 3) ? exp2_poly(x) : ptx::exp2_approx(x);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const int q = 32 * h + e;
+              const float ev = ptx::exp2_approx(fmaf(__uint_as_float(sr[e]), c2, -vl[q]));
+              pt[q] = (uint32_t)(cb + q) <= span ? ev : 0.f;
+            }
           }
-        }
-        {
-          uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = ptx::pack_bf16x2(pt[2 * e], pt[2 * e + 1]);
-          ptx::tmem_st32(tS, pk);
-          ptx::tmem_wait_st();
+          for (int e = 0; e < 16; ++e) pk[e] = ptx::pack_bf16x2(pt[32 * h + 2 * e], pt[32 * h + 2 * e + 1]);
+          ptx::tmem_st16(tS + 16 * h, pk);
         }
+        ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full);
         // ---- dS^T = P^T (dP^T - D)
         ok = __all_sync(0xffffffffu, bar_wait(&bars->dp_full, (cdp++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
-        {
-          uint32_t dr[2][32];
-          ptx::tmem_ld32(tDP, dr[0]);
-          ptx::tmem_ld32(tDP + 32, dr[1]);
-          ptx::tmem_wait_ld();
-          ptx::reg_fence(dr[0]);
-          ptx::reg_fence(dr[1]);
-          uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float d0 = pt[2 * e] * (__uint_as_float(dr[(2 * e) / 32][(2 * e) % 32]) - vd[2 * e]);
-            const float d1 =
-                pt[2 * e + 1] * (__uint_as_float(dr[(2 * e + 1) / 32][(2 * e + 1) % 32]) - vd[2 * e + 1]);
+        for (int h = 0; h < 2; ++h) {
+          uint32_t dr[32];
+          ptx::tmem_ld32(tDP + 32 * h, dr);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(dr);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int q = 32 * h + 2 * e;
+            const float d0 = pt[q] * (__uint_as_float(dr[2 * e]) - vd[q]);
+            const float d1 = pt[q + 1] * (__uint_as_float(dr[2 * e + 1]) - vd[q + 1]);
             pk[e] = ptx::pack_bf16x2(d0, d1);
           }
-          ptx::tmem_st32(tDP, pk);
-          ptx::tmem_wait_st();
+          ptx::tmem_st16(tDP + 16 * h, pk);
         }
+        ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->ds_full);
       }

@@ -5,6 +5,7 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include "fastexp.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
 

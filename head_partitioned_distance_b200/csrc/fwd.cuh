@@ -405,27 +405,42 @@ __global__ void __launch_bounds__(320, 1)
           ptx::tmem_wait_ld();
           ptx::reg_fence(sr);
           uint32_t pk[16];
-          const int cb = q * 32 - clo;
+          if (interior) {
+            // every key permitted; one exponential in four on the FMA pipe
 #pragma unroll
-          for (int e = 0; e < 32; e += 4) {
-            float x0 = fmaf(__uint_as_float(sr[e]), c2, mneg);
-            float x1 = fmaf(__uint_as_float(sr[e + 1]), c2, mneg);
-            float x2 = fmaf(__uint_as_float(sr[e + 2]), c2, mneg);
-            float x3 = fmaf(__uint_as_float(sr[e + 3]), c2, mneg);
-            if (!interior) {
+            for (int e = 0; e < 32; e += 4) {
+              const float p0 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e]), c2, mneg));
+              const float p1 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 1]), c2, mneg));
+              const float p2 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 2]), c2, mneg));
+              const float p3 = exp2_poly(fmaf(__uint_as_float(sr[e + 3]), c2, mneg));
+              sm0 += p0;
+              sm1 += p1;
+              sm2 += p2;
+              sm3 += p3;
+              pk[e / 2] = ptx::pack_bf16x2(p0, p1);
+              pk[e / 2 + 1] = ptx::pack_bf16x2(p2, p3);
+            }
+          } else {
+            const int cb = q * 32 - clo;
+#pragma unroll
+            for (int e = 0; e < 32; e += 4) {
+              float x0 = fmaf(__uint_as_float(sr[e]), c2, mneg);
+              float x1 = fmaf(__uint_as_float(sr[e + 1]), c2, mneg);
+              float x2 = fmaf(__uint_as_float(sr[e + 2]), c2, mneg);
+              float x3 = fmaf(__uint_as_float(sr[e + 3]), c2, mneg);
               x0 = (uint32_t)(cb + e) <= span ? x0 : -INFINITY;
               x1 = (uint32_t)(cb + e + 1) <= span ? x1 : -INFINITY;
               x2 = (uint32_t)(cb + e + 2) <= span ? x2 : -INFINITY;
               x3 = (uint32_t)(cb + e + 3) <= span ? x3 : -INFINITY;
+              const float p0 = ptx::exp2_approx(x0), p1 = ptx::exp2_approx(x1);
+              const float p2 = ptx::exp2_approx(x2), p3 = ptx::exp2_approx(x3);
+              sm0 += p0;
+              sm1 += p1;
+              sm2 += p2;
+              sm3 += p3;
+              pk[e / 2] = ptx::pack_bf16x2(p0, p1);
+              pk[e / 2 + 1] = ptx::pack_bf16x2(p2, p3);
             }
-            const float p0 = ptx::exp2_approx(x0), p1 = ptx::exp2_approx(x1);
-            const float p2 = ptx::exp2_approx(x2), p3 = ptx::exp2_approx(x3);
-            sm0 += p0;
-            sm1 += p1;
-            sm2 += p2;
-            sm3 += p3;
-            pk[e / 2] = ptx::pack_bf16x2(p0, p1);
-            pk[e / 2 + 1] = ptx::pack_bf16x2(p2, p3);
           }
           ptx::tmem_st16(tS + q * 16, pk);
         }

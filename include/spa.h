@@ -199,6 +199,14 @@ SPA_API int spa_tile_classes_device(int64_t N, int H, const int32_t* lo, const i
                             int Bk, uint8_t* tile_class_dev, void* stream);
 
 /*
+ * Test hook: y[i] = the kernels' FMA-pipe 2^x (Cody-Waite range reduction and
+ * a degree-3 minimax polynomial; relative error below 1.5e-4 for
+ * -126 <= x <= 127, inputs below -126 clamped) for n floats.  x, y: DEVICE
+ * buffers of n floats; asynchronous on `stream`.
+ */
+SPA_API int spa_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
+
+/*
  * Synchronises `stream` and returns the library's device error word, then
  * clears it: SPA_OK, or SPA_ERR_TIMEOUT when a kernel gave up on a wait (the
  * kernel then wrote incomplete outputs and released its tensor memory).
