@@ -79,8 +79,9 @@ struct DkvCfg {
   static constexpr uint32_t OFF_V = OFF_K + KT_BYTES;
   static constexpr uint32_t OFF_Q = OFF_V + KT_BYTES;
   static constexpr uint32_t OFF_DO = OFF_Q + NS * QT_BYTES;
-  static constexpr uint32_t OFF_VEC = OFF_DO + NS * QT_BYTES;  // [NS][2][BQ] floats: lse2, D
-  static constexpr uint32_t OFF_BAR = OFF_VEC + NS * 2 * BQ * 4;
+  // [2 warpgroups][2 buffers][128 floats]: lse2 then D of the warpgroup's 64 queries
+  static constexpr uint32_t OFF_VEC = OFF_DO + NS * QT_BYTES;
+  static constexpr uint32_t OFF_BAR = OFF_VEC + 2 * 2 * 128 * 4;
   static constexpr uint32_t SMEM_BYTES =
       (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
   static constexpr int NTHREADS = 320;
@@ -90,7 +91,7 @@ struct DkvCfg {
 
 struct DkvBars {
   uint64_t kv_full, kv_empty;
-  uint64_t q_full[2], q_empty[2], vec_full[2];
+  uint64_t q_full[2], q_empty[2];
   uint64_t s_full, dp_full, p_full, ds_full;
   uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
@@ -154,7 +155,6 @@ __global__ void __launch_bounds__(320, 1)
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars->q_full[s], 1);
       ptx::mbar_init(&bars->q_empty[s], 1);
-      ptx::mbar_init(&bars->vec_full[s], 1);
     }
     ptx::mbar_init(&bars->s_full, 1);
     ptx::mbar_init(&bars->dp_full, 1);
@@ -180,9 +180,9 @@ __global__ void __launch_bounds__(320, 1)
     // ------------------------------------------------------------ producer warp
     int nkv = 0, gq = 0, armed[2] = {0, 0};
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+    for (int u = blockIdx.x; ok && lane == 0 && u < num_units; u += gridDim.x) {
       const DkvUnit U = dkv_decode(u, p);
-      ok = __all_sync(0xffffffffu, bar_wait(&bars->kv_empty, (nkv & 1) ^ 1, abort_flag));
+      ok = bar_wait(&bars->kv_empty, (nkv & 1) ^ 1, abort_flag);
       if (!ok) break;
       if (lane == 0) {
         ptx::mbar_arrive_expect_tx(&bars->kv_full, 2 * C::KT_BYTES);
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(320, 1)
       ++nkv;
       for (int qt = U.qa; qt <= U.qb; ++qt, ++gq) {
         const int s = gq % C::NS;
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->q_empty[s], ((gq / C::NS) & 1) ^ 1, abort_flag));
+        ok = bar_wait(&bars->q_empty[s], ((gq / C::NS) & 1) ^ 1, abort_flag);
         if (!ok) break;
         const int64_t i0 = (int64_t)qt * C::BQ;
         if (lane == 0) {
@@ -206,18 +206,6 @@ __global__ void __launch_bounds__(320, 1)
                              &bars->q_full[s], c * 64, (int)i0, U.bh);
           }
         }
-        // lse (base 2) and D of this step's queries, for the element-wise
-        // warps; behind their own barrier so the tile copies above go first
-        float* vl = vec + s * 2 * C::BQ;
-        float* vd = vl + C::BQ;
-        for (int c = lane; c < C::BQ; c += 32) {
-          const int64_t i = i0 + c;
-          const bool in = i < N;
-          vl[c] = in ? p.lse[(int64_t)U.bh * N + i] * kLog2e : 0.f;
-          vd[c] = in ? p.delta[(int64_t)U.bh * N + i] : 0.f;
-        }
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bars->vec_full[s]);
         ++armed[s];
       }
     }
@@ -307,14 +295,37 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tS = tmem + lane_base + C::TM_ST + 64 * w;
     const uint32_t tDP = tmem + lane_base + C::TM_DPT + 64 * w;
     const float c2 = p.scale_log2;
+    float* vecw = vec + w * 256;                     // this warpgroup's two vector buffers
+    // Thread r fetches one value of the (lse2, D) vector a query tile needs:
+    // lse2 of query 64w + r for r < 64, else D of query 64w + r - 64.
+    auto fetch = [&](int bh, int64_t i0) -> float {
+      const int64_t i = i0 + 64 * w + (r & 63);
+      if (i >= N) return 0.f;
+      return r < 64 ? p.lse[(int64_t)bh * N + i] * kLog2e : p.delta[(int64_t)bh * N + i];
+    };
     int gq = 0, cs = 0, cdp = 0, cacc = 0;
     bool ok = true;
+    if (blockIdx.x < num_units) {
+      const DkvUnit U0 = dkv_decode(blockIdx.x, p);
+      vecw[r] = fetch(U0.bh, (int64_t)U0.qa * C::BQ);
+    }
+    ptx::named_bar_sync(1 + w, 128);
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
       const DkvUnit U = dkv_decode(u, p);
       const int64_t j = U.j0 + r;
       for (int qt = U.qa; qt <= U.qb; ++qt, ++gq) {
-        const int s = gq % C::NS;
         const int64_t i0 = (int64_t)qt * C::BQ;
+        // prefetch the vectors of the next query tile (this unit's or the next unit's first)
+        float pre = 0.f;
+        bool has_next = true;
+        if (qt < U.qb) {
+          pre = fetch(U.bh, i0 + C::BQ);
+        } else if (u + (int)gridDim.x < num_units) {
+          const DkvUnit Un = dkv_decode(u + gridDim.x, p);
+          pre = fetch(Un.bh, (int64_t)Un.qa * C::BQ);
+        } else {
+          has_next = false;
+        }
         const bool interior = tile_is_interior(N, U.lo, U.hi, i0, C::BQ, U.j0, C::BK);
         // Edge tile: query column q (0..127) is permitted for this key iff
         // qlo <= q <= qlo + span.
@@ -331,69 +342,72 @@ __global__ void __launch_bounds__(320, 1)
             span = (uint32_t)(q_last - q_first);
           }
         }
-        const float* vl = vec + s * 2 * C::BQ + 64 * w;
-        const float* vd = vl + C::BQ;
+        const float* vl = vecw + (gq & 1) * 128;
+        const float* vd = vl + 64;
         const int cb = 64 * w - qlo;
-        // ---- P^T = exp2(S^T c - lse2), two 32-column chunks; chunk h writes its
-        // bf16 pairs to columns [16h, 16h + 16), inside chunk 0 (already read)
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->vec_full[s], (gq / C::NS) & 1, abort_flag) &&
-                                         bar_wait(&bars->s_full, (cs++) & 1, abort_flag));
+        // ---- P^T = exp2(S^T c - lse2); bf16 pairs to columns [0, 32) of the
+        // warpgroup's 64 (already read)
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, (cs++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
         float pt[64];
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t sr[32];
-          ptx::tmem_ld32(tS + 32 * h, sr);
+        {
+          uint32_t sr[2][32];
+          ptx::tmem_ld32(tS, sr[0]);
+          ptx::tmem_ld32(tS + 32, sr[1]);
           ptx::tmem_wait_ld();
-          ptx::reg_fence(sr);
-          uint32_t pk[16];
+          ptx::reg_fence(sr[0]);
+          ptx::reg_fence(sr[1]);
           if (interior) {
             // every query permitted; one exponential in four on the FMA pipe
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int q = 32 * h + e;
-              const float x = fmaf(__uint_as_float(sr[e]), c2, -vl[q]);
-              pt[q] = ((e & 3) == 3) ? exp2_poly(x) : ptx::exp2_approx(x);
+            for (int q = 0; q < 64; ++q) {
+              const float x = fmaf(__uint_as_float(sr[q / 32][q % 32]), c2, -vl[q]);
+              pt[q] = ((q & 3) == 3) ? exp2_poly(x) : ptx::exp2_approx(x);
             }
           } else {
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int q = 32 * h + e;
-              const float ev = ptx::exp2_approx(fmaf(__uint_as_float(sr[e]), c2, -vl[q]));
+            for (int q = 0; q < 64; ++q) {
+              const float ev = ptx::exp2_approx(fmaf(__uint_as_float(sr[q / 32][q % 32]), c2, -vl[q]));
               pt[q] = (uint32_t)(cb + q) <= span ? ev : 0.f;
             }
           }
+          uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) pk[e] = ptx::pack_bf16x2(pt[32 * h + 2 * e], pt[32 * h + 2 * e + 1]);
-          ptx::tmem_st16(tS + 16 * h, pk);
+          for (int e = 0; e < 32; ++e) pk[e] = ptx::pack_bf16x2(pt[2 * e], pt[2 * e + 1]);
+          ptx::tmem_st32(tS, pk);
+          ptx::tmem_wait_st();
         }
-        ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full);
         // ---- dS^T = P^T (dP^T - D)
         ok = __all_sync(0xffffffffu, bar_wait(&bars->dp_full, (cdp++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t dr[32];
-          ptx::tmem_ld32(tDP + 32 * h, dr);
+        {
+          uint32_t dr[2][32];
+          ptx::tmem_ld32(tDP, dr[0]);
+          ptx::tmem_ld32(tDP + 32, dr[1]);
           ptx::tmem_wait_ld();
-          ptx::reg_fence(dr);
-          uint32_t pk[16];
+          ptx::reg_fence(dr[0]);
+          ptx::reg_fence(dr[1]);
+          uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int q = 32 * h + 2 * e;
-            const float d0 = pt[q] * (__uint_as_float(dr[2 * e]) - vd[q]);
-            const float d1 = pt[q + 1] * (__uint_as_float(dr[2 * e + 1]) - vd[q + 1]);
+          for (int e = 0; e < 32; ++e) {
+            const int q = 2 * e;
+            const float d0 = pt[q] * (__uint_as_float(dr[q / 32][q % 32]) - vd[q]);
+            const float d1 = pt[q + 1] * (__uint_as_float(dr[(q + 1) / 32][(q + 1) % 32]) - vd[q + 1]);
             pk[e] = ptx::pack_bf16x2(d0, d1);
           }
-          ptx::tmem_st16(tDP + 16 * h, pk);
+          ptx::tmem_st32(tDP, pk);
+          ptx::tmem_wait_st();
         }
-        ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->ds_full);
+        // publish the prefetched vectors; every thread of the warpgroup is past
+        // its last read of that buffer (the previous tile)
+        if (has_next) vecw[((gq + 1) & 1) * 128 + r] = pre;
+        ptx::named_bar_sync(1 + w, 128);
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
@@ -404,15 +418,17 @@ __global__ void __launch_bounds__(320, 1)
       const float mul = (w == 0) ? 1.f : p.scale;
       uint16_t* grow = static_cast<uint16_t*>(w == 0 ? p.dv : p.dk) + ((int64_t)U.bh * N + j) * D;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t g[32];
-        ptx::tmem_ld32(src + c, g);
+      for (int c = 0; c < D; c += 64) {
+        uint32_t g[2][32];
+        ptx::tmem_ld32(src + c, g[0]);
+        ptx::tmem_ld32(src + c + 32, g[1]);
         ptx::tmem_wait_ld();
-        ptx::reg_fence(g);
+        ptx::reg_fence(g[0]);
+        ptx::reg_fence(g[1]);
         if (j < N) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float* f = reinterpret_cast<const float*>(&g[8 * q]);
+          for (int q = 0; q < 8; ++q) {
+            const float* f = reinterpret_cast<const float*>(&g[q / 4][8 * (q % 4)]);
             ptx::st_global_v4(grow + c + 8 * q, ptx::pack_bf16x2(f[0] * mul, f[1] * mul),
                               ptx::pack_bf16x2(f[2] * mul, f[3] * mul),
                               ptx::pack_bf16x2(f[4] * mul, f[5] * mul),
