@@ -84,7 +84,11 @@ struct DkvCfg {
   static constexpr uint32_t OFF_BAR = OFF_VEC + 2 * 2 * 128 * 4;
   static constexpr uint32_t SMEM_BYTES =
       (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
-  static constexpr int NTHREADS = 320;
+  static constexpr int NTHREADS = 384;
+  // register split: 384 threads launch with 168 registers each; the two
+  // element-wise warpgroups take 192, the producer/MMA warpgroup 120.
+  static constexpr uint32_t LAUNCH_REGS = 168, EW_REGS = 192, CONTROL_REGS = 120;
+  static_assert(2 * EW_REGS + CONTROL_REGS <= 3 * LAUNCH_REGS, "register split over budget");
   static constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 384;
   static constexpr uint32_t TMEM_COLS = 512;
 };
@@ -131,7 +135,7 @@ __device__ __forceinline__ DkvUnit dkv_decode(int u, const AttnParams& p) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     spa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ AttnParams p) {
@@ -176,7 +180,11 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
 
-  if (warp == 8) {
+  if (warp >= 8) {
+    ptx::regs_dec<C::CONTROL_REGS>();
+  if (warp >= 10) {
+    // idle warps of the control warpgroup
+  } else if (warp == 8) {
     // ------------------------------------------------------------ producer warp
     int nkv = 0, gq = 0, armed[2] = {0, 0};
     bool ok = true;
@@ -223,23 +231,30 @@ __global__ void __launch_bounds__(320, 1)
       int nkv = 0, gq = 0, cp = 0, cds = 0, cacc = 0;
       bool ok = true;
       auto qstage = [&](int g) { return g % C::NS; };
-      auto issue_nt = [&](uint32_t dst, uint32_t a_base, int g) {  // dst = A (keys) x B^T (queries)
-        const uint32_t bb = (a_base == sK ? sQ : sDO) + qstage(g) * C::QT_BYTES;
+      // descriptors of every operand buffer, built once
+      const uint64_t dK = ptx::sdesc_sw128(sK, 0, 1024), dV = ptx::sdesc_sw128(sV, 0, 1024);
+      // K-major (B of S^T/dP^T) and MN-major (B of dK/dV) views of both Q/dO stages
+      const uint64_t dQk0 = ptx::sdesc_sw128(sQ, 0, 1024), dQk1 = ptx::sdesc_sw128(sQ + C::QT_BYTES, 0, 1024);
+      const uint64_t dOk0 = ptx::sdesc_sw128(sDO, 0, 1024), dOk1 = ptx::sdesc_sw128(sDO + C::QT_BYTES, 0, 1024);
+      const uint64_t dQm0 = ptx::sdesc_sw128(sQ, C::BQ * 128, 1024);
+      const uint64_t dQm1 = ptx::sdesc_sw128(sQ + C::QT_BYTES, C::BQ * 128, 1024);
+      const uint64_t dOm0 = ptx::sdesc_sw128(sDO, C::BQ * 128, 1024);
+      const uint64_t dOm1 = ptx::sdesc_sw128(sDO + C::QT_BYTES, C::BQ * 128, 1024);
+      auto dQk = [&](int st) { return st ? dQk1 : dQk0; };
+      auto dOk = [&](int st) { return st ? dOk1 : dOk0; };
+      auto dQm = [&](int st) { return st ? dQm1 : dQm0; };
+      auto dOm = [&](int st) { return st ? dOm1 : dOm0; };
+      auto issue_nt = [&](uint32_t dst, uint64_t da, uint64_t db) {  // dst = A (keys) x B^T (queries)
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = a_base + (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
-          const uint32_t b = bb + (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-          ptx::mma_bf16(tmem + dst, ptx::sdesc_sw128(a, 0, 1024), ptx::sdesc_sw128(b, 0, 1024), idesc_s, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          ptx::mma_bf16(tmem + dst, ptx::sdesc_advance(da, (kk / 4) * (C::BK * 128) + (kk % 4) * 32),
+                        ptx::sdesc_advance(db, (kk / 4) * (C::BQ * 128) + (kk % 4) * 32), idesc_s, kk > 0);
       };
-      auto issue_grad = [&](uint32_t dst, uint32_t a_col, uint32_t b_base, int g, bool first) {
-        const uint32_t bb = b_base + qstage(g) * C::QT_BYTES;
+      auto issue_grad = [&](uint32_t dst, uint32_t a_col, uint64_t db, bool first) {
 #pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk) {
-          const uint32_t acol = a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
-          ptx::mma_bf16_ts(tmem + dst, tmem + acol, ptx::sdesc_sw128(bb + kk * (16 * 128), C::BQ * 128, 1024),
-                           idesc_g, (!first || kk > 0));
-        }
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          ptx::mma_bf16_ts(tmem + dst, tmem + a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
+                           ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (!first || kk > 0));
       };
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
         const DkvUnit U = dkv_decode(u, p);
@@ -249,9 +264,9 @@ __global__ void __launch_bounds__(320, 1)
              bar_wait(&bars->q_full[qstage(g0)], (g0 / C::NS) & 1, abort_flag);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_nt(C::TM_ST, sK, g0);
+        issue_nt(C::TM_ST, dK, dQk(qstage(g0)));
         ptx::mma_commit(&bars->s_full);
-        issue_nt(C::TM_DPT, sV, g0);
+        issue_nt(C::TM_DPT, dV, dOk(qstage(g0)));
         ptx::mma_commit(&bars->dp_full);
         for (int j = 0; j < nq; ++j) {
           const int g = g0 + j;
@@ -259,21 +274,21 @@ __global__ void __launch_bounds__(320, 1)
           if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
-          issue_grad(C::TM_DV, C::TM_ST, sDO, g, j == 0);          // dV += P^T dO
+          issue_grad(C::TM_DV, C::TM_ST, dOm(qstage(g)), j == 0);   // dV += P^T dO
           if (j + 1 < nq) {
             ok = bar_wait(&bars->q_full[qstage(g + 1)], ((g + 1) / C::NS) & 1, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_nt(C::TM_ST, sK, g + 1);                         // S^T of the next tile
+            issue_nt(C::TM_ST, dK, dQk(qstage(g + 1)));            // S^T of the next tile
             ptx::mma_commit(&bars->s_full);
           }
           ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
-          issue_grad(C::TM_DK, C::TM_DPT, sQ, g, j == 0);          // dK += dS^T Q
+          issue_grad(C::TM_DK, C::TM_DPT, dQm(qstage(g)), j == 0);  // dK += dS^T Q
           ptx::mma_commit(&bars->q_empty[qstage(g)]);
           if (j + 1 < nq) {
-            issue_nt(C::TM_DPT, sV, g + 1);                        // dP^T of the next tile
+            issue_nt(C::TM_DPT, dV, dOk(qstage(g + 1)));           // dP^T of the next tile
             ptx::mma_commit(&bars->dp_full);
           }
         }
@@ -287,7 +302,9 @@ __global__ void __launch_bounds__(320, 1)
       bar_drain(&bars->drain, 0);
     }
     __syncwarp();
+  }
   } else {
+    ptx::regs_inc<C::EW_REGS>();
     // ------------------------------------------------------------ element-wise warpgroups
     const int w = warp / 4;                          // query columns [64w, 64w+64)
     const int r = threadIdx.x - 128 * w;             // key row = TMEM lane
@@ -296,18 +313,21 @@ __global__ void __launch_bounds__(320, 1)
     const uint32_t tDP = tmem + lane_base + C::TM_DPT + 64 * w;
     const float c2 = p.scale_log2;
     float* vecw = vec + w * 256;                     // this warpgroup's two vector buffers
-    // Thread r fetches one value of the (lse2, D) vector a query tile needs:
-    // lse2 of query 64w + r for r < 64, else D of query 64w + r - 64.
+    // Thread r fetches one value of the vectors a query tile needs: lse of
+    // query 64w + r for r < 64, else D of query 64w + r - 64.  The shared
+    // copy holds -lse * log2(e) and -D (see publish()), ready for fused
+    // multiply-adds; the conversion waits until the load has long landed.
     auto fetch = [&](int bh, int64_t i0) -> float {
       const int64_t i = i0 + 64 * w + (r & 63);
       if (i >= N) return 0.f;
-      return r < 64 ? p.lse[(int64_t)bh * N + i] * kLog2e : p.delta[(int64_t)bh * N + i];
+      return r < 64 ? p.lse[(int64_t)bh * N + i] : p.delta[(int64_t)bh * N + i];
     };
+    auto publish = [&](float raw) { return r < 64 ? -raw * kLog2e : -raw; };
     int gq = 0, cs = 0, cdp = 0, cacc = 0;
     bool ok = true;
     if (blockIdx.x < num_units) {
       const DkvUnit U0 = dkv_decode(blockIdx.x, p);
-      vecw[r] = fetch(U0.bh, (int64_t)U0.qa * C::BQ);
+      vecw[r] = publish(fetch(U0.bh, (int64_t)U0.qa * C::BQ));
     }
     ptx::named_bar_sync(1 + w, 128);
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
@@ -358,18 +378,47 @@ __global__ void __launch_bounds__(320, 1)
           ptx::tmem_wait_ld();
           ptx::reg_fence(sr[0]);
           ptx::reg_fence(sr[1]);
+          // vl holds -lse2 of the 64 queries: x = s * c2 - lse2 in pairs
+          const float4* nl4 = reinterpret_cast<const float4*>(vl);
+          const float2 c2v = make_float2(c2, c2);
           if (interior) {
-            // every query permitted; one exponential in four on the FMA pipe
+            // every query permitted; one exponential pair in four on the FMA pipe
 #pragma unroll
-            for (int q = 0; q < 64; ++q) {
-              const float x = fmaf(__uint_as_float(sr[q / 32][q % 32]), c2, -vl[q]);
-              pt[q] = ((q & 3) == 3) ? exp2_poly(x) : ptx::exp2_approx(x);
+            for (int q4 = 0; q4 < 16; ++q4) {
+              const float4 nl = nl4[q4];
+              const int q = 4 * q4;
+              const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[q / 32][q % 32]),
+                                                       __uint_as_float(sr[q / 32][q % 32 + 1])),
+                                           c2v, make_float2(nl.x, nl.y));
+              const float2 xb = __ffma2_rn(make_float2(__uint_as_float(sr[q / 32][q % 32 + 2]),
+                                                       __uint_as_float(sr[q / 32][q % 32 + 3])),
+                                           c2v, make_float2(nl.z, nl.w));
+              pt[q] = ptx::exp2_approx(xa.x);
+              pt[q + 1] = ptx::exp2_approx(xa.y);
+              if ((q4 & 1) == 1) {
+                const float2 pb = exp2_poly2(xb);
+                pt[q + 2] = pb.x;
+                pt[q + 3] = pb.y;
+              } else {
+                pt[q + 2] = ptx::exp2_approx(xb.x);
+                pt[q + 3] = ptx::exp2_approx(xb.y);
+              }
             }
           } else {
 #pragma unroll
-            for (int q = 0; q < 64; ++q) {
-              const float ev = ptx::exp2_approx(fmaf(__uint_as_float(sr[q / 32][q % 32]), c2, -vl[q]));
-              pt[q] = (uint32_t)(cb + q) <= span ? ev : 0.f;
+            for (int q4 = 0; q4 < 16; ++q4) {
+              const float4 nl = nl4[q4];
+              const int q = 4 * q4;
+              const float2 xa = __ffma2_rn(make_float2(__uint_as_float(sr[q / 32][q % 32]),
+                                                       __uint_as_float(sr[q / 32][q % 32 + 1])),
+                                           c2v, make_float2(nl.x, nl.y));
+              const float2 xb = __ffma2_rn(make_float2(__uint_as_float(sr[q / 32][q % 32 + 2]),
+                                                       __uint_as_float(sr[q / 32][q % 32 + 3])),
+                                           c2v, make_float2(nl.z, nl.w));
+              pt[q] = (uint32_t)(cb + q) <= span ? ptx::exp2_approx(xa.x) : 0.f;
+              pt[q + 1] = (uint32_t)(cb + q + 1) <= span ? ptx::exp2_approx(xa.y) : 0.f;
+              pt[q + 2] = (uint32_t)(cb + q + 2) <= span ? ptx::exp2_approx(xb.x) : 0.f;
+              pt[q + 3] = (uint32_t)(cb + q + 3) <= span ? ptx::exp2_approx(xb.y) : 0.f;
             }
           }
           uint32_t pk[32];
@@ -391,13 +440,23 @@ __global__ void __launch_bounds__(320, 1)
           ptx::tmem_wait_ld();
           ptx::reg_fence(dr[0]);
           ptx::reg_fence(dr[1]);
+          // vd holds -D of the 64 queries: dS = P (dP - D) in pairs
+          const float4* nd4 = reinterpret_cast<const float4*>(vd);
           uint32_t pk[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const int q = 2 * e;
-            const float d0 = pt[q] * (__uint_as_float(dr[q / 32][q % 32]) - vd[q]);
-            const float d1 = pt[q + 1] * (__uint_as_float(dr[(q + 1) / 32][(q + 1) % 32]) - vd[q + 1]);
-            pk[e] = ptx::pack_bf16x2(d0, d1);
+          for (int q4 = 0; q4 < 16; ++q4) {
+            const float4 nd = nd4[q4];
+            const int q = 4 * q4;
+            const float2 da = __fmul2_rn(make_float2(pt[q], pt[q + 1]),
+                                         __fadd2_rn(make_float2(__uint_as_float(dr[q / 32][q % 32]),
+                                                                __uint_as_float(dr[q / 32][q % 32 + 1])),
+                                                    make_float2(nd.x, nd.y)));
+            const float2 db = __fmul2_rn(make_float2(pt[q + 2], pt[q + 3]),
+                                         __fadd2_rn(make_float2(__uint_as_float(dr[q / 32][q % 32 + 2]),
+                                                                __uint_as_float(dr[q / 32][q % 32 + 3])),
+                                                    make_float2(nd.z, nd.w)));
+            pk[2 * q4] = ptx::pack_bf16x2(da.x, da.y);
+            pk[2 * q4 + 1] = ptx::pack_bf16x2(db.x, db.y);
           }
           ptx::tmem_st32(tDP, pk);
           ptx::tmem_wait_st();
@@ -406,7 +465,7 @@ __global__ void __launch_bounds__(320, 1)
         ptx::mbar_arrive(&bars->ds_full);
         // publish the prefetched vectors; every thread of the warpgroup is past
         // its last read of that buffer (the previous tile)
-        if (has_next) vecw[((gq + 1) & 1) * 128 + r] = pre;
+        if (has_next) vecw[((gq + 1) & 1) * 128 + r] = publish(pre);
         ptx::named_bar_sync(1 + w, 128);
       }
       if (!ok) break;
@@ -426,14 +485,8 @@ __global__ void __launch_bounds__(320, 1)
         ptx::reg_fence(g[0]);
         ptx::reg_fence(g[1]);
         if (j < N) {
-#pragma unroll
-          for (int q = 0; q < 8; ++q) {
-            const float* f = reinterpret_cast<const float*>(&g[q / 4][8 * (q % 4)]);
-            ptx::st_global_v4(grow + c + 8 * q, ptx::pack_bf16x2(f[0] * mul, f[1] * mul),
-                              ptx::pack_bf16x2(f[2] * mul, f[3] * mul),
-                              ptx::pack_bf16x2(f[4] * mul, f[5] * mul),
-                              ptx::pack_bf16x2(f[6] * mul, f[7] * mul));
-          }
+          ptx::store_row32_bf16(grow + c, g[0], mul);
+          ptx::store_row32_bf16(grow + c + 32, g[1], mul);
         }
       }
       ptx::tc_fence_before();
@@ -499,7 +552,11 @@ struct DqCfg {
   static constexpr uint32_t OFF_BAR = OFF_V + NS * KT_BYTES;
   static constexpr uint32_t SMEM_BYTES =
       (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
-  static constexpr int NTHREADS = 320;
+  static constexpr int NTHREADS = 384;
+  // register split: 384 threads launch with 168 registers each; the two
+  // element-wise warpgroups take 192, the producer/MMA warpgroup 120.
+  static constexpr uint32_t LAUNCH_REGS = 168, EW_REGS = 192, CONTROL_REGS = 120;
+  static_assert(2 * EW_REGS + CONTROL_REGS <= 3 * LAUNCH_REGS, "register split over budget");
   static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_DP = 256, TM_DQ = 384;
   static constexpr uint32_t TMEM_COLS = 512;
 };
@@ -542,7 +599,7 @@ __device__ __forceinline__ DqUnit dq_decode(int u, const AttnParams& p) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     spa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                       const __grid_constant__ AttnParams p) {
@@ -587,7 +644,11 @@ __global__ void __launch_bounds__(320, 1)
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
 
-  if (warp == 8) {
+  if (warp >= 8) {
+    ptx::regs_dec<C::CONTROL_REGS>();
+  if (warp >= 10) {
+    // idle warps of the control warpgroup
+  } else if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int nq = 0, g = 0, armed[2] = {0, 0};
@@ -633,13 +694,21 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t idesc_g = ptx::idesc_bf16_f32(128, D, false, true);
       int nq = 0, g = 0, gs = 0, cds = 0, cacc = 0;
       bool ok = true;
-      auto issue_nt = [&](uint32_t dst, uint32_t a_base, uint32_t b_base) {
+      // descriptors of every operand buffer, built once
+      const uint64_t dQd = ptx::sdesc_sw128(sQ, 0, 1024), dOd = ptx::sdesc_sw128(sDO, 0, 1024);
+      // K-major (B of S/dP) and MN-major K (B of dQ) views of both K/V stages
+      const uint64_t dKk0 = ptx::sdesc_sw128(sK, 0, 1024), dKk1 = ptx::sdesc_sw128(sK + C::KT_BYTES, 0, 1024);
+      const uint64_t dVk0 = ptx::sdesc_sw128(sV, 0, 1024), dVk1 = ptx::sdesc_sw128(sV + C::KT_BYTES, 0, 1024);
+      const uint64_t dKm0 = ptx::sdesc_sw128(sK, C::BK * 128, 1024);
+      const uint64_t dKm1 = ptx::sdesc_sw128(sK + C::KT_BYTES, C::BK * 128, 1024);
+      auto dKk = [&](int st) { return st ? dKk1 : dKk0; };
+      auto dVk = [&](int st) { return st ? dVk1 : dVk0; };
+      auto dKm = [&](int st) { return st ? dKm1 : dKm0; };
+      auto issue_nt = [&](uint32_t dst, uint64_t da, uint64_t db) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = a_base + (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-          const uint32_t b = b_base + (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
-          ptx::mma_bf16(tmem + dst, ptx::sdesc_sw128(a, 0, 1024), ptx::sdesc_sw128(b, 0, 1024), idesc_s, kk > 0);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          ptx::mma_bf16(tmem + dst, ptx::sdesc_advance(da, (kk / 4) * (C::BQ * 128) + (kk % 4) * 32),
+                        ptx::sdesc_advance(db, (kk / 4) * (C::BK * 128) + (kk % 4) * 32), idesc_s, kk > 0);
       };
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
         const DqUnit U = dq_decode(u, p);
@@ -652,19 +721,19 @@ __global__ void __launch_bounds__(320, 1)
         ok = bar_wait(&bars->q_full, (nq++) & 1, abort_flag) && bar_wait(&bars->k_full[slot(0)], par(0), abort_flag);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_nt(sbuf(0), sQ, sK + slot(0) * C::KT_BYTES);
+        issue_nt(sbuf(0), dQd, dKk(slot(0)));
         ptx::mma_commit(sbar(0));
         ok = bar_wait(&bars->v_full[slot(0)], par(0), abort_flag);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_nt(C::TM_DP, sDO, sV + slot(0) * C::KT_BYTES);
+        issue_nt(C::TM_DP, dOd, dVk(slot(0)));
         ptx::mma_commit(&bars->dp_full);
         for (int j = 0; j < nk; ++j) {
           if (j + 1 < nk) {
             ok = bar_wait(&bars->k_full[slot(j + 1)], par(j + 1), abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_nt(sbuf(j + 1), sQ, sK + slot(j + 1) * C::KT_BYTES);  // S of the next key tile
+            issue_nt(sbuf(j + 1), dQd, dKk(slot(j + 1)));              // S of the next key tile
             ptx::mma_commit(sbar(j + 1));
           }
           ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
@@ -674,21 +743,19 @@ __global__ void __launch_bounds__(320, 1)
           {
             // dQ += dS K: A = dS (bf16 pairs over S buffer j, key halves at +0 / +64),
             // B = K tile MN-major along d
-            const uint32_t kb = sK + slot(j) * C::KT_BYTES;
+            const uint64_t db = dKm(slot(j));
+            const uint32_t abase = tmem + sbuf(j);
 #pragma unroll
-            for (int kk = 0; kk < C::BK / 16; ++kk) {
-              const uint32_t acol = sbuf(j) + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8);
-              ptx::mma_bf16_ts(tmem + C::TM_DQ, tmem + acol,
-                               ptx::sdesc_sw128(kb + kk * (16 * 128), C::BK * 128, 1024), idesc_g,
-                               (j > 0 || kk > 0));
-            }
+            for (int kk = 0; kk < C::BK / 16; ++kk)
+              ptx::mma_bf16_ts(tmem + C::TM_DQ, abase + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
+                               ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (j > 0 || kk > 0));
           }
           ptx::mma_commit(&bars->kv_empty[slot(j)]);
           if (j + 1 < nk) {
             ok = bar_wait(&bars->v_full[slot(j + 1)], par(j + 1), abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_nt(C::TM_DP, sDO, sV + slot(j + 1) * C::KT_BYTES);  // dP of the next key tile
+            issue_nt(C::TM_DP, dOd, dVk(slot(j + 1)));                // dP of the next key tile
             ptx::mma_commit(&bars->dp_full);
           }
         }
@@ -703,7 +770,9 @@ __global__ void __launch_bounds__(320, 1)
       bar_drain(&bars->drain, 0);
     }
     __syncwarp();
+  }
   } else {
+    ptx::regs_inc<C::EW_REGS>();
     // ------------------------------------------------------------ element-wise warpgroups
     const int w = warp / 4;                      // key columns [64w, 64w+64)
     const int r = threadIdx.x - 128 * w;         // query row = TMEM lane
@@ -791,16 +860,7 @@ __global__ void __launch_bounds__(320, 1)
         ptx::tmem_ld32(tmem + lane_base + C::TM_DQ + c, g);
         ptx::tmem_wait_ld();
         ptx::reg_fence(g);
-        if (in) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float* f = reinterpret_cast<const float*>(&g[8 * q]);
-            ptx::st_global_v4(grow + c + 8 * q, ptx::pack_bf16x2(f[0] * mul, f[1] * mul),
-                              ptx::pack_bf16x2(f[2] * mul, f[3] * mul),
-                              ptx::pack_bf16x2(f[4] * mul, f[5] * mul),
-                              ptx::pack_bf16x2(f[6] * mul, f[7] * mul));
-          }
-        }
+        if (in) ptx::store_row32_bf16(grow + c, g, mul);
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->acc_free);

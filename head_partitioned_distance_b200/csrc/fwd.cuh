@@ -16,9 +16,11 @@
 // lse are written straight from registers; rows that precede their band get
 // o = 0 and lse = -inf.
 //
-// Warp roles (320 threads): warps 0-3 tile 0, warps 4-7 tile 1 (thread r of a
-// warpgroup owns row r = TMEM lane r), warp 8 TMA producer, warp 9 MMA issuer
-// and TMEM owner.  Every wait is bounded (common.cuh).
+// Warp roles (384 threads): warps 0-3 tile 0, warps 4-7 tile 1 (thread r of a
+// warpgroup owns row r = TMEM lane r), warp 8 TMA producer, warps 9 and 10
+// MMA issuers of tile 0 and tile 1 (warp 9 also owns TMEM), warp 11 idle; the
+// softmax warpgroups take most of the register file (setmaxnreg).  Every wait
+// is bounded (common.cuh).
 //
 // Softmax restricted to a permitted set: "Story of Attention -- Part 4",
 // section 1 (Sparse-Attention equation); bands: "Making Every Head Count",
@@ -47,7 +49,11 @@ struct FwdCfg {
   // columns) owns an SM even for d = 64
   static constexpr uint32_t SMEM_BYTES =
       (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
-  static constexpr int NTHREADS = 320;
+  static constexpr int NTHREADS = 384;
+  // register split: 384 threads launch with 168 registers each (64512); the
+  // two softmax warpgroups take 192, the producer/MMA warpgroup 120.
+  static constexpr uint32_t LAUNCH_REGS = 168, SOFTMAX_REGS = 192, CONTROL_REGS = 120;
+  static_assert(2 * SOFTMAX_REGS + CONTROL_REGS <= 3 * LAUNCH_REGS, "register split over budget");
   static constexpr uint32_t TMEM_COLS = 512;
   // tile t: S_t (and P_t over its first 64 columns) at t*256, O_t at t*256 + 128
   __host__ __device__ static constexpr uint32_t tm_s(int t) { return (uint32_t)t * 256u; }
@@ -59,7 +65,7 @@ struct FwdBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[2], v_full[2], kv_empty[2];
   uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
-  uint64_t drain;
+  uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
 };
@@ -110,7 +116,7 @@ __device__ __forceinline__ FwdUnit fwd_decode(int u, const AttnParams& p) {
 }
 
 template <int D>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     spa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
   using C = FwdCfg<D>;
@@ -131,13 +137,14 @@ __global__ void __launch_bounds__(320, 1)
       ptx::mbar_init(&bars->q_empty[i], 1);
       ptx::mbar_init(&bars->k_full[i], 1);
       ptx::mbar_init(&bars->v_full[i], 1);
-      ptx::mbar_init(&bars->kv_empty[i], 1);
+      ptx::mbar_init(&bars->kv_empty[i], 2);  // one release per MMA issuer
       ptx::mbar_init(&bars->s_full[i], 1);
       ptx::mbar_init(&bars->p_full[i], 128);
       ptx::mbar_init(&bars->o_done[i], 1);
       ptx::mbar_init(&bars->o_free[i], 128);
     }
-    ptx::mbar_init(&bars->drain, 1);
+    ptx::mbar_init(&bars->drain[0], 1);
+    ptx::mbar_init(&bars->drain[1], 1);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -155,8 +162,11 @@ __global__ void __launch_bounds__(320, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = bars->tmem_base;
   volatile int* abort_flag = &bars->abort;
-
-  if (warp == 8) {
+  if (warp >= 8) {
+    ptx::regs_dec<C::CONTROL_REGS>();
+  if (warp == 11) {
+    // idle warp of the control warpgroup
+  } else if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       int nq[2] = {0, 0}, armed[2] = {0, 0};
@@ -200,103 +210,99 @@ __global__ void __launch_bounds__(320, 1)
         }
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else {
+    // ------------------------------------------------------------ MMA issuers
+    // warp 9 issues every MMA of Q tile 0, warp 10 those of Q tile 1; both
+    // walk the unit's whole key range in the same order, so they agree on the
+    // K/V ring, and each releases a K/V stage once (kv_empty counts two).
+    const int t = warp - 9;
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BK, false, false);
       constexpr uint32_t idesc_o = ptx::idesc_bf16_f32(128, D, false, true);
-      int cq0 = 0, cq1 = 0, cp0 = 0, cp1 = 0, co0 = 0, co1 = 0;
+      // descriptors of every operand buffer, built once; a K-step only adds
+      // a constant offset to the start address
+      const uint64_t dq = ptx::sdesc_sw128(sQ + t * C::Q_BYTES, 0, 1024);
+      const uint64_t dk0 = ptx::sdesc_sw128(sK, 0, 1024), dk1 = ptx::sdesc_sw128(sK + C::KV_BYTES, 0, 1024);
+      const uint64_t dv0 = ptx::sdesc_sw128(sV, C::BK * 128, 1024);
+      const uint64_t dv1 = ptx::sdesc_sw128(sV + C::KV_BYTES, C::BK * 128, 1024);
+      const uint32_t tS = tmem + C::tm_s(t), tO = tmem + C::tm_o(t);
+      uint64_t* s_full = &bars->s_full[t];
+      uint64_t* p_full = &bars->p_full[t];
+      int cq = 0, cp = 0, co = 0;
       int g = 0;
       bool ok = true;
-      auto issue_s = [&](int t, int slot) {
-        const uint32_t kb = sK + slot * C::KV_BYTES;
-        const uint32_t qb = sQ + t * C::Q_BYTES;
+      auto issue_s = [&](int slot) {
+        const uint64_t db = slot ? dk1 : dk0;
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = qb + (kk / 4) * (C::BQ * 128) + (kk % 4) * 32;
-          const uint32_t bb = kb + (kk / 4) * (C::BK * 128) + (kk % 4) * 32;
-          ptx::mma_bf16(tmem + C::tm_s(t), ptx::sdesc_sw128(a, 0, 1024), ptx::sdesc_sw128(bb, 0, 1024),
-                        idesc_s, kk > 0);
-        }
-        ptx::mma_commit(&bars->s_full[t]);
+        for (int kk = 0; kk < D / 16; ++kk)
+          ptx::mma_bf16(tS, ptx::sdesc_advance(dq, (kk / 4) * (C::BQ * 128) + (kk % 4) * 32),
+                        ptx::sdesc_advance(db, (kk / 4) * (C::BK * 128) + (kk % 4) * 32), idesc_s, kk > 0);
+        ptx::mma_commit(s_full);
       };
-      auto issue_pv = [&](int t, int slot, bool first) {
-        const uint32_t vb = sV + slot * C::KV_BYTES;
+      auto issue_pv = [&](int slot, bool first) {
+        const uint64_t db = slot ? dv1 : dv0;
+        ptx::mma_bf16_ts(tO, tS, db, idesc_o, !first);
 #pragma unroll
-        for (int kk = 0; kk < C::BK / 16; ++kk)
-          ptx::mma_bf16_ts(tmem + C::tm_o(t), tmem + C::tm_s(t) + kk * 8,
-                           ptx::sdesc_sw128(vb + kk * (16 * 128), C::BK * 128, 1024), idesc_o,
-                           (!first || kk > 0));
+        for (int kk = 1; kk < C::BK / 16; ++kk)
+          ptx::mma_bf16_ts(tO, tS + kk * 8, ptx::sdesc_advance(db, kk * (16 * 128)), idesc_o, 1);
       };
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
         const FwdUnit U = fwd_decode<D>(u, p);
         if (U.u1 < U.u0) continue;
-        auto act = [&](int t, int it) { return U.act[t] && it >= U.a[t] && it <= U.b[t]; };
+        const bool act_t = t ? U.act[1] : U.act[0];
+        const int a_t = t ? U.a[1] : U.a[0];
+        const int b_t = t ? U.b[1] : U.b[0];
+        auto act = [&](int it) { return act_t && it >= a_t && it <= b_t; };
         const int g0 = g;
         auto slot = [&](int it) { return (g0 + it - U.u0) % C::NS; };
         auto ring_par = [&](int it) { return (uint32_t)(((g0 + it - U.u0) / C::NS) & 1); };
-        if (U.act[0]) ok = bar_wait(&bars->q_full[0], (cq0++) & 1, abort_flag);
-        if (ok && U.act[1]) ok = bar_wait(&bars->q_full[1], (cq1++) & 1, abort_flag);
-        bool first0 = true, first1 = true;
+        if (act_t) ok = bar_wait(&bars->q_full[t], (cq++) & 1, abort_flag);
+        bool first = true;
         ok = ok && bar_wait(&bars->k_full[slot(U.u0)], ring_par(U.u0), abort_flag);
         if (!ok) break;
         ptx::tc_fence_after();
-        if (act(0, U.u0)) {
-          issue_s(0, slot(U.u0));
-          if (U.u0 == U.b[0]) ptx::mma_commit(&bars->q_empty[0]);
-        }
-        if (act(1, U.u0)) {
-          issue_s(1, slot(U.u0));
-          if (U.u0 == U.b[1]) ptx::mma_commit(&bars->q_empty[1]);
+        if (act(U.u0)) {
+          issue_s(slot(U.u0));
+          if (U.u0 == b_t) ptx::mma_commit(&bars->q_empty[t]);
         }
         for (int it = U.u0; ok && it <= U.u1; ++it) {
           const int s = slot(it);
-          const bool nxt = it + 1 <= U.u1;
           ok = bar_wait(&bars->v_full[s], ring_par(it), abort_flag);
           if (!ok) break;
-          // tile 0: O_0 += P_0 V, then S_0 for the next key tile
-          if (act(0, it)) {
-            ok = bar_wait(&bars->p_full[0], (cp0++) & 1, abort_flag);
-            if (ok && first0) ok = bar_wait(&bars->o_free[0], ((co0++) & 1) ^ 1, abort_flag);
+          if (act(it)) {
+            // O_t += P_t V, then release the stage (this tile's reads of it are issued)
+            ok = bar_wait(p_full, (cp++) & 1, abort_flag);
+            if (ok && first) ok = bar_wait(&bars->o_free[t], ((co++) & 1) ^ 1, abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_pv(0, s, first0);
-            first0 = false;
-            if (it == U.b[0]) ptx::mma_commit(&bars->o_done[0]);
+            issue_pv(s, first);
+            first = false;
+            if (it == b_t) ptx::mma_commit(&bars->o_done[t]);
+            ptx::mma_commit(&bars->kv_empty[s]);
+          } else {
+            ptx::mbar_arrive(&bars->kv_empty[s]);  // this tile does not use the stage
           }
-          if (nxt) {
+          if (it + 1 <= U.u1) {
+            // S_t of the next key tile
             ok = bar_wait(&bars->k_full[slot(it + 1)], ring_par(it + 1), abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            if (act(0, it + 1)) {
-              issue_s(0, slot(it + 1));
-              if (it + 1 == U.b[0]) ptx::mma_commit(&bars->q_empty[0]);
+            if (act(it + 1)) {
+              issue_s(slot(it + 1));
+              if (it + 1 == b_t) ptx::mma_commit(&bars->q_empty[t]);
             }
-          }
-          // tile 1: O_1 += P_1 V, release the K/V stage, then S_1 for the next key tile
-          if (act(1, it)) {
-            ok = bar_wait(&bars->p_full[1], (cp1++) & 1, abort_flag);
-            if (ok && first1) ok = bar_wait(&bars->o_free[1], ((co1++) & 1) ^ 1, abort_flag);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            issue_pv(1, s, first1);
-            first1 = false;
-            if (it == U.b[1]) ptx::mma_commit(&bars->o_done[1]);
-          }
-          ptx::mma_commit(&bars->kv_empty[s]);
-          if (nxt && act(1, it + 1)) {
-            issue_s(1, slot(it + 1));
-            if (it + 1 == U.b[1]) ptx::mma_commit(&bars->q_empty[1]);
           }
         }
         g = g0 + (U.u1 - U.u0 + 1);
       }
       // Exit path: every MMA this thread issued has completed.
-      ptx::mma_commit(&bars->drain);
-      bar_drain(&bars->drain, 0);
+      ptx::mma_commit(&bars->drain[t]);
+      bar_drain(&bars->drain[t], 0);
     }
     __syncwarp();
+  }
   } else {
+    ptx::regs_inc<C::SOFTMAX_REGS>();
     // ------------------------------------------------------------ softmax warpgroups
     const int t = warp / 4;                    // Q tile of this warpgroup
     const int r = threadIdx.x - 128 * t;       // row within the tile = TMEM lane
@@ -343,108 +349,175 @@ __global__ void __launch_bounds__(320, 1)
             span = (uint32_t)(c_last - c_first);
           }
         }
-        // pass 1: row max of the raw scores (scale > 0 commutes with max)
-        float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t sr[32];
-          ptx::tmem_ld32(tS + q * 32, sr);
+        // Fast path, for every tile after a row's first: exponentiate against
+        // the current reference max while tracking this tile's max, keeping P
+        // packed in registers.  Only if some row's max rose past the reference
+        // by more than 2^8 is the tile redone by the two-pass path below (S is
+        // still intact then: nothing has been stored over it).
+        bool done = false;
+        if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
+          const float2 c2v = make_float2(p.scale_log2, p.scale_log2);
+          const float2 mnv = make_float2(-m_ref, -m_ref);
+          float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
+          float mx0 = -INFINITY, mx1 = -INFINITY;
+          uint32_t pk[2][32];
+          uint32_t sr[2][32];
+          ptx::tmem_ld32(tS, sr[0]);
           ptx::tmem_wait_ld();
-          ptx::reg_fence(sr);
+          ptx::reg_fence(sr[0]);
+          // chunk q of the row: masked scores become -inf on edge tiles;
+          // interior tiles send half of the exponentials to the FMA pipe
+#define SPA_FWD_FAST_CHUNKS(INTERIOR)                                                              \
+  _Pragma("unroll") for (int q = 0; q < 4; ++q) {                                                  \
+    if (q < 3) ptx::tmem_ld32(tS + (q + 1) * 32, sr[(q + 1) & 1]); /* next chunk in flight */      \
+    const uint32_t* cur = sr[q & 1];                                                               \
+    const int cb = q * 32 - clo;                                                                   \
+    _Pragma("unroll") for (int e = 0; e < 32; e += 4) {                                            \
+      float s0 = __uint_as_float(cur[e]), s1 = __uint_as_float(cur[e + 1]);                        \
+      float s2 = __uint_as_float(cur[e + 2]), s3 = __uint_as_float(cur[e + 3]);                    \
+      if (!(INTERIOR)) {                                                                           \
+        s0 = (uint32_t)(cb + e) <= span ? s0 : -INFINITY;                                          \
+        s1 = (uint32_t)(cb + e + 1) <= span ? s1 : -INFINITY;                                      \
+        s2 = (uint32_t)(cb + e + 2) <= span ? s2 : -INFINITY;                                      \
+        s3 = (uint32_t)(cb + e + 3) <= span ? s3 : -INFINITY;                                      \
+      }                                                                                            \
+      mx0 = ptx::fmax3(mx0, s0, s1);                                                               \
+      mx1 = ptx::fmax3(mx1, s2, s3);                                                               \
+      const float2 x01 = __ffma2_rn(make_float2(s0, s1), c2v, mnv);                                \
+      const float2 x23 = __ffma2_rn(make_float2(s2, s3), c2v, mnv);                                \
+      const float2 p01 = make_float2(ptx::exp2_approx(x01.x), ptx::exp2_approx(x01.y));            \
+      const float2 p23 = (INTERIOR) ? exp2_poly2(x23)                                              \
+                                    : make_float2(ptx::exp2_approx(x23.x), ptx::exp2_approx(x23.y)); \
+      sa = __fadd2_rn(sa, p01);                                                                    \
+      sb = __fadd2_rn(sb, p23);                                                                    \
+      pk[q / 2][(q % 2) * 16 + e / 2] = ptx::pack_bf16x2(p01.x, p01.y);                            \
+      pk[q / 2][(q % 2) * 16 + e / 2 + 1] = ptx::pack_bf16x2(p23.x, p23.y);                        \
+    }                                                                                              \
+    if (q < 3) {                                                                                   \
+      ptx::tmem_wait_ld();                                                                         \
+      ptx::reg_fence(sr[(q + 1) & 1]);                                                             \
+    }                                                                                              \
+  }
           if (interior) {
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              mx0 = fmaxf(mx0, __uint_as_float(sr[e]));
-              mx1 = fmaxf(mx1, __uint_as_float(sr[e + 1]));
-              mx2 = fmaxf(mx2, __uint_as_float(sr[e + 2]));
-              mx3 = fmaxf(mx3, __uint_as_float(sr[e + 3]));
-            }
+            SPA_FWD_FAST_CHUNKS(true)
           } else {
-            const int cb = q * 32 - clo;
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              mx0 = fmaxf(mx0, (uint32_t)(cb + e) <= span ? __uint_as_float(sr[e]) : -INFINITY);
-              mx1 = fmaxf(mx1, (uint32_t)(cb + e + 1) <= span ? __uint_as_float(sr[e + 1]) : -INFINITY);
-              mx2 = fmaxf(mx2, (uint32_t)(cb + e + 2) <= span ? __uint_as_float(sr[e + 2]) : -INFINITY);
-              mx3 = fmaxf(mx3, (uint32_t)(cb + e + 3) <= span ? __uint_as_float(sr[e + 3]) : -INFINITY);
-            }
+            SPA_FWD_FAST_CHUNKS(false)
+          }
+#undef SPA_FWD_FAST_CHUNKS
+          const float c2 = p.scale_log2;
+          const float sm0 = sa.x, sm1 = sa.y, sm2 = sb.x, sm3 = sb.y;
+          const bool over = fmaxf(mx0, mx1) * c2 > m_ref + 8.f;
+          if (!__any_sync(0xffffffffu, over)) {
+            ptx::tmem_st32(tS, pk[0]);
+            ptx::tmem_st32(tS + 32, pk[1]);
+            l += (sm0 + sm1) + (sm2 + sm3);
+            done = true;
           }
         }
-        const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2);
-        const bool need = m_new > m_ref + 8.f;   // also true for a row's first finite max
-        const bool need_o = need && (m_ref != -INFINITY);
-        float alpha = 1.f;
-        if (need) {
-          alpha = ptx::exp2_approx(m_ref - m_new);  // 0 while the row had seen nothing
-          l *= alpha;
-          m_ref = m_new;
-        }
-        if (__any_sync(0xffffffffu, need_o)) {
-          // O_t is stable: the PV of the previous key tile completed before S_t did
-          const float a = need_o ? alpha : 1.f;
-#pragma unroll 1
-          for (int c = 0; c < D; c += 32) {
-            uint32_t o[32];
-            ptx::tmem_ld32(tO + c, o);
+        if (!done) {
+          // pass 1: row max of the raw scores (scale > 0 commutes with max)
+          float mx0 = -INFINITY, mx1 = -INFINITY, mx2 = -INFINITY, mx3 = -INFINITY;
+  #pragma unroll 1
+          for (int q = 0; q < 4; ++q) {
+            uint32_t sr[32];
+            ptx::tmem_ld32(tS + q * 32, sr);
             ptx::tmem_wait_ld();
-            ptx::reg_fence(o);
-#pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
-            ptx::tmem_st32(tO + c, o);
-          }
-        }
-        // pass 2: p = exp2(s * scale_log2 - m), bf16 pairs over the first half
-        // of S_t (chunk q of P covers columns [16q, 16q+16), already read)
-        const float c2 = p.scale_log2;
-        const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
-        float sm0 = 0.f, sm1 = 0.f, sm2 = 0.f, sm3 = 0.f;
-#pragma unroll 1
-        for (int q = 0; q < 4; ++q) {
-          uint32_t sr[32];
-          ptx::tmem_ld32(tS + q * 32, sr);
-          ptx::tmem_wait_ld();
-          ptx::reg_fence(sr);
-          uint32_t pk[16];
-          if (interior) {
-            // every key permitted; one exponential in four on the FMA pipe
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              const float p0 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e]), c2, mneg));
-              const float p1 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 1]), c2, mneg));
-              const float p2 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 2]), c2, mneg));
-              const float p3 = exp2_poly(fmaf(__uint_as_float(sr[e + 3]), c2, mneg));
-              sm0 += p0;
-              sm1 += p1;
-              sm2 += p2;
-              sm3 += p3;
-              pk[e / 2] = ptx::pack_bf16x2(p0, p1);
-              pk[e / 2 + 1] = ptx::pack_bf16x2(p2, p3);
-            }
-          } else {
-            const int cb = q * 32 - clo;
-#pragma unroll
-            for (int e = 0; e < 32; e += 4) {
-              float x0 = fmaf(__uint_as_float(sr[e]), c2, mneg);
-              float x1 = fmaf(__uint_as_float(sr[e + 1]), c2, mneg);
-              float x2 = fmaf(__uint_as_float(sr[e + 2]), c2, mneg);
-              float x3 = fmaf(__uint_as_float(sr[e + 3]), c2, mneg);
-              x0 = (uint32_t)(cb + e) <= span ? x0 : -INFINITY;
-              x1 = (uint32_t)(cb + e + 1) <= span ? x1 : -INFINITY;
-              x2 = (uint32_t)(cb + e + 2) <= span ? x2 : -INFINITY;
-              x3 = (uint32_t)(cb + e + 3) <= span ? x3 : -INFINITY;
-              const float p0 = ptx::exp2_approx(x0), p1 = ptx::exp2_approx(x1);
-              const float p2 = ptx::exp2_approx(x2), p3 = ptx::exp2_approx(x3);
-              sm0 += p0;
-              sm1 += p1;
-              sm2 += p2;
-              sm3 += p3;
-              pk[e / 2] = ptx::pack_bf16x2(p0, p1);
-              pk[e / 2 + 1] = ptx::pack_bf16x2(p2, p3);
+            ptx::reg_fence(sr);
+            if (interior) {
+  #pragma unroll
+              for (int e = 0; e < 32; e += 4) {
+                mx0 = fmaxf(mx0, __uint_as_float(sr[e]));
+                mx1 = fmaxf(mx1, __uint_as_float(sr[e + 1]));
+                mx2 = fmaxf(mx2, __uint_as_float(sr[e + 2]));
+                mx3 = fmaxf(mx3, __uint_as_float(sr[e + 3]));
+              }
+            } else {
+              const int cb = q * 32 - clo;
+  #pragma unroll
+              for (int e = 0; e < 32; e += 4) {
+                mx0 = fmaxf(mx0, (uint32_t)(cb + e) <= span ? __uint_as_float(sr[e]) : -INFINITY);
+                mx1 = fmaxf(mx1, (uint32_t)(cb + e + 1) <= span ? __uint_as_float(sr[e + 1]) : -INFINITY);
+                mx2 = fmaxf(mx2, (uint32_t)(cb + e + 2) <= span ? __uint_as_float(sr[e + 2]) : -INFINITY);
+                mx3 = fmaxf(mx3, (uint32_t)(cb + e + 3) <= span ? __uint_as_float(sr[e + 3]) : -INFINITY);
+              }
             }
           }
-          ptx::tmem_st16(tS + q * 16, pk);
+          const float m_new = fmaxf(m_ref, fmaxf(fmaxf(mx0, mx1), fmaxf(mx2, mx3)) * p.scale_log2);
+          const bool need = m_new > m_ref + 8.f;   // also true for a row's first finite max
+          const bool need_o = need && (m_ref != -INFINITY);
+          float alpha = 1.f;
+          if (need) {
+            alpha = ptx::exp2_approx(m_ref - m_new);  // 0 while the row had seen nothing
+            l *= alpha;
+            m_ref = m_new;
+          }
+          if (__any_sync(0xffffffffu, need_o)) {
+            // O_t is stable: the PV of the previous key tile completed before S_t did
+            const float a = need_o ? alpha : 1.f;
+  #pragma unroll 1
+            for (int c = 0; c < D; c += 32) {
+              uint32_t o[32];
+              ptx::tmem_ld32(tO + c, o);
+              ptx::tmem_wait_ld();
+              ptx::reg_fence(o);
+  #pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * a);
+              ptx::tmem_st32(tO + c, o);
+            }
+          }
+          // pass 2: p = exp2(s * scale_log2 - m), bf16 pairs over the first half
+          // of S_t (chunk q of P covers columns [16q, 16q+16), already read)
+          const float c2 = p.scale_log2;
+          const float mneg = (m_ref == -INFINITY) ? 0.f : -m_ref;
+          float sm0 = 0.f, sm1 = 0.f, sm2 = 0.f, sm3 = 0.f;
+  #pragma unroll 1
+          for (int q = 0; q < 4; ++q) {
+            uint32_t sr[32];
+            ptx::tmem_ld32(tS + q * 32, sr);
+            ptx::tmem_wait_ld();
+            ptx::reg_fence(sr);
+            uint32_t pk[16];
+            if (interior) {
+              // every key permitted; one exponential in four on the FMA pipe
+  #pragma unroll
+              for (int e = 0; e < 32; e += 4) {
+                const float p0 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e]), c2, mneg));
+                const float p1 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 1]), c2, mneg));
+                const float p2 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 2]), c2, mneg));
+                const float p3 = exp2_poly(fmaf(__uint_as_float(sr[e + 3]), c2, mneg));
+                sm0 += p0;
+                sm1 += p1;
+                sm2 += p2;
+                sm3 += p3;
+                pk[e / 2] = ptx::pack_bf16x2(p0, p1);
+                pk[e / 2 + 1] = ptx::pack_bf16x2(p2, p3);
+              }
+            } else {
+              const int cb = q * 32 - clo;
+  #pragma unroll
+              for (int e = 0; e < 32; e += 4) {
+                float x0 = fmaf(__uint_as_float(sr[e]), c2, mneg);
+                float x1 = fmaf(__uint_as_float(sr[e + 1]), c2, mneg);
+                float x2 = fmaf(__uint_as_float(sr[e + 2]), c2, mneg);
+                float x3 = fmaf(__uint_as_float(sr[e + 3]), c2, mneg);
+                x0 = (uint32_t)(cb + e) <= span ? x0 : -INFINITY;
+                x1 = (uint32_t)(cb + e + 1) <= span ? x1 : -INFINITY;
+                x2 = (uint32_t)(cb + e + 2) <= span ? x2 : -INFINITY;
+                x3 = (uint32_t)(cb + e + 3) <= span ? x3 : -INFINITY;
+                const float p0 = ptx::exp2_approx(x0), p1 = ptx::exp2_approx(x1);
+                const float p2 = ptx::exp2_approx(x2), p3 = ptx::exp2_approx(x3);
+                sm0 += p0;
+                sm1 += p1;
+                sm2 += p2;
+                sm3 += p3;
+                pk[e / 2] = ptx::pack_bf16x2(p0, p1);
+                pk[e / 2 + 1] = ptx::pack_bf16x2(p2, p3);
+              }
+            }
+            ptx::tmem_st16(tS + q * 16, pk);
+          }
+          l += (sm0 + sm1) + (sm2 + sm3);
         }
-        l += (sm0 + sm1) + (sm2 + sm3);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full[t]);
@@ -461,16 +534,7 @@ __global__ void __launch_bounds__(320, 1)
         ptx::tmem_ld32(tO + c, o);
         ptx::tmem_wait_ld();
         ptx::reg_fence(o);
-        if (i < N) {
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float* f = reinterpret_cast<const float*>(&o[8 * q]);
-            ptx::st_global_v4(orow + c + 8 * q, ptx::pack_bf16x2(f[0] * inv, f[1] * inv),
-                              ptx::pack_bf16x2(f[2] * inv, f[3] * inv),
-                              ptx::pack_bf16x2(f[4] * inv, f[5] * inv),
-                              ptx::pack_bf16x2(f[6] * inv, f[7] * inv));
-          }
-        }
+        if (i < N) ptx::store_row32_bf16(orow + c, o, inv);
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->o_free[t]);

@@ -97,6 +97,21 @@ int prepare_kernel(K kernel, uint32_t smem_bytes, std::atomic<uint64_t>& done_ma
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? SPA_OK : SPA_ERR_CUDA; }
 
+// A kernel that re-splits its registers between warpgroups (setmaxnreg) must
+// have been compiled to exactly the per-thread count the split was budgeted
+// for; otherwise an increase could wait for registers that never come.
+template <typename K>
+int check_regs(K kernel, int want, std::atomic<int>& verdict) {
+  int v = verdict.load(std::memory_order_acquire);
+  if (v == 0) {
+    cudaFuncAttributes a;
+    if (cudaFuncGetAttributes(&a, kernel) != cudaSuccess) return SPA_ERR_CUDA;
+    v = (a.numRegs == want) ? 1 : 2;
+    verdict.store(v, std::memory_order_release);
+  }
+  return v == 1 ? SPA_OK : SPA_ERR_UNSUPPORTED;
+}
+
 int sm_count(int* n) {
   static std::atomic<int> cache[64];
   int dev = 0;
@@ -124,6 +139,8 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, A
       (st = make_map(&mv, v, p.N, BH, D, C::BK)))
     return st;
   if ((st = prepare_kernel(spa::spa_fwd_kernel<D>, C::SMEM_BYTES, prepared))) return st;
+  static std::atomic<int> regs_ok{0};
+  if ((st = check_regs(spa::spa_fwd_kernel<D>, (int)C::LAUNCH_REGS, regs_ok))) return st;
   // Work list of the persistent grid: per batch, every 256-row block of every
   // head from the one holding lo_h on (units), and the blocks before it (fills).
   const int64_t nblk = (p.N + C::BU - 1) / C::BU;
@@ -178,6 +195,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
         (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)))
       return st;
     if ((st = prepare_kernel(spa::spa_bwd_dkdv_kernel<D>, KC::SMEM_BYTES, prepared_kv))) return st;
+    static std::atomic<int> regs_kv{0};
+    if ((st = check_regs(spa::spa_bwd_dkdv_kernel<D>, (int)KC::LAUNCH_REGS, regs_kv))) return st;
     const int64_t nkt = (p.N + 127) / 128;
     int64_t upb = 0;
     for (int h = 0; h < p.H; ++h) upb += (p.N - 1 - p.lo[h]) / 128 + 1;
@@ -200,6 +219,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
         (st = make_map(&qv, v, p.N, BH, D, QC::BK)) || (st = make_map(&qdo, dout, p.N, BH, D, QC::BQ)))
       return st;
     if ((st = prepare_kernel(spa::spa_bwd_dq_kernel<D>, QC::SMEM_BYTES, prepared_q))) return st;
+    static std::atomic<int> regs_q{0};
+    if ((st = check_regs(spa::spa_bwd_dq_kernel<D>, (int)QC::LAUNCH_REGS, regs_q))) return st;
     const int64_t nqt = (p.N + 127) / 128;
     int64_t upb = 0, fpb = 0;
     for (int h = 0; h < p.H; ++h) {
