@@ -52,7 +52,8 @@ __device__ int g_spa_status;
 // Bounded wait on one mbarrier phase.  Returns false when the CTA aborted:
 // either this wait ran past kWaitLimitNs (it then raises the CTA's abort flag
 // and the device error word) or another thread already raised the flag.
-__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                         uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = ptx::smem_u32(bar);
   if (ptx::mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = ptx::globaltimer_ns();
@@ -61,7 +62,7 @@ __device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, volatil
     for (int n = 0; n < 32; ++n)
       if (ptx::mbar_try_wait(a, parity)) return true;
     if (*abort_flag) return false;
-    if (ptx::globaltimer_ns() - t0 > kWaitLimitNs) {
+    if (ptx::globaltimer_ns() - t0 > limit_ns) {
       *abort_flag = 1;
       atomicExch(&g_spa_status, kStatusTimeout);
       return false;

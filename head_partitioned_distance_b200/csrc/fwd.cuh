@@ -65,6 +65,7 @@ struct FwdBars {
   uint64_t q_full[2], q_empty[2];
   uint64_t k_full[2], v_full[2], kv_empty[2];
   uint64_t s_full[2], p_full[2], o_done[2], o_free[2];
+  uint64_t turn[2];  // turn[t]: softmax warpgroup t may start its next step
   uint64_t drain[2];
   uint32_t tmem_base;
   int abort;
@@ -142,6 +143,7 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_init(&bars->p_full[i], 128);
       ptx::mbar_init(&bars->o_done[i], 1);
       ptx::mbar_init(&bars->o_free[i], 128);
+      ptx::mbar_init(&bars->turn[i], 128);
     }
     ptx::mbar_init(&bars->drain[0], 1);
     ptx::mbar_init(&bars->drain[1], 1);
@@ -311,8 +313,18 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tmem + lane_base + C::tm_o(t);
     int cs = 0, cd = 0;
     bool ok = true;
+    // The two warpgroups take turns: their softmax steps run one at a time in
+    // the order (key tile it, tile 0), (it, tile 1), (it + 1, tile 0), ...
+    // so each one's special-function work overlaps the tensor core's work on
+    // the other tile instead of both competing at once.  At every change of
+    // owner the finishing warpgroup arrives on the other's turn barrier.
+    int last_owner = -1;  // owner of the previous step in this CTA's order
+    int turns = 0;        // waits on this warpgroup's turn barrier so far
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
       const FwdUnit U = fwd_decode<D>(u, p);
+      auto actv = [&](int tt, int it) {
+        return tt ? (U.act[1] && it >= U.a[1] && it <= U.b[1]) : (U.act[0] && it >= U.a[0] && it <= U.b[0]);
+      };
       const int64_t it0 = U.i0 + (int64_t)t * C::BQ;
       const int64_t i = it0 + r;
       const bool act_t = t ? U.act[1] : U.act[0];
@@ -325,11 +337,18 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < D; c += 8) ptx::st_global_v4(orow + c, 0u, 0u, 0u, 0u);
           p.lse[(int64_t)U.bh * N + i] = -INFINITY;
         }
+        last_owner = 1 - t;  // every step of this unit belongs to the other tile
         continue;
       }
       float m_ref = -INFINITY, l = 0.f;  // running max (base-2 units) and sum
       for (int it = a_t; it <= b_t; ++it) {
+        int prev;
+        if (t == 1 && actv(0, it)) prev = 0;
+        else if (actv(1, it - 1)) prev = 1;
+        else if (actv(0, it - 1)) prev = 0;
+        else prev = last_owner;
         ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[t], (cs++) & 1, abort_flag));
+        if (ok && prev == 1 - t) ok = __all_sync(0xffffffffu, bar_wait(&bars->turn[t], (turns++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
         const int64_t j0 = (int64_t)it * C::BK;
@@ -521,7 +540,18 @@ __global__ void __launch_bounds__(384, 1)
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full[t]);
+        // hand the turn over if the next step belongs to the other tile
+        int nxt = -1;
+        if (t == 0 && actv(1, it)) nxt = 1;
+        else if (actv(0, it + 1)) nxt = 0;
+        else if (actv(1, it + 1)) nxt = 1;
+        else if (u + (int)gridDim.x < num_units) {
+          const FwdUnit V = fwd_decode<D>(u + gridDim.x, p);
+          nxt = (V.act[0] && V.a[0] == V.u0) ? 0 : 1;
+        }
+        if (nxt == 1 - t) ptx::mbar_arrive(&bars->turn[1 - t]);
       }
+      last_owner = U.act[1] ? 1 : 0;
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
       ok = __all_sync(0xffffffffu, bar_wait(&bars->o_done[t], (cd++) & 1, abort_flag));

@@ -306,6 +306,22 @@ __global__ void tile_class_kernel(int64_t N, int H, int Bq, int Bk, int nqt, int
   }
 }
 
+// One warp waits on an mbarrier that nothing ever arrives on, with the given
+// limit: the bounded-wait path every kernel uses, exercised on purpose.
+__global__ void wait_timeout_kernel(uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    spa::ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    spa::ptx::fence_mbar_init();
+  }
+  __syncthreads();
+  const bool ok = spa::bar_wait(&bar, 0, &abort_flag, limit_ns);
+  __syncwarp();
+  if (threadIdx.x == 0 && ok) atomicExch(&spa::g_spa_status, -1);  // cannot happen: nothing arrives
+}
+
 __global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
   for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
     y[e] = spa::exp2_poly(x[e]);
@@ -484,6 +500,12 @@ int spa_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
   if (!x || !y || n < 0) return SPA_ERR_INVAL;
   if (n == 0) return SPA_OK;
   exp2_poly_kernel<<<148 * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
+  return launch_status();
+}
+
+int spa_debug_wait_timeout(int64_t limit_ns, void* stream) {
+  if (limit_ns < 1 || limit_ns > 1000000000LL) return SPA_ERR_INVAL;
+  wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)limit_ns);
   return launch_status();
 }
 

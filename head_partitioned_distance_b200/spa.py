@@ -49,6 +49,7 @@ EXPORTS = {
                           _int),
     "spa_tile_classes_device": ([_i64, _int, _i32p, _i32p, _int, _int, _vp, _vp], _int),
     "spa_debug_exp2_poly": ([_vp, _vp, _i64, _vp], _int),
+    "spa_debug_wait_timeout": ([_i64, _vp], _int),
     "spa_device_status": ([_vp], _int),
 }
 for _name, (_args, _res) in EXPORTS.items():
@@ -240,6 +241,11 @@ def spa_debug_exp2_poly(x: torch.Tensor, y: torch.Tensor, stream=None):
     _check(_lib.spa_debug_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(stream)),
            "spa_debug_exp2_poly")
     return y
+
+
+def spa_debug_wait_timeout(limit_ns: int, stream=None):
+    """Make one device wait run out of time (see spa.h); check with spa_device_status()."""
+    _check(_lib.spa_debug_wait_timeout(limit_ns, _stream_ptr(stream)), "spa_debug_wait_timeout")
 
 
 def spa_device_status(stream=None) -> int:

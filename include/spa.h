@@ -207,6 +207,16 @@ SPA_API int spa_tile_classes_device(int64_t N, int H, const int32_t* lo, const i
 SPA_API int spa_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
 
 /*
+ * Test hook for failure detection: launches one warp that waits on an
+ * mbarrier nothing ever arrives on, through the same bounded wait every
+ * kernel uses, with a limit of limit_ns nanoseconds (1 ns .. 1 s).  The wait
+ * gives up, raises the device error word and the kernel returns normally, so
+ * the next spa_device_status() reports SPA_ERR_TIMEOUT and the context stays
+ * usable.  Asynchronous on `stream`.
+ */
+SPA_API int spa_debug_wait_timeout(int64_t limit_ns, void* stream);
+
+/*
  * Synchronises `stream` and returns the library's device error word, then
  * clears it: SPA_OK, or SPA_ERR_TIMEOUT when a kernel gave up on a wait (the
  * kernel then wrote incomplete outputs and released its tensor memory).

@@ -151,3 +151,9 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
 def test_workspace_size():
     assert spa.spa_attn_bwd_workspace_bytes(4, 32, 8192) == 4 * 32 * 8192 * 4
     assert spa.spa_attn_bwd_workspace_bytes(0, 1, 1) == 0
+
+
+def test_timeout_hook_rejects_bad_limits():
+    L = spa._lib
+    assert L.spa_debug_wait_timeout(0, None) == spa.SPA_ERR_INVAL
+    assert L.spa_debug_wait_timeout(2_000_000_000, None) == spa.SPA_ERR_INVAL

@@ -248,3 +248,15 @@ def test_fma_pipe_exp2_error_bound(spa):
     out = torch.empty_like(lo)
     spa.spa_debug_exp2_poly(lo, out)
     assert torch.all(out >= 0) and torch.all(out < 2e-38) and not torch.isnan(out).any()
+
+
+def test_device_wait_timeout_reports_and_recovers(spa):
+    # a wait that nothing completes gives up after its limit: the kernel
+    # returns, the status word says so once, and the context keeps working
+    assert spa.spa_device_status() == spa.SPA_OK
+    spa.spa_debug_wait_timeout(20_000_000)  # 20 ms
+    assert spa.spa_device_status() == spa.SPA_ERR_TIMEOUT
+    assert spa.spa_device_status() == spa.SPA_OK  # cleared by the read
+    w = synth.WORKLOADS["b1_h4_n256_d64"]
+    q, k, v, do = synth.workload_inputs(w)
+    _full_check(spa, q, k, v, do, w.scale)
