@@ -382,7 +382,7 @@ __global__ void __launch_bounds__(384, 1)
           const float4* nl4 = reinterpret_cast<const float4*>(vl);
           const float2 c2v = make_float2(c2, c2);
           if (interior) {
-            // every query permitted; one exponential pair in four on the FMA pipe
+            // every query permitted
 #pragma unroll
             for (int q4 = 0; q4 < 16; ++q4) {
               const float4 nl = nl4[q4];
@@ -395,14 +395,8 @@ __global__ void __launch_bounds__(384, 1)
                                            c2v, make_float2(nl.z, nl.w));
               pt[q] = ptx::exp2_approx(xa.x);
               pt[q + 1] = ptx::exp2_approx(xa.y);
-              if ((q4 & 1) == 1) {
-                const float2 pb = exp2_poly2(xb);
-                pt[q + 2] = pb.x;
-                pt[q + 3] = pb.y;
-              } else {
-                pt[q + 2] = ptx::exp2_approx(xb.x);
-                pt[q + 3] = ptx::exp2_approx(xb.y);
-              }
+              pt[q + 2] = ptx::exp2_approx(xb.x);
+              pt[q + 3] = ptx::exp2_approx(xb.y);
             }
           } else {
 #pragma unroll
@@ -818,10 +812,28 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tmem_wait_ld();
           ptx::reg_fence(sr[0]);
           ptx::reg_fence(sr[1]);
+          // x = s * c2 - lse2 in pairs
+          const float2 c2v = make_float2(c2, c2);
+          const float2 nlv = make_float2(nlse2, nlse2);
+          if (interior) {
+            // every key permitted
 #pragma unroll
-          for (int e = 0; e < 64; ++e) {
-            const float ev = ptx::exp2_approx(fmaf(__uint_as_float(sr[e / 32][e % 32]), c2, nlse2));
-            pv[e] = (interior || (uint32_t)(cb + e) <= span) ? ev : 0.f;
+            for (int e = 0; e < 64; e += 2) {
+              const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[e / 32][e % 32]),
+                                                      __uint_as_float(sr[e / 32][e % 32 + 1])),
+                                          c2v, nlv);
+              pv[e] = ptx::exp2_approx(x.x);
+              pv[e + 1] = ptx::exp2_approx(x.y);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 64; e += 2) {
+              const float2 x = __ffma2_rn(make_float2(__uint_as_float(sr[e / 32][e % 32]),
+                                                      __uint_as_float(sr[e / 32][e % 32 + 1])),
+                                          c2v, nlv);
+              pv[e] = (uint32_t)(cb + e) <= span ? ptx::exp2_approx(x.x) : 0.f;
+              pv[e + 1] = (uint32_t)(cb + e + 1) <= span ? ptx::exp2_approx(x.y) : 0.f;
+            }
           }
         }
         ok = __all_sync(0xffffffffu, bar_wait(&bars->dp_full, (cdp++) & 1, abort_flag));
@@ -834,12 +846,16 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tmem_wait_ld();
           ptx::reg_fence(dr[0]);
           ptx::reg_fence(dr[1]);
+          // dS = P (dP - D) in pairs
+          const float2 ndv = make_float2(-Di, -Di);
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) {
-            const float d0 = pv[2 * e] * (__uint_as_float(dr[(2 * e) / 32][(2 * e) % 32]) - Di);
-            const float d1 = pv[2 * e + 1] * (__uint_as_float(dr[(2 * e + 1) / 32][(2 * e + 1) % 32]) - Di);
-            pk[e] = ptx::pack_bf16x2(d0, d1);
+            const float2 d = __fmul2_rn(make_float2(pv[2 * e], pv[2 * e + 1]),
+                                        __fadd2_rn(make_float2(__uint_as_float(dr[e / 16][(2 * e) % 32]),
+                                                               __uint_as_float(dr[e / 16][(2 * e) % 32 + 1])),
+                                                   ndv));
+            pk[e] = ptx::pack_bf16x2(d.x, d.y);
           }
           ptx::tmem_st32(tS, pk);
           ptx::tmem_wait_st();

@@ -52,7 +52,7 @@ struct FwdCfg {
   static constexpr int NTHREADS = 384;
   // register split: 384 threads launch with 168 registers each (64512); the
   // two softmax warpgroups take 192, the producer/MMA warpgroup 120.
-  static constexpr uint32_t LAUNCH_REGS = 168, SOFTMAX_REGS = 192, CONTROL_REGS = 120;
+  static constexpr uint32_t LAUNCH_REGS = 168, SOFTMAX_REGS = 200, CONTROL_REGS = 104;
   static_assert(2 * SOFTMAX_REGS + CONTROL_REGS <= 3 * LAUNCH_REGS, "register split over budget");
   static constexpr uint32_t TMEM_COLS = 512;
   // tile t: S_t (and P_t over its first 64 columns) at t*256, O_t at t*256 + 128
@@ -384,8 +384,7 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tmem_ld32(tS, sr[0]);
           ptx::tmem_wait_ld();
           ptx::reg_fence(sr[0]);
-          // chunk q of the row: masked scores become -inf on edge tiles;
-          // interior tiles send half of the exponentials to the FMA pipe
+          // chunk q of the row: masked scores become -inf on edge tiles
 #define SPA_FWD_FAST_CHUNKS(INTERIOR)                                                              \
   _Pragma("unroll") for (int q = 0; q < 4; ++q) {                                                  \
     if (q < 3) ptx::tmem_ld32(tS + (q + 1) * 32, sr[(q + 1) & 1]); /* next chunk in flight */      \
@@ -405,8 +404,7 @@ __global__ void __launch_bounds__(384, 1)
       const float2 x01 = __ffma2_rn(make_float2(s0, s1), c2v, mnv);                                \
       const float2 x23 = __ffma2_rn(make_float2(s2, s3), c2v, mnv);                                \
       const float2 p01 = make_float2(ptx::exp2_approx(x01.x), ptx::exp2_approx(x01.y));            \
-      const float2 p23 = (INTERIOR) ? exp2_poly2(x23)                                              \
-                                    : make_float2(ptx::exp2_approx(x23.x), ptx::exp2_approx(x23.y)); \
+      const float2 p23 = make_float2(ptx::exp2_approx(x23.x), ptx::exp2_approx(x23.y));            \
       sa = __fadd2_rn(sa, p01);                                                                    \
       sb = __fadd2_rn(sb, p23);                                                                    \
       pk[q / 2][(q % 2) * 16 + e / 2] = ptx::pack_bf16x2(p01.x, p01.y);                            \
@@ -497,13 +495,13 @@ __global__ void __launch_bounds__(384, 1)
             ptx::reg_fence(sr);
             uint32_t pk[16];
             if (interior) {
-              // every key permitted; one exponential in four on the FMA pipe
+              // every key permitted
   #pragma unroll
               for (int e = 0; e < 32; e += 4) {
                 const float p0 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e]), c2, mneg));
                 const float p1 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 1]), c2, mneg));
                 const float p2 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 2]), c2, mneg));
-                const float p3 = exp2_poly(fmaf(__uint_as_float(sr[e + 3]), c2, mneg));
+                const float p3 = ptx::exp2_approx(fmaf(__uint_as_float(sr[e + 3]), c2, mneg));
                 sm0 += p0;
                 sm1 += p1;
                 sm2 += p2;
