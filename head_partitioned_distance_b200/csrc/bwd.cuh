@@ -55,17 +55,19 @@ __global__ void __launch_bounds__(256) spa_bwd_delta_kernel(const uint16_t* __re
 // the 128-query tiles its band reaches.  Per query tile:
 //   S^T  = K Q^T      SS MMA -> TMEM [0,128)
 //   dP^T = V dO^T     SS MMA -> TMEM [128,256)
-//   P^T  = exp2(S^T c - lse2), masked on edge tiles; written as bf16 over S^T
+//   P^T  = exp2(S^T c - lse2), masked on edge tiles; bf16 to a shared tile
 //   dS^T = P^T (dP^T - D);                          written as bf16 over dP^T
-//   dV  += P^T dO     TS MMA (A = P^T from TMEM) -> TMEM [256,384)
+//   dV  += P^T dO     SS MMA (A = P^T from shared memory) -> TMEM [256,384)
 //   dK  += dS^T Q     TS MMA (A = dS^T from TMEM) -> TMEM [384,512)
 // Two warpgroups share each tile: warpgroup w owns query columns
-// [64w, 64w+64) of every key row (thread r = key row r = TMEM lane r) and
-// writes its bf16 pairs to columns [64w, 64w+32) of the region it read, so
-// the two never touch each other's unread columns.  S^T of the next query
-// tile is issued right after dV (which read P^T) and dP^T right after dK, so
-// the tensor core runs while the warpgroups work.  Epilogue: warpgroup 0
-// writes dV, warpgroup 1 writes scale * dK, straight from TMEM to global.
+// [64w, 64w+64) of every key row (thread r = key row r = TMEM lane r); its P^T
+// goes to 64-query block w of the shared tile and its dS^T pairs to columns
+// [64w, 64w+32) of the dP^T region it read.  S^T of the next query tile is
+// issued as soon as the warpgroups hold this one in registers (P^T does not
+// live in TMEM), so it overlaps their exponentials; dP^T of the next tile
+// follows dK.  K and V are released after their last S^T/dP^T so the next
+// unit's loads overlap the last step.  Epilogue: warpgroup 0 writes dV,
+// warpgroup 1 writes scale * dK, straight from TMEM to global.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DkvCfg {
@@ -79,15 +81,22 @@ struct DkvCfg {
   static constexpr uint32_t OFF_V = OFF_K + KT_BYTES;
   static constexpr uint32_t OFF_Q = OFF_V + KT_BYTES;
   static constexpr uint32_t OFF_DO = OFF_Q + NS * QT_BYTES;
+  // P^T of the current step, bf16 [keys x queries] K-major (A of dV = P^T dO)
+  static constexpr uint32_t OFF_P = OFF_DO + NS * QT_BYTES;
+  static constexpr uint32_t PT_BYTES = BK * BQ * 2;
   // [2 warpgroups][2 buffers][128 floats]: lse2 then D of the warpgroup's 64 queries
-  static constexpr uint32_t OFF_VEC = OFF_DO + NS * QT_BYTES;
+  static constexpr uint32_t OFF_VEC = OFF_P + PT_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_VEC + 2 * 2 * 128 * 4;
+  static constexpr uint32_t USED_BYTES = OFF_BAR + 256;
+  // The tiles want a 1024-byte aligned base; the launch adds that much slack
+  // where the per-block limit allows and the kernel checks the rest.
   static constexpr uint32_t SMEM_BYTES =
-      (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
+      USED_BYTES + 1024 < kMaxSmemPerBlock ? USED_BYTES + 1024 : kMaxSmemPerBlock;
+  static_assert(USED_BYTES <= kMaxSmemPerBlock, "dK/dV tiles exceed shared memory");
   static constexpr int NTHREADS = 384;
   // register split: 384 threads launch with 168 registers each; the two
-  // element-wise warpgroups take 192, the producer/MMA warpgroup 120.
-  static constexpr uint32_t LAUNCH_REGS = 168, EW_REGS = 192, CONTROL_REGS = 120;
+  // element-wise warpgroups take 200, the producer/MMA warpgroup 104.
+  static constexpr uint32_t LAUNCH_REGS = 168, EW_REGS = 200, CONTROL_REGS = 104;
   static_assert(2 * EW_REGS + CONTROL_REGS <= 3 * LAUNCH_REGS, "register split over budget");
   static constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 384;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -96,7 +105,7 @@ struct DkvCfg {
 struct DkvBars {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full, dp_full, p_full, ds_full;
+  uint64_t s_full, s_free, dp_full, p_full, p_empty, ds_full;
   uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
   int abort;
@@ -117,17 +126,12 @@ struct DkvUnit {
 __device__ __forceinline__ DkvUnit dkv_decode(int u, const AttnParams& p) {
   DkvUnit U;
   const int b = u / p.units_per_batch;
-  int r = u % p.units_per_batch;
-  int h = 0;
-  for (; h < p.H; ++h) {
-    const int cnt = dkv_units_of_head(p.N, p.lo[h]);
-    if (r < cnt) break;
-    r -= cnt;
-  }
+  const int r = u % p.units_per_batch;
+  const int h = head_of(p.unit_start, p.H, r);
   U.bh = b * p.H + h;
   U.lo = p.lo[h];
   U.hi = p.hi[h];
-  U.j0 = (int64_t)r * 128;
+  U.j0 = (int64_t)(r - p.unit_start[h]) * 128;
   const Strip s = query_strip(p.N, U.lo, U.hi, U.j0, 128, 128);
   U.qa = s.begin;
   U.qb = s.end;
@@ -142,6 +146,7 @@ __global__ void __launch_bounds__(384, 1)
   using C = DkvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
+  if (!smem_fits(smem_raw, smem, C::USED_BYTES)) return;
   DkvBars* bars = reinterpret_cast<DkvBars*>(smem + C::OFF_BAR);
   float* vec = reinterpret_cast<float*>(smem + C::OFF_VEC);
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
@@ -152,6 +157,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t sV = ptx::smem_u32(smem + C::OFF_V);
   const uint32_t sQ = ptx::smem_u32(smem + C::OFF_Q);
   const uint32_t sDO = ptx::smem_u32(smem + C::OFF_DO);
+  const uint32_t sP = ptx::smem_u32(smem + C::OFF_P);
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars->kv_full, 1);
@@ -161,8 +167,10 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_init(&bars->q_empty[s], 1);
     }
     ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->s_free, 256);
     ptx::mbar_init(&bars->dp_full, 1);
     ptx::mbar_init(&bars->p_full, 256);
+    ptx::mbar_init(&bars->p_empty, 1);
     ptx::mbar_init(&bars->ds_full, 256);
     ptx::mbar_init(&bars->acc_done, 1);
     ptx::mbar_init(&bars->acc_free, 256);
@@ -228,9 +236,10 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idesc_g = ptx::idesc_bf16_f32(128, D, false, true);
-      int nkv = 0, gq = 0, cp = 0, cds = 0, cacc = 0;
+      int nkv = 0, gq = 0, cf = 0, cp = 0, cds = 0, cacc = 0;
       bool ok = true;
       auto qstage = [&](int g) { return g % C::NS; };
+      const uint64_t dPk = ptx::sdesc_sw128(sP, 0, 1024);  // P^T, K-major (A of dV)
       // descriptors of every operand buffer, built once
       const uint64_t dK = ptx::sdesc_sw128(sK, 0, 1024), dV = ptx::sdesc_sw128(sV, 0, 1024);
       // K-major (B of S^T/dP^T) and MN-major (B of dK/dV) views of both Q/dO stages
@@ -256,6 +265,12 @@ __global__ void __launch_bounds__(384, 1)
           ptx::mma_bf16_ts(tmem + dst, tmem + a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
                            ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (!first || kk > 0));
       };
+      auto issue_dv = [&](uint64_t db, bool first) {  // dV += P^T dO, both from shared memory
+#pragma unroll
+        for (int kk = 0; kk < C::BQ / 16; ++kk)
+          ptx::mma_bf16(tmem + C::TM_DV, ptx::sdesc_advance(dPk, (kk / 4) * (C::BK * 128) + (kk % 4) * 32),
+                        ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (!first || kk > 0));
+      };
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
         const DkvUnit U = dkv_decode(u, p);
         const int nq = U.qb - U.qa + 1;
@@ -268,20 +283,26 @@ __global__ void __launch_bounds__(384, 1)
         ptx::mma_commit(&bars->s_full);
         issue_nt(C::TM_DPT, dV, dOk(qstage(g0)));
         ptx::mma_commit(&bars->dp_full);
+        if (nq == 1) ptx::mma_commit(&bars->kv_empty);           // K and V read for the last time
         for (int j = 0; j < nq; ++j) {
           const int g = g0 + j;
-          ok = bar_wait(&bars->p_full, (cp++) & 1, abort_flag);
+          // the warpgroups hold S^T of this tile in registers: S^T of the next
+          // one goes into the same columns while they exponentiate
+          ok = bar_wait(&bars->s_free, (cf++) & 1, abort_flag);
+          if (ok && j + 1 < nq) {
+            ok = bar_wait(&bars->q_full[qstage(g + 1)], ((g + 1) / C::NS) & 1, abort_flag);
+            if (ok) {
+              ptx::tc_fence_after();
+              issue_nt(C::TM_ST, dK, dQk(qstage(g + 1)));
+              ptx::mma_commit(&bars->s_full);
+            }
+          }
+          if (ok) ok = bar_wait(&bars->p_full, (cp++) & 1, abort_flag);
           if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
-          issue_grad(C::TM_DV, C::TM_ST, dOm(qstage(g)), j == 0);   // dV += P^T dO
-          if (j + 1 < nq) {
-            ok = bar_wait(&bars->q_full[qstage(g + 1)], ((g + 1) / C::NS) & 1, abort_flag);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            issue_nt(C::TM_ST, dK, dQk(qstage(g + 1)));            // S^T of the next tile
-            ptx::mma_commit(&bars->s_full);
-          }
+          issue_dv(dOm(qstage(g)), j == 0);                        // dV += P^T dO
+          ptx::mma_commit(&bars->p_empty);
           ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
@@ -290,12 +311,12 @@ __global__ void __launch_bounds__(384, 1)
           if (j + 1 < nq) {
             issue_nt(C::TM_DPT, dV, dOk(qstage(g + 1)));           // dP^T of the next tile
             ptx::mma_commit(&bars->dp_full);
+            if (j + 2 == nq) ptx::mma_commit(&bars->kv_empty);     // K and V read for the last time
           }
         }
         if (!ok) break;
         ++cacc;
         ptx::mma_commit(&bars->acc_done);
-        ptx::mma_commit(&bars->kv_empty);
         gq = g0 + nq;
       }
       ptx::mma_commit(&bars->drain);
@@ -365,8 +386,7 @@ __global__ void __launch_bounds__(384, 1)
         const float* vl = vecw + (gq & 1) * 128;
         const float* vd = vl + 64;
         const int cb = 64 * w - qlo;
-        // ---- P^T = exp2(S^T c - lse2); bf16 pairs to columns [0, 32) of the
-        // warpgroup's 64 (already read)
+        // ---- P^T = exp2(S^T c - lse2), bf16 to the shared P^T tile (A of dV)
         ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, (cs++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
@@ -378,6 +398,9 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tmem_wait_ld();
           ptx::reg_fence(sr[0]);
           ptx::reg_fence(sr[1]);
+          // S^T is in registers: its columns may take the next tile's S^T
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&bars->s_free);
           // vl holds -lse2 of the 64 queries: x = s * c2 - lse2 in pairs
           const float4* nl4 = reinterpret_cast<const float4*>(vl);
           const float2 c2v = make_float2(c2, c2);
@@ -418,10 +441,17 @@ __global__ void __launch_bounds__(384, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = ptx::pack_bf16x2(pt[2 * e], pt[2 * e + 1]);
-          ptx::tmem_st32(tS, pk);
-          ptx::tmem_wait_st();
+          // the tile is free once dV of the previous step has read it
+          ok = __all_sync(0xffffffffu, bar_wait(&bars->p_empty, (gq & 1) ^ 1, abort_flag));
+          if (!ok) break;
+          // row r of the warpgroup's 64-query block, 128-byte swizzle
+          const uint32_t prow = sP + (uint32_t)w * (C::BK * 128) + (uint32_t)r * 128;
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            ptx::st_shared_v4(prow + ((k ^ (r & 7)) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
+                              pk[4 * k + 3]);
+          ptx::fence_proxy_async_smem();
         }
-        ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full);
         // ---- dS^T = P^T (dP^T - D)
         ok = __all_sync(0xffffffffu, bar_wait(&bars->dp_full, (cdp++) & 1, abort_flag));
@@ -491,17 +521,11 @@ __global__ void __launch_bounds__(384, 1)
   // ------------------------------------------------------------ keys no query reaches
   {
     const int num_fill = p.B * p.fills_per_batch;
-    const int nkt = (int)((N + 127) / 128);
     for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
       const int b = f / p.fills_per_batch;
-      int r = f % p.fills_per_batch;
-      int h = 0;
-      for (; h < p.H; ++h) {
-        const int cnt = nkt - dkv_units_of_head(N, p.lo[h]);
-        if (r < cnt) break;
-        r -= cnt;
-      }
-      const int64_t kt = dkv_units_of_head(N, p.lo[h]) + r;
+      const int r = f % p.fills_per_batch;
+      const int h = head_of(p.fill_start, p.H, r);
+      const int64_t kt = dkv_units_of_head(N, p.lo[h]) + (r - p.fill_start[h]);
       const int64_t row0 = (int64_t)(b * p.H + h) * N + kt * 128;
       const int64_t rows = min64(kt * 128 + 128, N) - kt * 128;
       zero_rows_bf16(static_cast<uint16_t*>(p.dk) + row0 * D, rows, D);
@@ -573,19 +597,13 @@ struct DqUnit {
 
 __device__ __forceinline__ DqUnit dq_decode(int u, const AttnParams& p) {
   DqUnit U;
-  const int nqt = (int)((p.N + 127) / 128);
   const int b = u / p.units_per_batch;
-  int r = u % p.units_per_batch;
-  int h = 0;
-  for (; h < p.H; ++h) {
-    const int cnt = nqt - p.lo[h] / 128;
-    if (r < cnt) break;
-    r -= cnt;
-  }
+  const int r = u % p.units_per_batch;
+  const int h = head_of(p.unit_start, p.H, r);
   U.bh = b * p.H + h;
   U.lo = p.lo[h];
   U.hi = p.hi[h];
-  U.i0 = (int64_t)(p.lo[h] / 128 + r) * 128;
+  U.i0 = (int64_t)(p.lo[h] / 128 + (r - p.unit_start[h])) * 128;
   const Strip s = key_strip(p.N, U.lo, U.hi, U.i0, 128, 128);
   U.ka = s.begin;
   U.kb = s.end;
@@ -888,14 +906,9 @@ __global__ void __launch_bounds__(384, 1)
     const int num_fill = p.B * p.fills_per_batch;
     for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
       const int b = f / p.fills_per_batch;
-      int r = f % p.fills_per_batch;
-      int h = 0;
-      for (; h < p.H; ++h) {
-        const int cnt = p.lo[h] / 128;
-        if (r < cnt) break;
-        r -= cnt;
-      }
-      const int64_t row0 = (int64_t)(b * p.H + h) * N + (int64_t)r * 128;
+      const int r = f % p.fills_per_batch;
+      const int h = head_of(p.fill_start, p.H, r);
+      const int64_t row0 = (int64_t)(b * p.H + h) * N + (int64_t)(r - p.fill_start[h]) * 128;
       zero_rows_bf16(static_cast<uint16_t*>(p.dq) + row0 * D, 128, D);
     }
   }

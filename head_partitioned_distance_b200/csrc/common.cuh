@@ -15,7 +15,11 @@ constexpr int kMaxHeads = 256;
 
 // Status codes mirrored from spa.h (kept numerically identical).
 constexpr int kStatusOk = 0;
+constexpr int kStatusUnsupported = 2;
 constexpr int kStatusTimeout = 4;
+
+// Opt-in dynamic shared memory per block on sm_100 (227 KB).
+constexpr uint32_t kMaxSmemPerBlock = 232448;
 
 // Longest a thread waits on one mbarrier phase before the kernel gives up.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;
@@ -28,7 +32,10 @@ struct AttnParams {
   int64_t N;
   float scale;        // multiplies q.k
   float scale_log2;   // scale * log2(e): scores in base-2 units
-  // persistent forward: units (non-empty 256-row blocks) and all-empty blocks per batch
+  // Work list of a persistent grid, per batch: the kernel's units (tiles it
+  // computes) and fills (tiles it only zeroes), head by head.  The units of
+  // head h are numbers [unit_start[h], unit_start[h + 1]) of the batch, the
+  // fills [fill_start[h], fill_start[h + 1]); unit_start[H] = units_per_batch.
   int units_per_batch;
   int fills_per_batch;
   // forward: lse is written; backward: lse (read) and delta (workspace)
@@ -43,7 +50,26 @@ struct AttnParams {
   const void* dout;
   int32_t lo[kMaxHeads];
   int32_t hi[kMaxHeads];
+  int32_t unit_start[kMaxHeads + 1];
+  int32_t fill_start[kMaxHeads + 1];
 };
+
+// Head whose range [start[h], start[h + 1]) holds r, for 0 <= r < start[H]:
+// the number of k in [1, H] with start[k] <= r (start is non-decreasing).
+// Eight independent parameter loads per round rather than a dependent chain
+// of one load per head.
+__device__ __forceinline__ int head_of(const int32_t* start, int H, int r) {
+  int h = 0;
+#pragma unroll 1
+  for (int base = 1; base <= H; base += 8) {
+    int n = 0;
+#pragma unroll
+    for (int k = 0; k < 8; ++k) n += start[min(base + k, H)] <= r ? 1 : 0;
+    h += n;
+    if (n < 8) break;
+  }
+  return h;
+}
 
 // The library's device error word: a kernel that times out on a wait stores
 // kStatusTimeout here; spa_device_status() reads and clears it.
@@ -85,6 +111,18 @@ __device__ __forceinline__ bool bar_drain(uint64_t* bar, uint32_t parity) {
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
   return reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(p) + 1023) & ~uintptr_t(1023));
+}
+
+// True when `used` bytes from the aligned base stay inside the launch's
+// dynamic shared memory.  Otherwise the device error word becomes
+// kStatusUnsupported and the caller returns before touching shared memory
+// (the condition is the same for every thread of the block).
+__device__ __forceinline__ bool smem_fits(const uint8_t* raw, const uint8_t* aligned, uint32_t used) {
+  uint32_t dyn;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(dyn));
+  const bool fits = (uint32_t)(aligned - raw) + used <= dyn;
+  if (!fits && threadIdx.x == 0) atomicExch(&g_spa_status, kStatusUnsupported);
+  return fits;
 }
 
 // Zero `rows` rows of a [.., d] bf16 matrix starting at `base` (16-byte

@@ -85,20 +85,13 @@ template <int D>
 __device__ __forceinline__ FwdUnit fwd_decode(int u, const AttnParams& p) {
   using C = FwdCfg<D>;
   FwdUnit U;
-  const int nblk = (int)((p.N + C::BU - 1) / C::BU);
   const int b = u / p.units_per_batch;
-  int r = u % p.units_per_batch;
-  int h = 0;
-  for (; h < p.H; ++h) {
-    const int first = p.lo[h] / C::BU;
-    const int cnt = nblk - first;
-    if (r < cnt) break;
-    r -= cnt;
-  }
+  const int r = u % p.units_per_batch;
+  const int h = head_of(p.unit_start, p.H, r);
   U.bh = b * p.H + h;
   U.lo = p.lo[h];
   U.hi = p.hi[h];
-  U.i0 = (int64_t)(p.lo[h] / C::BU + r) * C::BU;
+  U.i0 = (int64_t)(p.lo[h] / C::BU + (r - p.unit_start[h])) * C::BU;
   U.u0 = 1 << 30;
   U.u1 = -1;
   for (int t = 0; t < 2; ++t) {
@@ -577,14 +570,9 @@ __global__ void __launch_bounds__(384, 1)
     const int num_fill = p.B * p.fills_per_batch;
     for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
       const int b = f / p.fills_per_batch;
-      int r = f % p.fills_per_batch;
-      int h = 0;
-      for (; h < p.H; ++h) {
-        const int cnt = p.lo[h] / C::BU;
-        if (r < cnt) break;
-        r -= cnt;
-      }
-      const int64_t row0 = (int64_t)(b * p.H + h) * N + (int64_t)r * C::BU;
+      const int r = f % p.fills_per_batch;
+      const int h = head_of(p.fill_start, p.H, r);
+      const int64_t row0 = (int64_t)(b * p.H + h) * N + (int64_t)(r - p.fill_start[h]) * C::BU;
       zero_rows_bf16(static_cast<uint16_t*>(p.o) + row0 * D, C::BU, D);
       for (int e = threadIdx.x; e < C::BU; e += blockDim.x) p.lse[row0 + e] = -INFINITY;
     }

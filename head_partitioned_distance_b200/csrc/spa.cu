@@ -127,6 +127,26 @@ int sm_count(int* n) {
   return SPA_OK;
 }
 
+// Per-head work lists of a persistent grid: unit and fill counts of head h
+// from units_of(h) and fills_of(h), stored as prefix sums in p.
+template <class Units, class Fills>
+int set_work_lists(AttnParams& p, Units units_of, Fills fills_of) {
+  int64_t u = 0, f = 0;
+  for (int h = 0; h < p.H; ++h) {
+    p.unit_start[h] = (int32_t)u;
+    p.fill_start[h] = (int32_t)f;
+    u += units_of(h);
+    f += fills_of(h);
+    if (u > 2147483647LL || f > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+  }
+  if ((int64_t)p.B * u > 2147483647LL || (int64_t)p.B * f > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+  p.unit_start[p.H] = (int32_t)u;
+  p.fill_start[p.H] = (int32_t)f;
+  p.units_per_batch = (int)u;
+  p.fills_per_batch = (int)f;
+  return SPA_OK;
+}
+
 template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, AttnParams& p,
              cudaStream_t stream) {
@@ -144,14 +164,10 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, A
   // Work list of the persistent grid: per batch, every 256-row block of every
   // head from the one holding lo_h on (units), and the blocks before it (fills).
   const int64_t nblk = (p.N + C::BU - 1) / C::BU;
-  int64_t upb = 0, fpb = 0;
-  for (int h = 0; h < p.H; ++h) {
-    upb += nblk - p.lo[h] / C::BU;
-    fpb += p.lo[h] / C::BU;
-  }
-  if ((int64_t)p.B * upb > 2147483647LL || (int64_t)p.B * fpb > 2147483647LL) return SPA_ERR_UNSUPPORTED;
-  p.units_per_batch = (int)upb;
-  p.fills_per_batch = (int)fpb;
+  if ((st = set_work_lists(
+           p, [&](int h) { return nblk - p.lo[h] / C::BU; }, [&](int h) { return (int64_t)(p.lo[h] / C::BU); })))
+    return st;
+  const int64_t upb = p.units_per_batch;
   p.lse = lse;
   p.o = o;
   int sms = 0;
@@ -198,12 +214,12 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     static std::atomic<int> regs_kv{0};
     if ((st = check_regs(spa::spa_bwd_dkdv_kernel<D>, (int)KC::LAUNCH_REGS, regs_kv))) return st;
     const int64_t nkt = (p.N + 127) / 128;
-    int64_t upb = 0;
-    for (int h = 0; h < p.H; ++h) upb += (p.N - 1 - p.lo[h]) / 128 + 1;
-    const int64_t fpb = (int64_t)p.H * nkt - upb;
     if ((int64_t)p.B * p.H * nkt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
-    p.units_per_batch = (int)upb;
-    p.fills_per_batch = (int)fpb;
+    if ((st = set_work_lists(
+             p, [&](int h) { return (p.N - 1 - p.lo[h]) / 128 + 1; },
+             [&](int h) { return nkt - ((p.N - 1 - p.lo[h]) / 128 + 1); })))
+      return st;
+    const int64_t upb = p.units_per_batch;
     int sms = 0;
     if ((st = sm_count(&sms))) return st;
     const int64_t units = (int64_t)p.B * upb;
@@ -222,14 +238,11 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     static std::atomic<int> regs_q{0};
     if ((st = check_regs(spa::spa_bwd_dq_kernel<D>, (int)QC::LAUNCH_REGS, regs_q))) return st;
     const int64_t nqt = (p.N + 127) / 128;
-    int64_t upb = 0, fpb = 0;
-    for (int h = 0; h < p.H; ++h) {
-      upb += nqt - p.lo[h] / 128;
-      fpb += p.lo[h] / 128;
-    }
     if ((int64_t)p.B * p.H * nqt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
-    p.units_per_batch = (int)upb;
-    p.fills_per_batch = (int)fpb;
+    if ((st = set_work_lists(
+             p, [&](int h) { return nqt - p.lo[h] / 128; }, [&](int h) { return (int64_t)(p.lo[h] / 128); })))
+      return st;
+    const int64_t upb = p.units_per_batch;
     int sms = 0;
     if ((st = sm_count(&sms))) return st;
     const int64_t units = (int64_t)p.B * upb;
@@ -517,7 +530,8 @@ int spa_device_status(void* stream) {
     const int z = 0;
     if (cudaMemcpyToSymbol(spa::g_spa_status, &z, sizeof(int)) != cudaSuccess) return SPA_ERR_CUDA;
   }
-  return v == 0 ? SPA_OK : SPA_ERR_TIMEOUT;
+  if (v == 0) return SPA_OK;
+  return v == spa::kStatusUnsupported ? SPA_ERR_UNSUPPORTED : SPA_ERR_TIMEOUT;
 }
 
 }  // extern "C"

@@ -218,8 +218,11 @@ SPA_API int spa_debug_wait_timeout(int64_t limit_ns, void* stream);
 
 /*
  * Synchronises `stream` and returns the library's device error word, then
- * clears it: SPA_OK, or SPA_ERR_TIMEOUT when a kernel gave up on a wait (the
- * kernel then wrote incomplete outputs and released its tensor memory).
+ * clears it: SPA_OK; SPA_ERR_TIMEOUT when a kernel gave up on a wait (the
+ * kernel then wrote incomplete outputs and released its tensor memory); or
+ * SPA_ERR_UNSUPPORTED when a kernel found its dynamic shared memory too
+ * small for its tiles after aligning the base to 1024 bytes (it returned
+ * without writing its outputs).
  */
 SPA_API int spa_device_status(void* stream);
 
