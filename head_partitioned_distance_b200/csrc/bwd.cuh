@@ -84,7 +84,8 @@ struct DkvCfg {
   // P^T of the current step, bf16 [keys x queries] K-major (A of dV = P^T dO)
   static constexpr uint32_t OFF_P = OFF_DO + NS * QT_BYTES;
   static constexpr uint32_t PT_BYTES = BK * BQ * 2;
-  // [2 warpgroups][2 buffers][128 floats]: lse2 then D of the warpgroup's 64 queries
+  // vectors of a query tile, [2 stages][256 floats]: -lse * log2(e) of its
+  // 128 queries, then -D of them
   static constexpr uint32_t OFF_VEC = OFF_P + PT_BYTES;
   static constexpr uint32_t OFF_BAR = OFF_VEC + 2 * 2 * 128 * 4;
   static constexpr uint32_t USED_BYTES = OFF_BAR + 256;
@@ -106,6 +107,7 @@ struct DkvBars {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full, s_free, dp_full, p_full, p_empty, ds_full;
+  uint64_t vec_full[2], vec_empty[2];
   uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
   int abort;
@@ -165,6 +167,8 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars->q_full[s], 1);
       ptx::mbar_init(&bars->q_empty[s], 1);
+      ptx::mbar_init(&bars->vec_full[s], 1);
+      ptx::mbar_init(&bars->vec_empty[s], 256);
     }
     ptx::mbar_init(&bars->s_full, 1);
     ptx::mbar_init(&bars->s_free, 256);
@@ -194,11 +198,13 @@ __global__ void __launch_bounds__(384, 1)
     // idle warps of the control warpgroup
   } else if (warp == 8) {
     // ------------------------------------------------------------ producer warp
+    // Lane 0 issues the tile copies; all lanes load the query tiles' lse and D
+    // into the shared vector ring.
     int nkv = 0, gq = 0, armed[2] = {0, 0};
     bool ok = true;
-    for (int u = blockIdx.x; ok && lane == 0 && u < num_units; u += gridDim.x) {
+    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
       const DkvUnit U = dkv_decode(u, p);
-      ok = bar_wait(&bars->kv_empty, (nkv & 1) ^ 1, abort_flag);
+      ok = __all_sync(0xffffffffu, bar_wait(&bars->kv_empty, (nkv & 1) ^ 1, abort_flag));
       if (!ok) break;
       if (lane == 0) {
         ptx::mbar_arrive_expect_tx(&bars->kv_full, 2 * C::KT_BYTES);
@@ -210,7 +216,7 @@ __global__ void __launch_bounds__(384, 1)
       ++nkv;
       for (int qt = U.qa; qt <= U.qb; ++qt, ++gq) {
         const int s = gq % C::NS;
-        ok = bar_wait(&bars->q_empty[s], ((gq / C::NS) & 1) ^ 1, abort_flag);
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->q_empty[s], ((gq / C::NS) & 1) ^ 1, abort_flag));
         if (!ok) break;
         const int64_t i0 = (int64_t)qt * C::BQ;
         if (lane == 0) {
@@ -223,6 +229,26 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         ++armed[s];
+        // -lse * log2(e) and -D of the tile's queries (rows past N: 0)
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->vec_empty[s], ((gq / C::NS) & 1) ^ 1, abort_flag));
+        if (!ok) break;
+        float* vs = vec + s * 256;
+        const float* lrow = p.lse + (int64_t)U.bh * N;
+        const float* drow = p.delta + (int64_t)U.bh * N;
+        float lv[4], dv[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int64_t i = i0 + lane + 32 * e;
+          lv[e] = i < N ? lrow[i] : 0.f;
+          dv[e] = i < N ? drow[i] : 0.f;
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          vs[lane + 32 * e] = -lv[e] * kLog2e;
+          vs[128 + lane + 32 * e] = -dv[e];
+        }
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bars->vec_full[s]);
       }
     }
     if (lane == 0) {
@@ -333,40 +359,13 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tS = tmem + lane_base + C::TM_ST + 64 * w;
     const uint32_t tDP = tmem + lane_base + C::TM_DPT + 64 * w;
     const float c2 = p.scale_log2;
-    float* vecw = vec + w * 256;                     // this warpgroup's two vector buffers
-    // Thread r fetches one value of the vectors a query tile needs: lse of
-    // query 64w + r for r < 64, else D of query 64w + r - 64.  The shared
-    // copy holds -lse * log2(e) and -D (see publish()), ready for fused
-    // multiply-adds; the conversion waits until the load has long landed.
-    auto fetch = [&](int bh, int64_t i0) -> float {
-      const int64_t i = i0 + 64 * w + (r & 63);
-      if (i >= N) return 0.f;
-      return r < 64 ? p.lse[(int64_t)bh * N + i] : p.delta[(int64_t)bh * N + i];
-    };
-    auto publish = [&](float raw) { return r < 64 ? -raw * kLog2e : -raw; };
     int gq = 0, cs = 0, cdp = 0, cacc = 0;
     bool ok = true;
-    if (blockIdx.x < num_units) {
-      const DkvUnit U0 = dkv_decode(blockIdx.x, p);
-      vecw[r] = publish(fetch(U0.bh, (int64_t)U0.qa * C::BQ));
-    }
-    ptx::named_bar_sync(1 + w, 128);
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
       const DkvUnit U = dkv_decode(u, p);
       const int64_t j = U.j0 + r;
       for (int qt = U.qa; qt <= U.qb; ++qt, ++gq) {
         const int64_t i0 = (int64_t)qt * C::BQ;
-        // prefetch the vectors of the next query tile (this unit's or the next unit's first)
-        float pre = 0.f;
-        bool has_next = true;
-        if (qt < U.qb) {
-          pre = fetch(U.bh, i0 + C::BQ);
-        } else if (u + (int)gridDim.x < num_units) {
-          const DkvUnit Un = dkv_decode(u + gridDim.x, p);
-          pre = fetch(Un.bh, (int64_t)Un.qa * C::BQ);
-        } else {
-          has_next = false;
-        }
         const bool interior = tile_is_interior(N, U.lo, U.hi, i0, C::BQ, U.j0, C::BK);
         // Edge tile: query column q (0..127) is permitted for this key iff
         // qlo <= q <= qlo + span.
@@ -383,11 +382,13 @@ __global__ void __launch_bounds__(384, 1)
             span = (uint32_t)(q_last - q_first);
           }
         }
-        const float* vl = vecw + (gq & 1) * 128;
-        const float* vd = vl + 64;
+        // this warpgroup's 64 queries in vector stage gq % 2
+        const float* vl = vec + (gq % C::NS) * 256 + 64 * w;
+        const float* vd = vl + 128;
         const int cb = 64 * w - qlo;
         // ---- P^T = exp2(S^T c - lse2), bf16 to the shared P^T tile (A of dV)
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, (cs++) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, (cs++) & 1, abort_flag) &&
+                                         bar_wait(&bars->vec_full[gq % C::NS], (gq / C::NS) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
         float pt[64];
@@ -487,10 +488,7 @@ __global__ void __launch_bounds__(384, 1)
         }
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->ds_full);
-        // publish the prefetched vectors; every thread of the warpgroup is past
-        // its last read of that buffer (the previous tile)
-        if (has_next) vecw[((gq + 1) & 1) * 128 + r] = publish(pre);
-        ptx::named_bar_sync(1 + w, 128);
+        ptx::mbar_arrive(&bars->vec_empty[gq % C::NS]);  // last read of this vector stage
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
