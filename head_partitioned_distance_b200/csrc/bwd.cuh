@@ -541,17 +541,22 @@ __global__ void __launch_bounds__(384, 1)
 
 // ---------------------------------------------------------------------------
 // dQ: persistent grid; a unit is (b, h, query tile of 128 rows), walking the
-// same 128-key strip as the forward.  Per key tile j:
-//   S_j = Q K^T      SS MMA -> TMEM S buffer j % 2 ([0,128) or [128,256))
-//   dP  = dO V^T     SS MMA -> TMEM [256,384)
+// same 128-key strip as the forward.  Q and dO of the unit are fixed, so they
+// sit in TMEM as bf16 A operands and the two products of each key tile read
+// only K or V from shared memory:
+//   S   = Q K^T      TS MMA (A = Q from TMEM [384, 384 + D/2))   -> TMEM [0,128)
+//   dP  = dO V^T     TS MMA (A = dO from TMEM [384 + D/2, 512))  -> TMEM [128,256)
 //   dS  = P (dP - D), P = exp2(S c - lse2) masked on edge tiles; written as
-//                    bf16 over S buffer j % 2
-//   dQ += dS K       TS MMA (A = dS from TMEM, B = K MN-major) -> TMEM [384,512)
+//                    bf16 over dP
+//   dQ += dS K       TS MMA (A = dS from TMEM, B = K MN-major)   -> TMEM [256,384)
 // Two warpgroups share each tile: warpgroup w owns key columns [64w, 64w+64)
 // of every query row (thread r = row r = TMEM lane r).  S of the next key
-// tile goes to the other buffer before dQ of this one, so the tensor core
-// runs while the warpgroups work.  Epilogue: scale * dQ straight from TMEM to
-// global, warpgroup w writing head dims [D/2 w, D/2 (w+1)).
+// tile is issued as soon as the warpgroups hold this one in registers, so it
+// overlaps their exponentials; dP of the next tile follows dQ.  At a unit's
+// start warpgroup 0 copies Q and warpgroup 1 copies dO from the staging tiles
+// the copy engine filled into TMEM, which frees the staging tiles for the next
+// unit.  Epilogue: scale * dQ straight from TMEM to global, warpgroup w
+// writing head dims [D/2 w, D/2 (w+1)).
 // ---------------------------------------------------------------------------
 template <int D>
 struct DqCfg {
@@ -573,14 +578,15 @@ struct DqCfg {
   // element-wise warpgroups take 192, the producer/MMA warpgroup 120.
   static constexpr uint32_t LAUNCH_REGS = 168, EW_REGS = 192, CONTROL_REGS = 120;
   static_assert(2 * EW_REGS + CONTROL_REGS <= 3 * LAUNCH_REGS, "register split over budget");
-  static constexpr uint32_t TM_S0 = 0, TM_S1 = 128, TM_DP = 256, TM_DQ = 384;
+  static constexpr uint32_t TM_S = 0, TM_DP = 128, TM_DQ = 256, TM_QA = 384, TM_DOA = 384 + D / 2;
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
 struct DqBars {
-  uint64_t q_full, q_empty;
+  uint64_t q_full, q_empty;  // staging tiles of Q and dO
   uint64_t k_full[2], v_full[2], kv_empty[2];
-  uint64_t s_full[2], dp_full, ds_full;  // s_full[b]: S buffer b written
+  uint64_t qa_full;          // Q and dO of the unit copied into TMEM
+  uint64_t s_full, s_free, dp_full, ds_full;
   uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
   int abort;
@@ -628,14 +634,15 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars->q_full, 1);
-    ptx::mbar_init(&bars->q_empty, 1);
+    ptx::mbar_init(&bars->q_empty, 256);
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars->k_full[s], 1);
       ptx::mbar_init(&bars->v_full[s], 1);
       ptx::mbar_init(&bars->kv_empty[s], 1);
     }
-    ptx::mbar_init(&bars->s_full[0], 1);
-    ptx::mbar_init(&bars->s_full[1], 1);
+    ptx::mbar_init(&bars->qa_full, 256);
+    ptx::mbar_init(&bars->s_full, 1);
+    ptx::mbar_init(&bars->s_free, 256);
     ptx::mbar_init(&bars->dp_full, 1);
     ptx::mbar_init(&bars->ds_full, 256);
     ptx::mbar_init(&bars->acc_done, 1);
@@ -665,6 +672,8 @@ __global__ void __launch_bounds__(384, 1)
       bool ok = true;
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
         const DqUnit U = dq_decode(u, p);
+        // the staging tiles are free once the warpgroups copied the previous
+        // unit's Q and dO into TMEM
         ok = bar_wait(&bars->q_empty, (nq & 1) ^ 1, abort_flag);
         if (!ok) break;
         ++nq;
@@ -702,10 +711,8 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BK, false, false);
       constexpr uint32_t idesc_g = ptx::idesc_bf16_f32(128, D, false, true);
-      int nq = 0, g = 0, gs = 0, cds = 0, cacc = 0;
+      int nq = 0, g = 0, cf = 0, cds = 0, cacc = 0;
       bool ok = true;
-      // descriptors of every operand buffer, built once
-      const uint64_t dQd = ptx::sdesc_sw128(sQ, 0, 1024), dOd = ptx::sdesc_sw128(sDO, 0, 1024);
       // K-major (B of S/dP) and MN-major K (B of dQ) views of both K/V stages
       const uint64_t dKk0 = ptx::sdesc_sw128(sK, 0, 1024), dKk1 = ptx::sdesc_sw128(sK + C::KT_BYTES, 0, 1024);
       const uint64_t dVk0 = ptx::sdesc_sw128(sV, 0, 1024), dVk1 = ptx::sdesc_sw128(sV + C::KT_BYTES, 0, 1024);
@@ -714,11 +721,12 @@ __global__ void __launch_bounds__(384, 1)
       auto dKk = [&](int st) { return st ? dKk1 : dKk0; };
       auto dVk = [&](int st) { return st ? dVk1 : dVk0; };
       auto dKm = [&](int st) { return st ? dKm1 : dKm0; };
-      auto issue_nt = [&](uint32_t dst, uint64_t da, uint64_t db) {
+      // dst = A (queries, bf16 pairs in TMEM at a_col) x B^T (keys, K-major in shared memory)
+      auto issue_nt = [&](uint32_t dst, uint32_t a_col, uint64_t db) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          ptx::mma_bf16(tmem + dst, ptx::sdesc_advance(da, (kk / 4) * (C::BQ * 128) + (kk % 4) * 32),
-                        ptx::sdesc_advance(db, (kk / 4) * (C::BK * 128) + (kk % 4) * 32), idesc_s, kk > 0);
+          ptx::mma_bf16_ts(tmem + dst, tmem + a_col + kk * 8,
+                           ptx::sdesc_advance(db, (kk / 4) * (C::BK * 128) + (kk % 4) * 32), idesc_s, kk > 0);
       };
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
         const DqUnit U = dq_decode(u, p);
@@ -726,35 +734,37 @@ __global__ void __launch_bounds__(384, 1)
         const int g0 = g;
         auto slot = [&](int jj) { return (g0 + jj) % C::NS; };
         auto par = [&](int jj) { return (uint32_t)(((g0 + jj) / C::NS) & 1); };
-        auto sbuf = [&](int jj) { return ((gs + jj) & 1) ? C::TM_S1 : C::TM_S0; };
-        auto sbar = [&](int jj) { return &bars->s_full[(gs + jj) & 1]; };
-        ok = bar_wait(&bars->q_full, (nq++) & 1, abort_flag) && bar_wait(&bars->k_full[slot(0)], par(0), abort_flag);
+        ok = bar_wait(&bars->qa_full, (nq++) & 1, abort_flag) && bar_wait(&bars->k_full[slot(0)], par(0), abort_flag);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_nt(sbuf(0), dQd, dKk(slot(0)));
-        ptx::mma_commit(sbar(0));
+        issue_nt(C::TM_S, C::TM_QA, dKk(slot(0)));
+        ptx::mma_commit(&bars->s_full);
         ok = bar_wait(&bars->v_full[slot(0)], par(0), abort_flag);
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_nt(C::TM_DP, dOd, dVk(slot(0)));
+        issue_nt(C::TM_DP, C::TM_DOA, dVk(slot(0)));
         ptx::mma_commit(&bars->dp_full);
         for (int j = 0; j < nk; ++j) {
-          if (j + 1 < nk) {
+          // the warpgroups hold S of this key tile in registers: S of the
+          // next one goes into the same columns while they exponentiate
+          ok = bar_wait(&bars->s_free, (cf++) & 1, abort_flag);
+          if (ok && j + 1 < nk) {
             ok = bar_wait(&bars->k_full[slot(j + 1)], par(j + 1), abort_flag);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            issue_nt(sbuf(j + 1), dQd, dKk(slot(j + 1)));              // S of the next key tile
-            ptx::mma_commit(sbar(j + 1));
+            if (ok) {
+              ptx::tc_fence_after();
+              issue_nt(C::TM_S, C::TM_QA, dKk(slot(j + 1)));
+              ptx::mma_commit(&bars->s_full);
+            }
           }
-          ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
+          if (ok) ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
           if (ok && j == 0) ok = bar_wait(&bars->acc_free, (cacc & 1) ^ 1, abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
           {
-            // dQ += dS K: A = dS (bf16 pairs over S buffer j, key halves at +0 / +64),
+            // dQ += dS K: A = dS (bf16 pairs over dP, key halves at +0 / +64),
             // B = K tile MN-major along d
             const uint64_t db = dKm(slot(j));
-            const uint32_t abase = tmem + sbuf(j);
+            const uint32_t abase = tmem + C::TM_DP;
 #pragma unroll
             for (int kk = 0; kk < C::BK / 16; ++kk)
               ptx::mma_bf16_ts(tmem + C::TM_DQ, abase + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
@@ -765,16 +775,14 @@ __global__ void __launch_bounds__(384, 1)
             ok = bar_wait(&bars->v_full[slot(j + 1)], par(j + 1), abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_nt(C::TM_DP, dOd, dVk(slot(j + 1)));                // dP of the next key tile
+            issue_nt(C::TM_DP, C::TM_DOA, dVk(slot(j + 1)));  // dP of the next key tile
             ptx::mma_commit(&bars->dp_full);
           }
         }
         if (!ok) break;
         ++cacc;
         ptx::mma_commit(&bars->acc_done);
-        ptx::mma_commit(&bars->q_empty);
         g = g0 + nk;
-        gs += nk;
       }
       ptx::mma_commit(&bars->drain);
       bar_drain(&bars->drain, 0);
@@ -787,19 +795,56 @@ __global__ void __launch_bounds__(384, 1)
     const int w = warp / 4;                      // key columns [64w, 64w+64)
     const int r = threadIdx.x - 128 * w;         // query row = TMEM lane
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + C::TM_S + 64 * w;
+    const uint32_t tDP = tmem + lane_base + C::TM_DP + 64 * w;
     const float c2 = p.scale_log2;
-    int gs = 0, cdp = 0, cacc = 0;
+    int cq = 0, cs = 0, cdp = 0, cacc = 0;
     bool ok = true;
-    for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-      const DqUnit U = dq_decode(u, p);
+    // Row r of the staged Q (warpgroup 0) or dO (warpgroup 1), 128-byte
+    // swizzled, into the warpgroup's TMEM operand as bf16 pairs along d.
+    auto stage_operands = [&]() -> bool {
+      if (!__all_sync(0xffffffffu, bar_wait(&bars->q_full, (cq++) & 1, abort_flag))) return false;
+      const uint32_t src = (w == 0 ? sQ : sDO) + (uint32_t)r * 128;
+      const uint32_t dst = tmem + lane_base + (w == 0 ? C::TM_QA : C::TM_DOA);
+#pragma unroll
+      for (int c = 0; c < C::DB; ++c) {
+        uint32_t v[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          ptx::ld_shared_v4(src + c * (C::BQ * 128) + ((k ^ (r & 7)) << 4), v[4 * k], v[4 * k + 1],
+                            v[4 * k + 2], v[4 * k + 3]);
+        ptx::tmem_st32(dst + 32 * c, v);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars->q_empty);
+      ptx::mbar_arrive(&bars->qa_full);
+      return true;
+    };
+    // The unit and the raw lse, D of row r; the loads land while other work runs.
+    DqUnit U{};
+    float lraw = 0.f, draw = 0.f;
+    auto fetch_unit = [&](int uu) {
+      U = dq_decode(uu, p);
+      const int64_t i = U.i0 + r;
+      lraw = 0.f;
+      draw = 0.f;
+      if (i < N) {
+        lraw = p.lse[(int64_t)U.bh * N + i];
+        draw = p.delta[(int64_t)U.bh * N + i];
+      }
+    };
+    int u = blockIdx.x;
+    if (u < num_units) {
+      ok = stage_operands();
+      fetch_unit(u);
+    }
+    for (; ok && u < num_units; u += gridDim.x) {
       const int64_t i = U.i0 + r;
       const bool in = i < N;
-      const float lse2 = in ? p.lse[(int64_t)U.bh * N + i] * kLog2e : 0.f;
-      const float Di = in ? p.delta[(int64_t)U.bh * N + i] : 0.f;
-      const float nlse2 = -lse2;
-      for (int kt = U.ka; kt <= U.kb; ++kt, ++gs) {
-        const uint32_t tS = tmem + lane_base + ((gs & 1) ? C::TM_S1 : C::TM_S0) + 64 * w;
-        const uint32_t tDP = tmem + lane_base + C::TM_DP + 64 * w;
+      const float nlse2 = -lraw * kLog2e;
+      const float Di = draw;
+      for (int kt = U.ka; kt <= U.kb; ++kt) {
         const int64_t j0 = (int64_t)kt * C::BK;
         const bool interior = tile_is_interior(N, U.lo, U.hi, U.i0, C::BQ, j0, C::BK);
         int clo = 0;
@@ -816,8 +861,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         const int cb = 64 * w - clo;
-        // buffer gs & 1 is used for the (gs >> 1)-th time
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[gs & 1], (gs >> 1) & 1, abort_flag));
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, (cs++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
         float pv[64];
@@ -828,6 +872,9 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tmem_wait_ld();
           ptx::reg_fence(sr[0]);
           ptx::reg_fence(sr[1]);
+          // S is in registers: its columns may take the next key tile's S
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&bars->s_free);
           // x = s * c2 - lse2 in pairs
           const float2 c2v = make_float2(c2, c2);
           const float2 nlv = make_float2(nlse2, nlse2);
@@ -862,7 +909,7 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tmem_wait_ld();
           ptx::reg_fence(dr[0]);
           ptx::reg_fence(dr[1]);
-          // dS = P (dP - D) in pairs
+          // dS = P (dP - D) in pairs, bf16 over the first half of the columns read
           const float2 ndv = make_float2(-Di, -Di);
           uint32_t pk[32];
 #pragma unroll
@@ -873,18 +920,26 @@ __global__ void __launch_bounds__(384, 1)
                                                    ndv));
             pk[e] = ptx::pack_bf16x2(d.x, d.y);
           }
-          ptx::tmem_st32(tS, pk);
+          ptx::tmem_st32(tDP, pk);
           ptx::tmem_wait_st();
         }
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->ds_full);
       }
       if (!ok) break;
+      const int bh = U.bh;
+      // the next unit's Q and dO go into TMEM while the last dQ products run
+      // (S and dP of this unit, their last readers, have completed)
+      if (u + (int)gridDim.x < num_units) {
+        ok = stage_operands();
+        if (!ok) break;
+        fetch_unit(u + gridDim.x);
+      }
       // ---------------------------------------------------------- epilogue
       ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
       if (!ok) break;
       ptx::tc_fence_after();
-      uint16_t* grow = static_cast<uint16_t*>(p.dq) + ((int64_t)U.bh * N + i) * D;
+      uint16_t* grow = static_cast<uint16_t*>(p.dq) + ((int64_t)bh * N + i) * D;
       const float mul = p.scale;
 #pragma unroll 1
       for (int c = w * (D / 2); c < (w + 1) * (D / 2); c += 32) {
