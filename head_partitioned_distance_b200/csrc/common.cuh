@@ -5,7 +5,6 @@
 #include <cuda.h>
 #include <stdint.h>
 
-#include "fastexp.cuh"
 #include "ptx.cuh"
 #include "sched.cuh"
 

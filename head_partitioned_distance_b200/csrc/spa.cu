@@ -335,11 +335,6 @@ __global__ void wait_timeout_kernel(uint64_t limit_ns) {
   if (threadIdx.x == 0 && ok) atomicExch(&spa::g_spa_status, -1);  // cannot happen: nothing arrives
 }
 
-__global__ void exp2_poly_kernel(const float* x, float* y, int64_t n) {
-  for (int64_t e = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; e < n; e += (int64_t)gridDim.x * blockDim.x)
-    y[e] = spa::exp2_poly(x[e]);
-}
-
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -507,13 +502,6 @@ int spa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
   // it, so the scratch needs no clearing between calls.
   return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, scratch, B, H, N, d, scale, nullptr, nullptr,
                    stream, kStepAll);
-}
-
-int spa_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream) {
-  if (!x || !y || n < 0) return SPA_ERR_INVAL;
-  if (n == 0) return SPA_OK;
-  exp2_poly_kernel<<<148 * 4, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n);
-  return launch_status();
 }
 
 int spa_debug_wait_timeout(int64_t limit_ns, void* stream) {

@@ -48,7 +48,6 @@ EXPORTS = {
     "spa_tile_schedule": ([_i64, _int, _i32p, _i32p, _int, _int, _i32p, _i32p, _u8p, _i32p, _i32p],
                           _int),
     "spa_tile_classes_device": ([_i64, _int, _i32p, _i32p, _int, _int, _vp, _vp], _int),
-    "spa_debug_exp2_poly": ([_vp, _vp, _i64, _vp], _int),
     "spa_debug_wait_timeout": ([_i64, _vp], _int),
     "spa_device_status": ([_vp], _int),
 }
@@ -232,15 +231,6 @@ def spa_tile_classes_device(N: int, H: int, Bq: int, Bk: int, out: torch.Tensor,
     _check(_lib.spa_tile_classes_device(N, H, lo_a, hi_a, Bq, Bk, out.data_ptr(), _stream_ptr(stream)),
            "spa_tile_classes_device")
     return out
-
-
-def spa_debug_exp2_poly(x: torch.Tensor, y: torch.Tensor, stream=None):
-    """y = the kernels' FMA-pipe 2^x, elementwise (float32 CUDA tensors)."""
-    if x.dtype != torch.float32 or y.dtype != torch.float32 or x.numel() != y.numel() or not x.is_cuda:
-        raise ValueError("x, y: float32 CUDA tensors of equal size")
-    _check(_lib.spa_debug_exp2_poly(x.data_ptr(), y.data_ptr(), x.numel(), _stream_ptr(stream)),
-           "spa_debug_exp2_poly")
-    return y
 
 
 def spa_debug_wait_timeout(limit_ns: int, stream=None):

@@ -199,14 +199,6 @@ SPA_API int spa_tile_classes_device(int64_t N, int H, const int32_t* lo, const i
                             int Bk, uint8_t* tile_class_dev, void* stream);
 
 /*
- * Test hook: y[i] = the kernels' FMA-pipe 2^x (Cody-Waite range reduction and
- * a degree-3 minimax polynomial; relative error below 1.5e-4 for
- * -126 <= x <= 127, inputs below -126 clamped) for n floats.  x, y: DEVICE
- * buffers of n floats; asynchronous on `stream`.
- */
-SPA_API int spa_debug_exp2_poly(const float* x, float* y, int64_t n, void* stream);
-
-/*
  * Test hook for failure detection: launches one warp that waits on an
  * mbarrier nothing ever arrives on, through the same bounded wait every
  * kernel uses, with a limit of limit_ns nanoseconds (1 ns .. 1 s).  The wait
