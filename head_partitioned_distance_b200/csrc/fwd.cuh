@@ -51,7 +51,7 @@ struct FwdCfg {
       (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
   static constexpr int NTHREADS = 384;
   // register split: 384 threads launch with 168 registers each (64512); the
-  // two softmax warpgroups take 192, the producer/MMA warpgroup 120.
+  // two softmax warpgroups take 200, the producer/MMA warpgroup 104.
   static constexpr uint32_t LAUNCH_REGS = 168, SOFTMAX_REGS = 200, CONTROL_REGS = 104;
   static_assert(2 * SOFTMAX_REGS + CONTROL_REGS <= 3 * LAUNCH_REGS, "register split over budget");
   static constexpr uint32_t TMEM_COLS = 512;
