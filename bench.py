@@ -45,7 +45,9 @@ METRIC = "band-sparse attn fwd+bwd useful TFLOP/s and % of B200 bf16 tensor peak
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "b1_h32_n32768_d128"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS = ("spa_fwd_kernel", "spa_bwd_delta_kernel", "spa_bwd_dkdv_kernel", "spa_bwd_dq_kernel")
+# one step = the forward, the dQ pass (which also forms the row sums D) and the
+# dK/dV pass, in launch order
+KERNELS = ("spa_fwd_kernel", "spa_bwd_dq_kernel", "spa_bwd_dkdv_kernel")
 
 
 # --------------------------------------------------------------------- counting
@@ -66,9 +68,8 @@ def kernel_work(w, pairs: int):
     rows = w.B * w.H * w.N
     return {
         "spa_fwd_kernel": ("tensor", 4 * d * pairs),            # S = QK^T, O += PV
-        "spa_bwd_delta_kernel": ("hbm", 2 * rows * d * 2 + rows * 4),  # read O, dO; write D
         "spa_bwd_dkdv_kernel": ("tensor", 8 * d * pairs),       # S^T, dP^T, dV, dK
-        "spa_bwd_dq_kernel": ("tensor", 6 * d * pairs),         # S, dP, dQ
+        "spa_bwd_dq_kernel": ("tensor", 6 * d * pairs),         # S, dP, dQ (and D = rowsum(dO * O))
     }
 
 
@@ -303,15 +304,12 @@ def run_spa(args):
         spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, stream=stream)
         if ev is not None:
             ev[0].record(stream)
-        spa.spa_attn_bwd_preprocess(o, dod, ws, stream=stream)
+        spa.spa_attn_bwd_dq_delta(qd, kd, vd, o, dod, lse, ws, dq, scale, stream=stream)
         if ev is not None:
             ev[1].record(stream)
         spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, ws, dk, dv, scale, stream=stream)
         if ev is not None:
             ev[2].record(stream)
-        spa.spa_attn_bwd_dq(qd, kd, vd, dod, lse, ws, dq, scale, stream=stream)
-        if ev is not None:
-            ev[3].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -324,7 +322,7 @@ def run_spa(args):
     sampler.start()
     K = args.steps
     t_start = torch.cuda.Event(enable_timing=True)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS))] for _ in range(K)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize(device)
@@ -339,16 +337,15 @@ def run_spa(args):
     clocks = sampler.stop()
     if spa.spa_device_status(stream) != spa.SPA_OK:
         raise SystemExit("device status not OK after the timed region")
-    elapsed_ms = t_start.elapsed_time(evs[-1][3])
+    elapsed_ms = t_start.elapsed_time(evs[-1][-1])
     per_kernel_ms = {name: 0.0 for name in KERNELS}
     prev = t_start
     for s in range(K):
         e = evs[s]
         per_kernel_ms["spa_fwd_kernel"] += prev.elapsed_time(e[0])
-        per_kernel_ms["spa_bwd_delta_kernel"] += e[0].elapsed_time(e[1])
+        per_kernel_ms["spa_bwd_dq_kernel"] += e[0].elapsed_time(e[1])
         per_kernel_ms["spa_bwd_dkdv_kernel"] += e[1].elapsed_time(e[2])
-        per_kernel_ms["spa_bwd_dq_kernel"] += e[2].elapsed_time(e[3])
-        prev = e[3]
+        prev = e[2]
     max_ms = reduce_max(elapsed_ms, device)
     value = aggregate(useful, K, world, max_ms)
 
@@ -436,7 +433,7 @@ def run_spa(args):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": e2e_ms / E},
-            "gpu_launches": 4 * K,
+            "gpu_launches": len(KERNELS) * K,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)

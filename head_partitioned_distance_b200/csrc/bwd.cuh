@@ -555,8 +555,13 @@ __global__ void __launch_bounds__(384, 1)
 // overlaps their exponentials; dP of the next tile follows dQ.  At a unit's
 // start warpgroup 0 copies Q and warpgroup 1 copies dO from the staging tiles
 // the copy engine filled into TMEM, which frees the staging tiles for the next
-// unit.  Epilogue: scale * dQ straight from TMEM to global, warpgroup w
-// writing head dims [D/2 w, D/2 (w+1)).
+// unit.  When the kernel is given o (AttnParams::o_in), the copy engine also
+// stages the unit's O tile and warpgroup 1 forms D_i = sum_c dO_ic O_ic from
+// the staged rows while it copies dO (fp32, the definition in the backward
+// of spa.h), writes D to the workspace for the dK/dV pass and hands it to
+// warpgroup 0 through shared memory; otherwise D is read from the workspace.
+// Epilogue: scale * dQ straight from TMEM to global, warpgroup w writing head
+// dims [D/2 w, D/2 (w+1)).
 // ---------------------------------------------------------------------------
 template <int D>
 struct DqCfg {
@@ -568,9 +573,11 @@ struct DqCfg {
   static constexpr uint32_t KT_BYTES = BK * D * 2;
   static constexpr uint32_t OFF_Q = 0;
   static constexpr uint32_t OFF_DO = OFF_Q + QT_BYTES;
-  static constexpr uint32_t OFF_K = OFF_DO + QT_BYTES;
+  static constexpr uint32_t OFF_O = OFF_DO + QT_BYTES;    // O staging (D formed in this kernel)
+  static constexpr uint32_t OFF_K = OFF_O + QT_BYTES;
   static constexpr uint32_t OFF_V = OFF_K + NS * KT_BYTES;
-  static constexpr uint32_t OFF_BAR = OFF_V + NS * KT_BYTES;
+  static constexpr uint32_t OFF_DVEC = OFF_V + NS * KT_BYTES;  // D of the unit's 128 rows
+  static constexpr uint32_t OFF_BAR = OFF_DVEC + BQ * 4;
   static constexpr uint32_t SMEM_BYTES =
       (OFF_BAR + 256 + 1024) > 116u * 1024 ? (OFF_BAR + 256 + 1024) : 116u * 1024;
   static constexpr int NTHREADS = 384;
@@ -586,6 +593,7 @@ struct DqBars {
   uint64_t q_full, q_empty;  // staging tiles of Q and dO
   uint64_t k_full[2], v_full[2], kv_empty[2];
   uint64_t qa_full;          // Q and dO of the unit copied into TMEM
+  uint64_t dvec_full;        // D of the unit's rows in shared memory (when formed here)
   uint64_t s_full, s_free, dp_full, ds_full;
   uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
@@ -618,7 +626,7 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
     spa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                      const __grid_constant__ AttnParams p) {
+                      const __grid_constant__ CUtensorMap tm_o, const __grid_constant__ AttnParams p) {
   using C = DqCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -626,9 +634,12 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x / 32, lane = threadIdx.x % 32;
   const int64_t N = p.N;
   const int num_units = p.B * p.units_per_batch;
+  const bool fuse_d = p.o_in != nullptr;  // form D here rather than read it
 
   const uint32_t sQ = ptx::smem_u32(smem + C::OFF_Q);
   const uint32_t sDO = ptx::smem_u32(smem + C::OFF_DO);
+  const uint32_t sO = ptx::smem_u32(smem + C::OFF_O);
+  float* dvec = reinterpret_cast<float*>(smem + C::OFF_DVEC);
   const uint32_t sK = ptx::smem_u32(smem + C::OFF_K);
   const uint32_t sV = ptx::smem_u32(smem + C::OFF_V);
 
@@ -641,6 +652,7 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_init(&bars->kv_empty[s], 1);
     }
     ptx::mbar_init(&bars->qa_full, 256);
+    ptx::mbar_init(&bars->dvec_full, 128);
     ptx::mbar_init(&bars->s_full, 1);
     ptx::mbar_init(&bars->s_free, 256);
     ptx::mbar_init(&bars->dp_full, 1);
@@ -677,10 +689,12 @@ __global__ void __launch_bounds__(384, 1)
         ok = bar_wait(&bars->q_empty, (nq & 1) ^ 1, abort_flag);
         if (!ok) break;
         ++nq;
-        ptx::mbar_arrive_expect_tx(&bars->q_full, 2 * C::QT_BYTES);
+        ptx::mbar_arrive_expect_tx(&bars->q_full, (fuse_d ? 3 : 2) * C::QT_BYTES);
         for (int c = 0; c < C::DB; ++c) {
           ptx::tma_load_3d(smem + C::OFF_Q + c * (C::BQ * 128), &tm_q, &bars->q_full, c * 64, (int)U.i0, U.bh);
           ptx::tma_load_3d(smem + C::OFF_DO + c * (C::BQ * 128), &tm_do, &bars->q_full, c * 64, (int)U.i0, U.bh);
+          if (fuse_d)
+            ptx::tma_load_3d(smem + C::OFF_O + c * (C::BQ * 128), &tm_o, &bars->q_full, c * 64, (int)U.i0, U.bh);
         }
         for (int kt = U.ka; ok && kt <= U.kb; ++kt, ++g) {
           const int s = g % C::NS;
@@ -802,26 +816,8 @@ __global__ void __launch_bounds__(384, 1)
     bool ok = true;
     // Row r of the staged Q (warpgroup 0) or dO (warpgroup 1), 128-byte
     // swizzled, into the warpgroup's TMEM operand as bf16 pairs along d.
-    auto stage_operands = [&]() -> bool {
-      if (!__all_sync(0xffffffffu, bar_wait(&bars->q_full, (cq++) & 1, abort_flag))) return false;
-      const uint32_t src = (w == 0 ? sQ : sDO) + (uint32_t)r * 128;
-      const uint32_t dst = tmem + lane_base + (w == 0 ? C::TM_QA : C::TM_DOA);
-#pragma unroll
-      for (int c = 0; c < C::DB; ++c) {
-        uint32_t v[32];
-#pragma unroll
-        for (int k = 0; k < 8; ++k)
-          ptx::ld_shared_v4(src + c * (C::BQ * 128) + ((k ^ (r & 7)) << 4), v[4 * k], v[4 * k + 1],
-                            v[4 * k + 2], v[4 * k + 3]);
-        ptx::tmem_st32(dst + 32 * c, v);
-      }
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->q_empty);
-      ptx::mbar_arrive(&bars->qa_full);
-      return true;
-    };
-    // The unit and the raw lse, D of row r; the loads land while other work runs.
+    // The unit and the raw lse, D of row r; the loads land while other work
+    // runs (D only when it is not formed here).
     DqUnit U{};
     float lraw = 0.f, draw = 0.f;
     auto fetch_unit = [&](int uu) {
@@ -831,13 +827,63 @@ __global__ void __launch_bounds__(384, 1)
       draw = 0.f;
       if (i < N) {
         lraw = p.lse[(int64_t)U.bh * N + i];
-        draw = p.delta[(int64_t)U.bh * N + i];
+        if (!fuse_d) draw = p.delta[(int64_t)U.bh * N + i];
       }
+    };
+    // Row r of the staged Q (warpgroup 0) or dO (warpgroup 1), 128-byte
+    // swizzled, into the warpgroup's TMEM operand as bf16 pairs along d;
+    // the staging tiles are then free.  With fuse_d, warpgroup 1 also forms
+    // D_r from the staged dO and O rows of unit U (decoded just before).
+    auto stage_operands = [&]() -> bool {
+      if (!__all_sync(0xffffffffu, bar_wait(&bars->q_full, (cq++) & 1, abort_flag))) return false;
+      const uint32_t src = (w == 0 ? sQ : sDO) + (uint32_t)r * 128;
+      const uint32_t dst = tmem + lane_base + (w == 0 ? C::TM_QA : C::TM_DOA);
+      const bool form_d = fuse_d && w == 1;
+      float2 acc = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int c = 0; c < C::DB; ++c) {
+        uint32_t v[32];
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          ptx::ld_shared_v4(src + c * (C::BQ * 128) + ((k ^ (r & 7)) << 4), v[4 * k], v[4 * k + 1],
+                            v[4 * k + 2], v[4 * k + 3]);
+        ptx::tmem_st32(dst + 32 * c, v);
+        if (form_d) {
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            uint32_t o4[4];
+            ptx::ld_shared_v4(sO + (uint32_t)r * 128 + c * (C::BQ * 128) + ((k ^ (r & 7)) << 4), o4[0], o4[1],
+                              o4[2], o4[3]);
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              acc = __ffma2_rn(ptx::bf16x2_to_float2(v[4 * k + e]), ptx::bf16x2_to_float2(o4[e]), acc);
+          }
+        }
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&bars->q_empty);
+      ptx::mbar_arrive(&bars->qa_full);
+      if (fuse_d) {
+        if (w == 1) {
+          draw = acc.x + acc.y;
+          dvec[r] = draw;
+          ptx::mbar_arrive(&bars->dvec_full);
+          const int64_t i = U.i0 + r;
+          if (i < N) p.delta[(int64_t)U.bh * N + i] = draw;
+        } else {
+          // this unit's D from warpgroup 1 (it rewrites the array only after
+          // every step of the unit, each of which waits for both warpgroups)
+          if (!__all_sync(0xffffffffu, bar_wait(&bars->dvec_full, (cq - 1) & 1, abort_flag))) return false;
+          draw = dvec[r];
+        }
+      }
+      return true;
     };
     int u = blockIdx.x;
     if (u < num_units) {
-      ok = stage_operands();
       fetch_unit(u);
+      ok = stage_operands();
     }
     for (; ok && u < num_units; u += gridDim.x) {
       const int64_t i = U.i0 + r;
@@ -931,9 +977,9 @@ __global__ void __launch_bounds__(384, 1)
       // the next unit's Q and dO go into TMEM while the last dQ products run
       // (S and dP of this unit, their last readers, have completed)
       if (u + (int)gridDim.x < num_units) {
+        fetch_unit(u + gridDim.x);
         ok = stage_operands();
         if (!ok) break;
-        fetch_unit(u + gridDim.x);
       }
       // ---------------------------------------------------------- epilogue
       ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));

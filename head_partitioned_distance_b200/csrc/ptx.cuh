@@ -305,6 +305,12 @@ __device__ __forceinline__ void store_row32_bf16(uint16_t* dst, const uint32_t (
   st_global_v8(dst + 16, pk + 8);
 }
 
+// Two bf16 values packed in a 32-bit word (the lower address in the low
+// half) as floats: a bf16 is the upper half of the fp32 with the same value.
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
+  return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,
                                              uint32_t& d) {
   asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"

@@ -44,6 +44,11 @@ EncodeTiledFn encode_fn() {
 int make_map(CUtensorMap* m, const void* ptr, int64_t N, int64_t BH, int d, int box_rows) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return SPA_ERR_CUDA;
+  // The encoder is a driver call and needs a current context; a thread that
+  // has made no runtime call yet (an autograd worker, say) has none.
+  // cudaSetDevice makes the device's primary context current for the thread.
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return SPA_ERR_CUDA;
   cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)N, (cuuint64_t)BH};
   cuuint64_t strides[2] = {(cuuint64_t)d * 2, (cuuint64_t)N * (cuuint64_t)d * 2};
   cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
@@ -178,7 +183,10 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, A
   return launch_status();
 }
 
-enum BwdStep { kStepDelta = 1, kStepDkDv = 2, kStepDq = 4, kStepAll = 7 };
+// Backward steps.  The full backward runs the dQ pass first, forming D there
+// (kStepDqDelta), then the dK/dV pass reading it; the separate D kernel
+// serves the three-step entry points.
+enum BwdStep { kStepDelta = 1, kStepDkDv = 2, kStepDq = 4, kStepDqDelta = 8, kStepAll = kStepDqDelta | kStepDkDv };
 
 template <int D>
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -203,6 +211,33 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
         static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), delta, rows);
     if ((st = launch_status())) return st;
   }
+  if (steps & (kStepDq | kStepDqDelta)) {
+    // persistent grid over query tiles of 128 with a row inside its band; the
+    // whole tiles before the band only get zero rows.  With kStepDqDelta the
+    // kernel also forms D (from o and dout) and writes it to the workspace.
+    const bool fuse_d = (steps & kStepDqDelta) != 0;
+    CUtensorMap qq, qk, qv, qdo, qo;
+    if ((st = make_map(&qq, q, p.N, BH, D, QC::BQ)) || (st = make_map(&qk, k, p.N, BH, D, QC::BK)) ||
+        (st = make_map(&qv, v, p.N, BH, D, QC::BK)) || (st = make_map(&qdo, dout, p.N, BH, D, QC::BQ)) ||
+        (st = make_map(&qo, fuse_d ? o : dout, p.N, BH, D, QC::BQ)))
+      return st;
+    p.o_in = fuse_d ? o : nullptr;
+    if ((st = prepare_kernel(spa::spa_bwd_dq_kernel<D>, QC::SMEM_BYTES, prepared_q))) return st;
+    static std::atomic<int> regs_q{0};
+    if ((st = check_regs(spa::spa_bwd_dq_kernel<D>, (int)QC::LAUNCH_REGS, regs_q))) return st;
+    const int64_t nqt = (p.N + 127) / 128;
+    if ((int64_t)p.B * p.H * nqt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+    if ((st = set_work_lists(
+             p, [&](int h) { return nqt - p.lo[h] / 128; }, [&](int h) { return (int64_t)(p.lo[h] / 128); })))
+      return st;
+    const int64_t upb = p.units_per_batch;
+    int sms = 0;
+    if ((st = sm_count(&sms))) return st;
+    const int64_t units = (int64_t)p.B * upb;
+    const unsigned grid = (unsigned)(units < sms ? units : sms);
+    spa::spa_bwd_dq_kernel<D><<<grid, QC::NTHREADS, QC::SMEM_BYTES, stream>>>(qq, qk, qv, qdo, qo, p);
+    if ((st = launch_status())) return st;
+  }
   if (steps & kStepDkDv) {
     // persistent grid over key tiles of 128 that some query reaches; the
     // other key tiles only get zero rows
@@ -225,29 +260,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     const int64_t units = (int64_t)p.B * upb;
     const unsigned grid = (unsigned)(units < sms ? units : sms);
     spa::spa_bwd_dkdv_kernel<D><<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, p);
-    if ((st = launch_status())) return st;
-  }
-  if (steps & kStepDq) {
-    // persistent grid over query tiles of 128 with a row inside its band; the
-    // whole tiles before the band only get zero rows
-    CUtensorMap qq, qk, qv, qdo;
-    if ((st = make_map(&qq, q, p.N, BH, D, QC::BQ)) || (st = make_map(&qk, k, p.N, BH, D, QC::BK)) ||
-        (st = make_map(&qv, v, p.N, BH, D, QC::BK)) || (st = make_map(&qdo, dout, p.N, BH, D, QC::BQ)))
-      return st;
-    if ((st = prepare_kernel(spa::spa_bwd_dq_kernel<D>, QC::SMEM_BYTES, prepared_q))) return st;
-    static std::atomic<int> regs_q{0};
-    if ((st = check_regs(spa::spa_bwd_dq_kernel<D>, (int)QC::LAUNCH_REGS, regs_q))) return st;
-    const int64_t nqt = (p.N + 127) / 128;
-    if ((int64_t)p.B * p.H * nqt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
-    if ((st = set_work_lists(
-             p, [&](int h) { return nqt - p.lo[h] / 128; }, [&](int h) { return (int64_t)(p.lo[h] / 128); })))
-      return st;
-    const int64_t upb = p.units_per_batch;
-    int sms = 0;
-    if ((st = sm_count(&sms))) return st;
-    const int64_t units = (int64_t)p.B * upb;
-    const unsigned grid = (unsigned)(units < sms ? units : sms);
-    spa::spa_bwd_dq_kernel<D><<<grid, QC::NTHREADS, QC::SMEM_BYTES, stream>>>(qq, qk, qv, qdo, p);
     if ((st = launch_status())) return st;
   }
   return SPA_OK;
@@ -280,10 +292,10 @@ int bwd_entry(const void* q, const void* k, const void* v, const void* o, const 
   if (st) return st;
   // every step reads the workspace (D); each checks the tensors it touches
   if (!workspace) return SPA_ERR_INVAL;
-  if ((steps & kStepDelta) && (!o || !dout)) return SPA_ERR_INVAL;
-  if ((steps & (kStepDkDv | kStepDq)) && (!q || !k || !v || !dout || !lse)) return SPA_ERR_INVAL;
+  if ((steps & (kStepDelta | kStepDqDelta)) && (!o || !dout)) return SPA_ERR_INVAL;
+  if ((steps & (kStepDkDv | kStepDq | kStepDqDelta)) && (!q || !k || !v || !dout || !lse)) return SPA_ERR_INVAL;
   if ((steps & kStepDkDv) && (!dk || !dv)) return SPA_ERR_INVAL;
-  if ((steps & kStepDq) && !dq) return SPA_ERR_INVAL;
+  if ((steps & (kStepDq | kStepDqDelta)) && !dq) return SPA_ERR_INVAL;
   if (!std::isfinite(scale) || !(scale > 0.f)) return SPA_ERR_INVAL;
   for (const void* t : {q, k, v, o, dout, (const void*)dq, (const void*)dk, (const void*)dv})
     if (t && !aligned(t, 16)) return SPA_ERR_UNSUPPORTED;
@@ -443,6 +455,13 @@ int spa_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dou
                     const int32_t* lo, const int32_t* hi, void* stream) {
   return bwd_entry(q, k, v, nullptr, dout, lse, dq, nullptr, nullptr, const_cast<void*>(workspace), B, H,
                    N, d, scale, lo, hi, stream, kStepDq);
+}
+
+int spa_attn_bwd_dq_delta(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                          const float* lse, void* workspace, void* dq, int B, int H, int64_t N, int d,
+                          float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+  return bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, workspace, B, H, N, d, scale, lo, hi, stream,
+                   kStepDqDelta);
 }
 
 int spa_tile_schedule(int64_t N, int H, const int32_t* lo, const int32_t* hi, int Bq, int Bk,

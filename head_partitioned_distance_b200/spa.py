@@ -44,6 +44,7 @@ EXPORTS = {
     "spa_attn_bwd_preprocess": ([_vp, _vp, _vp, _int, _int, _i64, _int, _vp], _int),
     "spa_attn_bwd_dkdv": ([_vp] * 8 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_dq": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
+    "spa_attn_bwd_dq_delta": ([_vp] * 8 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_noalloc": ([_vp] * 9 + [_int, _int, _i64, _int, _f32, _vp], _int),
     "spa_tile_schedule": ([_i64, _int, _i32p, _i32p, _int, _int, _i32p, _i32p, _u8p, _i32p, _i32p],
                           _int),
@@ -199,6 +200,17 @@ def spa_attn_bwd_dq(q, k, v, dout, lse, workspace, dq, scale: float, lo=None, hi
     _check(_lib.spa_attn_bwd_dq(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
                                 lse.data_ptr(), workspace.data_ptr(), dq.data_ptr(), B, H, N, d, scale,
                                 lo_a, hi_a, _stream_ptr(stream)), "spa_attn_bwd_dq")
+
+
+def spa_attn_bwd_dq_delta(q, k, v, o, dout, lse, workspace, dq, scale: float, lo=None, hi=None,
+                          stream=None):
+    B, H, N, d = _dims(q)
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    _check(_lib.spa_attn_bwd_dq_delta(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
+                                      dout.data_ptr(), lse.data_ptr(), workspace.data_ptr(), dq.data_ptr(),
+                                      B, H, N, d, scale, lo_a, hi_a, _stream_ptr(stream)),
+           "spa_attn_bwd_dq_delta")
 
 
 def spa_tile_schedule(N: int, H: int, Bq: int, Bk: int, lo=None, hi=None):

@@ -132,6 +132,13 @@ SPA_API int spa_attn_bwd_ex(const void* q, const void* k, const void* v, const v
  *  3. spa_attn_bwd_dq:   dq from q, k, v, dout, lse and D (one CTA per query
  *     tile, walking the same key strip as the forward).
  * Steps 2 and 3 only read the workspace and may run concurrently.
+ *
+ * spa_attn_bwd_dq_delta is steps 1 and 3 in one pass, the way spa_attn_bwd
+ * runs them: the dq pass stages each 128-row block of o next to dout and
+ * forms D there (fp32 sums of bf16 products, the same definition as step 1),
+ * writes it to the workspace for every row of the query blocks the band
+ * reaches, and computes dq.  spa_attn_bwd_dkdv run after it on the same
+ * workspace completes the backward.
  */
 SPA_API int spa_attn_bwd_preprocess(const void* o, const void* dout, void* workspace, int B, int H,
                                     int64_t N, int d, void* stream);
@@ -143,6 +150,10 @@ SPA_API int spa_attn_bwd_dq(const void* q, const void* k, const void* v, const v
                             const float* lse, const void* workspace, void* dq, int B, int H,
                             int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi,
                             void* stream);
+SPA_API int spa_attn_bwd_dq_delta(const void* q, const void* k, const void* v, const void* o,
+                                  const void* dout, const float* lse, void* workspace, void* dq,
+                                  int B, int H, int64_t N, int d, float scale, const int32_t* lo,
+                                  const int32_t* hi, void* stream);
 
 /*
  * Backward pass that allocates nothing and takes no workspace argument.

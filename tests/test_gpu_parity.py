@@ -132,6 +132,51 @@ def test_explicit_bands(spa, kind):
     _full_check(spa, q, k, v, do, 0.125, [int(x) for x in lo], [int(x) for x in hi])
 
 
+@pytest.mark.parametrize("B,H,N,d", [(1, 8, 1001, 64), (2, 5, 777, 128), (1, 3, 129, 128), (1, 4, 300, 128)])
+def test_backward_step_entry_points(spa, B, H, N, d):
+    # The three-step entry points (D kernel, dk/dv pass, dq pass) and the
+    # fused dq pass that forms D itself, followed by the dk/dv pass, both give
+    # the oracle's gradients; the D each leaves in the workspace matches its
+    # definition evaluated in fp64 on the same bf16 o and dout.
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=31 + N + d)
+    scale = 1 / math.sqrt(d)
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = spa.attention_forward(qd, kd, vd, scale)
+    rows = B * H * N
+    ws3 = torch.full((spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4,), float("nan"), device=dev)
+    wsf = torch.full_like(ws3, float("nan"))
+    g3 = [torch.empty_like(qd) for _ in range(3)]  # dq, dk, dv
+    gf = [torch.empty_like(qd) for _ in range(3)]
+    spa.spa_attn_bwd_preprocess(o, dod, ws3)
+    spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, ws3, g3[1], g3[2], scale)
+    spa.spa_attn_bwd_dq(qd, kd, vd, dod, lse, ws3, g3[0], scale)
+    spa.spa_attn_bwd_dq_delta(qd, kd, vd, o, dod, lse, wsf, gf[0], scale)
+    spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, wsf, gf[1], gf[2], scale)
+    torch.cuda.synchronize()
+    assert spa.spa_device_status() == spa.SPA_OK
+
+    d_ref = (o.double() * dod.double()).sum(-1).reshape(-1).cpu().numpy()
+    d3 = ws3[:rows].double().cpu().numpy()
+    df = wsf[:rows].double().cpu().numpy()
+    tol = 1e-5 + 1e-5 * np.abs(d_ref)
+    assert (np.abs(d3 - d_ref) <= tol).all()
+    # the fused pass writes D for every row of the 128-row query blocks some
+    # band reaches: rows from 128 * floor(lo_h / 128) on
+    lo, _ = oracle.bands(N, H)
+    written = np.zeros((B, H, N), dtype=bool)
+    for h in range(H):
+        written[:, h, (int(lo[h]) // 128) * 128:] = True
+    written = written.reshape(-1)
+    assert (np.abs(df[written] - d_ref[written]) <= tol[written]).all()
+
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    refs = oracle.spa_bwd(qf, kf, vf, dof, scale)
+    for got in (g3, gf):
+        for g, ref, name in zip(got, refs, ("dq", "dk", "dv")):
+            _check_grad(_f64(g), ref, name)
+
+
 def test_dense_causal_equals_torch_sdpa_in_fp32(spa):
     # an independent library path: full bands on every head is causal attention
     B, H, N, d = 2, 4, 512, 128
@@ -164,6 +209,29 @@ def test_autograd_function(spa):
     for g, ref, n in zip((qd.grad, kd.grad, vd.grad), oracle.spa_bwd(qf, kf, vf, dof, d ** -0.5),
                          "qkv"):
         _check_grad(_f64(g), ref, n)
+
+
+def test_calls_from_a_fresh_thread(spa):
+    # a host thread that has made no CUDA call yet (as autograd's worker
+    # thread may be) gets the same results as the main thread
+    import threading
+    B, H, N, d = 1, 4, 300, 64
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=5)
+    want = _gpu_run(spa, q, k, v, do, 0.125)
+    got, errors = {}, []
+
+    def run():
+        try:
+            got.update(_gpu_run(spa, q, k, v, do, 0.125))
+        except Exception as e:  # reported below, in the test's own thread
+            errors.append(e)
+
+    t = threading.Thread(target=run)
+    t.start()
+    t.join()
+    assert not errors, errors
+    for name in ("o", "lse", "dq", "dk", "dv"):
+        assert np.array_equal(got[name], want[name]), name
 
 
 @pytest.mark.parametrize("N,H,Bq,Bk", [(1024, 8, 128, 128), (1001, 8, 64, 128), (1001, 8, 128, 64),
