@@ -37,6 +37,7 @@ ROOT = os.path.dirname(os.path.abspath(__file__))
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 
+import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
 from head_partitioned_distance_b200 import synth  # noqa: E402
@@ -273,6 +274,147 @@ def run_reference(args):
     return 0
 
 
+# --------------------------------------------------------------------- decode step
+DECODE_METRIC = "band-sparse decode step (one new token per sequence): GB/s of band K/V read"
+DECODE_CONFIG = {"workload": "decode_b16_h32_n32768_d128", "B": 16, "H": 32, "N": 32768, "d": 128}
+
+
+def decode_bytes(d, bands, positions):
+    """Algorithmic bytes of one decode call: the band's keys and values read
+    once per (b, h), q read, o and lse written."""
+    total = 0
+    for t in positions:
+        for lo, hi in zip(*bands):
+            jlo, jhi = max(0, t - hi + 1), t - lo
+            total += 2 * max(0, jhi - jlo + 1) * d * 2 + d * 2 + d * 2 + 4
+    return total
+
+
+def run_decode(args):
+    """One decode call per step on the B16 H32 N32768 d128 cache, every
+    sequence at its last position (each head reads its full band)."""
+    from head_partitioned_distance_b200 import spa
+
+    rank, local, world = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200); there is no CPU path")
+    dist = dist_init("nccl", local) if world > 1 else None
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    B, H, N, d = (DECODE_CONFIG[x] for x in ("B", "H", "N", "d"))
+    scale = d ** -0.5
+    bands = spa.spa_band_bounds(N, H)
+    # seeded synthetic inputs, generated on the device (the cache is 8.6 GB)
+    gen = torch.Generator(device=device).manual_seed(5000 + 7919 * rank)
+    kc = torch.randn((B, H, N, d), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+    vc = torch.randn((B, H, N, d), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+    q = torch.randn((B, H, d), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+    positions = [N - 1] * B
+    pos = torch.tensor(positions, dtype=torch.int32, device=device)
+    o = torch.empty((B, H, d), dtype=torch.bfloat16, device=device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=device)
+    ws = torch.empty(spa.spa_attn_decode_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    step = lambda: spa.spa_attn_decode(q, kc, vc, pos, o, lse, ws, scale, stream=stream)
+    nbytes = decode_bytes(d, bands, positions)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(device)
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after warm-up")
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(visible.split(",")[local] if visible else local)
+    sampler.start()
+    K = args.steps
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    sampler.mark_start()
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    sampler.mark_end()
+    clocks = sampler.stop()
+    max_ms = reduce_max(e0.elapsed_time(e1), device)
+    value = world * nbytes * K / (max_ms * 1e-3) / 1e9
+    # end to end: the new tokens' queries and positions from pinned host
+    # memory, o and lse back, inside the timed region
+    q_h, pos_h = q.cpu().pin_memory(), pos.cpu().pin_memory()
+    o_h, lse_h = torch.empty(o.shape, dtype=o.dtype).pin_memory(), torch.empty(lse.shape).pin_memory()
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        pos.copy_(pos_h, non_blocking=True)
+        step()
+        o_h.copy_(o, non_blocking=True)
+        lse_h.copy_(lse, non_blocking=True)
+
+    E = max(3, min(50, K))
+    e2e_step()
+    torch.cuda.synchronize(device)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    f0.record(stream)
+    for _ in range(E):
+        e2e_step()
+    f1.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = reduce_max(f0.elapsed_time(f1), device)
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after the timed region")
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        per_gpu = value / world
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            import oracle
+            # the oracle's forward rows on head 0's slice of the first
+            # sequence: the decode of that (b, h) at several positions
+            kf = kc[0, :1].unsqueeze(0).double().cpu().numpy()
+            vf = vc[0, :1].unsqueeze(0).double().cpu().numpy()
+            qf = np.zeros_like(kf)
+            rows = list(range(N - 1, -1, -1))
+            qf[0, 0, rows, :] = q[0, 0].double().cpu().numpy()
+            lo0, hi0 = [bands[0][0]], [bands[1][0]]
+            # repeat the N positions until about half the target CPU time
+            reps, secs = 0, 0.0
+            while secs < args.cpu_seconds / 2:
+                t0 = time.perf_counter()
+                oracle.spa_fwd_rows(qf, kf, vf, scale, rows, lo0, hi0)
+                secs += time.perf_counter() - t0
+                reps += 1
+            cb = reps * decode_bytes(d, (lo0, hi0), rows)
+            cpu = {"value": cb / secs / 1e9, "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                   "sample": f"oracle spa_fwd_rows (fp64) for all {N} decode positions of head 0 "
+                             f"(band [{lo0[0]}, {hi0[0]})) of sequence 0, {reps} times", "seconds": secs}
+        line = {
+            "metric": DECODE_METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": max_ms / K, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {**DECODE_CONFIG, "positions": "N - 1 for every sequence",
+                       "bands": "balanced distance partitioning", "bytes_per_call": nbytes,
+                       "l2": f"no flush: the bands' K/V ({nbytes / 2**20:.0f} MiB) exceed L2",
+                       "parallelism": f"{world} independent replicas"},
+            "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": per_gpu / peaks["hbm_gbs"], "traffic": None,
+                         "kernel": "spa_decode_chunk_kernel + spa_decode_merge_kernel",
+                         "peak_source": f"{peak_src} (hbm_gbs)"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": world * nbytes * E / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": q.numel() * 2 + B * 4, "d2h_bytes_per_step": o.numel() * 2 + lse.numel() * 4,
+                    "steps": E, "ms_per_step": e2e_ms / E},
+            "gpu_launches": 2 * K,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 # --------------------------------------------------------------------- GPU arm
 def run_spa(args):
     from head_partitioned_distance_b200 import spa
@@ -453,11 +595,15 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--decode", action="store_true",
+                    help="time the decode step (one new token per sequence) instead of fwd+bwd")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.impl == "reference":
         return run_reference(args)
+    if args.decode:
+        return run_decode(args)
     return run_spa(args)
 
 

@@ -4,6 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <cmath>
 #include <cstring>
@@ -13,6 +14,7 @@
 
 #include "bwd.cuh"
 #include "common.cuh"
+#include "decode.cuh"
 #include "fwd.cuh"
 #include "sched.cuh"
 
@@ -526,6 +528,67 @@ int spa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
 int spa_debug_wait_timeout(int64_t limit_ns, void* stream) {
   if (limit_ns < 1 || limit_ns > 1000000000LL) return SPA_ERR_INVAL;
   wait_timeout_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>((uint64_t)limit_ns);
+  return launch_status();
+}
+
+// Chunks of kDecodeChunk keys that the widest band needs.
+int64_t decode_chunks(const AttnParams& p, int H) {
+  int64_t w = 1;
+  for (int h = 0; h < H; ++h) w = std::max<int64_t>(w, (int64_t)p.hi[h] - p.lo[h]);
+  return (w + spa::kDecodeChunk - 1) / spa::kDecodeChunk;
+}
+
+size_t spa_attn_decode_workspace_bytes(int B, int H, int64_t N, int d, const int32_t* lo, const int32_t* hi) {
+  if (check_shape(B, H, N, d)) return 0;
+  static AttnParams zero{};
+  AttnParams p = zero;
+  if (fill_bands(p, H, N, lo, hi)) return 0;
+  return (size_t)B * H * decode_chunks(p, H) * (d + 2) * sizeof(float);
+}
+
+int spa_attn_decode(const void* q, const void* k, const void* v, const int32_t* pos, void* o, float* lse,
+                    void* workspace, int B, int H, int64_t N, int d, float scale, const int32_t* lo,
+                    const int32_t* hi, void* stream) {
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  if (!q || !k || !v || !pos || !o || !lse || !workspace) return SPA_ERR_INVAL;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return SPA_ERR_INVAL;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4) ||
+      !aligned(pos, 4) || !aligned(workspace, 4))
+    return SPA_ERR_UNSUPPORTED;
+  static AttnParams zero{};
+  AttnParams bands = zero;
+  if ((st = fill_bands(bands, H, N, lo, hi))) return st;
+  static spa::DecodeParams dzero{};
+  spa::DecodeParams p = dzero;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.d = d;
+  p.scale_log2 = scale * spa::kLog2e;
+  const int64_t nchunk = decode_chunks(bands, H);
+  if (nchunk > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+  p.nchunk = (int)nchunk;
+  p.q = static_cast<const uint16_t*>(q);
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.pos = pos;
+  p.o = static_cast<uint16_t*>(o);
+  p.lse = lse;
+  p.part = static_cast<float*>(workspace);
+  std::memcpy(p.lo, bands.lo, sizeof(p.lo));
+  std::memcpy(p.hi, bands.hi, sizeof(p.hi));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const dim3 grid_c((unsigned)nchunk, (unsigned)H, (unsigned)B), grid_m((unsigned)H, (unsigned)B);
+  if (d == 64) {
+    spa::spa_decode_chunk_kernel<64><<<grid_c, 128, 0, s>>>(p);
+    if ((st = launch_status())) return st;
+    spa::spa_decode_merge_kernel<64><<<grid_m, 128, 0, s>>>(p);
+  } else {
+    spa::spa_decode_chunk_kernel<128><<<grid_c, 128, 0, s>>>(p);
+    if ((st = launch_status())) return st;
+    spa::spa_decode_merge_kernel<128><<<grid_m, 128, 0, s>>>(p);
+  }
   return launch_status();
 }
 

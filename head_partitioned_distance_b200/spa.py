@@ -45,6 +45,8 @@ EXPORTS = {
     "spa_attn_bwd_dkdv": ([_vp] * 8 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_dq": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_dq_delta": ([_vp] * 8 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
+    "spa_attn_decode_workspace_bytes": ([_int, _int, _i64, _int, _i32p, _i32p], ctypes.c_size_t),
+    "spa_attn_decode": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_noalloc": ([_vp] * 9 + [_int, _int, _i64, _int, _f32, _vp], _int),
     "spa_tile_schedule": ([_i64, _int, _i32p, _i32p, _int, _int, _i32p, _i32p, _u8p, _i32p, _i32p],
                           _int),
@@ -262,6 +264,37 @@ def attention_forward(q, k, v, scale=None, lo=None, hi=None):
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
     return spa_attn_fwd(q, k, v, o, lse, scale, lo, hi)
+
+
+def spa_attn_decode_workspace_bytes(B: int, H: int, N: int, d: int, lo=None, hi=None) -> int:
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    return int(_lib.spa_attn_decode_workspace_bytes(B, H, N, d, lo_a, hi_a))
+
+
+def spa_attn_decode(q, k, v, pos, o, lse, workspace, scale: float, lo=None, hi=None, stream=None):
+    """One new token per sequence: q [B, H, d] at positions pos (int32 [B]) of
+    the caches k, v [B, H, N, d]; writes o [B, H, d] and lse [B, H]."""
+    B, H, N, d = _dims(k)
+    if q.shape != (B, H, d) or pos.dtype != torch.int32 or pos.numel() != B:
+        raise ValueError("q is [B, H, d] and pos int32 [B] for caches [B, H, N, d]")
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    _check(_lib.spa_attn_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), pos.data_ptr(), o.data_ptr(),
+                                lse.data_ptr(), workspace.data_ptr(), B, H, N, d, scale, lo_a, hi_a,
+                                _stream_ptr(stream)), "spa_attn_decode")
+    return o, lse
+
+
+def attention_decode(q, k_cache, v_cache, pos, scale=None, lo=None, hi=None):
+    """Allocate o / lse / workspace and run spa_attn_decode."""
+    B, H, N, d = _dims(k_cache)
+    scale = d ** -0.5 if scale is None else scale
+    o = torch.empty((B, H, d), dtype=q.dtype, device=q.device)
+    lse = torch.empty((B, H), dtype=torch.float32, device=q.device)
+    nbytes = spa_attn_decode_workspace_bytes(B, H, N, d, lo, hi)
+    ws = torch.empty(max(nbytes // 4, 1), dtype=torch.float32, device=q.device)
+    return spa_attn_decode(q, k_cache, v_cache, pos, o, lse, ws, scale, lo, hi)
 
 
 def attention_backward(q, k, v, o, dout, lse, scale=None, lo=None, hi=None):

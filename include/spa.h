@@ -182,6 +182,39 @@ SPA_API int spa_attn_bwd_noalloc(const void* q, const void* k, const void* v, co
                                  int B, int H, int64_t N, int d, float scale, void* stream);
 
 /*
+ * Decode step: one new token per sequence.  Each head attends only to its
+ * own band of causal distances ("Making Every Head Count", abstract and
+ * Figure 1 caption), so the query at position t of head h reads just the
+ * cached keys j with lo_h <= t - j < hi_h -- at most the band's width,
+ * whatever t is -- with the softmax over that set ("Story of Attention --
+ * Part 4", section 1, the Sparse-Attention equation).
+ *   q:         DEVICE bf16 [B][H][d], the new tokens' queries
+ *   k, v:      DEVICE bf16 [B][H][N][d], the key/value cache (row j holds
+ *              position j; only the band's rows are read)
+ *   pos:       DEVICE int32 [B], the position of each sequence's new token;
+ *              a position outside [0, N) gives that sequence o = 0, lse = -inf
+ *   o:         DEVICE bf16 [B][H][d]
+ *   lse:       DEVICE fp32 [B][H], natural log; -inf when the band holds no
+ *              key yet (pos < lo_h), with o = 0
+ *   workspace: DEVICE buffer of spa_attn_decode_workspace_bytes(B, H, N, d,
+ *              lo, hi) bytes, caller-owned, overwritten
+ *   lo, hi:    HOST band arrays (rules of spa_attn_fwd_ex) or both NULL for
+ *              the Balanced Distance Partitioning bands of length N
+ * Equals row pos[b] of spa_attn_fwd on the sequence whose row pos[b] holds q.
+ * Two launches (a split over 256-key chunks, then their merge), asynchronous
+ * on `stream`; nothing is allocated.  SPA_ERR_INVAL for null pointers, bad
+ * bands or a scale that is not finite and > 0; SPA_ERR_UNSUPPORTED for
+ * d not in {64, 128}, H > 256, B > 65535 or misaligned buffers (16 bytes for
+ * q, k, v, o; 4 for pos, lse, workspace).  The workspace size is 0 for
+ * arguments the call would reject.
+ */
+SPA_API size_t spa_attn_decode_workspace_bytes(int B, int H, int64_t N, int d, const int32_t* lo,
+                                               const int32_t* hi);
+SPA_API int spa_attn_decode(const void* q, const void* k, const void* v, const int32_t* pos, void* o,
+                            float* lse, void* workspace, int B, int H, int64_t N, int d, float scale,
+                            const int32_t* lo, const int32_t* hi, void* stream);
+
+/*
  * Band tile schedule, as the kernels walk it (host evaluation of the same
  * code the device runs).  Query tile t covers rows [t*Bq, t*Bq + Bq), key
  * tile u keys [u*Bk, u*Bk + Bk); positions >= N are not permitted.

@@ -153,6 +153,29 @@ def test_workspace_size():
     assert spa.spa_attn_bwd_workspace_bytes(0, 1, 1) == 0
 
 
+def test_decode_rejects_bad_arguments_and_sizes_its_workspace():
+    L = spa._lib
+    p = _fake(1 << 20)  # never dereferenced: every call below fails its checks first
+    f = lambda *a: L.spa_attn_decode(p, p, p, p, p, p, p, *a, None, None, None)
+    assert f(1, 4, 256, 96, 0.1) == spa.SPA_ERR_UNSUPPORTED      # d
+    assert f(1, 300, 400, 64, 0.1) == spa.SPA_ERR_UNSUPPORTED    # H > 256
+    assert f(1, 8, 4, 64, 0.1) == spa.SPA_ERR_INVAL              # H > N
+    assert f(1, 4, 256, 64, float("inf")) == spa.SPA_ERR_INVAL   # scale
+    assert f(1, 4, 256, 64, 0.0) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_decode(p, p, p, None, p, p, p, 1, 4, 256, 64, 0.1, None, None, None) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_decode(p, p, p, p, p, p, None, 1, 4, 256, 64, 0.1, None, None, None) == spa.SPA_ERR_INVAL
+    odd = _fake((1 << 20) + 2)
+    assert L.spa_attn_decode(p, p, p, odd, p, p, p, 1, 4, 256, 64, 0.1, None, None, None) == spa.SPA_ERR_UNSUPPORTED
+    a, b = (ctypes.c_int32 * 2)(3, 1), (ctypes.c_int32 * 2)(2, 9)     # reversed band
+    assert L.spa_attn_decode(p, p, p, p, p, p, p, 1, 2, 256, 64, 0.1, a, b, None) == spa.SPA_ERR_INVAL
+    # workspace: one (o[d], m, l) partial per 256-key chunk of the widest band
+    assert spa.spa_attn_decode_workspace_bytes(2, 4, 4096, 128) == 2 * 4 * 4 * 130 * 4
+    assert spa.spa_attn_decode_workspace_bytes(1, 8, 1001, 64) == 8 * 1 * 66 * 4
+    assert spa.spa_attn_decode_workspace_bytes(1, 2, 700, 128, [0, 5], [600, 6]) == 2 * 3 * 130 * 4
+    assert spa.spa_attn_decode_workspace_bytes(1, 4, 256, 96) == 0
+    assert spa.spa_attn_decode_workspace_bytes(1, 2, 700, 128, [3, 1], [2, 9]) == 0
+
+
 def test_timeout_hook_rejects_bad_limits():
     L = spa._lib
     assert L.spa_debug_wait_timeout(0, None) == spa.SPA_ERR_INVAL

@@ -211,6 +211,49 @@ def test_autograd_function(spa):
         _check_grad(_f64(g), ref, n)
 
 
+@pytest.mark.parametrize("B,H,N,d,explicit", [(3, 4, 1000, 64, False), (2, 8, 4096, 128, False),
+                                             (2, 3, 700, 128, True), (1, 32, 2048, 128, False)])
+def test_decode_matches_the_forward_row(spa, B, H, N, d, explicit):
+    # One new token per sequence: the result equals the oracle's forward row
+    # pos[b] of the sequence whose row pos[b] holds the token's query.
+    q, k, v, _ = synth.make_inputs(B, H, N, d, seed=41 + N + d)
+    tok = synth.make_inputs(B, H, 1, d, seed=43 + N)[0][:, :, 0, :].contiguous()  # [B, H, d]
+    lo, hi = (None, None)
+    if explicit:
+        lo, hi = [0, 5, 300], [700, 6, 457]
+    blo = np.array(oracle.bands(N, H)[0] if lo is None else lo)
+    scale = 1 / math.sqrt(d)
+    dev = torch.device("cuda:0")
+    kd, vd, tokd = k.to(dev), v.to(dev), tok.to(dev)
+    rng = np.random.default_rng(N)
+    # positions: start, the band edges, the end, random ones
+    cands = sorted({0, 1, int(blo.max()) - 1, int(blo.max()), int(blo[1]) if H > 1 else 1, N - 2, N - 1}
+                   | set(int(x) for x in rng.integers(0, N, 6)))
+    cands = [c for c in cands if 0 <= c < N]
+    for start in range(0, len(cands), B):
+        pos = np.array([cands[(start + b) % len(cands)] for b in range(B)], dtype=np.int32)
+        o, lse = spa.attention_decode(tokd, kd, vd, torch.from_numpy(pos).to(dev), scale, lo, hi)
+        torch.cuda.synchronize()
+        assert spa.spa_device_status() == spa.SPA_OK
+        qfull = q.clone()
+        for b in range(B):
+            qfull[b, :, pos[b], :] = tok[b]
+        rows = [(b * H + h) * N + int(pos[b]) for b in range(B) for h in range(H)]
+        o_ref, lse_ref = oracle.spa_fwd_rows(_f64(qfull), _f64(k), _f64(v), scale, rows,
+                                             None if lo is None else np.array(lo),
+                                             None if hi is None else np.array(hi))
+        got_o = _f64(o).reshape(B * H, d)
+        assert not np.isnan(got_o).any()
+        assert np.abs(got_o - o_ref).max() <= O_TOL
+        _check_lse(_f64(lse).reshape(-1), lse_ref)
+    # positions outside [0, N): o = 0, lse = -inf
+    pos = torch.tensor([N, -1][:B] + [0] * max(0, B - 2), dtype=torch.int32, device=dev)
+    o, lse = spa.attention_decode(tokd, kd, vd, pos, scale, lo, hi)
+    torch.cuda.synchronize()
+    for b in range(min(B, 2)):
+        assert torch.all(o[b] == 0) and torch.all(torch.isneginf(lse[b]))
+
+
 def test_calls_from_a_fresh_thread(spa):
     # a host thread that has made no CUDA call yet (as autograd's worker
     # thread may be) gets the same results as the main thread
