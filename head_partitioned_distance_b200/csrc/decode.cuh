@@ -92,16 +92,40 @@ __global__ void __launch_bounds__(128) spa_decode_chunk_kernel(const __grid_cons
   for (int g8 = 0; g8 < kDecodeChunk / kDecodeWarps; g8 += 8) {
     const int64_t kb = w0 + g8;  // keys kb .. kb + 7 of this group
     if (kb > c1) break;
-    // score of key kb + lane / 4 (masked past c1)
-    const int64_t j = kb + lane / 4;
-    float s = -INFINITY;
+    // every load of the group first (keys past c1 read as zero), so one
+    // memory latency covers both the scores and the values
+    const int64_t j = kb + lane / 4;  // this lane's key for the score
+    uint4 kq[QD / 8];
+#pragma unroll
+    for (int x = 0; x < QD / 8; ++x) kq[x] = make_uint4(0u, 0u, 0u, 0u);
     if (j <= c1) {
       const uint4* kp = reinterpret_cast<const uint4*>(kh + j * D + (lane % 4) * QD);
+#pragma unroll
+      for (int x = 0; x < QD / 8; ++x) kq[x] = kp[x];
+    }
+    uint32_t vw[8][OD / 2];  // this lane's OD value columns of the group's 8 keys
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+#pragma unroll
+      for (int e = 0; e < OD / 2; ++e) vw[kk][e] = 0u;
+      if (kb + kk <= c1) {
+        const uint16_t* vr = vh + (kb + kk) * D + OD * lane;
+        if (OD == 4) {
+          const uint2 u = *reinterpret_cast<const uint2*>(vr);
+          vw[kk][0] = u.x;
+          vw[kk][1 % (OD / 2)] = u.y;
+        } else {
+          vw[kk][0] = *reinterpret_cast<const uint32_t*>(vr);
+        }
+      }
+    }
+    // score of key j (masked past c1)
+    float s = -INFINITY;
+    if (j <= c1) {
       float2 a = make_float2(0.f, 0.f);
 #pragma unroll
       for (int x = 0; x < QD / 8; ++x) {
-        const uint4 u = kp[x];
-        const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+        const uint32_t w4[4] = {kq[x].x, kq[x].y, kq[x].z, kq[x].w};
 #pragma unroll
         for (int y = 0; y < 4; ++y)
           a = __ffma2_rn(ptx::bf16x2_to_float2(w4[y]), make_float2(qv[8 * x + 2 * y], qv[8 * x + 2 * y + 1]), a);
@@ -132,22 +156,12 @@ __global__ void __launch_bounds__(128) spa_decode_chunk_kernel(const __grid_cons
     // o += p_j v_j over the group's keys; lane owns dims [OD lane, OD lane + OD)
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-      const float pk = __shfl_sync(0xffffffffu, pj, 4 * kk);
-      if (kb + kk <= c1) {
-        const uint16_t* vr = vh + (kb + kk) * D + OD * lane;
-        if (OD == 4) {
-          const uint2 u = *reinterpret_cast<const uint2*>(vr);
-          const float2 f0 = ptx::bf16x2_to_float2(u.x), f1 = ptx::bf16x2_to_float2(u.y);
-          acc[0] = fmaf(pk, f0.x, acc[0]);
-          acc[1] = fmaf(pk, f0.y, acc[1]);
-          acc[2 % OD] = fmaf(pk, f1.x, acc[2 % OD]);
-          acc[3 % OD] = fmaf(pk, f1.y, acc[3 % OD]);
-        } else {
-          const uint32_t u = *reinterpret_cast<const uint32_t*>(vr);
-          const float2 f0 = ptx::bf16x2_to_float2(u);
-          acc[0] = fmaf(pk, f0.x, acc[0]);
-          acc[1 % OD] = fmaf(pk, f0.y, acc[1 % OD]);
-        }
+      const float pk = __shfl_sync(0xffffffffu, pj, 4 * kk);  // 0 past c1
+#pragma unroll
+      for (int e = 0; e < OD / 2; ++e) {
+        const float2 f = ptx::bf16x2_to_float2(vw[kk][e]);
+        acc[2 * e] = fmaf(pk, f.x, acc[2 * e]);
+        acc[2 * e + 1] = fmaf(pk, f.y, acc[2 * e + 1]);
       }
     }
   }
