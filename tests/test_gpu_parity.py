@@ -254,6 +254,30 @@ def test_decode_matches_the_forward_row(spa, B, H, N, d, explicit):
         assert torch.all(o[b] == 0) and torch.all(torch.isneginf(lse[b]))
 
 
+def test_decode_full_size_sampled_heads(spa):
+    # The decode bench's cache shape (H32, N32768, d128), two sequences at
+    # different positions; sampled heads are checked against the oracle's
+    # forward row on that head's slice of the cache.
+    B, H, N, d = 2, 32, 32768, 128
+    q, k, v, _ = synth.make_inputs(B, H, N, d, seed=77)
+    tok = q[:, :, 0, :].contiguous()
+    dev = torch.device("cuda:0")
+    pos = np.array([N - 1, 20011], dtype=np.int32)
+    scale = 1 / math.sqrt(d)
+    o, lse = spa.attention_decode(tok.to(dev), k.to(dev), v.to(dev), torch.from_numpy(pos).to(dev), scale)
+    torch.cuda.synchronize()
+    assert spa.spa_device_status() == spa.SPA_OK
+    lo, hi = oracle.bands(N, H)
+    for b in range(B):
+        for h in (0, 1, 13, 30, 31):
+            ks, vs = _f64(k[b:b + 1, h:h + 1]), _f64(v[b:b + 1, h:h + 1])
+            qs = np.zeros_like(ks)
+            qs[0, 0, pos[b]] = _f64(tok[b, h])
+            o_ref, lse_ref = oracle.spa_fwd_rows(qs, ks, vs, scale, [int(pos[b])], [int(lo[h])], [int(hi[h])])
+            assert np.abs(_f64(o[b, h]) - o_ref[0]).max() <= O_TOL, (b, h)
+            _check_lse(_f64(lse[b, h]).reshape(1), lse_ref)
+
+
 def test_calls_from_a_fresh_thread(spa):
     # a host thread that has made no CUDA call yet (as autograd's worker
     # thread may be) gets the same results as the main thread
