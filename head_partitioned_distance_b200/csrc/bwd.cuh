@@ -144,6 +144,7 @@ template <int D>
 __global__ void __launch_bounds__(384, 1)
     spa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                        const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
                         const __grid_constant__ AttnParams p) {
   using C = DkvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
@@ -442,7 +443,10 @@ __global__ void __launch_bounds__(384, 1)
           uint32_t pk[32];
 #pragma unroll
           for (int e = 0; e < 32; ++e) pk[e] = ptx::pack_bf16x2(pt[2 * e], pt[2 * e + 1]);
-          // the tile is free once dV of the previous step has read it
+          // the tile is free once dV of the previous step has read it and, at
+          // a unit's first step, once this warp's bulk stores of the last
+          // unit's dV and dK have read their staging rows in it
+          if (qt == U.qa) ptx::bulk_wait_group_read_all();
           ok = __all_sync(0xffffffffu, bar_wait(&bars->p_empty, (gq & 1) ^ 1, abort_flag));
           if (!ok) break;
           // row r of the warpgroup's 64-query block, 128-byte swizzle
@@ -492,28 +496,59 @@ __global__ void __launch_bounds__(384, 1)
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
+      // Warp (w, wq) owns key rows [32 wq, 32 wq + 32) and, for d = 128,
+      // head dims [64 w, 64 w + 64) of both dV and dK (for d = 64: all of dV
+      // if w = 0, all of dK if w = 1).  It reads them from TMEM (which then
+      // goes back to the MMA warp) and stages each as bf16 in its own 4 KB
+      // slice of the P^T tile (the rows it writes P^T into, 128-byte swizzle)
+      // for a bulk tensor store of a 32 x 64 box.  The next unit's P^T write
+      // waits for those stores to have read the slice.
       ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
       if (!ok) break;
       ptx::tc_fence_after();
-      const uint32_t src = tmem + lane_base + (w == 0 ? C::TM_DV : C::TM_DK);
-      const float mul = (w == 0) ? 1.f : p.scale;
-      uint16_t* grow = static_cast<uint16_t*>(w == 0 ? p.dv : p.dk) + ((int64_t)U.bh * N + j) * D;
-#pragma unroll 1
-      for (int c = 0; c < D; c += 64) {
+      constexpr int NJ = D / 64;
+      const int x0 = NJ == 2 ? 64 * w : 0;
+      uint32_t pk[NJ][32];
+#pragma unroll
+      for (int t = 0; t < NJ; ++t) {
+        const bool is_dk = NJ == 2 ? t == 1 : w == 1;
+        const uint32_t src = tmem + lane_base + (is_dk ? C::TM_DK : C::TM_DV) + x0;
+        const float mul = is_dk ? p.scale : 1.f;
         uint32_t g[2][32];
-        ptx::tmem_ld32(src + c, g[0]);
-        ptx::tmem_ld32(src + c + 32, g[1]);
+        ptx::tmem_ld32(src, g[0]);
+        ptx::tmem_ld32(src + 32, g[1]);
         ptx::tmem_wait_ld();
-        ptx::reg_fence(g[0]);
-        ptx::reg_fence(g[1]);
-        if (j < N) {
-          ptx::store_row32_bf16(grow + c, g[0], mul);
-          ptx::store_row32_bf16(grow + c + 32, g[1], mul);
+        if (t == NJ - 1) {
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&bars->acc_free);
+        }
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          pk[t][e] = ptx::pack_bf16x2(__uint_as_float(g[e / 16][(2 * e) % 32]) * mul,
+                                      __uint_as_float(g[e / 16][(2 * e) % 32 + 1]) * mul);
+      }
+      const int wq = warp % 4;
+      const uint32_t slice = (uint32_t)w * (C::BK * 128) + (uint32_t)wq * (32 * 128);
+      const uint32_t srow = sP + (uint32_t)w * (C::BK * 128) + (uint32_t)r * 128;
+      const int64_t row0 = U.j0 + 32 * wq;
+#pragma unroll
+      for (int t = 0; t < NJ; ++t) {
+        const bool is_dk = NJ == 2 ? t == 1 : w == 1;
+        if (t > 0 && lane == 0) ptx::bulk_wait_group_read_all();
+        __syncwarp();
+#pragma unroll
+        for (int k = 0; k < 8; ++k)
+          ptx::st_shared_v4(srow + ((k ^ (r & 7)) << 4), pk[t][4 * k], pk[t][4 * k + 1], pk[t][4 * k + 2],
+                            pk[t][4 * k + 3]);
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0 && row0 < N) {  // rows past N in the box are clipped
+          ptx::tma_store_3d(is_dk ? &tm_dk : &tm_dv, smem + C::OFF_P + slice, x0, (int)row0, U.bh);
+          ptx::bulk_commit_group();
         }
       }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->acc_free);
     }
+    ptx::bulk_wait_group_all();
   }
 
   // ------------------------------------------------------------ keys no query reaches

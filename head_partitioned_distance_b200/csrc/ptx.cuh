@@ -92,6 +92,12 @@ __device__ __forceinline__ void bulk_wait_group_all() {
   asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// The thread's bulk stores have finished reading their shared-memory source
+// (the global writes may still be in flight).
+__device__ __forceinline__ void bulk_wait_group_read_all() {
+  asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
 // Generic-proxy writes to shared memory become visible to the async proxy
 // (TMA and the tensor core read shared memory through it).
 __device__ __forceinline__ void fence_proxy_async_smem() {

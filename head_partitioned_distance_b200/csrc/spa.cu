@@ -243,9 +243,11 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   if (steps & kStepDkDv) {
     // persistent grid over key tiles of 128 that some query reaches; the
     // other key tiles only get zero rows
-    CUtensorMap kq, kk, kv, kdo;
+    // dk and dv leave through bulk tensor stores of 32-row boxes
+    CUtensorMap kq, kk, kv, kdo, kdk, kdv;
     if ((st = make_map(&kq, q, p.N, BH, D, KC::BQ)) || (st = make_map(&kk, k, p.N, BH, D, KC::BK)) ||
-        (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)))
+        (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)) ||
+        (st = make_map(&kdk, dk, p.N, BH, D, 32)) || (st = make_map(&kdv, dv, p.N, BH, D, 32)))
       return st;
     if ((st = prepare_kernel(spa::spa_bwd_dkdv_kernel<D>, KC::SMEM_BYTES, prepared_kv))) return st;
     static std::atomic<int> regs_kv{0};
@@ -261,7 +263,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if ((st = sm_count(&sms))) return st;
     const int64_t units = (int64_t)p.B * upb;
     const unsigned grid = (unsigned)(units < sms ? units : sms);
-    spa::spa_bwd_dkdv_kernel<D><<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, p);
+    spa::spa_bwd_dkdv_kernel<D><<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
     if ((st = launch_status())) return st;
   }
   return SPA_OK;
