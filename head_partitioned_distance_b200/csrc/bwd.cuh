@@ -55,19 +55,21 @@ __global__ void __launch_bounds__(256) spa_bwd_delta_kernel(const uint16_t* __re
 // the 128-query tiles its band reaches.  Per query tile:
 //   S^T  = K Q^T      SS MMA -> TMEM [0,128)
 //   dP^T = V dO^T     SS MMA -> TMEM [128,256)
-//   P^T  = exp2(S^T c - lse2), masked on edge tiles; bf16 to a shared tile
-//   dS^T = P^T (dP^T - D);                          written as bf16 over dP^T
-//   dV  += P^T dO     SS MMA (A = P^T from shared memory) -> TMEM [256,384)
+//   P^T  = exp2(S^T c - lse2), masked on edge tiles; bf16 over dP^T
+//   dS^T = P^T (dP^T - D);                          bf16 over dP^T
+//   dV  += P^T dO     TS MMA (A = P^T from TMEM)  -> TMEM [256,384)
 //   dK  += dS^T Q     TS MMA (A = dS^T from TMEM) -> TMEM [384,512)
 // Two warpgroups share each tile: warpgroup w owns query columns
-// [64w, 64w+64) of every key row (thread r = key row r = TMEM lane r); its P^T
-// goes to 64-query block w of the shared tile and its dS^T pairs to columns
-// [64w, 64w+32) of the dP^T region it read.  S^T of the next query tile is
-// issued as soon as the warpgroups hold this one in registers (P^T does not
-// live in TMEM), so it overlaps their exponentials; dP^T of the next tile
-// follows dK.  K and V are released after their last S^T/dP^T so the next
-// unit's loads overlap the last step.  Epilogue: warpgroup 0 writes dV,
-// warpgroup 1 writes scale * dK, straight from TMEM to global.
+// [64w, 64w+64) of every key row (thread r = key row r = TMEM lane r).  Once
+// it holds its 64 columns of dP^T in registers it writes its P^T pairs to the
+// first 32 of them and its dS^T pairs to the other 32, so both gradient
+// products read their A operand from TMEM and shared memory carries only the
+// tiles the copy engine brings (the SS products of N = 128 need all of its
+// bandwidth).  S^T of the next query tile is issued as soon as the
+// warpgroups hold this one in registers, so it overlaps their exponentials;
+// dP^T of the next tile follows dK.  K and V are released after their last
+// S^T/dP^T so the next unit's loads overlap the last step.  Epilogue: bulk
+// tensor stores of dV and scale * dK staged through shared memory.
 // ---------------------------------------------------------------------------
 template <int D>
 struct DkvCfg {
@@ -81,9 +83,10 @@ struct DkvCfg {
   static constexpr uint32_t OFF_V = OFF_K + KT_BYTES;
   static constexpr uint32_t OFF_Q = OFF_V + KT_BYTES;
   static constexpr uint32_t OFF_DO = OFF_Q + NS * QT_BYTES;
-  // P^T of the current step, bf16 [keys x queries] K-major (A of dV = P^T dO)
+  // epilogue staging: dV and dK of the unit as bf16, [keys x 64 head dims]
+  // per warpgroup, 128-byte swizzle, for the bulk tensor stores
   static constexpr uint32_t OFF_P = OFF_DO + NS * QT_BYTES;
-  static constexpr uint32_t PT_BYTES = BK * BQ * 2;
+  static constexpr uint32_t PT_BYTES = BK * 128 * 2;
   // vectors of a query tile, [2 stages][256 floats]: -lse * log2(e) of its
   // 128 queries, then -D of them
   static constexpr uint32_t OFF_VEC = OFF_P + PT_BYTES;
@@ -96,17 +99,21 @@ struct DkvCfg {
   static_assert(USED_BYTES <= kMaxSmemPerBlock, "dK/dV tiles exceed shared memory");
   static constexpr int NTHREADS = 384;
   // register split: 384 threads launch with 168 registers each; the two
-  // element-wise warpgroups take 200, the producer/MMA warpgroup 104.
-  static constexpr uint32_t LAUNCH_REGS = 168, EW_REGS = 200, CONTROL_REGS = 104;
+  // element-wise warpgroups take 192, the producer/MMA warpgroup 120.
+  static constexpr uint32_t LAUNCH_REGS = 168, EW_REGS = 192, CONTROL_REGS = 120;
   static_assert(2 * EW_REGS + CONTROL_REGS <= 3 * LAUNCH_REGS, "register split over budget");
   static constexpr uint32_t TM_ST = 0, TM_DPT = 128, TM_DV = 256, TM_DK = 384;
+  // Once the warpgroups hold dP^T in registers, its columns take P^T and
+  // dS^T as bf16 pairs (A operands of dV and dK): warpgroup w's 64 queries
+  // at TM_DPT + 64 w + [0, 32) (P^T) and + [32, 64) (dS^T).
+  static constexpr uint32_t TM_PT = TM_DPT, TM_DST = TM_DPT + 32;
   static constexpr uint32_t TMEM_COLS = 512;
 };
 
 struct DkvBars {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2];
-  uint64_t s_full, s_free, dp_full, p_full, p_empty, ds_full;
+  uint64_t s_full, s_free, dp_full, p_full, ds_full;
   uint64_t vec_full[2], vec_empty[2];
   uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
@@ -175,7 +182,6 @@ __global__ void __launch_bounds__(384, 1)
     ptx::mbar_init(&bars->s_free, 256);
     ptx::mbar_init(&bars->dp_full, 1);
     ptx::mbar_init(&bars->p_full, 256);
-    ptx::mbar_init(&bars->p_empty, 1);
     ptx::mbar_init(&bars->ds_full, 256);
     ptx::mbar_init(&bars->acc_done, 1);
     ptx::mbar_init(&bars->acc_free, 256);
@@ -266,7 +272,6 @@ __global__ void __launch_bounds__(384, 1)
       int nkv = 0, gq = 0, cf = 0, cp = 0, cds = 0, cacc = 0;
       bool ok = true;
       auto qstage = [&](int g) { return g % C::NS; };
-      const uint64_t dPk = ptx::sdesc_sw128(sP, 0, 1024);  // P^T, K-major (A of dV)
       // descriptors of every operand buffer, built once
       const uint64_t dK = ptx::sdesc_sw128(sK, 0, 1024), dV = ptx::sdesc_sw128(sV, 0, 1024);
       // K-major (B of S^T/dP^T) and MN-major (B of dK/dV) views of both Q/dO stages
@@ -291,12 +296,6 @@ __global__ void __launch_bounds__(384, 1)
         for (int kk = 0; kk < C::BQ / 16; ++kk)
           ptx::mma_bf16_ts(tmem + dst, tmem + a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
                            ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (!first || kk > 0));
-      };
-      auto issue_dv = [&](uint64_t db, bool first) {  // dV += P^T dO, both from shared memory
-#pragma unroll
-        for (int kk = 0; kk < C::BQ / 16; ++kk)
-          ptx::mma_bf16(tmem + C::TM_DV, ptx::sdesc_advance(dPk, (kk / 4) * (C::BK * 128) + (kk % 4) * 32),
-                        ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (!first || kk > 0));
       };
       for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
         const DkvUnit U = dkv_decode(u, p);
@@ -328,12 +327,11 @@ __global__ void __launch_bounds__(384, 1)
           if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
-          issue_dv(dOm(qstage(g)), j == 0);                        // dV += P^T dO
-          ptx::mma_commit(&bars->p_empty);
+          issue_grad(C::TM_DV, C::TM_PT, dOm(qstage(g)), j == 0);   // dV += P^T dO
           ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
-          issue_grad(C::TM_DK, C::TM_DPT, dQm(qstage(g)), j == 0);  // dK += dS^T Q
+          issue_grad(C::TM_DK, C::TM_DST, dQm(qstage(g)), j == 0);  // dK += dS^T Q
           ptx::mma_commit(&bars->q_empty[qstage(g)]);
           if (j + 1 < nq) {
             issue_nt(C::TM_DPT, dV, dOk(qstage(g + 1)));           // dP^T of the next tile
@@ -359,6 +357,8 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t lane_base = (uint32_t)((warp % 4) * 32) << 16;
     const uint32_t tS = tmem + lane_base + C::TM_ST + 64 * w;
     const uint32_t tDP = tmem + lane_base + C::TM_DPT + 64 * w;
+    const uint32_t tPT = tmem + lane_base + C::TM_PT + 64 * w;
+    const uint32_t tDST = tmem + lane_base + C::TM_DST + 64 * w;
     const float c2 = p.scale_log2;
     int gq = 0, cs = 0, cdp = 0, cacc = 0;
     bool ok = true;
@@ -387,7 +387,7 @@ __global__ void __launch_bounds__(384, 1)
         const float* vl = vec + (gq % C::NS) * 256 + 64 * w;
         const float* vd = vl + 128;
         const int cb = 64 * w - qlo;
-        // ---- P^T = exp2(S^T c - lse2), bf16 to the shared P^T tile (A of dV)
+        // ---- P^T = exp2(S^T c - lse2)
         ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full, (cs++) & 1, abort_flag) &&
                                          bar_wait(&bars->vec_full[gq % C::NS], (gq / C::NS) & 1, abort_flag));
         if (!ok) break;
@@ -440,36 +440,31 @@ __global__ void __launch_bounds__(384, 1)
               pt[q + 3] = (uint32_t)(cb + q + 3) <= span ? ptx::exp2_approx(xb.y) : 0.f;
             }
           }
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) pk[e] = ptx::pack_bf16x2(pt[2 * e], pt[2 * e + 1]);
-          // the tile is free once dV of the previous step has read it and, at
-          // a unit's first step, once this warp's bulk stores of the last
-          // unit's dV and dK have read their staging rows in it
-          if (qt == U.qa) ptx::bulk_wait_group_read_all();
-          ok = __all_sync(0xffffffffu, bar_wait(&bars->p_empty, (gq & 1) ^ 1, abort_flag));
-          if (!ok) break;
-          // row r of the warpgroup's 64-query block, 128-byte swizzle
-          const uint32_t prow = sP + (uint32_t)w * (C::BK * 128) + (uint32_t)r * 128;
-#pragma unroll
-          for (int k = 0; k < 8; ++k)
-            ptx::st_shared_v4(prow + ((k ^ (r & 7)) << 4), pk[4 * k], pk[4 * k + 1], pk[4 * k + 2],
-                              pk[4 * k + 3]);
-          ptx::fence_proxy_async_smem();
         }
-        ptx::mbar_arrive(&bars->p_full);
-        // ---- dS^T = P^T (dP^T - D)
+        // ---- dP^T into registers; its columns take P^T (A of dV), then dS^T
         ok = __all_sync(0xffffffffu, bar_wait(&bars->dp_full, (cdp++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
         {
+          // the first 32 columns of dP^T take P^T: read them first, the
+          // other 32 (where dS^T goes) after P^T is written
           uint32_t dr[2][32];
           ptx::tmem_ld32(tDP, dr[0]);
-          ptx::tmem_ld32(tDP + 32, dr[1]);
           ptx::tmem_wait_ld();
           ptx::reg_fence(dr[0]);
+          {
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) pk[e] = ptx::pack_bf16x2(pt[2 * e], pt[2 * e + 1]);
+            ptx::tmem_st32(tPT, pk);
+            ptx::tmem_wait_st();
+          }
+          ptx::tc_fence_before();
+          ptx::mbar_arrive(&bars->p_full);
+          ptx::tmem_ld32(tDP + 32, dr[1]);
+          ptx::tmem_wait_ld();
           ptx::reg_fence(dr[1]);
-          // vd holds -D of the 64 queries: dS = P (dP - D) in pairs
+          // ---- dS^T = P^T (dP^T - D); vd holds -D of the 64 queries, in pairs
           const float4* nd4 = reinterpret_cast<const float4*>(vd);
           uint32_t pk[32];
 #pragma unroll
@@ -487,7 +482,7 @@ __global__ void __launch_bounds__(384, 1)
             pk[2 * q4] = ptx::pack_bf16x2(da.x, da.y);
             pk[2 * q4 + 1] = ptx::pack_bf16x2(db.x, db.y);
           }
-          ptx::tmem_st32(tDP, pk);
+          ptx::tmem_st32(tDST, pk);
           ptx::tmem_wait_st();
         }
         ptx::tc_fence_before();
@@ -500,9 +495,8 @@ __global__ void __launch_bounds__(384, 1)
       // head dims [64 w, 64 w + 64) of both dV and dK (for d = 64: all of dV
       // if w = 0, all of dK if w = 1).  It reads them from TMEM (which then
       // goes back to the MMA warp) and stages each as bf16 in its own 4 KB
-      // slice of the P^T tile (the rows it writes P^T into, 128-byte swizzle)
-      // for a bulk tensor store of a 32 x 64 box.  The next unit's P^T write
-      // waits for those stores to have read the slice.
+      // slice of the staging tile (128-byte swizzle)
+      // for a bulk tensor store of a 32 x 64 box.
       ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
       if (!ok) break;
       ptx::tc_fence_after();
@@ -534,7 +528,8 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
       for (int t = 0; t < NJ; ++t) {
         const bool is_dk = NJ == 2 ? t == 1 : w == 1;
-        if (t > 0 && lane == 0) ptx::bulk_wait_group_read_all();
+        // the slice is free once this warp's previous bulk store has read it
+        if (lane == 0) ptx::bulk_wait_group_read_all();
         __syncwarp();
 #pragma unroll
         for (int k = 0; k < 8; ++k)
