@@ -275,7 +275,8 @@ int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (st) return st;
   if (!q || !k || !v || !o || !lse) return SPA_ERR_INVAL;
   if (!std::isfinite(scale) || !(scale > 0.f)) return SPA_ERR_INVAL;
-  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(lse, 4))
+  // o leaves in 32-byte stores
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 32) || !aligned(lse, 4))
     return SPA_ERR_UNSUPPORTED;
   static AttnParams zero{};
   AttnParams p = zero;
@@ -301,8 +302,11 @@ int bwd_entry(const void* q, const void* k, const void* v, const void* o, const 
   if ((steps & kStepDkDv) && (!dk || !dv)) return SPA_ERR_INVAL;
   if ((steps & (kStepDq | kStepDqDelta)) && !dq) return SPA_ERR_INVAL;
   if (!std::isfinite(scale) || !(scale > 0.f)) return SPA_ERR_INVAL;
-  for (const void* t : {q, k, v, o, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+  for (const void* t : {q, k, v, o, dout})
     if (t && !aligned(t, 16)) return SPA_ERR_UNSUPPORTED;
+  // the gradients leave in 32-byte stores
+  for (const void* t : {(const void*)dq, (const void*)dk, (const void*)dv})
+    if (t && !aligned(t, 32)) return SPA_ERR_UNSUPPORTED;
   if ((lse && !aligned(lse, 4)) || !aligned(workspace, 4)) return SPA_ERR_UNSUPPORTED;
   static AttnParams zero{};
   AttnParams p = zero;

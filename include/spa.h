@@ -14,8 +14,10 @@
  *
  * Conventions shared by every entry point:
  *  - Tensors q, k, v, o, dout, dq, dk, dv are bf16, layout [B][H][N][d]
- *    row-major contiguous, in DEVICE memory, 16-byte aligned.  lse and the
- *    backward workspace are fp32 [B][H][N], device memory, 4-byte aligned.
+ *    row-major contiguous, in DEVICE memory, 16-byte aligned; the outputs
+ *    o of the forward and dq, dk, dv of the backward 32-byte aligned (they
+ *    are written in 32-byte stores).  lse and the backward workspace are
+ *    fp32 [B][H][N], device memory, 4-byte aligned.
  *  - The caller owns every buffer; no call allocates device memory (the
  *    one library-owned buffer is the static scratch array of
  *    spa_attn_bwd_noalloc, below).

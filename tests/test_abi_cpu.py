@@ -142,6 +142,13 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
         b = (ctypes.c_int32 * 2)(*hi)
         assert L.spa_attn_fwd_ex(p, p, p, p, p, 1, 2, 256, 64, 0.1, a, b, None) == spa.SPA_ERR_INVAL
     assert L.spa_attn_fwd_ex(p, p, p, p, p, 1, 2, 256, 64, 0.1, None, None, None) == spa.SPA_ERR_INVAL
+    # outputs written in 32-byte stores: 16-byte aligned is not enough
+    half = _fake((1 << 20) + 16)
+    assert L.spa_attn_fwd(p, p, p, half, p, 1, 4, 256, 64, 0.1, None) == spa.SPA_ERR_UNSUPPORTED
+    for pos in (6, 7, 8):  # dq, dk, dv of spa_attn_bwd
+        args = [p] * 10
+        args[pos] = half
+        assert L.spa_attn_bwd(*args, 1, 4, 256, 64, 0.1, None) == spa.SPA_ERR_UNSUPPORTED
     g = lambda *a: L.spa_attn_bwd(p, p, p, p, p, p, p, p, p, p, *a, None)
     assert g(1, 4, 256, 80, 0.1) == spa.SPA_ERR_UNSUPPORTED
     assert g(1, 8, 4, 64, 0.1) == spa.SPA_ERR_INVAL
