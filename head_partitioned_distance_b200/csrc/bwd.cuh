@@ -171,10 +171,10 @@ __global__ void __launch_bounds__(384, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(&bars->kv_full, 1);
-    ptx::mbar_init(&bars->kv_empty, 1);
+    ptx::mbar_init(&bars->kv_empty, 2);  // one commit from each MMA issuer
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars->q_full[s], 1);
-      ptx::mbar_init(&bars->q_empty[s], 1);
+      ptx::mbar_init(&bars->q_empty[s], 2);
       ptx::mbar_init(&bars->vec_full[s], 1);
       ptx::mbar_init(&bars->vec_empty[s], 256);
     }
@@ -185,7 +185,7 @@ __global__ void __launch_bounds__(384, 1)
     ptx::mbar_init(&bars->ds_full, 256);
     ptx::mbar_init(&bars->acc_done, 1);
     ptx::mbar_init(&bars->acc_free, 256);
-    ptx::mbar_init(&bars->drain, 1);
+    ptx::mbar_init(&bars->drain, 2);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -201,8 +201,8 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     ptx::regs_dec<C::CONTROL_REGS>();
-  if (warp >= 10) {
-    // idle warps of the control warpgroup
+  if (warp >= 11) {
+    // idle warp of the control warpgroup
   } else if (warp == 8) {
     // ------------------------------------------------------------ producer warp
     // Lane 0 issues the tile copies; all lanes load the query tiles' lse and D
@@ -264,14 +264,22 @@ __global__ void __launch_bounds__(384, 1)
         if (armed[s] > 0) bar_drain(&bars->q_full[s], (armed[s] - 1) & 1);
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 10 issues S^T of every query tile, warp 9 dV, dK and dP^T.  The
+    // issuing thread blocks in each group of MMAs for about as long as the
+    // tensor core takes to run it, so one issuer leaves the tensor core idle
+    // while it waits for the warpgroups; with two, S^T of the next tile fills
+    // the gaps of the gradient chain.  The two write disjoint TMEM columns
+    // (S^T vs dP^T, dV, dK); Q stages and K/V are released by one commit
+    // from each.
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idesc_g = ptx::idesc_bf16_f32(128, D, false, true);
-      int nkv = 0, gq = 0, cf = 0, cp = 0, cds = 0, cacc = 0;
+      int nkv = 0, gq = 0;
       bool ok = true;
       auto qstage = [&](int g) { return g % C::NS; };
+      auto qphase = [&](int g) { return (uint32_t)((g / C::NS) & 1); };
       // descriptors of every operand buffer, built once
       const uint64_t dK = ptx::sdesc_sw128(sK, 0, 1024), dV = ptx::sdesc_sw128(sV, 0, 1024);
       // K-major (B of S^T/dP^T) and MN-major (B of dK/dV) views of both Q/dO stages
@@ -297,52 +305,70 @@ __global__ void __launch_bounds__(384, 1)
           ptx::mma_bf16_ts(tmem + dst, tmem + a_col + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
                            ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (!first || kk > 0));
       };
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const DkvUnit U = dkv_decode(u, p);
-        const int nq = U.qb - U.qa + 1;
-        const int g0 = gq;
-        ok = bar_wait(&bars->kv_full, (nkv++) & 1, abort_flag) &&
-             bar_wait(&bars->q_full[qstage(g0)], (g0 / C::NS) & 1, abort_flag);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        issue_nt(C::TM_ST, dK, dQk(qstage(g0)));
-        ptx::mma_commit(&bars->s_full);
-        issue_nt(C::TM_DPT, dV, dOk(qstage(g0)));
-        ptx::mma_commit(&bars->dp_full);
-        if (nq == 1) ptx::mma_commit(&bars->kv_empty);           // K and V read for the last time
-        for (int j = 0; j < nq; ++j) {
-          const int g = g0 + j;
-          // the warpgroups hold S^T of this tile in registers: S^T of the next
-          // one goes into the same columns while they exponentiate
-          ok = bar_wait(&bars->s_free, (cf++) & 1, abort_flag);
-          if (ok && j + 1 < nq) {
-            ok = bar_wait(&bars->q_full[qstage(g + 1)], ((g + 1) / C::NS) & 1, abort_flag);
-            if (ok) {
+      if (warp == 10) {
+        // ---- S^T of each query tile, as soon as the warpgroups hold the last
+        // one in registers
+        int cf = 0;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+          const DkvUnit U = dkv_decode(u, p);
+          const int nq = U.qb - U.qa + 1;
+          const int g0 = gq;
+          for (int j = 0; ok && j < nq; ++j) {
+            const int g = g0 + j;
+            // S^T of the previous tile is in registers (for j = 0: the
+            // previous unit's last tile, if any)
+            if (g > 0) ok = bar_wait(&bars->s_free, (cf++) & 1, abort_flag);
+            if (ok && j == 0) ok = bar_wait(&bars->kv_full, (nkv++) & 1, abort_flag);
+            if (ok) ok = bar_wait(&bars->q_full[qstage(g)], qphase(g), abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_nt(C::TM_ST, dK, dQk(qstage(g)));
+            ptx::mma_commit(&bars->s_full);
+            ptx::mma_commit(&bars->q_empty[qstage(g)]);
+            if (j + 1 == nq) ptx::mma_commit(&bars->kv_empty);      // K read for the last time
+          }
+          gq = g0 + nq;
+        }
+      } else {
+        // ---- dV, dK of each query tile and dP^T of the next
+        int cp = 0, cds = 0, cacc = 0;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+          const DkvUnit U = dkv_decode(u, p);
+          const int nq = U.qb - U.qa + 1;
+          const int g0 = gq;
+          ok = bar_wait(&bars->kv_full, (nkv++) & 1, abort_flag) &&
+               bar_wait(&bars->q_full[qstage(g0)], qphase(g0), abort_flag);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_nt(C::TM_DPT, dV, dOk(qstage(g0)));
+          ptx::mma_commit(&bars->dp_full);
+          if (nq == 1) ptx::mma_commit(&bars->kv_empty);           // V read for the last time
+          for (int j = 0; j < nq; ++j) {
+            const int g = g0 + j;
+            ok = bar_wait(&bars->p_full, (cp++) & 1, abort_flag);
+            if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_grad(C::TM_DV, C::TM_PT, dOm(qstage(g)), j == 0);   // dV += P^T dO
+            ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_grad(C::TM_DK, C::TM_DST, dQm(qstage(g)), j == 0);  // dK += dS^T Q
+            ptx::mma_commit(&bars->q_empty[qstage(g)]);
+            if (j + 1 < nq) {
+              ok = bar_wait(&bars->q_full[qstage(g + 1)], qphase(g + 1), abort_flag);
+              if (!ok) break;
               ptx::tc_fence_after();
-              issue_nt(C::TM_ST, dK, dQk(qstage(g + 1)));
-              ptx::mma_commit(&bars->s_full);
+              issue_nt(C::TM_DPT, dV, dOk(qstage(g + 1)));           // dP^T of the next tile
+              ptx::mma_commit(&bars->dp_full);
+              if (j + 2 == nq) ptx::mma_commit(&bars->kv_empty);     // V read for the last time
             }
           }
-          if (ok) ok = bar_wait(&bars->p_full, (cp++) & 1, abort_flag);
-          if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
           if (!ok) break;
-          ptx::tc_fence_after();
-          issue_grad(C::TM_DV, C::TM_PT, dOm(qstage(g)), j == 0);   // dV += P^T dO
-          ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          issue_grad(C::TM_DK, C::TM_DST, dQm(qstage(g)), j == 0);  // dK += dS^T Q
-          ptx::mma_commit(&bars->q_empty[qstage(g)]);
-          if (j + 1 < nq) {
-            issue_nt(C::TM_DPT, dV, dOk(qstage(g + 1)));           // dP^T of the next tile
-            ptx::mma_commit(&bars->dp_full);
-            if (j + 2 == nq) ptx::mma_commit(&bars->kv_empty);     // K and V read for the last time
-          }
+          ++cacc;
+          ptx::mma_commit(&bars->acc_done);
+          gq = g0 + nq;
         }
-        if (!ok) break;
-        ++cacc;
-        ptx::mma_commit(&bars->acc_done);
-        gq = g0 + nq;
       }
       ptx::mma_commit(&bars->drain);
       bar_drain(&bars->drain, 0);
