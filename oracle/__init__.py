@@ -18,6 +18,11 @@ follows, is written at the top of ``oracle.c``:
   S_i^h = {j : lo_h <= i - j < hi_h, j <= i}; empty rows give o = 0,
   lse = -inf; gradients derived by hand (the pages give none).
 * ``tile_classes``     -- brute-force per-element classification of tiles.
+* ``union_fwd``/``union_bwd`` (and ``union_fwd_rows``) -- each head's band
+  plus a local window [0, w) shared by every head, S_i^h = {j <= i :
+  i - j < w or lo_h <= i - j < hi_h}: a reading of the "local sharing" that
+  Figure 2(b) of "Making Every Head Count" says the EBALL ablation removes
+  (the pages do not define it).
 
 Parity status: every function is pinned by ``tests/test_oracle_pins.py``
 (worked example of the blog post, band invariants, reduction to dense causal
@@ -88,6 +93,12 @@ def _load():
                                                  ctypes.c_double, _i64p, _i64p, _i64p,
                                                  _i64, _d, _d]
         lib.oracle_tile_classes.argtypes = [_i64, _i64, _i64p, _i64p, _i64, _i64, _u8p]
+        lib.oracle_union_fwd.argtypes = [_d, _d, _d, _i64, _i64, _i64, _i64, ctypes.c_double, _i64,
+                                         _i64p, _i64p, _d, _d]
+        lib.oracle_union_fwd_rows.argtypes = [_d, _d, _d, _i64, _i64, _i64, _i64, ctypes.c_double,
+                                              _i64, _i64p, _i64p, _i64p, _i64, _d, _d]
+        lib.oracle_union_bwd.argtypes = [_d, _d, _d, _d, _i64, _i64, _i64, _i64, ctypes.c_double,
+                                         _i64, _i64p, _i64p, _d, _d, _d]
         _lib = lib
         return lib
 
@@ -231,3 +242,39 @@ def tile_classes(N: int, lo, hi, Bq: int, Bk: int) -> np.ndarray:
     cls = np.zeros((H, nqt, nkt), np.uint8)
     _load().oracle_tile_classes(N, H, _pi(lo), _pi(hi), Bq, Bk, cls.ctypes.data_as(_u8p))
     return cls
+
+
+def union_fwd(q, k, v, scale: float, window: int, lo=None, hi=None):
+    """Band plus shared local window [0, window).  Returns (o, lse) like spa_fwd."""
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    lo, hi = _bands_arg(N, H, lo, hi)
+    o = np.zeros_like(q)
+    lse = np.zeros((B, H, N))
+    _load().oracle_union_fwd(_pd(q), _pd(k), _pd(v), B, H, N, d, scale, int(window), _pi(lo), _pi(hi),
+                             _pd(o), _pd(lse))
+    return o, lse
+
+
+def union_fwd_rows(q, k, v, scale: float, window: int, rows, lo=None, hi=None):
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, N, d = q.shape
+    lo, hi = _bands_arg(N, H, lo, hi)
+    rows = _i64arr(rows)
+    o = np.zeros((len(rows), d))
+    lse = np.zeros(len(rows))
+    _load().oracle_union_fwd_rows(_pd(q), _pd(k), _pd(v), B, H, N, d, scale, int(window), _pi(lo),
+                                  _pi(hi), _pi(rows), len(rows), _pd(o), _pd(lse))
+    return o, lse
+
+
+def union_bwd(q, k, v, dout, scale: float, window: int, lo=None, hi=None):
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, N, d = q.shape
+    lo, hi = _bands_arg(N, H, lo, hi)
+    dq = np.zeros_like(q)
+    dk = np.zeros_like(q)
+    dv = np.zeros_like(q)
+    _load().oracle_union_bwd(_pd(q), _pd(k), _pd(v), _pd(dout), B, H, N, d, scale, int(window),
+                             _pi(lo), _pi(hi), _pd(dq), _pd(dk), _pd(dv))
+    return dq, dk, dv

@@ -275,6 +275,108 @@ void oracle_spa_bwd(const double* q, const double* k, const double* v, const dou
   }
 }
 
+/* ------------------------------------------------------------------------ */
+/* Exclusive bands plus a local window shared by every head: the reading    */
+/* of Figure 2(b) of "Making Every Head Count", where the EBALL ablation is  */
+/* said to remove "local sharing".  The pages never define the shared part; */
+/* here head h attends to S_i = { j <= i : i - j < w  or  lo_h <= i - j <   */
+/* hi_h }, enumerated one key at a time.  w = 0 is the plain band.          */
+/* ------------------------------------------------------------------------ */
+static int union_permitted(int64_t i, int64_t j, int64_t w, int64_t lo, int64_t hi) {
+  if (j < 0 || j > i) return 0;
+  return (i - j < w) || ((i - j >= lo) && (i - j < hi));
+}
+
+static double union_row_fwd(const double* qh, const double* kh, const double* vh,
+                            int64_t d, double scale, int64_t w, int64_t lo, int64_t hi,
+                            int64_t i, double* o_i) {
+  for (int64_t c = 0; c < d; ++c) o_i[c] = 0.0;
+  double m = -INFINITY;
+  int64_t count = 0;
+  for (int64_t j = 0; j <= i; ++j) {
+    if (!union_permitted(i, j, w, lo, hi)) continue;
+    double s = scale * dot(qh + i * d, kh + j * d, d);
+    if (s > m) m = s;
+    ++count;
+  }
+  if (count == 0) return -INFINITY;
+  double l = 0.0;
+  for (int64_t j = 0; j <= i; ++j)
+    if (union_permitted(i, j, w, lo, hi)) l += exp(scale * dot(qh + i * d, kh + j * d, d) - m);
+  double lse = m + log(l);
+  for (int64_t j = 0; j <= i; ++j) {
+    if (!union_permitted(i, j, w, lo, hi)) continue;
+    double p = exp(scale * dot(qh + i * d, kh + j * d, d) - lse);
+    for (int64_t c = 0; c < d; ++c) o_i[c] += p * vh[j * d + c];
+  }
+  return lse;
+}
+
+void oracle_union_fwd(const double* q, const double* k, const double* v,
+                      int64_t B, int64_t H, int64_t N, int64_t d, double scale, int64_t w,
+                      const int64_t* lo, const int64_t* hi, double* o, double* lse) {
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t flat = 0; flat < B * H * N; ++flat) {
+    int64_t bh = flat / N, i = flat % N, h = bh % H;
+    lse[flat] = union_row_fwd(q + bh * N * d, k + bh * N * d, v + bh * N * d, d, scale, w,
+                              lo[h], hi[h], i, o + flat * d);
+  }
+}
+
+void oracle_union_fwd_rows(const double* q, const double* k, const double* v,
+                           int64_t B, int64_t H, int64_t N, int64_t d, double scale, int64_t w,
+                           const int64_t* lo, const int64_t* hi, const int64_t* rows,
+                           int64_t nrows, double* o_rows, double* lse_rows) {
+  (void)B;
+#pragma omp parallel for schedule(dynamic, 16)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t flat = rows[r];
+    int64_t bh = flat / N, i = flat % N, h = bh % H;
+    lse_rows[r] = union_row_fwd(q + bh * N * d, k + bh * N * d, v + bh * N * d, d, scale, w,
+                                lo[h], hi[h], i, o_rows + r * d);
+  }
+}
+
+/* Gradients of L = sum(O * dout) for the union above (same derivation as
+ * oracle_spa_bwd, over the union's permitted set). */
+void oracle_union_bwd(const double* q, const double* k, const double* v, const double* dout,
+                      int64_t B, int64_t H, int64_t N, int64_t d, double scale, int64_t w,
+                      const int64_t* lo, const int64_t* hi, double* dq, double* dk, double* dv) {
+  memset(dq, 0, sizeof(double) * (size_t)(B * H * N * d));
+  memset(dk, 0, sizeof(double) * (size_t)(B * H * N * d));
+  memset(dv, 0, sizeof(double) * (size_t)(B * H * N * d));
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t bh = 0; bh < B * H; ++bh) {
+    int64_t h = bh % H;
+    const double* qh = q + bh * N * d;
+    const double* kh = k + bh * N * d;
+    const double* vh = v + bh * N * d;
+    const double* doh = dout + bh * N * d;
+    double* dqh = dq + bh * N * d;
+    double* dkh = dk + bh * N * d;
+    double* dvh = dv + bh * N * d;
+    double* o_i = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int64_t i = 0; i < N; ++i) {
+      double lse = union_row_fwd(qh, kh, vh, d, scale, w, lo[h], hi[h], i, o_i);
+      if (isinf(lse)) continue;
+      double Di = dot(doh + i * d, o_i, d);
+      for (int64_t j = 0; j <= i; ++j) {
+        if (!union_permitted(i, j, w, lo[h], hi[h])) continue;
+        double s = scale * dot(qh + i * d, kh + j * d, d);
+        double p = exp(s - lse);
+        double dp = dot(doh + i * d, vh + j * d, d);
+        double ds = p * (dp - Di);
+        for (int64_t c = 0; c < d; ++c) {
+          dqh[i * d + c] += scale * ds * kh[j * d + c];
+          dkh[j * d + c] += scale * ds * qh[i * d + c];
+          dvh[j * d + c] += p * doh[i * d + c];
+        }
+      }
+    }
+    free(o_i);
+  }
+}
+
 /* dQ for a list of query rows (flat ids as in oracle_spa_fwd_rows). */
 void oracle_spa_bwd_dq_rows(const double* q, const double* k, const double* v,
                             const double* dout, int64_t B, int64_t H, int64_t N, int64_t d,
