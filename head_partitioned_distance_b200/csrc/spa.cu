@@ -17,6 +17,7 @@
 #include "decode.cuh"
 #include "fwd.cuh"
 #include "sched.cuh"
+#include "union.cuh"
 
 namespace {
 
@@ -322,6 +323,63 @@ int bwd_entry(const void* q, const void* k, const void* v, const void* o, const 
                  : bwd_impl<128>(q, k, v, o, dout, lse, dq, dk, dv, delta, p, s, steps);
 }
 
+// ---------------------------------------------------------------------------
+// Band plus shared window (union.cuh): each head's permitted distances
+// [0, w) u [lo_h, hi_h) as two disjoint, non-empty parts [a1, b1), [a2, b2):
+// the window and the band when they do not touch, else the two halves of
+// [0, max(w, hi_h)).
+struct UnionParts {
+  int32_t a1[spa::kMaxHeads], b1[spa::kMaxHeads], a2[spa::kMaxHeads], b2[spa::kMaxHeads];
+};
+
+int union_parts(int H, int64_t N, int64_t window, const int32_t* lo, const int32_t* hi, UnionParts& u) {
+  if (window < 1 || window > N) return SPA_ERR_INVAL;
+  static AttnParams zero{};
+  AttnParams p = zero;
+  int st = fill_bands(p, H, N, lo, hi);
+  if (st) return st;
+  for (int h = 0; h < H; ++h) {
+    if (window < p.lo[h]) {
+      u.a1[h] = 0;
+      u.b1[h] = (int32_t)window;
+      u.a2[h] = p.lo[h];
+      u.b2[h] = p.hi[h];
+    } else {
+      const int64_t len = window > p.hi[h] ? window : p.hi[h];
+      if (len < 2) return SPA_ERR_UNSUPPORTED;  // one distance cannot be split
+      const int64_t m = (len + 1) / 2;
+      u.a1[h] = 0;
+      u.b1[h] = (int32_t)m;
+      u.a2[h] = (int32_t)m;
+      u.b2[h] = (int32_t)len;
+    }
+  }
+  return SPA_OK;
+}
+
+size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
+
+// Workspace of the union passes: fp32 [B H N] (lse of part 2, or D), then
+// three bf16 [B H N d] tensors (o of part 2, or dq, dk, dv of part 2).
+struct UnionWs {
+  float* vec;
+  uint16_t* t[3];
+};
+
+UnionWs union_ws(void* ws, int64_t rows, int d) {
+  UnionWs w;
+  uint8_t* b = static_cast<uint8_t*>(ws);
+  w.vec = reinterpret_cast<float*>(b);
+  b += align256((size_t)rows * 4);
+  for (int i = 0; i < 3; ++i) {
+    w.t[i] = reinterpret_cast<uint16_t*>(b);
+    b += align256((size_t)rows * d * 2);
+  }
+  return w;
+}
+
+int union_launch_status() { return cudaGetLastError() == cudaSuccess ? SPA_OK : SPA_ERR_CUDA; }
+
 struct BandArgs {
   int32_t lo[spa::kMaxHeads];
   int32_t hi[spa::kMaxHeads];
@@ -596,6 +654,69 @@ int spa_attn_decode(const void* q, const void* k, const void* v, const int32_t* 
     spa::spa_decode_merge_kernel<128><<<grid_m, 128, 0, s>>>(p);
   }
   return launch_status();
+}
+
+size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d) {
+  if (check_shape(B, H, N, d)) return 0;
+  const size_t rows = (size_t)B * H * N;
+  return align256(rows * 4) + 3 * align256(rows * (size_t)d * 2);
+}
+
+int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
+                       int B, int H, int64_t N, int d, float scale, int64_t window, const int32_t* lo,
+                       const int32_t* hi, void* stream) {
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  if (!workspace) return SPA_ERR_INVAL;
+  if (!aligned(workspace, 32)) return SPA_ERR_UNSUPPORTED;
+  static UnionParts zero{};
+  UnionParts u = zero;
+  if ((st = union_parts(H, N, window, lo, hi, u))) return st;
+  const int64_t rows = (int64_t)B * H * N;
+  UnionWs w = union_ws(workspace, rows, d);
+  if ((st = fwd_entry(q, k, v, o, lse, B, H, N, d, scale, u.a1, u.b1, stream))) return st;
+  if ((st = fwd_entry(q, k, v, w.t[0], w.vec, B, H, N, d, scale, u.a2, u.b2, stream))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t threads = rows * (d / 8);
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  if (d == 64)
+    spa::spa_union_merge_kernel<64><<<blocks, 256, 0, s>>>(static_cast<uint16_t*>(o), lse, w.t[0], w.vec, rows);
+  else
+    spa::spa_union_merge_kernel<128><<<blocks, 256, 0, s>>>(static_cast<uint16_t*>(o), lse, w.t[0], w.vec, rows);
+  return union_launch_status();
+}
+
+int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int H, int64_t N,
+                       int d, float scale, int64_t window, const int32_t* lo, const int32_t* hi, void* stream) {
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  if (!workspace || !dq || !dk || !dv) return SPA_ERR_INVAL;
+  if (!aligned(workspace, 32)) return SPA_ERR_UNSUPPORTED;
+  static UnionParts zero{};
+  UnionParts u = zero;
+  if ((st = union_parts(H, N, window, lo, hi, u))) return st;
+  const int64_t rows = (int64_t)B * H * N;
+  UnionWs w = union_ws(workspace, rows, d);
+  // part 1 starts at distance 0, so its dQ pass forms D for every row
+  if ((st = bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, w.vec, B, H, N, d, scale, u.a1, u.b1,
+                      stream, kStepDqDelta)) ||
+      (st = bwd_entry(q, k, v, o, dout, lse, nullptr, dk, dv, w.vec, B, H, N, d, scale, u.a1, u.b1, stream,
+                      kStepDkDv)) ||
+      (st = bwd_entry(q, k, v, o, dout, lse, w.t[0], nullptr, nullptr, w.vec, B, H, N, d, scale, u.a2, u.b2,
+                      stream, kStepDq)) ||
+      (st = bwd_entry(q, k, v, o, dout, lse, nullptr, w.t[1], w.t[2], w.vec, B, H, N, d, scale, u.a2, u.b2,
+                      stream, kStepDkDv)))
+    return st;
+  int sms = 0;
+  if ((st = sm_count(&sms))) return st;
+  const int64_t n16 = rows * d / 8;
+  const int64_t want = (3 * n16 + 255) / 256;
+  const unsigned blocks = (unsigned)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  spa::spa_add3_bf16_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint16_t*>(dq), static_cast<uint16_t*>(dk), static_cast<uint16_t*>(dv), w.t[0], w.t[1], w.t[2],
+      n16);
+  return union_launch_status();
 }
 
 int spa_device_status(void* stream) {

@@ -48,6 +48,9 @@ EXPORTS = {
     "spa_attn_decode_workspace_bytes": ([_int, _int, _i64, _int, _i32p, _i32p], ctypes.c_size_t),
     "spa_attn_decode": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_noalloc": ([_vp] * 9 + [_int, _int, _i64, _int, _f32, _vp], _int),
+    "spa_attn_union_workspace_bytes": ([_int, _int, _i64, _int], ctypes.c_size_t),
+    "spa_attn_fwd_union": ([_vp] * 6 + [_int, _int, _i64, _int, _f32, _i64, _i32p, _i32p, _vp], _int),
+    "spa_attn_bwd_union": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i64, _i32p, _i32p, _vp], _int),
     "spa_tile_schedule": ([_i64, _int, _i32p, _i32p, _int, _int, _i32p, _i32p, _u8p, _i32p, _i32p],
                           _int),
     "spa_tile_classes_device": ([_i64, _int, _i32p, _i32p, _int, _int, _vp, _vp], _int),
@@ -329,3 +332,71 @@ def spattention(q, k, v, scale=None, lo=None, hi=None):
     Distance Partitioning band (or the explicit bands lo/hi)."""
     scale = q.shape[-1] ** -0.5 if scale is None else scale
     return SPAttentionFunction.apply(q, k, v, scale, lo, hi)
+
+
+# ------------------------------------------------------------- band + shared window
+def spa_attn_union_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib.spa_attn_union_workspace_bytes(B, H, N, d))
+
+
+def _union_ws(workspace, B, H, N, d):
+    need = spa_attn_union_workspace_bytes(B, H, N, d)
+    if not workspace.is_cuda or workspace.numel() * workspace.element_size() < need:
+        raise ValueError("workspace: CUDA tensor of spa_attn_union_workspace_bytes(B, H, N, d) bytes")
+
+
+def spa_attn_fwd_union(q, k, v, o, lse, workspace, scale: float, window: int, lo=None, hi=None,
+                       stream=None):
+    """Each head attends to its band and to the distances [0, window) that every
+    head shares; writes o [B,H,N,d] bf16 and lse [B,H,N] fp32."""
+    B, H, N, d = _dims(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    _need(lse, (B, H, N), torch.float32, "lse")
+    _union_ws(workspace, B, H, N, d)
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    _check(_lib.spa_attn_fwd_union(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   workspace.data_ptr(), B, H, N, d, scale, int(window), lo_a, hi_a,
+                                   _stream_ptr(stream)), "spa_attn_fwd_union")
+    return o, lse
+
+
+def spa_attn_bwd_union(q, k, v, o, dout, lse, dq, dk, dv, workspace, scale: float, window: int, lo=None,
+                       hi=None, stream=None):
+    """Gradients of sum(o * dout) for spa_attn_fwd_union (o, lse from it)."""
+    B, H, N, d = _dims(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    _need(lse, (B, H, N), torch.float32, "lse")
+    _union_ws(workspace, B, H, N, d)
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    ptrs = [t.data_ptr() for t in (q, k, v, o, dout, lse, dq, dk, dv, workspace)]
+    _check(_lib.spa_attn_bwd_union(*ptrs, B, H, N, d, scale, int(window), lo_a, hi_a, _stream_ptr(stream)),
+           "spa_attn_bwd_union")
+    return dq, dk, dv
+
+
+def _union_workspace(q):
+    B, H, N, d = _dims(q)
+    nbytes = spa_attn_union_workspace_bytes(B, H, N, d)
+    return torch.empty(max(nbytes // 4, 1), dtype=torch.float32, device=q.device)
+
+
+def attention_forward_union(q, k, v, window: int, scale=None, lo=None, hi=None):
+    """Allocate o / lse / workspace and run spa_attn_fwd_union."""
+    B, H, N, d = _dims(q)
+    scale = d ** -0.5 if scale is None else scale
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
+    return spa_attn_fwd_union(q, k, v, o, lse, _union_workspace(q), scale, window, lo, hi)
+
+
+def attention_backward_union(q, k, v, o, dout, lse, window: int, scale=None, lo=None, hi=None):
+    """Allocate dq / dk / dv / workspace and run spa_attn_bwd_union."""
+    B, H, N, d = _dims(q)
+    scale = d ** -0.5 if scale is None else scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    return spa_attn_bwd_union(q, k, v, o, dout, lse, dq, dk, dv, _union_workspace(q), scale, window, lo, hi)

@@ -217,6 +217,41 @@ SPA_API int spa_attn_decode(const void* q, const void* k, const void* v, const i
                             const int32_t* lo, const int32_t* hi, void* stream);
 
 /*
+ * Band plus a local window shared by every head.  "Making Every Head Count",
+ * Figure 2(b), presents its EBALL ablation as the exclusive bands with local
+ * sharing taken out; the pages never define the shared part, and the reading
+ * built here gives every head h the permitted set
+ *   S_i^h = { j <= i : i - j < window  or  lo_h <= i - j < hi_h },
+ * with the softmax over S_i^h as in spa_attn_fwd.  Every row attends at least
+ * to itself (window >= 1), so no row is empty.
+ *   window:    1 <= window <= N, the shared distances [0, window)
+ *   lo, hi:    HOST band arrays (rules of spa_attn_fwd_ex) or both NULL for the
+ *              Balanced Distance Partitioning bands
+ *   workspace: DEVICE buffer of spa_attn_union_workspace_bytes(B, H, N, d)
+ *              bytes, 32-byte aligned, caller-owned, overwritten
+ * Other arguments, layouts and alignment as in spa_attn_fwd / spa_attn_bwd.
+ * Each head's set is split into two disjoint, non-empty distance intervals
+ * and the band kernels run once per part; the forward merges the two
+ * partial softmaxes through their lse (one more launch), the backward runs
+ * the dQ and dK/dV passes of each part with the joint lse and D and adds the
+ * second part's gradients to the first's (one more launch).  lse and o
+ * passed to spa_attn_bwd_union must come from spa_attn_fwd_union.
+ * SPA_ERR_INVAL for a window outside [1, N], bad bands, null pointers or a
+ * bad scale; SPA_ERR_UNSUPPORTED where spa_attn_fwd / spa_attn_bwd would
+ * return it, for a misaligned workspace, or when some head's set is a single
+ * distance (it cannot be split).  The workspace size is 0 for shapes the
+ * calls reject.
+ */
+SPA_API size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d);
+SPA_API int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, float* lse,
+                               void* workspace, int B, int H, int64_t N, int d, float scale,
+                               int64_t window, const int32_t* lo, const int32_t* hi, void* stream);
+SPA_API int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               void* workspace, int B, int H, int64_t N, int d, float scale,
+                               int64_t window, const int32_t* lo, const int32_t* hi, void* stream);
+
+/*
  * Band tile schedule, as the kernels walk it (host evaluation of the same
  * code the device runs).  Query tile t covers rows [t*Bq, t*Bq + Bq), key
  * tile u keys [u*Bk, u*Bk + Bk); positions >= N are not permitted.

@@ -20,8 +20,8 @@ follows, is written at the top of ``oracle.c``:
 * ``tile_classes``     -- brute-force per-element classification of tiles.
 * ``union_fwd``/``union_bwd`` (and ``union_fwd_rows``) -- each head's band
   plus a local window [0, w) shared by every head, S_i^h = {j <= i :
-  i - j < w or lo_h <= i - j < hi_h}: a reading of the "local sharing" that
-  Figure 2(b) of "Making Every Head Count" says the EBALL ablation removes
+  i - j < w or lo_h <= i - j < hi_h}: a reading of the local sharing that
+  the EBALL ablation of "Making Every Head Count" (Figure 2(b)) takes out
   (the pages do not define it).
 
 Parity status: every function is pinned by ``tests/test_oracle_pins.py``
@@ -99,6 +99,10 @@ def _load():
                                               _i64, _i64p, _i64p, _i64p, _i64, _d, _d]
         lib.oracle_union_bwd.argtypes = [_d, _d, _d, _d, _i64, _i64, _i64, _i64, ctypes.c_double,
                                          _i64, _i64p, _i64p, _d, _d, _d]
+        lib.oracle_union_bwd_dq_rows.argtypes = [_d, _d, _d, _d, _i64, _i64, _i64, _i64, ctypes.c_double,
+                                                 _i64, _i64p, _i64p, _i64p, _i64, _d]
+        lib.oracle_union_bwd_dkdv_rows.argtypes = [_d, _d, _d, _d, _i64, _i64, _i64, _i64,
+                                                   ctypes.c_double, _i64, _i64p, _i64p, _i64p, _i64, _d, _d]
         _lib = lib
         return lib
 
@@ -278,3 +282,26 @@ def union_bwd(q, k, v, dout, scale: float, window: int, lo=None, hi=None):
     _load().oracle_union_bwd(_pd(q), _pd(k), _pd(v), _pd(dout), B, H, N, d, scale, int(window),
                              _pi(lo), _pi(hi), _pd(dq), _pd(dk), _pd(dv))
     return dq, dk, dv
+
+
+def union_bwd_dq_rows(q, k, v, dout, scale: float, window: int, rows, lo=None, hi=None):
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, N, d = q.shape
+    lo, hi = _bands_arg(N, H, lo, hi)
+    rows = _i64arr(rows)
+    dq = np.zeros((len(rows), d))
+    _load().oracle_union_bwd_dq_rows(_pd(q), _pd(k), _pd(v), _pd(dout), B, H, N, d, scale, int(window),
+                                     _pi(lo), _pi(hi), _pi(rows), len(rows), _pd(dq))
+    return dq
+
+
+def union_bwd_dkdv_rows(q, k, v, dout, scale: float, window: int, rows, lo=None, hi=None):
+    q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
+    B, H, N, d = q.shape
+    lo, hi = _bands_arg(N, H, lo, hi)
+    rows = _i64arr(rows)
+    dk = np.zeros((len(rows), d))
+    dv = np.zeros((len(rows), d))
+    _load().oracle_union_bwd_dkdv_rows(_pd(q), _pd(k), _pd(v), _pd(dout), B, H, N, d, scale, int(window),
+                                       _pi(lo), _pi(hi), _pi(rows), len(rows), _pd(dk), _pd(dv))
+    return dk, dv

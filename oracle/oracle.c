@@ -276,9 +276,9 @@ void oracle_spa_bwd(const double* q, const double* k, const double* v, const dou
 }
 
 /* ------------------------------------------------------------------------ */
-/* Exclusive bands plus a local window shared by every head: the reading    */
-/* of Figure 2(b) of "Making Every Head Count", where the EBALL ablation is  */
-/* said to remove "local sharing".  The pages never define the shared part; */
+/* Exclusive bands plus a local window shared by every head: a reading of   */
+/* Figure 2(b) of "Making Every Head Count", whose EBALL ablation takes     */
+/* local sharing out.  The pages never define the shared part;              */
 /* here head h attends to S_i = { j <= i : i - j < w  or  lo_h <= i - j <   */
 /* hi_h }, enumerated one key at a time.  w = 0 is the plain band.          */
 /* ------------------------------------------------------------------------ */
@@ -371,6 +371,72 @@ void oracle_union_bwd(const double* q, const double* k, const double* v, const d
           dkh[j * d + c] += scale * ds * qh[i * d + c];
           dvh[j * d + c] += p * doh[i * d + c];
         }
+      }
+    }
+    free(o_i);
+  }
+}
+
+/* dQ of the union for a list of query rows (flat ids as in oracle_spa_fwd_rows). */
+void oracle_union_bwd_dq_rows(const double* q, const double* k, const double* v,
+                              const double* dout, int64_t B, int64_t H, int64_t N, int64_t d,
+                              double scale, int64_t w, const int64_t* lo, const int64_t* hi,
+                              const int64_t* rows, int64_t nrows, double* dq_rows) {
+  (void)B;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t flat = rows[r];
+    int64_t bh = flat / N, i = flat % N, h = bh % H;
+    const double* qh = q + bh * N * d;
+    const double* kh = k + bh * N * d;
+    const double* vh = v + bh * N * d;
+    const double* doh = dout + bh * N * d;
+    double* out = dq_rows + r * d;
+    for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
+    double* o_i = (double*)malloc(sizeof(double) * (size_t)d);
+    double lse = union_row_fwd(qh, kh, vh, d, scale, w, lo[h], hi[h], i, o_i);
+    if (!isinf(lse)) {
+      double Di = dot(doh + i * d, o_i, d);
+      for (int64_t j = 0; j <= i; ++j) {
+        if (!union_permitted(i, j, w, lo[h], hi[h])) continue;
+        double p = exp(scale * dot(qh + i * d, kh + j * d, d) - lse);
+        double ds = p * (dot(doh + i * d, vh + j * d, d) - Di);
+        for (int64_t c = 0; c < d; ++c) out[c] += scale * ds * kh[j * d + c];
+      }
+    }
+    free(o_i);
+  }
+}
+
+/* dK and dV of the union for a list of key rows r = (b*H + h)*N + j: every
+ * query i >= j whose set holds key j, its forward row recomputed first. */
+void oracle_union_bwd_dkdv_rows(const double* q, const double* k, const double* v,
+                                const double* dout, int64_t B, int64_t H, int64_t N, int64_t d,
+                                double scale, int64_t w, const int64_t* lo, const int64_t* hi,
+                                const int64_t* rows, int64_t nrows, double* dk_rows,
+                                double* dv_rows) {
+  (void)B;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int64_t r = 0; r < nrows; ++r) {
+    int64_t flat = rows[r];
+    int64_t bh = flat / N, j = flat % N, h = bh % H;
+    const double* qh = q + bh * N * d;
+    const double* kh = k + bh * N * d;
+    const double* vh = v + bh * N * d;
+    const double* doh = dout + bh * N * d;
+    double* dkr = dk_rows + r * d;
+    double* dvr = dv_rows + r * d;
+    for (int64_t c = 0; c < d; ++c) dkr[c] = dvr[c] = 0.0;
+    double* o_i = (double*)malloc(sizeof(double) * (size_t)d);
+    for (int64_t i = j; i < N; ++i) {
+      if (!union_permitted(i, j, w, lo[h], hi[h])) continue;
+      double lse = union_row_fwd(qh, kh, vh, d, scale, w, lo[h], hi[h], i, o_i);
+      double Di = dot(doh + i * d, o_i, d);
+      double p = exp(scale * dot(qh + i * d, kh + j * d, d) - lse);
+      double ds = p * (dot(doh + i * d, vh + j * d, d) - Di);
+      for (int64_t c = 0; c < d; ++c) {
+        dkr[c] += scale * ds * qh[i * d + c];
+        dvr[c] += p * doh[i * d + c];
       }
     }
     free(o_i);

@@ -187,3 +187,32 @@ def test_timeout_hook_rejects_bad_limits():
     L = spa._lib
     assert L.spa_debug_wait_timeout(0, None) == spa.SPA_ERR_INVAL
     assert L.spa_debug_wait_timeout(2_000_000_000, None) == spa.SPA_ERR_INVAL
+
+
+def test_union_entry_points_reject_bad_arguments_before_any_launch():
+    L = spa._lib
+    p = _fake(1 << 20)  # never dereferenced: every call below fails its checks first
+    B, H, N, d = 1, 4, 256, 64
+    args = (B, H, N, d, 0.1)
+
+    def fwd(ws, w, lo=None, hi=None, shape=args):
+        return L.spa_attn_fwd_union(p, p, p, p, p, ws, *shape, w, lo, hi, None)
+
+    def bwd(ws, w, lo=None, hi=None, shape=args):
+        return L.spa_attn_bwd_union(p, p, p, p, p, p, p, p, p, ws, *shape, w, lo, hi, None)
+
+    for call in (fwd, bwd):
+        assert call(p, 0) == spa.SPA_ERR_INVAL            # window must be >= 1
+        assert call(p, N + 1) == spa.SPA_ERR_INVAL        # and <= N
+        assert call(None, 8) == spa.SPA_ERR_INVAL         # workspace
+        assert call(_fake((1 << 20) + 16), 8) == spa.SPA_ERR_UNSUPPORTED  # 32-byte aligned
+        assert call(p, 8, shape=(B, H, N, 96, 0.1)) == spa.SPA_ERR_UNSUPPORTED
+        bad_lo = (ctypes.c_int32 * H)(0, 9, 5, 7)
+        bad_hi = (ctypes.c_int32 * H)(4, 3, 6, 300)     # reversed and out-of-range bands
+        assert call(p, 8, bad_lo, bad_hi) == spa.SPA_ERR_INVAL
+        # H = N with window 1: head 0's set is the single distance 0
+        assert call(p, 1, shape=(1, 16, 16, 64, 0.1)) == spa.SPA_ERR_UNSUPPORTED
+    assert L.spa_attn_bwd_union(p, p, p, p, p, p, None, p, p, p, *args, 8, None, None, None) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_union_workspace_bytes(1, 4, 256, 96) == 0
+    rows = 1 * 4 * 256
+    assert L.spa_attn_union_workspace_bytes(1, 4, 256, 64) == rows * 4 + 3 * rows * 64 * 2

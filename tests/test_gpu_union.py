@@ -1,0 +1,126 @@
+"""GPU parity of band-plus-shared-window attention (spa_attn_fwd_union /
+spa_attn_bwd_union through the C ABI) against the fp64 oracle's union
+entries, on the same seeded bf16 inputs.  Tolerances as in
+test_gpu_parity.py: |o - o_ref| <= 2e-2, |lse - lse_ref| <= 1e-3, each
+gradient max-abs error <= 5e-2 of the reference's max-abs value."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from head_partitioned_distance_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+O_TOL, LSE_TOL, GRAD_TOL = 2e-2, 1e-3, 5e-2
+
+
+@pytest.fixture(scope="module")
+def spa():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    from head_partitioned_distance_b200 import spa as mod
+    return mod
+
+
+def _f64(t):
+    return t.detach().to("cpu", torch.float64).numpy()
+
+
+def _check_grad(g, ref, name):
+    assert not np.isnan(g).any(), name
+    err = np.abs(g - ref).max()
+    assert err / np.abs(ref).max() <= GRAD_TOL, (name, err)
+
+
+def _gpu(spa, q, k, v, do, scale, window, lo=None, hi=None):
+    dev = torch.device("cuda:0")
+    qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
+    o, lse = spa.attention_forward_union(qd, kd, vd, window, scale, lo, hi)
+    dq, dk, dv = spa.attention_backward_union(qd, kd, vd, o, dod, lse, window, scale, lo, hi)
+    torch.cuda.synchronize()
+    assert spa.spa_device_status() == spa.SPA_OK
+    return {n: _f64(t) for n, t in (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+
+
+CASES = [
+    (1, 4, 600, 64, 1),      # window = the diagonal only
+    (1, 4, 600, 64, 100),    # window apart from every band but head 0's
+    (1, 4, 600, 64, 200),    # window overlapping head 1's band
+    (1, 4, 600, 64, 600),    # window covering every distance: dense causal
+    (2, 5, 777, 128, 37),
+    (1, 8, 1001, 64, 64),
+    (1, 3, 129, 128, 5),
+    (1, 32, 2048, 128, 256),
+]
+
+
+@pytest.mark.parametrize("B,H,N,d,w", CASES)
+def test_union_every_element(spa, B, H, N, d, w):
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=101 + N + w)
+    scale = 1 / math.sqrt(d)
+    got = _gpu(spa, q, k, v, do, scale, w)
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    o_ref, lse_ref = oracle.union_fwd(qf, kf, vf, scale, w)
+    assert np.isfinite(got["lse"]).all()  # distance 0 is in every set
+    assert np.abs(got["o"] - o_ref).max() <= O_TOL
+    assert np.abs(got["lse"] - lse_ref).max() <= LSE_TOL
+    for name, ref in zip(("dq", "dk", "dv"), oracle.union_bwd(qf, kf, vf, dof, scale, w)):
+        _check_grad(got[name], ref, name)
+
+
+def test_union_with_explicit_bands(spa):
+    B, H, N, d, w = 1, 4, 600, 64, 50
+    lo, hi = [0, 3, 257, 40], [1, 400, 300, 600]
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=77)
+    got = _gpu(spa, q, k, v, do, 0.125, w, lo, hi)
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    o_ref, lse_ref = oracle.union_fwd(qf, kf, vf, 0.125, w, np.array(lo), np.array(hi))
+    assert np.abs(got["o"] - o_ref).max() <= O_TOL
+    assert np.abs(got["lse"] - lse_ref).max() <= LSE_TOL
+    refs = oracle.union_bwd(qf, kf, vf, dof, 0.125, w, np.array(lo), np.array(hi))
+    for name, ref in zip(("dq", "dk", "dv"), refs):
+        _check_grad(got[name], ref, name)
+
+
+def test_union_full_size_sampled_rows(spa):
+    # the benchmark's union workload: B1 H32 N32768 d128, window 256
+    w = synth.WORKLOADS["b1_h32_n32768_d128"]
+    window = 256
+    q, k, v, do = synth.workload_inputs(w)
+    got = _gpu(spa, q, k, v, do, w.scale, window)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    lo, hi = oracle.bands(N, H)
+    per_head = [[0, window - 1, window, int(lo[h]), int(lo[h]) + 1, N - 1] for h in range(H)]
+    rows = synth.sample_rows(B, H, N, 32, seed=w.seed + 7, per_head=per_head)
+    key_rows = [N - 1, 0, window, (H - 1) * N + N - 1 - int(lo[H - 1]), 5 * N + 1000]
+    flat = lambda x: x.reshape(B * H * N, -1)
+    res = {n: ([], []) for n in ("o", "lse", "dq", "dk", "dv")}
+    for bh in sorted(set(r // N for r in rows) | set(r // N for r in key_rows)):
+        h = bh % H
+        sl = lambda t: _f64(t.reshape(B * H, N, d)[bh])[None, None]
+        qh, kh, vh, doh = sl(q), sl(k), sl(v), sl(do)
+        blo, bhi = lo[h:h + 1], hi[h:h + 1]
+        rs = [r % N for r in rows if r // N == bh]
+        if rs:
+            o_r, l_r = oracle.union_fwd_rows(qh, kh, vh, w.scale, window, rs, blo, bhi)
+            dq_r = oracle.union_bwd_dq_rows(qh, kh, vh, doh, w.scale, window, rs, blo, bhi)
+            idx = [bh * N + i for i in rs]
+            for n, g, r in (("o", flat(got["o"])[idx], o_r), ("dq", flat(got["dq"])[idx], dq_r),
+                            ("lse", got["lse"].reshape(-1)[idx], l_r)):
+                res[n][0].append(g)
+                res[n][1].append(r)
+        ks = [r % N for r in key_rows if r // N == bh]
+        if ks:
+            dk_r, dv_r = oracle.union_bwd_dkdv_rows(qh, kh, vh, doh, w.scale, window, ks, blo, bhi)
+            idx = [bh * N + j for j in ks]
+            for n, g, r in (("dk", flat(got["dk"])[idx], dk_r), ("dv", flat(got["dv"])[idx], dv_r)):
+                res[n][0].append(g)
+                res[n][1].append(r)
+    cat = lambda xs: np.concatenate(xs, axis=0)
+    assert np.abs(cat(res["o"][0]) - cat(res["o"][1])).max() <= O_TOL
+    assert np.abs(cat(res["lse"][0]) - cat(res["lse"][1])).max() <= LSE_TOL
+    for name in ("dq", "dk", "dv"):
+        _check_grad(cat(res[name][0]), cat(res[name][1]), name)

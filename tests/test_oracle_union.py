@@ -1,7 +1,7 @@
 """Pins for the oracle's band-plus-shared-window attention (each head attends
 to its band [lo_h, hi_h) and to the distances [0, w) that every head shares;
-a reading of the "local sharing" that Figure 2(b) of "Making Every Head
-Count" says the EBALL ablation removes).  The checks reduce it to the band
+a reading of the local sharing that the EBALL ablation of "Making Every Head
+Count", Figure 2(b), takes out).  The checks reduce it to the band
 oracle (w = 0), to dense causal attention (w >= N), to torch's fp64
 scaled_dot_product_attention with the union written as an explicit mask
 (forward and autograd backward), and to the log-sum-exp merge of its two
@@ -97,11 +97,18 @@ def test_disjoint_parts_merge_through_their_lse():
         np.testing.assert_allclose(o[0, h], w1 * o1[0, h] + w2 * o2[0, h], atol=1e-12, rtol=0)
 
 
-def test_row_entry_matches_full_tensor():
+def test_row_entries_match_full_tensor():
     B, H, N, d = 2, 3, 40, 4
-    q, k, v = (_rand((B, H, N, d), s) for s in (15, 16, 17))
+    q, k, v, do = (_rand((B, H, N, d), s) for s in (15, 16, 17, 18))
     o, lse = oracle.union_fwd(q, k, v, 0.5, 7)
+    dq, dk, dv = oracle.union_bwd(q, k, v, do, 0.5, 7)
     rows = list(range(0, B * H * N, 5)) + [B * H * N - 1]
+    flat = lambda t: t.reshape(B * H * N, -1)
     orow, lrow = oracle.union_fwd_rows(q, k, v, 0.5, 7, rows)
-    np.testing.assert_array_equal(orow, o.reshape(B * H * N, d)[rows])
+    np.testing.assert_array_equal(orow, flat(o)[rows])
     np.testing.assert_array_equal(lrow, lse.reshape(-1)[rows])
+    np.testing.assert_allclose(oracle.union_bwd_dq_rows(q, k, v, do, 0.5, 7, rows), flat(dq)[rows],
+                               atol=1e-12, rtol=0)
+    dkr, dvr = oracle.union_bwd_dkdv_rows(q, k, v, do, 0.5, 7, rows)
+    np.testing.assert_allclose(dkr, flat(dk)[rows], atol=1e-12, rtol=0)
+    np.testing.assert_allclose(dvr, flat(dv)[rows], atol=1e-12, rtol=0)
