@@ -62,6 +62,18 @@ def workload_pairs(N: int, bands) -> int:
     return sum(band_pairs_prefix(N, lo, hi) for lo, hi in zip(*bands))
 
 
+def union_pairs(N: int, window: int, bands) -> int:
+    """Pairs of the band-plus-shared-window sets: distances [0, window) and
+    [lo_h, hi_h), each distance counted once."""
+    total = 0
+    for lo, hi in zip(*bands):
+        total += band_pairs_prefix(N, 0, window) + band_pairs_prefix(N, lo, hi)
+        a, b = max(0, lo), min(window, hi)
+        if b > a:
+            total -= band_pairs_prefix(N, a, b)
+    return total
+
+
 def kernel_work(w, pairs: int):
     """Algorithmic work per launch of each kernel (FLOPs over permitted pairs,
     or bytes for the row-sum kernel)."""
@@ -228,6 +240,34 @@ def oracle_sample(w, bands, prefix_rows: int):
     desc = (f"oracle spa_fwd + spa_bwd (fp64, OpenMP) on head 0, query rows [0, {prefix_rows}) "
             f"of the {w.name} workload (band [{lo[0]}, {hi[0]}), d={w.d}); {pairs} pairs")
     return 14 * w.d * pairs, secs, oracle.num_threads(), desc
+
+
+def oracle_union_sample(w, bands, window: int, prefix_rows: int):
+    """The union oracle's forward + backward on a causal prefix of head 1 of
+    batch 0 (its band and the window do not touch there).  Returns (useful
+    flops, seconds, threads, description)."""
+    import oracle
+    q, k, v, do = synth.make_inputs(1, 1, prefix_rows, w.d, seed=w.seed)
+    f = lambda t: t.to(torch.float64).numpy()
+    h = 1 if len(bands[0]) > 1 else 0
+    lo, hi = [bands[0][h]], [bands[1][h]]
+    t0 = time.perf_counter()
+    oracle.union_fwd(f(q), f(k), f(v), w.scale, window, lo, hi)
+    oracle.union_bwd(f(q), f(k), f(v), f(do), w.scale, window, lo, hi)
+    secs = time.perf_counter() - t0
+    pairs = union_pairs(prefix_rows, window, (lo, hi))
+    desc = (f"oracle union_fwd + union_bwd (fp64, OpenMP) on head {h}, query rows [0, {prefix_rows}) of the "
+            f"{w.name} workload (band [{lo[0]}, {hi[0]}), window {window}, d={w.d}); {pairs} pairs")
+    return 14 * w.d * pairs, secs, oracle.num_threads(), desc
+
+
+def calibrate_union_prefix(w, bands, window: int, target_s: float, start: int = 1024):
+    P = min(start, w.N)
+    while True:
+        fl, secs, cores, desc = oracle_union_sample(w, bands, window, P)
+        if secs >= target_s / 2 or P >= w.N:
+            return P, fl, secs, cores, desc
+        P = min(2 * P, w.N)
 
 
 def calibrate_prefix(w, bands, target_s: float, start: int = 256):
@@ -436,6 +476,63 @@ def run_decode(args):
 
 
 # --------------------------------------------------------------------- GPU arm
+E2E_SCHEDULE = ("H2D, compute and D2H on three streams with two device buffer sets: each step's copies "
+                "overlap its neighbours' compute and copies")
+
+
+def pipelined_e2e(device, stream, host, dev0, out_names, compute, E, dist):
+    """End-to-end time of E steps through the public API with host buffers.
+    Every step copies its inputs (``host``: name -> CPU tensor, same names in
+    ``dev0``) in from pinned host memory and its outputs (``out_names``) back.
+    As a caller streaming batches would, the copies of neighbouring steps
+    overlap the compute: H2D, compute and D2H run on three streams over two
+    device buffer sets, so PCIe carries both directions at once.  ``compute``
+    launches one step on a buffer set (a dict like ``dev0``) on ``stream``.
+    Returns (max-over-ranks ms for the E steps, H2D bytes, D2H bytes per step)."""
+    pin = {n: t.pin_memory() for n, t in host.items()}
+    out_h = {n: torch.empty(dev0[n].shape, dtype=dev0[n].dtype).pin_memory() for n in out_names}
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_h.values())
+    sets = [dev0, {n: torch.empty_like(t) for n, t in dev0.items()}]
+    s_h2d, s_d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    ev = lambda: torch.cuda.Event()
+    h2d_done, cmp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+
+    def run(steps):
+        for s_ in range(steps):
+            x = s_ % 2
+            S = sets[x]
+            if s_ >= 2:
+                s_h2d.wait_event(cmp_done[x])  # step s - 2 has read this set's inputs
+            with torch.cuda.stream(s_h2d):
+                for n in pin:
+                    S[n].copy_(pin[n], non_blocking=True)
+                h2d_done[x].record(s_h2d)
+            stream.wait_event(h2d_done[x])
+            if s_ >= 2:
+                stream.wait_event(d2h_done[x])  # step s - 2's outputs have left this set
+            compute(S)
+            cmp_done[x].record(stream)
+            s_d2h.wait_event(cmp_done[x])
+            with torch.cuda.stream(s_d2h):
+                for n in out_h:
+                    out_h[n].copy_(S[n], non_blocking=True)
+                d2h_done[x].record(s_d2h)
+
+    run(2)
+    torch.cuda.synchronize(device)
+    if dist:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(s_h2d)
+    stream.wait_event(e0)
+    run(E)
+    s_d2h.wait_event(cmp_done[(E - 1) % 2])
+    e1.record(s_d2h)
+    torch.cuda.synchronize(device)
+    return reduce_max(e0.elapsed_time(e1), device), h2d, d2h
+
+
 def run_spa(args):
     from head_partitioned_distance_b200 import spa
 
@@ -512,58 +609,16 @@ def run_spa(args):
     value = aggregate(useful, K, world, max_ms)
 
     # ------------------------------------------------ end to end, host buffers
-    # Every step copies its inputs in from pinned host memory and its
-    # outputs back.  As a caller streaming batches would, the copies of
-    # neighbouring steps overlap the compute: H2D, compute and D2H run on
-    # three streams over two device buffer sets, so PCIe carries both
-    # directions at once.
     E = max(4, min(16, K))
-    pin = {n: t.pin_memory() for n, t in host.items()}
-    out_h = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in
-             (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
-    h2d = sum(t.numel() * t.element_size() for t in pin.values())
-    d2h = sum(t.numel() * t.element_size() for t in out_h.values())
-    sets = [dict(q=qd, k=kd, v=vd, do=dod, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)]
-    sets.append({n: torch.empty_like(t) for n, t in sets[0].items()})
-    s_h2d, s_d2h = torch.cuda.Stream(device), torch.cuda.Stream(device)
-    ev = lambda: torch.cuda.Event()
-    h2d_done, cmp_done, d2h_done = [ev(), ev()], [ev(), ev()], [ev(), ev()]
+    dev0 = dict(q=qd, k=kd, v=vd, do=dod, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)
 
-    def e2e_run(steps):
-        for s_ in range(steps):
-            x = s_ % 2
-            S = sets[x]
-            if s_ >= 2:
-                s_h2d.wait_event(cmp_done[x])  # step s - 2 has read this set's inputs
-            with torch.cuda.stream(s_h2d):
-                for n in ("q", "k", "v", "do"):
-                    S[n].copy_(pin[n], non_blocking=True)
-                h2d_done[x].record(s_h2d)
-            stream.wait_event(h2d_done[x])
-            if s_ >= 2:
-                stream.wait_event(d2h_done[x])  # step s - 2's outputs have left this set
-            spa.spa_attn_fwd(S["q"], S["k"], S["v"], S["o"], S["lse"], scale, stream=stream)
-            spa.spa_attn_bwd(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"],
-                             S["ws"], scale, stream=stream)
-            cmp_done[x].record(stream)
-            s_d2h.wait_event(cmp_done[x])
-            with torch.cuda.stream(s_d2h):
-                for n in ("o", "lse", "dq", "dk", "dv"):
-                    out_h[n].copy_(S[n], non_blocking=True)
-                d2h_done[x].record(s_d2h)
+    def compute(S):
+        spa.spa_attn_fwd(S["q"], S["k"], S["v"], S["o"], S["lse"], scale, stream=stream)
+        spa.spa_attn_bwd(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"],
+                         S["ws"], scale, stream=stream)
 
-    e2e_run(2)
-    torch.cuda.synchronize(device)
-    if dist:
-        dist.barrier()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(s_h2d)
-    stream.wait_event(e0)
-    e2e_run(E)
-    s_d2h.wait_event(cmp_done[(E - 1) % 2])
-    e1.record(s_d2h)
-    torch.cuda.synchronize(device)
-    e2e_ms = reduce_max(e0.elapsed_time(e1), device)
+    e2e_ms, h2d, d2h = pipelined_e2e(device, stream, host, dev0, ("o", "lse", "dq", "dk", "dv"), compute, E,
+                                     dist)
     e2e_value = aggregate(useful, E, world, e2e_ms)
     if spa.spa_device_status(stream) != spa.SPA_OK:
         raise SystemExit("device status not OK after the end-to-end region")
@@ -619,9 +674,170 @@ def run_spa(args):
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": e2e_ms / E,
-                    "schedule": "H2D, compute and D2H on three streams with two device buffer sets: "
-                                "each step's copies overlap its neighbours' compute and copies"},
+                    "schedule": E2E_SCHEDULE},
             "gpu_launches": len(KERNELS) * K,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+# one union step, launch by launch: (name, what it runs)
+UNION_LAUNCHES = ("fwd part 1", "fwd part 2", "merge", "dq+D part 1", "dk/dv part 1", "dq part 2",
+                  "dk/dv part 2", "add grads")
+UNION_KERNEL_OF = {"fwd part 1": "spa_fwd_kernel", "fwd part 2": "spa_fwd_kernel",
+                   "merge": "spa_union_merge_kernel", "dq+D part 1": "spa_bwd_dq_kernel",
+                   "dk/dv part 1": "spa_bwd_dkdv_kernel", "dq part 2": "spa_bwd_dq_kernel",
+                   "dk/dv part 2": "spa_bwd_dkdv_kernel", "add grads": "spa_add3_bf16_kernel"}
+
+
+def run_union(args):
+    """Band plus a local window [0, W) shared by every head (spa_attn_fwd_union
+    + spa_attn_bwd_union) on the same workload; useful FLOPs over the union's
+    pairs."""
+    from head_partitioned_distance_b200 import spa
+
+    rank, local, world = dist_setup()
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device (B200); there is no CPU path")
+    dist = dist_init("nccl", local) if world > 1 else None
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    w = synth.WORKLOADS[args.workload]
+    B, H, N, d = w.B, w.H, w.N, w.d
+    W = args.union
+    bands = spa.spa_band_bounds(N, H)
+    a1, b1, a2, b2 = spa.spa_union_parts(N, H, W)
+    pairs = B * union_pairs(N, W, bands)
+    pairs1 = B * workload_pairs(N, (a1, b1))
+    pairs2 = B * workload_pairs(N, (a2, b2))
+    assert pairs1 + pairs2 == pairs
+    useful = 14 * d * pairs
+
+    q, k, v, do = synth.make_inputs(B, H, N, d, w.seed + 7919 * rank, w.qkv_mult, w.rms_qk, w.do_mult)
+    host = {"q": q, "k": k, "v": v, "do": do}
+    qd, kd, vd, dod = (t.to(device) for t in (q, k, v, do))
+    o = torch.empty_like(qd)
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=device)
+    dq, dk, dv = torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd)
+    ws = torch.empty(spa.spa_attn_union_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32, device=device)
+    stream = torch.cuda.current_stream(device)
+    scale = w.scale
+
+    def step(S):
+        spa.spa_attn_fwd_union(S["q"], S["k"], S["v"], S["o"], S["lse"], S["ws"], scale, W, stream=stream)
+        spa.spa_attn_bwd_union(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"],
+                               S["ws"], scale, W, stream=stream)
+
+    dev0 = dict(q=qd, k=kd, v=vd, do=dod, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)
+    for _ in range(args.warmup):
+        step(dev0)
+    torch.cuda.synchronize(device)
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after warm-up")
+
+    visible = os.environ.get("CUDA_VISIBLE_DEVICES")
+    sampler = ClockSampler(visible.split(",")[local] if visible else local)
+    sampler.start()
+    K = args.steps
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(device)
+    sampler.mark_start()
+    t0.record(stream)
+    for _ in range(K):
+        step(dev0)
+    t1.record(stream)
+    torch.cuda.synchronize(device)
+    sampler.mark_end()
+    if dist:
+        dist.barrier()
+    clocks = sampler.stop()
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after the timed region")
+    max_ms = reduce_max(t0.elapsed_time(t1), device)
+    value = aggregate(useful, K, world, max_ms)
+
+    # the same launches one public call at a time, with an event after each:
+    # per-launch durations for the shares and the roofline
+    o2 = torch.empty_like(qd)
+    lse2 = torch.empty_like(lse)
+    dq2, dk2, dv2 = torch.empty_like(qd), torch.empty_like(qd), torch.empty_like(qd)
+    wsb = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=device)
+    calls = [
+        lambda: spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, a1, b1, stream=stream),
+        lambda: spa.spa_attn_fwd(qd, kd, vd, o2, lse2, scale, a2, b2, stream=stream),
+        lambda: spa.spa_attn_union_merge(o, lse, o2, lse2, stream=stream),
+        lambda: spa.spa_attn_bwd_dq_delta(qd, kd, vd, o, dod, lse, wsb, dq, scale, a1, b1, stream=stream),
+        lambda: spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, wsb, dk, dv, scale, a1, b1, stream=stream),
+        lambda: spa.spa_attn_bwd_dq(qd, kd, vd, dod, lse, wsb, dq2, scale, a2, b2, stream=stream),
+        lambda: spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, wsb, dk2, dv2, scale, a2, b2, stream=stream),
+        lambda: spa.spa_attn_union_add_grads(dq, dk, dv, dq2, dk2, dv2, stream=stream),
+    ]
+    Kd = max(3, min(K, 20))
+    for _ in range(2):
+        for c in calls:
+            c()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(calls) + 1)] for _ in range(Kd)]
+    for s_ in range(Kd):
+        evs[s_][0].record(stream)
+        for i, c in enumerate(calls):
+            c()
+            evs[s_][i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after the launch-by-launch pass")
+    launch_ms = {n: sum(e[i].elapsed_time(e[i + 1]) for e in evs) / Kd for i, n in enumerate(UNION_LAUNCHES)}
+    step_ms = sum(launch_ms.values())
+
+    E = max(4, min(16, K))
+    e2e_ms, h2d, d2h = pipelined_e2e(device, stream, host, dev0, ("o", "lse", "dq", "dk", "dv"), step, E, dist)
+    e2e_value = aggregate(useful, E, world, e2e_ms)
+    if spa.spa_device_status(stream) != spa.SPA_OK:
+        raise SystemExit("device status not OK after the end-to-end region")
+
+    if rank == 0:
+        peaks, peak_src = load_peaks()
+        kern = {}
+        for name in sorted(set(UNION_KERNEL_OF.values())):
+            ms = sum(launch_ms[n] for n in UNION_LAUNCHES if UNION_KERNEL_OF[n] == name)
+            kern[name] = {"ms_per_step": ms, "share": ms / step_ms,
+                          "launches_per_step": sum(1 for n in UNION_LAUNCHES if UNION_KERNEL_OF[n] == name)}
+        # dominant kernel: the dK/dV pass, over both parts' pairs
+        dk_ms = kern["spa_bwd_dkdv_kernel"]["ms_per_step"]
+        achieved = 8 * d * pairs / (dk_ms * 1e-3) / 1e12
+        roofline = {"bound": "tensor", "achieved": achieved, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                    "frac": achieved / peaks["bf16_tflops"], "traffic": None, "kernel": "spa_bwd_dkdv_kernel",
+                    "per": "both launches of one step (parts 1 and 2): 8 d x union pairs over their summed time",
+                    "peak_source": f"{peak_src} (bf16_tflops burst)"}
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            P, fl, secs, cores, desc = calibrate_union_prefix(w, bands, W, args.cpu_seconds)
+            cpu = {"value": fl / secs / 1e12, "unit": UNIT, "cores": cores, "kind": "oracle",
+                   "sample": desc, "seconds": secs}
+        line = {
+            "metric": METRIC + " (band plus shared local window)", "value": value, "unit": UNIT,
+            "n_gpus": world, "steps": K, "warmup": args.warmup, "ms_per_step": max_ms / K,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic",
+            "pct_of_bf16_peak": 100.0 * value / world / peaks["bf16_tflops"],
+            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d,
+                       "bands": "balanced distance partitioning", "window": W,
+                       "parts": "two disjoint distance intervals per head (spa_union_parts)",
+                       "pairs_per_rank": pairs, "useful_flops_per_rank_step": useful,
+                       "l2": "no flush: q, k, v, dout are each larger than L2",
+                       "parallelism": f"{world} independent replicas (one batch each)"},
+            "roofline": roofline,
+            "kernels": kern,
+            "launches_ms": launch_ms,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "steps": E, "ms_per_step": e2e_ms / E, "schedule": E2E_SCHEDULE},
+            "gpu_launches": len(UNION_LAUNCHES) * K,
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -641,6 +857,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--union", type=int, default=0, metavar="W",
+                    help="time band plus a local window [0, W) shared by every head instead")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (one new token per sequence) instead of fwd+bwd")
     args = ap.parse_args(argv)
@@ -650,6 +868,8 @@ def main(argv=None):
         return run_reference(args)
     if args.decode:
         return run_decode(args)
+    if args.union:
+        return run_union(args)
     return run_spa(args)
 
 

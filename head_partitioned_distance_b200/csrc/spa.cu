@@ -380,6 +380,44 @@ UnionWs union_ws(void* ws, int64_t rows, int d) {
 
 int union_launch_status() { return cudaGetLastError() == cudaSuccess ? SPA_OK : SPA_ERR_CUDA; }
 
+int union_merge(void* o, float* lse, const void* o2, const float* lse2, int B, int H, int64_t N, int d,
+                void* stream) {
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  if (!o || !lse || !o2 || !lse2) return SPA_ERR_INVAL;
+  if (!aligned(o, 16) || !aligned(o2, 16) || !aligned(lse, 4) || !aligned(lse2, 4)) return SPA_ERR_UNSUPPORTED;
+  const int64_t rows = (int64_t)B * H * N;
+  const int64_t threads = rows * (d / 8);
+  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d == 64)
+    spa::spa_union_merge_kernel<64><<<blocks, 256, 0, s>>>(static_cast<uint16_t*>(o), lse,
+                                                           static_cast<const uint16_t*>(o2), lse2, rows);
+  else
+    spa::spa_union_merge_kernel<128><<<blocks, 256, 0, s>>>(static_cast<uint16_t*>(o), lse,
+                                                            static_cast<const uint16_t*>(o2), lse2, rows);
+  return union_launch_status();
+}
+
+int union_add_grads(void* dq, void* dk, void* dv, const void* dq2, const void* dk2, const void* dv2, int B, int H,
+                    int64_t N, int d, void* stream) {
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  for (const void* t : {(const void*)dq, (const void*)dk, (const void*)dv, dq2, dk2, dv2}) {
+    if (!t) return SPA_ERR_INVAL;
+    if (!aligned(t, 16)) return SPA_ERR_UNSUPPORTED;
+  }
+  int sms = 0;
+  if ((st = sm_count(&sms))) return st;
+  const int64_t n16 = (int64_t)B * H * N * d / 8;
+  const int64_t want = (3 * n16 + 255) / 256;
+  const unsigned blocks = (unsigned)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
+  spa::spa_add3_bf16_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint16_t*>(dq), static_cast<uint16_t*>(dk), static_cast<uint16_t*>(dv),
+      static_cast<const uint16_t*>(dq2), static_cast<const uint16_t*>(dk2), static_cast<const uint16_t*>(dv2), n16);
+  return union_launch_status();
+}
+
 struct BandArgs {
   int32_t lo[spa::kMaxHeads];
   int32_t hi[spa::kMaxHeads];
@@ -656,6 +694,23 @@ int spa_attn_decode(const void* q, const void* k, const void* v, const int32_t* 
   return launch_status();
 }
 
+int spa_union_parts(int64_t N, int H, int64_t window, const int32_t* lo, const int32_t* hi, int32_t* a1,
+                    int32_t* b1, int32_t* a2, int32_t* b2) {
+  if (H < 1 || H > spa::kMaxHeads || N < 1 || N > 2147483647LL) return SPA_ERR_INVAL;
+  if (!a1 || !b1 || !a2 || !b2) return SPA_ERR_INVAL;
+  static UnionParts zero{};
+  UnionParts u = zero;
+  const int st = union_parts(H, N, window, lo, hi, u);
+  if (st) return st;
+  for (int h = 0; h < H; ++h) {
+    a1[h] = u.a1[h];
+    b1[h] = u.b1[h];
+    a2[h] = u.a2[h];
+    b2[h] = u.b2[h];
+  }
+  return SPA_OK;
+}
+
 size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d) {
   if (check_shape(B, H, N, d)) return 0;
   const size_t rows = (size_t)B * H * N;
@@ -676,14 +731,7 @@ int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, flo
   UnionWs w = union_ws(workspace, rows, d);
   if ((st = fwd_entry(q, k, v, o, lse, B, H, N, d, scale, u.a1, u.b1, stream))) return st;
   if ((st = fwd_entry(q, k, v, w.t[0], w.vec, B, H, N, d, scale, u.a2, u.b2, stream))) return st;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const int64_t threads = rows * (d / 8);
-  const unsigned blocks = (unsigned)((threads + 255) / 256);
-  if (d == 64)
-    spa::spa_union_merge_kernel<64><<<blocks, 256, 0, s>>>(static_cast<uint16_t*>(o), lse, w.t[0], w.vec, rows);
-  else
-    spa::spa_union_merge_kernel<128><<<blocks, 256, 0, s>>>(static_cast<uint16_t*>(o), lse, w.t[0], w.vec, rows);
-  return union_launch_status();
+  return union_merge(o, lse, w.t[0], w.vec, B, H, N, d, stream);
 }
 
 int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -708,15 +756,17 @@ int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* 
       (st = bwd_entry(q, k, v, o, dout, lse, nullptr, w.t[1], w.t[2], w.vec, B, H, N, d, scale, u.a2, u.b2,
                       stream, kStepDkDv)))
     return st;
-  int sms = 0;
-  if ((st = sm_count(&sms))) return st;
-  const int64_t n16 = rows * d / 8;
-  const int64_t want = (3 * n16 + 255) / 256;
-  const unsigned blocks = (unsigned)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
-  spa::spa_add3_bf16_kernel<<<blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(
-      static_cast<uint16_t*>(dq), static_cast<uint16_t*>(dk), static_cast<uint16_t*>(dv), w.t[0], w.t[1], w.t[2],
-      n16);
-  return union_launch_status();
+  return union_add_grads(dq, dk, dv, w.t[0], w.t[1], w.t[2], B, H, N, d, stream);
+}
+
+int spa_attn_union_merge(void* o, float* lse, const void* o2, const float* lse2, int B, int H, int64_t N, int d,
+                         void* stream) {
+  return union_merge(o, lse, o2, lse2, B, H, N, d, stream);
+}
+
+int spa_attn_union_add_grads(void* dq, void* dk, void* dv, const void* dq2, const void* dk2, const void* dv2,
+                             int B, int H, int64_t N, int d, void* stream) {
+  return union_add_grads(dq, dk, dv, dq2, dk2, dv2, B, H, N, d, stream);
 }
 
 int spa_device_status(void* stream) {

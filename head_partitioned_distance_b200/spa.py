@@ -49,6 +49,9 @@ EXPORTS = {
     "spa_attn_decode": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_noalloc": ([_vp] * 9 + [_int, _int, _i64, _int, _f32, _vp], _int),
     "spa_attn_union_workspace_bytes": ([_int, _int, _i64, _int], ctypes.c_size_t),
+    "spa_union_parts": ([_i64, _int, _i64, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p], _int),
+    "spa_attn_union_merge": ([_vp] * 4 + [_int, _int, _i64, _int, _vp], _int),
+    "spa_attn_union_add_grads": ([_vp] * 6 + [_int, _int, _i64, _int, _vp], _int),
     "spa_attn_fwd_union": ([_vp] * 6 + [_int, _int, _i64, _int, _f32, _i64, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_union": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i64, _i32p, _i32p, _vp], _int),
     "spa_tile_schedule": ([_i64, _int, _i32p, _i32p, _int, _int, _i32p, _i32p, _u8p, _i32p, _i32p],
@@ -339,6 +342,16 @@ def spa_attn_union_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
     return int(_lib.spa_attn_union_workspace_bytes(B, H, N, d))
 
 
+def spa_union_parts(N: int, H: int, window: int, lo=None, hi=None):
+    """The two disjoint distance intervals per head that the union calls run:
+    returns (a1, b1, a2, b2), lists of H ints."""
+    out = [(ctypes.c_int32 * H)() for _ in range(4)]
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    _check(_lib.spa_union_parts(N, H, int(window), lo_a, hi_a, *out), "spa_union_parts")
+    return tuple(list(a) for a in out)
+
+
 def _union_ws(workspace, B, H, N, d):
     need = spa_attn_union_workspace_bytes(B, H, N, d)
     if not workspace.is_cuda or workspace.numel() * workspace.element_size() < need:
@@ -400,3 +413,26 @@ def attention_backward_union(q, k, v, o, dout, lse, window: int, scale=None, lo=
     scale = d ** -0.5 if scale is None else scale
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     return spa_attn_bwd_union(q, k, v, o, dout, lse, dq, dk, dv, _union_workspace(q), scale, window, lo, hi)
+
+
+def spa_attn_union_merge(o, lse, o2, lse2, stream=None):
+    """(o, lse) <- softmax over the union of two disjoint parts' (o, lse), (o2, lse2)."""
+    B, H, N, d = _dims(o)
+    for t, n in ((o, "o"), (o2, "o2")):
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    for t, n in ((lse, "lse"), (lse2, "lse2")):
+        _need(t, (B, H, N), torch.float32, n)
+    _check(_lib.spa_attn_union_merge(o.data_ptr(), lse.data_ptr(), o2.data_ptr(), lse2.data_ptr(), B, H, N, d,
+                                     _stream_ptr(stream)), "spa_attn_union_merge")
+    return o, lse
+
+
+def spa_attn_union_add_grads(dq, dk, dv, dq2, dk2, dv2, stream=None):
+    """dq += dq2, dk += dk2, dv += dv2 (bf16)."""
+    B, H, N, d = _dims(dq)
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv"), (dq2, "dq2"), (dk2, "dk2"), (dv2, "dv2")):
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    _check(_lib.spa_attn_union_add_grads(dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), dq2.data_ptr(),
+                                         dk2.data_ptr(), dv2.data_ptr(), B, H, N, d, _stream_ptr(stream)),
+           "spa_attn_union_add_grads")
+    return dq, dk, dv

@@ -243,6 +243,28 @@ SPA_API int spa_attn_decode(const void* q, const void* k, const void* v, const i
  * calls reject.
  */
 SPA_API size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d);
+/* The split the two union calls use, on the host: head h's set is the
+ * distances [a1[h], b1[h]) u [a2[h], b2[h]), disjoint and non-empty -- the
+ * window and the band when window < lo_h, else the two halves of
+ * [0, max(window, hi_h)).  a1, b1, a2, b2: HOST arrays of H int32.  Same
+ * argument rules and errors as spa_attn_fwd_union's window and bands. */
+SPA_API int spa_union_parts(int64_t N, int H, int64_t window, const int32_t* lo, const int32_t* hi,
+                            int32_t* a1, int32_t* b1, int32_t* a2, int32_t* b2);
+/* The two steps the union calls add to the band kernels, callable alone
+ * (with spa_union_parts and the band entry points they make up the union
+ * calls launch by launch):
+ *  spa_attn_union_merge: o, lse (part 1, DEVICE, overwritten) and o2, lse2
+ *    (part 2, DEVICE) -> softmax over the union of the two disjoint sets:
+ *    L = log(e^lse + e^lse2), o = e^(lse - L) o + e^(lse2 - L) o2, lse = L
+ *    (a row empty in both parts stays o = 0, lse = -inf).
+ *  spa_attn_union_add_grads: dq += dq2, dk += dk2, dv += dv2 (DEVICE bf16
+ *    [B][H][N][d], summed in fp32 and rounded once).
+ * Tensors 16-byte aligned (lse, lse2: 4).  SPA_ERR_INVAL for null pointers or
+ * bad sizes, SPA_ERR_UNSUPPORTED as for spa_attn_fwd. */
+SPA_API int spa_attn_union_merge(void* o, float* lse, const void* o2, const float* lse2, int B, int H,
+                                 int64_t N, int d, void* stream);
+SPA_API int spa_attn_union_add_grads(void* dq, void* dk, void* dv, const void* dq2, const void* dk2,
+                                     const void* dv2, int B, int H, int64_t N, int d, void* stream);
 SPA_API int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, float* lse,
                                void* workspace, int B, int H, int64_t N, int d, float scale,
                                int64_t window, const int32_t* lo, const int32_t* hi, void* stream);

@@ -213,6 +213,26 @@ def test_union_entry_points_reject_bad_arguments_before_any_launch():
         # H = N with window 1: head 0's set is the single distance 0
         assert call(p, 1, shape=(1, 16, 16, 64, 0.1)) == spa.SPA_ERR_UNSUPPORTED
     assert L.spa_attn_bwd_union(p, p, p, p, p, p, None, p, p, p, *args, 8, None, None, None) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_union_merge(p, p, None, p, *args[:4], None) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_union_merge(p, p, _fake((1 << 20) + 8), p, *args[:4], None) == spa.SPA_ERR_UNSUPPORTED
+    assert L.spa_attn_union_merge(p, p, p, p, 1, 4, 256, 96, None) == spa.SPA_ERR_UNSUPPORTED
+    assert L.spa_attn_union_add_grads(p, p, p, p, None, p, *args[:4], None) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_union_add_grads(p, p, p, p, p, _fake((1 << 20) + 4), *args[:4], None) == \
+        spa.SPA_ERR_UNSUPPORTED
     assert L.spa_attn_union_workspace_bytes(1, 4, 256, 96) == 0
     rows = 1 * 4 * 256
     assert L.spa_attn_union_workspace_bytes(1, 4, 256, 64) == rows * 4 + 3 * rows * 64 * 2
+
+
+@pytest.mark.parametrize("N,H,w", [(600, 4, 100), (600, 4, 200), (600, 4, 600), (777, 5, 37), (32768, 32, 256),
+                                   (16, 16, 2), (1001, 8, 1)])
+def test_union_parts_split_each_head_into_two_disjoint_intervals(N, H, w):
+    a1, b1, a2, b2 = spa.spa_union_parts(N, H, w)
+    lo, hi = oracle.bands(N, H)
+    for h in range(H):
+        want = set(range(0, w)) | set(range(int(lo[h]), int(hi[h])))
+        p1, p2 = set(range(a1[h], b1[h])), set(range(a2[h], b2[h]))
+        assert p1 and p2 and not (p1 & p2)
+        assert p1 | p2 == want
+    with pytest.raises(spa.SpaError):
+        spa.spa_union_parts(16, 16, 1)  # head 0 is the single distance 0

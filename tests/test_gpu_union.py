@@ -124,3 +124,30 @@ def test_union_full_size_sampled_rows(spa):
     assert np.abs(cat(res["lse"][0]) - cat(res["lse"][1])).max() <= LSE_TOL
     for name in ("dq", "dk", "dv"):
         _check_grad(cat(res[name][0]), cat(res[name][1]), name)
+
+
+def test_launch_by_launch_composition_equals_the_union_calls(spa):
+    # spa_union_parts + the band entry points + the merge and gradient-sum
+    # steps, called one by one, are exactly what the two union calls launch
+    B, H, N, d, w = 1, 8, 1001, 64, 64
+    q, k, v, do = (t.to("cuda:0") for t in synth.make_inputs(B, H, N, d, seed=5))
+    scale = 0.125
+    o, lse = spa.attention_forward_union(q, k, v, w, scale)
+    dq, dk, dv = spa.attention_backward_union(q, k, v, o, do, lse, w, scale)
+    a1, b1, a2, b2 = spa.spa_union_parts(N, H, w)
+    o1, l1 = spa.attention_forward(q, k, v, scale, a1, b1)
+    o2, l2 = spa.attention_forward(q, k, v, scale, a2, b2)
+    spa.spa_attn_union_merge(o1, l1, o2, l2)
+    ws = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device="cuda:0")
+    g1 = [torch.empty_like(q) for _ in range(3)]
+    g2 = [torch.empty_like(q) for _ in range(3)]
+    spa.spa_attn_bwd_dq_delta(q, k, v, o1, do, l1, ws, g1[0], scale, a1, b1)
+    spa.spa_attn_bwd_dkdv(q, k, v, do, l1, ws, g1[1], g1[2], scale, a1, b1)
+    spa.spa_attn_bwd_dq(q, k, v, do, l1, ws, g2[0], scale, a2, b2)
+    spa.spa_attn_bwd_dkdv(q, k, v, do, l1, ws, g2[1], g2[2], scale, a2, b2)
+    spa.spa_attn_union_add_grads(*g1, *g2)
+    torch.cuda.synchronize()
+    assert spa.spa_device_status() == spa.SPA_OK
+    assert torch.equal(o, o1) and torch.equal(lse, l1)
+    for a, b in zip((dq, dk, dv), g1):
+        assert torch.equal(a, b)
