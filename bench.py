@@ -2,10 +2,12 @@
 """Benchmark: SPAttention band-sparse attention, forward + backward, on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl spa|reference]
+                    [--decode | --union W]
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-spa_attn_fwd (1 kernel) then the three backward steps (row sums D, the dK/dV
-pass, the dQ pass).  Inputs are resident in HBM when the timed region starts;
+spa_attn_fwd (1 kernel) then the backward as two passes (the dQ pass, which
+also forms the row sums D, and the dK/dV pass).  Inputs are resident in HBM
+when the timed region starts;
 each of q, k, v, dout is larger than the 126 MB L2, so no flush is needed
 between steps.  The metric is useful TFLOP/s: 14 * d * (permitted pairs) per
 step (forward 4 d, backward 10 d per pair -- the two GEMMs of the forward and
@@ -19,6 +21,11 @@ barrier and the max of the timings.
 --impl reference times the fp64 CPU oracle (the slow, plain implementation the
 tests check against) on a bounded sample of the same workload and prints the
 same line with "impl": "reference".
+
+--decode times the decode step instead (one new token per sequence against a
+KV cache, HBM roofline); --union W times the band plus a local window [0, W)
+shared by every head (spa_attn_fwd_union + spa_attn_bwd_union), useful FLOPs
+over the union's pairs.
 """
 from __future__ import annotations
 
