@@ -147,7 +147,9 @@ __device__ __forceinline__ DkvUnit dkv_decode(int u, const AttnParams& p) {
   return U;
 }
 
-template <int D>
+// ACC: add dk, dv to what the outputs hold (spa_attn_bwd_dkdv_add) and leave
+// the keys no query reaches untouched.
+template <int D, bool ACC = false>
 __global__ void __launch_bounds__(384, 1)
     spa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -522,12 +524,26 @@ __global__ void __launch_bounds__(384, 1)
       // if w = 0, all of dK if w = 1).  It reads them from TMEM (which then
       // goes back to the MMA warp) and stages each as bf16 in its own 4 KB
       // slice of the staging tile (128-byte swizzle)
-      // for a bulk tensor store of a 32 x 64 box.
+      // for a bulk tensor store of a 32 x 64 box.  When adding to the
+      // outputs, the row's 64 columns of each are read while the last
+      // products finish, and added before the rounding.
+      constexpr int NJ = D / 64;
+      const int x0 = NJ == 2 ? 64 * w : 0;
+      uint4 old[ACC ? NJ : 1][8];
+      if constexpr (ACC) {
+#pragma unroll
+        for (int t = 0; t < NJ; ++t) {
+          const bool is_dk = NJ == 2 ? t == 1 : w == 1;
+          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(is_dk ? p.dk : p.dv) +
+                                                            ((int64_t)U.bh * N + j) * D + x0);
+#pragma unroll
+          for (int e = 0; e < 8; ++e)  // rows past N: -0, the identity of the sum
+            old[t][e] = j < N ? src[e] : make_uint4(0x80008000u, 0x80008000u, 0x80008000u, 0x80008000u);
+        }
+      }
       ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
       if (!ok) break;
       ptx::tc_fence_after();
-      constexpr int NJ = D / 64;
-      const int x0 = NJ == 2 ? 64 * w : 0;
       uint32_t pk[NJ][32];
 #pragma unroll
       for (int t = 0; t < NJ; ++t) {
@@ -542,10 +558,19 @@ __global__ void __launch_bounds__(384, 1)
           ptx::tc_fence_before();
           ptx::mbar_arrive(&bars->acc_free);
         }
+        if constexpr (ACC) {
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          pk[t][e] = ptx::pack_bf16x2(__uint_as_float(g[e / 16][(2 * e) % 32]) * mul,
-                                      __uint_as_float(g[e / 16][(2 * e) % 32 + 1]) * mul);
+          for (int e = 0; e < 32; ++e) {
+            const float2 o = ptx::bf16x2_to_float2(ptx::word_of(old[t][e / 4], e % 4));
+            pk[t][e] = ptx::pack_bf16x2(fmaf(__uint_as_float(g[e / 16][(2 * e) % 32]), mul, o.x),
+                                        fmaf(__uint_as_float(g[e / 16][(2 * e) % 32 + 1]), mul, o.y));
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e)
+            pk[t][e] = ptx::pack_bf16x2(__uint_as_float(g[e / 16][(2 * e) % 32]) * mul,
+                                        __uint_as_float(g[e / 16][(2 * e) % 32 + 1]) * mul);
+        }
       }
       const int wq = warp % 4;
       const uint32_t slice = (uint32_t)w * (C::BK * 128) + (uint32_t)wq * (32 * 128);
@@ -573,8 +598,9 @@ __global__ void __launch_bounds__(384, 1)
   }
 
   // ------------------------------------------------------------ keys no query reaches
+  // (left as they are when adding to the output)
   {
-    const int num_fill = p.B * p.fills_per_batch;
+    const int num_fill = ACC ? 0 : p.B * p.fills_per_batch;
     for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
       const int b = f / p.fills_per_batch;
       const int r = f % p.fills_per_batch;
@@ -678,7 +704,9 @@ __device__ __forceinline__ DqUnit dq_decode(int u, const AttnParams& p) {
   return U;
 }
 
-template <int D>
+// ACC: add dq to what the output holds (spa_attn_bwd_dq_add) and leave the
+// rows before the band untouched.
+template <int D, bool ACC = false>
 __global__ void __launch_bounds__(384, 1)
     spa_bwd_dq_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                       const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -1038,18 +1066,40 @@ __global__ void __launch_bounds__(384, 1)
         if (!ok) break;
       }
       // ---------------------------------------------------------- epilogue
-      ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
-      if (!ok) break;
-      ptx::tc_fence_after();
       uint16_t* grow = static_cast<uint16_t*>(p.dq) + ((int64_t)bh * N + i) * D;
       const float mul = p.scale;
+      if constexpr (ACC) {
+        // the half row already in the output is read while the last products
+        // finish
+        uint4 old[D / 16];
+        if (in) {
+#pragma unroll
+          for (int e = 0; e < D / 16; ++e) old[e] = reinterpret_cast<const uint4*>(grow + w * (D / 2))[e];
+        }
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int cc = 0; cc < D / 64; ++cc) {
+          const int c = w * (D / 2) + 32 * cc;
+          uint32_t g[32];
+          ptx::tmem_ld32(tmem + lane_base + C::TM_DQ + c, g);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(g);
+          if (in) ptx::store_row32_bf16_add(grow + c, g, mul, old + 4 * cc);
+        }
+      } else {
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->acc_done, (cacc++) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
 #pragma unroll 1
-      for (int c = w * (D / 2); c < (w + 1) * (D / 2); c += 32) {
-        uint32_t g[32];
-        ptx::tmem_ld32(tmem + lane_base + C::TM_DQ + c, g);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence(g);
-        if (in) ptx::store_row32_bf16(grow + c, g, mul);
+        for (int c = w * (D / 2); c < (w + 1) * (D / 2); c += 32) {
+          uint32_t g[32];
+          ptx::tmem_ld32(tmem + lane_base + C::TM_DQ + c, g);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(g);
+          if (in) ptx::store_row32_bf16(grow + c, g, mul);
+        }
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(&bars->acc_free);
@@ -1057,8 +1107,9 @@ __global__ void __launch_bounds__(384, 1)
   }
 
   // ------------------------------------------------------------ rows before their band
+  // (left as they are when adding to the output)
   {
-    const int num_fill = p.B * p.fills_per_batch;
+    const int num_fill = ACC ? 0 : p.B * p.fills_per_batch;
     for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
       const int b = f / p.fills_per_batch;
       const int r = f % p.fills_per_batch;

@@ -311,10 +311,30 @@ __device__ __forceinline__ void store_row32_bf16(uint16_t* dst, const uint32_t (
   st_global_v8(dst + 16, pk + 8);
 }
 
+// Word e (0..3) of a 16-byte vector, e a compile-time constant after unrolling.
+__device__ __forceinline__ uint32_t word_of(const uint4& v, int e) {
+  return e == 0 ? v.x : (e == 1 ? v.y : (e == 2 ? v.z : v.w));
+}
+
 // Two bf16 values packed in a 32-bit word (the lower address in the low
 // half) as floats: a bf16 is the upper half of the fp32 with the same value.
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t v) {
   return make_float2(__uint_as_float(v << 16), __uint_as_float(v & 0xffff0000u));
+}
+
+// 32 fp32 values times `mul`, each added to the bf16 value already at that
+// position (`old`: the 64 bytes at dst, read earlier), rounded once to bf16
+// and stored at `dst` (64 bytes, 32-byte aligned).
+__device__ __forceinline__ void store_row32_bf16_add(uint16_t* dst, const uint32_t (&g)[32], float mul,
+                                                     const uint4* old) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int e = 0; e < 16; ++e) {
+    const float2 o = bf16x2_to_float2(word_of(old[e / 4], e % 4));
+    pk[e] = pack_bf16x2(fmaf(__uint_as_float(g[2 * e]), mul, o.x), fmaf(__uint_as_float(g[2 * e + 1]), mul, o.y));
+  }
+  st_global_v8(dst, pk);
+  st_global_v8(dst + 16, pk + 8);
 }
 
 __device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c,

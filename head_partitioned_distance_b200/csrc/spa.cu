@@ -188,8 +188,17 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, A
 
 // Backward steps.  The full backward runs the dQ pass first, forming D there
 // (kStepDqDelta), then the dK/dV pass reading it; the separate D kernel
-// serves the three-step entry points.
-enum BwdStep { kStepDelta = 1, kStepDkDv = 2, kStepDq = 4, kStepDqDelta = 8, kStepAll = kStepDqDelta | kStepDkDv };
+// serves the three-step entry points.  kStepAccumulate makes the dQ and dK/dV
+// passes add to their outputs (the second part of the band-plus-window
+// backward).
+enum BwdStep {
+  kStepDelta = 1,
+  kStepDkDv = 2,
+  kStepDq = 4,
+  kStepDqDelta = 8,
+  kStepAccumulate = 16,
+  kStepAll = kStepDqDelta | kStepDkDv
+};
 
 template <int D>
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -197,7 +206,10 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
              cudaStream_t stream, int steps) {
   using KC = spa::DkvCfg<D>;
   using QC = spa::DqCfg<D>;
-  static std::atomic<uint64_t> prepared_kv{0}, prepared_q{0};
+  // one (prepared, register check) pair per kernel instantiation: [adding]
+  static std::atomic<uint64_t> prepared_kv[2], prepared_q[2];
+  static std::atomic<int> regs_kv[2], regs_q[2];
+  const bool acc = (steps & kStepAccumulate) != 0;
   const int64_t BH = (int64_t)p.B * p.H;
   int st;
   p.lse = const_cast<float*>(lse);
@@ -225,9 +237,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
         (st = make_map(&qo, fuse_d ? o : dout, p.N, BH, D, QC::BQ)))
       return st;
     p.o_in = fuse_d ? o : nullptr;
-    if ((st = prepare_kernel(spa::spa_bwd_dq_kernel<D>, QC::SMEM_BYTES, prepared_q))) return st;
-    static std::atomic<int> regs_q{0};
-    if ((st = check_regs(spa::spa_bwd_dq_kernel<D>, (int)QC::LAUNCH_REGS, regs_q))) return st;
+    auto* kernel_q = acc ? spa::spa_bwd_dq_kernel<D, true> : spa::spa_bwd_dq_kernel<D, false>;
+    if ((st = prepare_kernel(kernel_q, QC::SMEM_BYTES, prepared_q[acc]))) return st;
+    if ((st = check_regs(kernel_q, (int)QC::LAUNCH_REGS, regs_q[acc]))) return st;
     const int64_t nqt = (p.N + 127) / 128;
     if ((int64_t)p.B * p.H * nqt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
     if ((st = set_work_lists(
@@ -238,7 +250,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if ((st = sm_count(&sms))) return st;
     const int64_t units = (int64_t)p.B * upb;
     const unsigned grid = (unsigned)(units < sms ? units : sms);
-    spa::spa_bwd_dq_kernel<D><<<grid, QC::NTHREADS, QC::SMEM_BYTES, stream>>>(qq, qk, qv, qdo, qo, p);
+    kernel_q<<<grid, QC::NTHREADS, QC::SMEM_BYTES, stream>>>(qq, qk, qv, qdo, qo, p);
     if ((st = launch_status())) return st;
   }
   if (steps & kStepDkDv) {
@@ -250,9 +262,9 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
         (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)) ||
         (st = make_map(&kdk, dk, p.N, BH, D, 32)) || (st = make_map(&kdv, dv, p.N, BH, D, 32)))
       return st;
-    if ((st = prepare_kernel(spa::spa_bwd_dkdv_kernel<D>, KC::SMEM_BYTES, prepared_kv))) return st;
-    static std::atomic<int> regs_kv{0};
-    if ((st = check_regs(spa::spa_bwd_dkdv_kernel<D>, (int)KC::LAUNCH_REGS, regs_kv))) return st;
+    auto* kernel_kv = acc ? spa::spa_bwd_dkdv_kernel<D, true> : spa::spa_bwd_dkdv_kernel<D, false>;
+    if ((st = prepare_kernel(kernel_kv, KC::SMEM_BYTES, prepared_kv[acc]))) return st;
+    if ((st = check_regs(kernel_kv, (int)KC::LAUNCH_REGS, regs_kv[acc]))) return st;
     const int64_t nkt = (p.N + 127) / 128;
     if ((int64_t)p.B * p.H * nkt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
     if ((st = set_work_lists(
@@ -264,7 +276,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if ((st = sm_count(&sms))) return st;
     const int64_t units = (int64_t)p.B * upb;
     const unsigned grid = (unsigned)(units < sms ? units : sms);
-    spa::spa_bwd_dkdv_kernel<D><<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
+    kernel_kv<<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
     if ((st = launch_status())) return st;
   }
   return SPA_OK;
@@ -359,22 +371,18 @@ int union_parts(int H, int64_t N, int64_t window, const int32_t* lo, const int32
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Workspace of the union passes: fp32 [B H N] (lse of part 2, or D), then
-// three bf16 [B H N d] tensors (o of part 2, or dq, dk, dv of part 2).
+// Workspace of the union passes: fp32 [B H N] (lse of part 2 in the
+// forward, D in the backward), then bf16 [B H N d] (o of part 2).
 struct UnionWs {
   float* vec;
-  uint16_t* t[3];
+  uint16_t* o2;
 };
 
-UnionWs union_ws(void* ws, int64_t rows, int d) {
+UnionWs union_ws(void* ws, int64_t rows) {
   UnionWs w;
   uint8_t* b = static_cast<uint8_t*>(ws);
   w.vec = reinterpret_cast<float*>(b);
-  b += align256((size_t)rows * 4);
-  for (int i = 0; i < 3; ++i) {
-    w.t[i] = reinterpret_cast<uint16_t*>(b);
-    b += align256((size_t)rows * d * 2);
-  }
+  w.o2 = reinterpret_cast<uint16_t*>(b + align256((size_t)rows * 4));
   return w;
 }
 
@@ -561,6 +569,20 @@ int spa_attn_bwd_dq(const void* q, const void* k, const void* v, const void* dou
                    N, d, scale, lo, hi, stream, kStepDq);
 }
 
+int spa_attn_bwd_dkdv_add(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                          const void* workspace, void* dk, void* dv, int B, int H, int64_t N, int d,
+                          float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+  return bwd_entry(q, k, v, nullptr, dout, lse, nullptr, dk, dv, const_cast<void*>(workspace), B, H, N,
+                   d, scale, lo, hi, stream, kStepDkDv | kStepAccumulate);
+}
+
+int spa_attn_bwd_dq_add(const void* q, const void* k, const void* v, const void* dout, const float* lse,
+                        const void* workspace, void* dq, int B, int H, int64_t N, int d, float scale,
+                        const int32_t* lo, const int32_t* hi, void* stream) {
+  return bwd_entry(q, k, v, nullptr, dout, lse, dq, nullptr, nullptr, const_cast<void*>(workspace), B, H,
+                   N, d, scale, lo, hi, stream, kStepDq | kStepAccumulate);
+}
+
 int spa_attn_bwd_dq_delta(const void* q, const void* k, const void* v, const void* o, const void* dout,
                           const float* lse, void* workspace, void* dq, int B, int H, int64_t N, int d,
                           float scale, const int32_t* lo, const int32_t* hi, void* stream) {
@@ -714,7 +736,7 @@ int spa_union_parts(int64_t N, int H, int64_t window, const int32_t* lo, const i
 size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d) {
   if (check_shape(B, H, N, d)) return 0;
   const size_t rows = (size_t)B * H * N;
-  return align256(rows * 4) + 3 * align256(rows * (size_t)d * 2);
+  return align256(rows * 4) + align256(rows * (size_t)d * 2);
 }
 
 int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
@@ -728,10 +750,10 @@ int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, flo
   UnionParts u = zero;
   if ((st = union_parts(H, N, window, lo, hi, u))) return st;
   const int64_t rows = (int64_t)B * H * N;
-  UnionWs w = union_ws(workspace, rows, d);
+  UnionWs w = union_ws(workspace, rows);
   if ((st = fwd_entry(q, k, v, o, lse, B, H, N, d, scale, u.a1, u.b1, stream))) return st;
-  if ((st = fwd_entry(q, k, v, w.t[0], w.vec, B, H, N, d, scale, u.a2, u.b2, stream))) return st;
-  return union_merge(o, lse, w.t[0], w.vec, B, H, N, d, stream);
+  if ((st = fwd_entry(q, k, v, w.o2, w.vec, B, H, N, d, scale, u.a2, u.b2, stream))) return st;
+  return union_merge(o, lse, w.o2, w.vec, B, H, N, d, stream);
 }
 
 int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -745,18 +767,19 @@ int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* 
   UnionParts u = zero;
   if ((st = union_parts(H, N, window, lo, hi, u))) return st;
   const int64_t rows = (int64_t)B * H * N;
-  UnionWs w = union_ws(workspace, rows, d);
-  // part 1 starts at distance 0, so its dQ pass forms D for every row
+  UnionWs w = union_ws(workspace, rows);
+  // part 1 starts at distance 0, so its dQ pass forms D for every row; part
+  // 2's passes add their gradients to part 1's in their epilogues
   if ((st = bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, w.vec, B, H, N, d, scale, u.a1, u.b1,
                       stream, kStepDqDelta)) ||
       (st = bwd_entry(q, k, v, o, dout, lse, nullptr, dk, dv, w.vec, B, H, N, d, scale, u.a1, u.b1, stream,
                       kStepDkDv)) ||
-      (st = bwd_entry(q, k, v, o, dout, lse, w.t[0], nullptr, nullptr, w.vec, B, H, N, d, scale, u.a2, u.b2,
-                      stream, kStepDq)) ||
-      (st = bwd_entry(q, k, v, o, dout, lse, nullptr, w.t[1], w.t[2], w.vec, B, H, N, d, scale, u.a2, u.b2,
-                      stream, kStepDkDv)))
+      (st = bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, w.vec, B, H, N, d, scale, u.a2, u.b2,
+                      stream, kStepDq | kStepAccumulate)) ||
+      (st = bwd_entry(q, k, v, o, dout, lse, nullptr, dk, dv, w.vec, B, H, N, d, scale, u.a2, u.b2, stream,
+                      kStepDkDv | kStepAccumulate)))
     return st;
-  return union_add_grads(dq, dk, dv, w.t[0], w.t[1], w.t[2], B, H, N, d, stream);
+  return SPA_OK;
 }
 
 int spa_attn_union_merge(void* o, float* lse, const void* o2, const float* lse2, int B, int H, int64_t N, int d,

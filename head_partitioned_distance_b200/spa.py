@@ -45,6 +45,8 @@ EXPORTS = {
     "spa_attn_bwd_dkdv": ([_vp] * 8 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_dq": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_dq_delta": ([_vp] * 8 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
+    "spa_attn_bwd_dkdv_add": ([_vp] * 8 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
+    "spa_attn_bwd_dq_add": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_decode_workspace_bytes": ([_int, _int, _i64, _int, _i32p, _i32p], ctypes.c_size_t),
     "spa_attn_decode": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_noalloc": ([_vp] * 9 + [_int, _int, _i64, _int, _f32, _vp], _int),
@@ -208,6 +210,28 @@ def spa_attn_bwd_dq(q, k, v, dout, lse, workspace, dq, scale: float, lo=None, hi
     _check(_lib.spa_attn_bwd_dq(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
                                 lse.data_ptr(), workspace.data_ptr(), dq.data_ptr(), B, H, N, d, scale,
                                 lo_a, hi_a, _stream_ptr(stream)), "spa_attn_bwd_dq")
+
+
+def spa_attn_bwd_dkdv_add(q, k, v, dout, lse, workspace, dk, dv, scale: float, lo=None, hi=None,
+                          stream=None):
+    """The dk/dv pass adding to dk, dv instead of overwriting them."""
+    B, H, N, d = _dims(q)
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    _check(_lib.spa_attn_bwd_dkdv_add(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                                      lse.data_ptr(), workspace.data_ptr(), dk.data_ptr(), dv.data_ptr(),
+                                      B, H, N, d, scale, lo_a, hi_a, _stream_ptr(stream)),
+           "spa_attn_bwd_dkdv_add")
+
+
+def spa_attn_bwd_dq_add(q, k, v, dout, lse, workspace, dq, scale: float, lo=None, hi=None, stream=None):
+    """The dq pass adding to dq instead of overwriting it."""
+    B, H, N, d = _dims(q)
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    _check(_lib.spa_attn_bwd_dq_add(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
+                                    lse.data_ptr(), workspace.data_ptr(), dq.data_ptr(), B, H, N, d, scale,
+                                    lo_a, hi_a, _stream_ptr(stream)), "spa_attn_bwd_dq_add")
 
 
 def spa_attn_bwd_dq_delta(q, k, v, o, dout, lse, workspace, dq, scale: float, lo=None, hi=None,

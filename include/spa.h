@@ -152,6 +152,24 @@ SPA_API int spa_attn_bwd_dq(const void* q, const void* k, const void* v, const v
                             const float* lse, const void* workspace, void* dq, int B, int H,
                             int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi,
                             void* stream);
+/*
+ * spa_attn_bwd_dkdv_add and spa_attn_bwd_dq_add: the dk/dv and dq passes,
+ * adding their gradients to what dk, dv (dq) hold -- each element read, the
+ * pass's fp32 value added, the sum rounded once to bf16 -- instead of
+ * overwriting them; rows the pass does not reach (keys no query of the band
+ * reaches, queries before the band) are left as they are.  For summing the
+ * passes of several disjoint bands that share one lse and D (the band plus
+ * shared window calls below use them for their second part).  Same
+ * arguments and errors as spa_attn_bwd_dkdv / spa_attn_bwd_dq.
+ */
+SPA_API int spa_attn_bwd_dkdv_add(const void* q, const void* k, const void* v, const void* dout,
+                                  const float* lse, const void* workspace, void* dk, void* dv, int B,
+                                  int H, int64_t N, int d, float scale, const int32_t* lo,
+                                  const int32_t* hi, void* stream);
+SPA_API int spa_attn_bwd_dq_add(const void* q, const void* k, const void* v, const void* dout,
+                                const float* lse, const void* workspace, void* dq, int B, int H,
+                                int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi,
+                                void* stream);
 SPA_API int spa_attn_bwd_dq_delta(const void* q, const void* k, const void* v, const void* o,
                                   const void* dout, const float* lse, void* workspace, void* dq,
                                   int B, int H, int64_t N, int d, float scale, const int32_t* lo,
@@ -233,9 +251,10 @@ SPA_API int spa_attn_decode(const void* q, const void* k, const void* v, const i
  * Each head's set is split into two disjoint, non-empty distance intervals
  * and the band kernels run once per part; the forward merges the two
  * partial softmaxes through their lse (one more launch), the backward runs
- * the dQ and dK/dV passes of each part with the joint lse and D and adds the
- * second part's gradients to the first's (one more launch).  lse and o
- * passed to spa_attn_bwd_union must come from spa_attn_fwd_union.
+ * the dQ and dK/dV passes of each part with the joint lse and D, the second
+ * part's passes adding their gradients to the first's in their epilogues
+ * (spa_attn_bwd_dq_add, spa_attn_bwd_dkdv_add).  lse and o passed to
+ * spa_attn_bwd_union must come from spa_attn_fwd_union.
  * SPA_ERR_INVAL for a window outside [1, N], bad bands, null pointers or a
  * bad scale; SPA_ERR_UNSUPPORTED where spa_attn_fwd / spa_attn_bwd would
  * return it, for a misaligned workspace, or when some head's set is a single
@@ -250,15 +269,17 @@ SPA_API size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d);
  * argument rules and errors as spa_attn_fwd_union's window and bands. */
 SPA_API int spa_union_parts(int64_t N, int H, int64_t window, const int32_t* lo, const int32_t* hi,
                             int32_t* a1, int32_t* b1, int32_t* a2, int32_t* b2);
-/* The two steps the union calls add to the band kernels, callable alone
- * (with spa_union_parts and the band entry points they make up the union
- * calls launch by launch):
+/* Two steps for composing bands by hand (with spa_union_parts, the band
+ * forward and spa_attn_union_merge make up spa_attn_fwd_union launch by
+ * launch; spa_attn_bwd_union is the band backward passes with the _add forms
+ * for its second part):
  *  spa_attn_union_merge: o, lse (part 1, DEVICE, overwritten) and o2, lse2
  *    (part 2, DEVICE) -> softmax over the union of the two disjoint sets:
  *    L = log(e^lse + e^lse2), o = e^(lse - L) o + e^(lse2 - L) o2, lse = L
  *    (a row empty in both parts stays o = 0, lse = -inf).
  *  spa_attn_union_add_grads: dq += dq2, dk += dk2, dv += dv2 (DEVICE bf16
- *    [B][H][N][d], summed in fp32 and rounded once).
+ *    [B][H][N][d], summed in fp32 and rounded once), for gradients of two
+ *    parts computed into separate buffers.
  * Tensors 16-byte aligned (lse, lse2: 4).  SPA_ERR_INVAL for null pointers or
  * bad sizes, SPA_ERR_UNSUPPORTED as for spa_attn_fwd. */
 SPA_API int spa_attn_union_merge(void* o, float* lse, const void* o2, const float* lse2, int B, int H,
