@@ -693,10 +693,10 @@ def run_spa(args):
 
 
 # one union step, launch by launch: (name, what it runs)
-UNION_LAUNCHES = ("fwd part 1", "fwd part 2", "merge", "dq+D part 1", "dk/dv part 1", "dq part 2 (adding)",
+UNION_LAUNCHES = ("fwd part 1", "fwd part 2 (merging)", "dq+D part 1", "dk/dv part 1", "dq part 2 (adding)",
                   "dk/dv part 2 (adding)")
-UNION_KERNEL_OF = {"fwd part 1": "spa_fwd_kernel", "fwd part 2": "spa_fwd_kernel",
-                   "merge": "spa_union_merge_kernel", "dq+D part 1": "spa_bwd_dq_kernel",
+UNION_KERNEL_OF = {"fwd part 1": "spa_fwd_kernel", "fwd part 2 (merging)": "spa_fwd_kernel",
+                   "dq+D part 1": "spa_bwd_dq_kernel",
                    "dk/dv part 1": "spa_bwd_dkdv_kernel", "dq part 2 (adding)": "spa_bwd_dq_kernel",
                    "dk/dv part 2 (adding)": "spa_bwd_dkdv_kernel"}
 
@@ -771,13 +771,10 @@ def run_union(args):
 
     # the same launches one public call at a time, with an event after each:
     # per-launch durations for the shares and the roofline
-    o2 = torch.empty_like(qd)
-    lse2 = torch.empty_like(lse)
     wsb = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=device)
     calls = [
         lambda: spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, a1, b1, stream=stream),
-        lambda: spa.spa_attn_fwd(qd, kd, vd, o2, lse2, scale, a2, b2, stream=stream),
-        lambda: spa.spa_attn_union_merge(o, lse, o2, lse2, stream=stream),
+        lambda: spa.spa_attn_fwd_merge(qd, kd, vd, o, lse, scale, a2, b2, stream=stream),
         lambda: spa.spa_attn_bwd_dq_delta(qd, kd, vd, o, dod, lse, wsb, dq, scale, a1, b1, stream=stream),
         lambda: spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, wsb, dk, dv, scale, a1, b1, stream=stream),
         lambda: spa.spa_attn_bwd_dq_add(qd, kd, vd, dod, lse, wsb, dq, scale, a2, b2, stream=stream),

@@ -109,7 +109,11 @@ __device__ __forceinline__ FwdUnit fwd_decode(int u, const AttnParams& p) {
   return U;
 }
 
-template <int D>
+// MERGE: o and lse hold, on entry, a softmax over another set of keys,
+// disjoint from this kernel's bands (spa_attn_fwd_merge); each row is
+// combined with it through the two lse values, and rows this kernel's bands
+// do not reach are left as they are.
+template <int D, bool MERGE = false>
 __global__ void __launch_bounds__(384, 1)
     spa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
@@ -326,7 +330,7 @@ __global__ void __launch_bounds__(384, 1)
       uint16_t* orow = static_cast<uint16_t*>(p.o) + ((int64_t)U.bh * N + i) * D;
       if (!act_t) {
         // rows of this tile precede their band (or lie past N)
-        if (i < N) {
+        if (!MERGE && i < N) {
           for (int c = 0; c < D; c += 8) ptx::st_global_v4(orow + c, 0u, 0u, 0u, 0u);
           p.lse[(int64_t)U.bh * N + i] = -INFINITY;
         }
@@ -545,29 +549,72 @@ __global__ void __launch_bounds__(384, 1)
       last_owner = U.act[1] ? 1 : 0;
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
-      ok = __all_sync(0xffffffffu, bar_wait(&bars->o_done[t], (cd++) & 1, abort_flag));
-      if (!ok) break;
-      ptx::tc_fence_after();
-      const float inv = (l > 0.f) ? 1.f / l : 0.f;
+      if constexpr (MERGE) {
+        // The row already in o (lse1, o1) is combined with this part's.  In
+        // base 2, with a = lse1 log2(e) and b = m + log2(l) this
+        // part's lse: L = log2(2^a + 2^b), o = 2^(a - L) o1 + 2^(b - L) O / l.
+        // A row this part leaves empty (l = 0) keeps o1 and lse1 unchanged.
+        const float lse1 = i < N ? p.lse[(int64_t)U.bh * N + i] : -INFINITY;
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->o_done[t], (cd++) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const float a = lse1 * 1.4426950408889634f;
+        const float b = (l > 0.f) ? m_ref + log2f(l) : -INFINITY;
+        const bool write = i < N && b != -INFINITY;
+        const float mx = fmaxf(a, b);
+        const float L = write ? mx + ptx::log2_approx(ptx::exp2_approx(a - mx) + ptx::exp2_approx(b - mx)) : 0.f;
+        const float w1 = write ? ptx::exp2_approx(a - L) : 0.f;
+        const float w2 = write ? ptx::exp2_approx(b - L) / l : 0.f;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tO + c, o);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(o);
+          if (write) {
+            uint4 o1[4];  // part 1's 32 columns
+#pragma unroll
+            for (int e = 0; e < 4; ++e) o1[e] = reinterpret_cast<const uint4*>(orow + c)[e];
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const float2 f1 = ptx::bf16x2_to_float2(ptx::word_of(o1[e / 4], e % 4));
+              pk[e] = ptx::pack_bf16x2(fmaf(__uint_as_float(o[2 * e]), w2, w1 * f1.x),
+                                       fmaf(__uint_as_float(o[2 * e + 1]), w2, w1 * f1.y));
+            }
+            ptx::st_global_v8(orow + c, pk);
+            ptx::st_global_v8(orow + c + 16, pk + 8);
+          }
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->o_free[t]);
+        if (write) p.lse[(int64_t)U.bh * N + i] = L * 0.69314718055994531f;
+      } else {
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->o_done[t], (cd++) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        const float inv = (l > 0.f) ? 1.f / l : 0.f;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        uint32_t o[32];
-        ptx::tmem_ld32(tO + c, o);
-        ptx::tmem_wait_ld();
-        ptx::reg_fence(o);
-        if (i < N) ptx::store_row32_bf16(orow + c, o, inv);
+        for (int c = 0; c < D; c += 32) {
+          uint32_t o[32];
+          ptx::tmem_ld32(tO + c, o);
+          ptx::tmem_wait_ld();
+          ptx::reg_fence(o);
+          if (i < N) ptx::store_row32_bf16(orow + c, o, inv);
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&bars->o_free[t]);
+        if (i < N)
+          p.lse[(int64_t)U.bh * N + i] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
       }
-      ptx::tc_fence_before();
-      ptx::mbar_arrive(&bars->o_free[t]);
-      if (i < N)
-        p.lse[(int64_t)U.bh * N + i] = (l > 0.f) ? (m_ref + log2f(l)) * 0.69314718055994531f : -INFINITY;
     }
   }
 
   // ------------------------------------------------------------ empty blocks
-  // Whole 256-row blocks that precede their head's band: o = 0, lse = -inf.
+  // Whole 256-row blocks that precede their head's band: o = 0, lse = -inf
+  // (left as they are when merging).
   {
-    const int num_fill = p.B * p.fills_per_batch;
+    const int num_fill = MERGE ? 0 : p.B * p.fills_per_batch;
     for (int f = blockIdx.x; f < num_fill; f += gridDim.x) {
       const int b = f / p.fills_per_batch;
       const int r = f % p.fills_per_batch;

@@ -157,18 +157,20 @@ int set_work_lists(AttnParams& p, Units units_of, Fills fills_of) {
 
 template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, AttnParams& p,
-             cudaStream_t stream) {
+             cudaStream_t stream, bool merge) {
   using C = spa::FwdCfg<D>;
-  static std::atomic<uint64_t> prepared{0};
+  // one (prepared, register check) pair per kernel instantiation: [merging]
+  static std::atomic<uint64_t> prepared[2];
+  static std::atomic<int> regs_ok[2];
+  auto* kernel = merge ? spa::spa_fwd_kernel<D, true> : spa::spa_fwd_kernel<D, false>;
   const int64_t BH = (int64_t)p.B * p.H;
   CUtensorMap mq, mk, mv;
   int st;
   if ((st = make_map(&mq, q, p.N, BH, D, C::BQ)) || (st = make_map(&mk, k, p.N, BH, D, C::BK)) ||
       (st = make_map(&mv, v, p.N, BH, D, C::BK)))
     return st;
-  if ((st = prepare_kernel(spa::spa_fwd_kernel<D>, C::SMEM_BYTES, prepared))) return st;
-  static std::atomic<int> regs_ok{0};
-  if ((st = check_regs(spa::spa_fwd_kernel<D>, (int)C::LAUNCH_REGS, regs_ok))) return st;
+  if ((st = prepare_kernel(kernel, C::SMEM_BYTES, prepared[merge]))) return st;
+  if ((st = check_regs(kernel, (int)C::LAUNCH_REGS, regs_ok[merge]))) return st;
   // Work list of the persistent grid: per batch, every 256-row block of every
   // head from the one holding lo_h on (units), and the blocks before it (fills).
   const int64_t nblk = (p.N + C::BU - 1) / C::BU;
@@ -182,7 +184,7 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, A
   if ((st = sm_count(&sms))) return st;
   const int64_t units = (int64_t)p.B * upb;
   const unsigned grid = (unsigned)(units < sms ? units : sms);
-  spa::spa_fwd_kernel<D><<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
+  kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(mq, mk, mv, p);
   return launch_status();
 }
 
@@ -283,7 +285,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
 }
 
 int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
-              int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+              int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi, void* stream,
+              bool merge = false) {
   int st = check_shape(B, H, N, d);
   if (st) return st;
   if (!q || !k || !v || !o || !lse) return SPA_ERR_INVAL;
@@ -300,7 +303,7 @@ int fwd_entry(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.scale_log2 = scale * spa::kLog2e;
   if ((st = fill_bands(p, H, N, lo, hi))) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d == 64 ? fwd_impl<64>(q, k, v, o, lse, p, s) : fwd_impl<128>(q, k, v, o, lse, p, s);
+  return d == 64 ? fwd_impl<64>(q, k, v, o, lse, p, s, merge) : fwd_impl<128>(q, k, v, o, lse, p, s, merge);
 }
 
 int bwd_entry(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -371,20 +374,8 @@ int union_parts(int H, int64_t N, int64_t window, const int32_t* lo, const int32
 
 size_t align256(size_t n) { return (n + 255) & ~size_t(255); }
 
-// Workspace of the union passes: fp32 [B H N] (lse of part 2 in the
-// forward, D in the backward), then bf16 [B H N d] (o of part 2).
-struct UnionWs {
-  float* vec;
-  uint16_t* o2;
-};
-
-UnionWs union_ws(void* ws, int64_t rows) {
-  UnionWs w;
-  uint8_t* b = static_cast<uint8_t*>(ws);
-  w.vec = reinterpret_cast<float*>(b);
-  w.o2 = reinterpret_cast<uint16_t*>(b + align256((size_t)rows * 4));
-  return w;
-}
+// Workspace of the union calls: the backward's row sums D, fp32 [B H N]
+// (the forward merges in place and needs none).
 
 int union_launch_status() { return cudaGetLastError() == cudaSuccess ? SPA_OK : SPA_ERR_CUDA; }
 
@@ -736,7 +727,7 @@ int spa_union_parts(int64_t N, int H, int64_t window, const int32_t* lo, const i
 size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d) {
   if (check_shape(B, H, N, d)) return 0;
   const size_t rows = (size_t)B * H * N;
-  return align256(rows * 4) + align256(rows * (size_t)d * 2);
+  return align256(rows * 4);
 }
 
 int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
@@ -750,10 +741,10 @@ int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, flo
   UnionParts u = zero;
   if ((st = union_parts(H, N, window, lo, hi, u))) return st;
   const int64_t rows = (int64_t)B * H * N;
-  UnionWs w = union_ws(workspace, rows);
+  (void)rows;
+  // part 2's forward merges into part 1's o and lse in its epilogue
   if ((st = fwd_entry(q, k, v, o, lse, B, H, N, d, scale, u.a1, u.b1, stream))) return st;
-  if ((st = fwd_entry(q, k, v, w.o2, w.vec, B, H, N, d, scale, u.a2, u.b2, stream))) return st;
-  return union_merge(o, lse, w.o2, w.vec, B, H, N, d, stream);
+  return fwd_entry(q, k, v, o, lse, B, H, N, d, scale, u.a2, u.b2, stream, true);
 }
 
 int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -767,19 +758,25 @@ int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* 
   UnionParts u = zero;
   if ((st = union_parts(H, N, window, lo, hi, u))) return st;
   const int64_t rows = (int64_t)B * H * N;
-  UnionWs w = union_ws(workspace, rows);
+  (void)rows;
+  float* D_ = static_cast<float*>(workspace);
   // part 1 starts at distance 0, so its dQ pass forms D for every row; part
   // 2's passes add their gradients to part 1's in their epilogues
-  if ((st = bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, w.vec, B, H, N, d, scale, u.a1, u.b1,
+  if ((st = bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, D_, B, H, N, d, scale, u.a1, u.b1,
                       stream, kStepDqDelta)) ||
-      (st = bwd_entry(q, k, v, o, dout, lse, nullptr, dk, dv, w.vec, B, H, N, d, scale, u.a1, u.b1, stream,
+      (st = bwd_entry(q, k, v, o, dout, lse, nullptr, dk, dv, D_, B, H, N, d, scale, u.a1, u.b1, stream,
                       kStepDkDv)) ||
-      (st = bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, w.vec, B, H, N, d, scale, u.a2, u.b2,
+      (st = bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, D_, B, H, N, d, scale, u.a2, u.b2,
                       stream, kStepDq | kStepAccumulate)) ||
-      (st = bwd_entry(q, k, v, o, dout, lse, nullptr, dk, dv, w.vec, B, H, N, d, scale, u.a2, u.b2, stream,
+      (st = bwd_entry(q, k, v, o, dout, lse, nullptr, dk, dv, D_, B, H, N, d, scale, u.a2, u.b2, stream,
                       kStepDkDv | kStepAccumulate)))
     return st;
   return SPA_OK;
+}
+
+int spa_attn_fwd_merge(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H, int64_t N,
+                       int d, float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+  return fwd_entry(q, k, v, o, lse, B, H, N, d, scale, lo, hi, stream, true);
 }
 
 int spa_attn_union_merge(void* o, float* lse, const void* o2, const float* lse2, int B, int H, int64_t N, int d,

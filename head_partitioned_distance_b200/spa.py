@@ -38,6 +38,7 @@ EXPORTS = {
     "spa_attn_fwd": ([_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _int, _f32, _vp], _int),
     "spa_attn_fwd_ex": ([_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _int, _f32, _i32p, _i32p, _vp],
                         _int),
+    "spa_attn_fwd_merge": ([_vp, _vp, _vp, _vp, _vp, _int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_workspace_bytes": ([_int, _int, _i64], ctypes.c_size_t),
     "spa_attn_bwd": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _vp], _int),
     "spa_attn_bwd_ex": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
@@ -137,6 +138,20 @@ def spa_attn_fwd(q, k, v, o, lse, scale: float, lo=None, hi=None, stream=None):
         st = _lib.spa_attn_fwd_ex(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
                                   lse.data_ptr(), B, H, N, d, scale, _i32(lo), _i32(hi), s)
         _check(st, "spa_attn_fwd_ex")
+    return o, lse
+
+
+def spa_attn_fwd_merge(q, k, v, o, lse, scale: float, lo=None, hi=None, stream=None):
+    """Forward over bands disjoint from the ones o, lse already hold a
+    softmax over; merges into o, lse (the softmax over both sets)."""
+    B, H, N, d = _dims(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    _need(lse, (B, H, N), torch.float32, "lse")
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    _check(_lib.spa_attn_fwd_merge(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                   B, H, N, d, scale, lo_a, hi_a, _stream_ptr(stream)), "spa_attn_fwd_merge")
     return o, lse
 
 

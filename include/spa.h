@@ -95,6 +95,20 @@ SPA_API int spa_attn_fwd_ex(const void* q, const void* k, const void* v, void* o
                     int B, int H, int64_t N, int d, float scale,
                     const int32_t* lo, const int32_t* hi, void* stream);
 
+/*
+ * Forward that merges: o and lse hold, on entry, the output and lse of a
+ * softmax over another set of keys per row (for example spa_attn_fwd_ex on
+ * other bands), disjoint from the bands given here; on return they hold the
+ * softmax over the union of the two sets:
+ *   L = log(e^lse + e^lse_here),  o = e^(lse - L) o + e^(lse_here - L) o_here,
+ * computed per row in the kernel's epilogue.  Rows these bands leave empty
+ * keep o and lse as they were.  Same arguments and rules as spa_attn_fwd_ex
+ * (lo, hi both NULL for the Balanced Distance Partitioning bands).
+ */
+SPA_API int spa_attn_fwd_merge(const void* q, const void* k, const void* v, void* o, float* lse,
+                               int B, int H, int64_t N, int d, float scale,
+                               const int32_t* lo, const int32_t* hi, void* stream);
+
 /* Bytes of device workspace that spa_attn_bwd needs: 4 * B * H * N (the fp32
  * row sums D_i = sum_c dout_ic * o_ic).  Returns 0 on bad sizes. */
 SPA_API size_t spa_attn_bwd_workspace_bytes(int B, int H, int64_t N);
@@ -246,14 +260,16 @@ SPA_API int spa_attn_decode(const void* q, const void* k, const void* v, const i
  *   lo, hi:    HOST band arrays (rules of spa_attn_fwd_ex) or both NULL for the
  *              Balanced Distance Partitioning bands
  *   workspace: DEVICE buffer of spa_attn_union_workspace_bytes(B, H, N, d)
- *              bytes, 32-byte aligned, caller-owned, overwritten
+ *              bytes (the backward's row sums D; the forward uses none),
+ *              32-byte aligned, caller-owned, overwritten
  * Other arguments, layouts and alignment as in spa_attn_fwd / spa_attn_bwd.
  * Each head's set is split into two disjoint, non-empty distance intervals
- * and the band kernels run once per part; the forward merges the two
- * partial softmaxes through their lse (one more launch), the backward runs
+ * and the band kernels run once per part: the forward of the second part
+ * merges into the first's o and lse (spa_attn_fwd_merge), the backward runs
  * the dQ and dK/dV passes of each part with the joint lse and D, the second
  * part's passes adding their gradients to the first's in their epilogues
- * (spa_attn_bwd_dq_add, spa_attn_bwd_dkdv_add).  lse and o passed to
+ * (spa_attn_bwd_dq_add, spa_attn_bwd_dkdv_add): two launches forward, four
+ * backward.  lse and o passed to
  * spa_attn_bwd_union must come from spa_attn_fwd_union.
  * SPA_ERR_INVAL for a window outside [1, N], bad bands, null pointers or a
  * bad scale; SPA_ERR_UNSUPPORTED where spa_attn_fwd / spa_attn_bwd would
@@ -269,10 +285,9 @@ SPA_API size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d);
  * argument rules and errors as spa_attn_fwd_union's window and bands. */
 SPA_API int spa_union_parts(int64_t N, int H, int64_t window, const int32_t* lo, const int32_t* hi,
                             int32_t* a1, int32_t* b1, int32_t* a2, int32_t* b2);
-/* Two steps for composing bands by hand (with spa_union_parts, the band
- * forward and spa_attn_union_merge make up spa_attn_fwd_union launch by
- * launch; spa_attn_bwd_union is the band backward passes with the _add forms
- * for its second part):
+/* Two steps for composing bands by hand from outputs computed into separate
+ * buffers (the union calls themselves merge and add inside the kernels'
+ * epilogues, spa_attn_fwd_merge and the _add passes):
  *  spa_attn_union_merge: o, lse (part 1, DEVICE, overwritten) and o2, lse2
  *    (part 2, DEVICE) -> softmax over the union of the two disjoint sets:
  *    L = log(e^lse + e^lse2), o = e^(lse - L) o + e^(lse2 - L) o2, lse = L

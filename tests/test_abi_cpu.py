@@ -221,7 +221,10 @@ def test_union_entry_points_reject_bad_arguments_before_any_launch():
         spa.SPA_ERR_UNSUPPORTED
     assert L.spa_attn_union_workspace_bytes(1, 4, 256, 96) == 0
     rows = 1 * 4 * 256
-    assert L.spa_attn_union_workspace_bytes(1, 4, 256, 64) == rows * 4 + rows * 64 * 2
+    assert L.spa_attn_union_workspace_bytes(1, 4, 256, 64) == rows * 4
+    assert L.spa_attn_fwd_merge(p, p, p, None, p, *args, None, None, None) == spa.SPA_ERR_INVAL
+    assert L.spa_attn_fwd_merge(p, p, p, _fake((1 << 20) + 16), p, *args, None, None, None) == \
+        spa.SPA_ERR_UNSUPPORTED
     # the adding backward passes check like the overwriting ones
     assert L.spa_attn_bwd_dkdv_add(p, p, p, p, p, p, None, p, *args, None, None, None) == spa.SPA_ERR_INVAL
     assert L.spa_attn_bwd_dq_add(p, p, p, p, p, p, None, *args, None, None, None) == spa.SPA_ERR_INVAL

@@ -127,10 +127,10 @@ def test_union_full_size_sampled_rows(spa):
 
 
 def test_launch_by_launch_composition_equals_the_union_calls(spa):
-    # spa_union_parts + the band entry points + the merge step and the adding
+    # spa_union_parts + the band forward, the merging forward and the adding
     # backward passes, called one by one, are exactly what the two union
-    # calls launch; summing part 2 computed into separate buffers with
-    # spa_attn_union_add_grads agrees to bf16 rounding
+    # calls launch; merging / summing part 2 computed into separate buffers
+    # (spa_attn_union_merge, spa_attn_union_add_grads) agrees to bf16 rounding
     B, H, N, d, w = 1, 8, 1001, 64, 64
     q, k, v, do = (t.to("cuda:0") for t in synth.make_inputs(B, H, N, d, seed=5))
     scale = 0.125
@@ -138,8 +138,10 @@ def test_launch_by_launch_composition_equals_the_union_calls(spa):
     dq, dk, dv = spa.attention_backward_union(q, k, v, o, do, lse, w, scale)
     a1, b1, a2, b2 = spa.spa_union_parts(N, H, w)
     o1, l1 = spa.attention_forward(q, k, v, scale, a1, b1)
+    om, lm = o1.clone(), l1.clone()
+    spa.spa_attn_fwd_merge(q, k, v, o1, l1, scale, a2, b2)
     o2, l2 = spa.attention_forward(q, k, v, scale, a2, b2)
-    spa.spa_attn_union_merge(o1, l1, o2, l2)
+    spa.spa_attn_union_merge(om, lm, o2, l2)
     ws = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device="cuda:0")
     g1 = [torch.empty_like(q) for _ in range(3)]
     spa.spa_attn_bwd_dq_delta(q, k, v, o1, do, l1, ws, g1[0], scale, a1, b1)
@@ -154,6 +156,9 @@ def test_launch_by_launch_composition_equals_the_union_calls(spa):
     torch.cuda.synchronize()
     assert spa.spa_device_status() == spa.SPA_OK
     assert torch.equal(o, o1) and torch.equal(lse, l1)
+    # merged in the epilogue vs merged from two bf16 outputs: two roundings against one
+    assert (o.float() - om.float()).abs().max() <= 2 ** -7 * o.float().abs().max()
+    assert (lse - lm).abs().max() <= 1e-4
     for a, b, c in zip((dq, dk, dv), g1, g2):
         assert torch.equal(a, b)
         # two roundings (part 2 to bf16, then the sum) against one
