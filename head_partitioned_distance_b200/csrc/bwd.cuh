@@ -733,7 +733,7 @@ __global__ void __launch_bounds__(384, 1)
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars->k_full[s], 1);
       ptx::mbar_init(&bars->v_full[s], 1);
-      ptx::mbar_init(&bars->kv_empty[s], 1);
+      ptx::mbar_init(&bars->kv_empty[s], 2);  // one commit from each MMA issuer
     }
     ptx::mbar_init(&bars->qa_full, 256);
     ptx::mbar_init(&bars->dvec_full, 128);
@@ -743,7 +743,7 @@ __global__ void __launch_bounds__(384, 1)
     ptx::mbar_init(&bars->ds_full, 256);
     ptx::mbar_init(&bars->acc_done, 1);
     ptx::mbar_init(&bars->acc_free, 256);
-    ptx::mbar_init(&bars->drain, 1);
+    ptx::mbar_init(&bars->drain, 2);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -759,7 +759,7 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     ptx::regs_dec<C::CONTROL_REGS>();
-  if (warp >= 10) {
+  if (warp >= 11) {
     // idle warps of the control warpgroup
   } else if (warp == 8) {
     // ------------------------------------------------------------ TMA producer
@@ -804,12 +804,16 @@ __global__ void __launch_bounds__(384, 1)
         }
     }
     __syncwarp();
-  } else if (warp == 9) {
-    // ------------------------------------------------------------ MMA issuer
+  } else {
+    // ------------------------------------------------------------ MMA issuers
+    // Warp 10 issues S of every key tile, warp 9 dQ and dP of the next tile
+    // (as in dK/dV: an issuing thread blocks for about the length of each
+    // group, so S of the next tile should not queue behind the waits of the
+    // dQ chain).  K stages are released by one commit from each.
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BK, false, false);
       constexpr uint32_t idesc_g = ptx::idesc_bf16_f32(128, D, false, true);
-      int nq = 0, g = 0, cf = 0, cds = 0, cacc = 0;
+      int nq = 0, g = 0;
       bool ok = true;
       // K-major (B of S/dP) and MN-major K (B of dQ) views of both K/V stages
       const uint64_t dKk0 = ptx::sdesc_sw128(sK, 0, 1024), dKk1 = ptx::sdesc_sw128(sK + C::KT_BYTES, 0, 1024);
@@ -826,61 +830,71 @@ __global__ void __launch_bounds__(384, 1)
           ptx::mma_bf16_ts(tmem + dst, tmem + a_col + kk * 8,
                            ptx::sdesc_advance(db, (kk / 4) * (C::BK * 128) + (kk % 4) * 32), idesc_s, kk > 0);
       };
-      for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
-        const DqUnit U = dq_decode(u, p);
-        const int nk = U.kb - U.ka + 1;
-        const int g0 = g;
-        auto slot = [&](int jj) { return (g0 + jj) % C::NS; };
-        auto par = [&](int jj) { return (uint32_t)(((g0 + jj) / C::NS) & 1); };
-        ok = bar_wait(&bars->qa_full, (nq++) & 1, abort_flag) && bar_wait(&bars->k_full[slot(0)], par(0), abort_flag);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        issue_nt(C::TM_S, C::TM_QA, dKk(slot(0)));
-        ptx::mma_commit(&bars->s_full);
-        ok = bar_wait(&bars->v_full[slot(0)], par(0), abort_flag);
-        if (!ok) break;
-        ptx::tc_fence_after();
-        issue_nt(C::TM_DP, C::TM_DOA, dVk(slot(0)));
-        ptx::mma_commit(&bars->dp_full);
-        for (int j = 0; j < nk; ++j) {
-          // the warpgroups hold S of this key tile in registers: S of the
-          // next one goes into the same columns while they exponentiate
-          ok = bar_wait(&bars->s_free, (cf++) & 1, abort_flag);
-          if (ok && j + 1 < nk) {
-            ok = bar_wait(&bars->k_full[slot(j + 1)], par(j + 1), abort_flag);
-            if (ok) {
-              ptx::tc_fence_after();
-              issue_nt(C::TM_S, C::TM_QA, dKk(slot(j + 1)));
-              ptx::mma_commit(&bars->s_full);
-            }
-          }
-          if (ok) ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
-          if (ok && j == 0) ok = bar_wait(&bars->acc_free, (cacc & 1) ^ 1, abort_flag);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          {
-            // dQ += dS K: A = dS (bf16 pairs over dP, key halves at +0 / +64),
-            // B = K tile MN-major along d
-            const uint64_t db = dKm(slot(j));
-            const uint32_t abase = tmem + C::TM_DP;
-#pragma unroll
-            for (int kk = 0; kk < C::BK / 16; ++kk)
-              ptx::mma_bf16_ts(tmem + C::TM_DQ, abase + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
-                               ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (j > 0 || kk > 0));
-          }
-          ptx::mma_commit(&bars->kv_empty[slot(j)]);
-          if (j + 1 < nk) {
-            ok = bar_wait(&bars->v_full[slot(j + 1)], par(j + 1), abort_flag);
+      if (warp == 10) {
+        // ---- S of each key tile, as soon as the warpgroups hold the last one
+        int cf = 0;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+          const DqUnit U = dq_decode(u, p);
+          const int nk = U.kb - U.ka + 1;
+          const int g0 = g;
+          for (int j = 0; ok && j < nk; ++j) {
+            const int gj = g0 + j;
+            const int st = gj % C::NS;
+            if (gj > 0) ok = bar_wait(&bars->s_free, (cf++) & 1, abort_flag);
+            if (ok && j == 0) ok = bar_wait(&bars->qa_full, (nq++) & 1, abort_flag);
+            if (ok) ok = bar_wait(&bars->k_full[st], (uint32_t)((gj / C::NS) & 1), abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
-            issue_nt(C::TM_DP, C::TM_DOA, dVk(slot(j + 1)));  // dP of the next key tile
-            ptx::mma_commit(&bars->dp_full);
+            issue_nt(C::TM_S, C::TM_QA, dKk(st));
+            ptx::mma_commit(&bars->s_full);
+            ptx::mma_commit(&bars->kv_empty[st]);
           }
+          g = g0 + nk;
         }
-        if (!ok) break;
-        ++cacc;
-        ptx::mma_commit(&bars->acc_done);
-        g = g0 + nk;
+      } else {
+        // ---- dQ of each key tile and dP of the next
+        int cds = 0, cacc = 0;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+          const DqUnit U = dq_decode(u, p);
+          const int nk = U.kb - U.ka + 1;
+          const int g0 = g;
+          auto slot = [&](int jj) { return (g0 + jj) % C::NS; };
+          auto par = [&](int jj) { return (uint32_t)(((g0 + jj) / C::NS) & 1); };
+          ok = bar_wait(&bars->qa_full, (nq++) & 1, abort_flag) && bar_wait(&bars->v_full[slot(0)], par(0), abort_flag);
+          if (!ok) break;
+          ptx::tc_fence_after();
+          issue_nt(C::TM_DP, C::TM_DOA, dVk(slot(0)));
+          ptx::mma_commit(&bars->dp_full);
+          for (int j = 0; j < nk; ++j) {
+            ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
+            if (ok && j == 0) ok = bar_wait(&bars->acc_free, (cacc & 1) ^ 1, abort_flag);
+            if (ok) ok = bar_wait(&bars->k_full[slot(j)], par(j), abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            {
+              // dQ += dS K: A = dS (bf16 pairs over dP, key halves at +0 / +64),
+              // B = K tile MN-major along d
+              const uint64_t db = dKm(slot(j));
+              const uint32_t abase = tmem + C::TM_DP;
+#pragma unroll
+              for (int kk = 0; kk < C::BK / 16; ++kk)
+                ptx::mma_bf16_ts(tmem + C::TM_DQ, abase + (kk < 4 ? kk * 8 : 64 + (kk - 4) * 8),
+                                 ptx::sdesc_advance(db, kk * (16 * 128)), idesc_g, (j > 0 || kk > 0));
+            }
+            ptx::mma_commit(&bars->kv_empty[slot(j)]);
+            if (j + 1 < nk) {
+              ok = bar_wait(&bars->v_full[slot(j + 1)], par(j + 1), abort_flag);
+              if (!ok) break;
+              ptx::tc_fence_after();
+              issue_nt(C::TM_DP, C::TM_DOA, dVk(slot(j + 1)));  // dP of the next key tile
+              ptx::mma_commit(&bars->dp_full);
+            }
+          }
+          if (!ok) break;
+          ++cacc;
+          ptx::mma_commit(&bars->acc_done);
+          g = g0 + nk;
+        }
       }
       ptx::mma_commit(&bars->drain);
       bar_drain(&bars->drain, 0);
