@@ -163,3 +163,39 @@ def test_launch_by_launch_composition_equals_the_union_calls(spa):
         assert torch.equal(a, b)
         # two roundings (part 2 to bf16, then the sum) against one
         assert (a.float() - c.float()).abs().max() <= 2 ** -7 * a.float().abs().max()
+
+
+@pytest.mark.parametrize("B,H,N,d", [(1, 4, 600, 64), (2, 3, 777, 128)])
+def test_split_bands_merge_and_add_to_the_whole_band(spa, B, H, N, d):
+    # every head's band [lo, hi) cut at an arbitrary distance m into [lo, m)
+    # and [m, hi): the forward of the first part then the merging forward of
+    # the second give the whole band's o and lse, and the backward passes of
+    # the first part then the adding passes of the second (with the whole
+    # band's lse and D) give its gradients; rows the second part leaves empty
+    # (i < m) keep the first part's values
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=17 + N)
+    scale = 1 / math.sqrt(d)
+    lo, hi = oracle.bands(N, H)
+    cut = [int(a + (b - a) // 3 + 1) for a, b in zip(lo, hi)]
+    lo1, hi1 = [int(x) for x in lo], cut
+    lo2, hi2 = cut, [int(x) for x in hi]
+    qd, kd, vd, dod = (t.to("cuda:0") for t in (q, k, v, do))
+    o, lse = spa.attention_forward(qd, kd, vd, scale, lo1, hi1)
+    spa.spa_attn_fwd_merge(qd, kd, vd, o, lse, scale, lo2, hi2)
+    ws = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device="cuda:0")
+    dq, dk, dv = (torch.empty_like(qd) for _ in range(3))
+    spa.spa_attn_bwd_dq_delta(qd, kd, vd, o, dod, lse, ws, dq, scale, lo1, hi1)
+    spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, ws, dk, dv, scale, lo1, hi1)
+    spa.spa_attn_bwd_dq_add(qd, kd, vd, dod, lse, ws, dq, scale, lo2, hi2)
+    spa.spa_attn_bwd_dkdv_add(qd, kd, vd, dod, lse, ws, dk, dv, scale, lo2, hi2)
+    torch.cuda.synchronize()
+    assert spa.spa_device_status() == spa.SPA_OK
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    o_ref, lse_ref = oracle.spa_fwd(qf, kf, vf, scale)
+    got_lse = _f64(lse)
+    neg = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(got_lse), neg)
+    assert np.abs(_f64(o) - o_ref).max() <= O_TOL
+    assert np.abs(got_lse[~neg] - lse_ref[~neg]).max() <= LSE_TOL
+    for name, g, ref in zip(("dq", "dk", "dv"), (dq, dk, dv), oracle.spa_bwd(qf, kf, vf, dof, scale)):
+        _check_grad(_f64(g), ref, name)
