@@ -114,6 +114,7 @@ struct DkvBars {
   uint64_t kv_full, kv_empty;
   uint64_t q_full[2], q_empty[2];
   uint64_t s_full, s_free, dp_full, p_full, ds_full;
+  uint64_t pt_read;  // dV of a query tile has read its P^T (dP^T of the next may overwrite it)
   uint64_t vec_full[2], vec_empty[2];
   uint64_t acc_done, acc_free, drain;
   uint32_t tmem_base;
@@ -176,7 +177,7 @@ __global__ void __launch_bounds__(384, 1)
     ptx::mbar_init(&bars->kv_empty, 2);  // one commit from each MMA issuer
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&bars->q_full[s], 1);
-      ptx::mbar_init(&bars->q_empty[s], 2);
+      ptx::mbar_init(&bars->q_empty[s], 3);  // one commit from each MMA issuer
       ptx::mbar_init(&bars->vec_full[s], 1);
       ptx::mbar_init(&bars->vec_empty[s], 256);
     }
@@ -185,9 +186,10 @@ __global__ void __launch_bounds__(384, 1)
     ptx::mbar_init(&bars->dp_full, 1);
     ptx::mbar_init(&bars->p_full, 256);
     ptx::mbar_init(&bars->ds_full, 256);
-    ptx::mbar_init(&bars->acc_done, 1);
+    ptx::mbar_init(&bars->pt_read, 1);
+    ptx::mbar_init(&bars->acc_done, 2);  // dK (warp 9) and dV (warp 11)
     ptx::mbar_init(&bars->acc_free, 256);
-    ptx::mbar_init(&bars->drain, 2);
+    ptx::mbar_init(&bars->drain, 3);
     bars->abort = 0;
     ptx::fence_mbar_init();
   }
@@ -203,9 +205,7 @@ __global__ void __launch_bounds__(384, 1)
 
   if (warp >= 8) {
     ptx::regs_dec<C::CONTROL_REGS>();
-  if (warp >= 11) {
-    // idle warp of the control warpgroup
-  } else if (warp == 8) {
+  if (warp == 8) {
     // ------------------------------------------------------------ producer warp
     // Lane 0 issues the tile copies; all lanes load the query tiles' lse and D
     // into the shared vector ring.
@@ -268,13 +268,15 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ MMA issuers
-    // Warp 10 issues S^T of every query tile, warp 9 dV, dK and dP^T.  The
-    // issuing thread blocks in each group of MMAs for about as long as the
-    // tensor core takes to run it, so one issuer leaves the tensor core idle
-    // while it waits for the warpgroups; with two, S^T of the next tile fills
-    // the gaps of the gradient chain.  The two write disjoint TMEM columns
-    // (S^T vs dP^T, dV, dK); Q stages and K/V are released by one commit
-    // from each.
+    // Warp 10 issues S^T of every query tile, warp 11 dV, warp 9 dK and dP^T
+    // of the next tile.  The issuing thread blocks in each group of MMAs for
+    // about as long as the tensor core takes to run it, so a single issuer
+    // leaves the tensor core idle while it waits for the warpgroups, and the
+    // dK -> dP^T chain would wait behind dV.  Each issuer writes its own
+    // TMEM columns (S^T; dV; dK and dP^T); dP^T of the next tile overwrites
+    // the P^T that dV reads, so warp 9 issues it only after warp 11's commit
+    // on pt_read.  Q/dO stages are released by one commit from each issuer,
+    // K/V by one from warps 10 and 9, the accumulators by one from 9 and 11.
     if (lane == 0) {
       constexpr uint32_t idesc_s = ptx::idesc_bf16_f32(128, C::BQ, false, false);
       constexpr uint32_t idesc_g = ptx::idesc_bf16_f32(128, D, false, true);
@@ -331,15 +333,40 @@ __global__ void __launch_bounds__(384, 1)
           }
           gq = g0 + nq;
         }
-      } else {
-        // ---- dV, dK of each query tile and dP^T of the next
-        int cp = 0, cds = 0, cacc = 0;
+      } else if (warp == 11) {
+        // ---- dV of each query tile, as soon as its P^T is in TMEM
+        int cp = 0, cacc = 0;
         for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
           const DkvUnit U = dkv_decode(u, p);
           const int nq = U.qb - U.qa + 1;
           const int g0 = gq;
+          for (int j = 0; ok && j < nq; ++j) {
+            const int g = g0 + j;
+            ok = bar_wait(&bars->p_full, (cp++) & 1, abort_flag);
+            if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
+            if (ok) ok = bar_wait(&bars->q_full[qstage(g)], qphase(g), abort_flag);
+            if (!ok) break;
+            ptx::tc_fence_after();
+            issue_grad(C::TM_DV, C::TM_PT, dOm(qstage(g)), j == 0);   // dV += P^T dO
+            ptx::mma_commit(&bars->pt_read);
+            ptx::mma_commit(&bars->q_empty[qstage(g)]);
+          }
+          if (!ok) break;
+          ++cacc;
+          ptx::mma_commit(&bars->acc_done);
+          gq = g0 + nq;
+        }
+      } else {
+        // ---- dK of each query tile and dP^T of the next
+        int cds = 0, cacc = 0, cpt = 0;
+        for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
+          const DkvUnit U = dkv_decode(u, p);
+          const int nq = U.qb - U.qa + 1;
+          const int g0 = gq;
+          // dP^T of tile g overwrites P^T of tile g - 1: wait for its dV
           ok = bar_wait(&bars->kv_full, (nkv++) & 1, abort_flag) &&
-               bar_wait(&bars->q_full[qstage(g0)], qphase(g0), abort_flag);
+               bar_wait(&bars->q_full[qstage(g0)], qphase(g0), abort_flag) &&
+               (g0 == 0 || bar_wait(&bars->pt_read, (cpt++) & 1, abort_flag));
           if (!ok) break;
           ptx::tc_fence_after();
           issue_nt(C::TM_DPT, dV, dOk(qstage(g0)));
@@ -347,18 +374,15 @@ __global__ void __launch_bounds__(384, 1)
           if (nq == 1) ptx::mma_commit(&bars->kv_empty);           // V read for the last time
           for (int j = 0; j < nq; ++j) {
             const int g = g0 + j;
-            ok = bar_wait(&bars->p_full, (cp++) & 1, abort_flag);
-            if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
-            if (!ok) break;
-            ptx::tc_fence_after();
-            issue_grad(C::TM_DV, C::TM_PT, dOm(qstage(g)), j == 0);   // dV += P^T dO
             ok = bar_wait(&bars->ds_full, (cds++) & 1, abort_flag);
+            if (ok && j == 0) ok = bar_wait(&bars->acc_free, ((cacc & 1) ^ 1), abort_flag);
             if (!ok) break;
             ptx::tc_fence_after();
             issue_grad(C::TM_DK, C::TM_DST, dQm(qstage(g)), j == 0);  // dK += dS^T Q
             ptx::mma_commit(&bars->q_empty[qstage(g)]);
             if (j + 1 < nq) {
-              ok = bar_wait(&bars->q_full[qstage(g + 1)], qphase(g + 1), abort_flag);
+              ok = bar_wait(&bars->q_full[qstage(g + 1)], qphase(g + 1), abort_flag) &&
+                   bar_wait(&bars->pt_read, (cpt++) & 1, abort_flag);
               if (!ok) break;
               ptx::tc_fence_after();
               issue_nt(C::TM_DPT, dV, dOk(qstage(g + 1)));           // dP^T of the next tile
