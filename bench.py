@@ -735,7 +735,7 @@ def run_union(args):
     scale = w.scale
 
     def step(S):
-        spa.spa_attn_fwd_union(S["q"], S["k"], S["v"], S["o"], S["lse"], S["ws"], scale, W, stream=stream)
+        spa.spa_attn_fwd_union(S["q"], S["k"], S["v"], S["o"], S["lse"], scale, W, stream=stream)
         spa.spa_attn_bwd_union(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"],
                                S["ws"], scale, W, stream=stream)
 

@@ -730,18 +730,14 @@ size_t spa_attn_union_workspace_bytes(int B, int H, int64_t N, int d) {
   return align256(rows * 4);
 }
 
-int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, float* lse, void* workspace,
-                       int B, int H, int64_t N, int d, float scale, int64_t window, const int32_t* lo,
-                       const int32_t* hi, void* stream) {
+int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, float* lse, int B, int H,
+                       int64_t N, int d, float scale, int64_t window, const int32_t* lo, const int32_t* hi,
+                       void* stream) {
   int st = check_shape(B, H, N, d);
   if (st) return st;
-  if (!workspace) return SPA_ERR_INVAL;
-  if (!aligned(workspace, 32)) return SPA_ERR_UNSUPPORTED;
   static UnionParts zero{};
   UnionParts u = zero;
   if ((st = union_parts(H, N, window, lo, hi, u))) return st;
-  const int64_t rows = (int64_t)B * H * N;
-  (void)rows;
   // part 2's forward merges into part 1's o and lse in its epilogue
   if ((st = fwd_entry(q, k, v, o, lse, B, H, N, d, scale, u.a1, u.b1, stream))) return st;
   return fwd_entry(q, k, v, o, lse, B, H, N, d, scale, u.a2, u.b2, stream, true);
@@ -757,8 +753,6 @@ int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* 
   static UnionParts zero{};
   UnionParts u = zero;
   if ((st = union_parts(H, N, window, lo, hi, u))) return st;
-  const int64_t rows = (int64_t)B * H * N;
-  (void)rows;
   float* D_ = static_cast<float*>(workspace);
   // part 1 starts at distance 0, so its dQ pass forms D for every row; part
   // 2's passes add their gradients to part 1's in their epilogues

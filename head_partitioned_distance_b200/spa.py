@@ -55,7 +55,7 @@ EXPORTS = {
     "spa_union_parts": ([_i64, _int, _i64, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p], _int),
     "spa_attn_union_merge": ([_vp] * 4 + [_int, _int, _i64, _int, _vp], _int),
     "spa_attn_union_add_grads": ([_vp] * 6 + [_int, _int, _i64, _int, _vp], _int),
-    "spa_attn_fwd_union": ([_vp] * 6 + [_int, _int, _i64, _int, _f32, _i64, _i32p, _i32p, _vp], _int),
+    "spa_attn_fwd_union": ([_vp] * 5 + [_int, _int, _i64, _int, _f32, _i64, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_union": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i64, _i32p, _i32p, _vp], _int),
     "spa_tile_schedule": ([_i64, _int, _i32p, _i32p, _int, _int, _i32p, _i32p, _u8p, _i32p, _i32p],
                           _int),
@@ -397,20 +397,18 @@ def _union_ws(workspace, B, H, N, d):
         raise ValueError("workspace: CUDA tensor of spa_attn_union_workspace_bytes(B, H, N, d) bytes")
 
 
-def spa_attn_fwd_union(q, k, v, o, lse, workspace, scale: float, window: int, lo=None, hi=None,
-                       stream=None):
+def spa_attn_fwd_union(q, k, v, o, lse, scale: float, window: int, lo=None, hi=None, stream=None):
     """Each head attends to its band and to the distances [0, window) that every
     head shares; writes o [B,H,N,d] bf16 and lse [B,H,N] fp32."""
     B, H, N, d = _dims(q)
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o")):
         _need(t, (B, H, N, d), torch.bfloat16, n)
     _need(lse, (B, H, N), torch.float32, "lse")
-    _union_ws(workspace, B, H, N, d)
     lo_a = None if lo is None else _i32(lo)
     hi_a = None if hi is None else _i32(hi)
     _check(_lib.spa_attn_fwd_union(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                   workspace.data_ptr(), B, H, N, d, scale, int(window), lo_a, hi_a,
-                                   _stream_ptr(stream)), "spa_attn_fwd_union")
+                                   B, H, N, d, scale, int(window), lo_a, hi_a, _stream_ptr(stream)),
+           "spa_attn_fwd_union")
     return o, lse
 
 
@@ -438,12 +436,12 @@ def _union_workspace(q):
 
 
 def attention_forward_union(q, k, v, window: int, scale=None, lo=None, hi=None):
-    """Allocate o / lse / workspace and run spa_attn_fwd_union."""
+    """Allocate o / lse and run spa_attn_fwd_union."""
     B, H, N, d = _dims(q)
     scale = d ** -0.5 if scale is None else scale
     o = torch.empty_like(q)
     lse = torch.empty((B, H, N), dtype=torch.float32, device=q.device)
-    return spa_attn_fwd_union(q, k, v, o, lse, _union_workspace(q), scale, window, lo, hi)
+    return spa_attn_fwd_union(q, k, v, o, lse, scale, window, lo, hi)
 
 
 def attention_backward_union(q, k, v, o, dout, lse, window: int, scale=None, lo=None, hi=None):

@@ -259,9 +259,9 @@ SPA_API int spa_attn_decode(const void* q, const void* k, const void* v, const i
  *   window:    1 <= window <= N, the shared distances [0, window)
  *   lo, hi:    HOST band arrays (rules of spa_attn_fwd_ex) or both NULL for the
  *              Balanced Distance Partitioning bands
- *   workspace: DEVICE buffer of spa_attn_union_workspace_bytes(B, H, N, d)
- *              bytes (the backward's row sums D; the forward uses none),
- *              32-byte aligned, caller-owned, overwritten
+ *   workspace: (backward only) DEVICE buffer of
+ *              spa_attn_union_workspace_bytes(B, H, N, d) bytes for the row
+ *              sums D, 32-byte aligned, caller-owned, overwritten
  * Other arguments, layouts and alignment as in spa_attn_fwd / spa_attn_bwd.
  * Each head's set is split into two disjoint, non-empty distance intervals
  * and the band kernels run once per part: the forward of the second part
@@ -302,8 +302,8 @@ SPA_API int spa_attn_union_merge(void* o, float* lse, const void* o2, const floa
 SPA_API int spa_attn_union_add_grads(void* dq, void* dk, void* dv, const void* dq2, const void* dk2,
                                      const void* dv2, int B, int H, int64_t N, int d, void* stream);
 SPA_API int spa_attn_fwd_union(const void* q, const void* k, const void* v, void* o, float* lse,
-                               void* workspace, int B, int H, int64_t N, int d, float scale,
-                               int64_t window, const int32_t* lo, const int32_t* hi, void* stream);
+                               int B, int H, int64_t N, int d, float scale, int64_t window,
+                               const int32_t* lo, const int32_t* hi, void* stream);
 SPA_API int spa_attn_bwd_union(const void* q, const void* k, const void* v, const void* o,
                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
                                void* workspace, int B, int H, int64_t N, int d, float scale,

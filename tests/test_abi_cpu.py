@@ -196,16 +196,17 @@ def test_union_entry_points_reject_bad_arguments_before_any_launch():
     args = (B, H, N, d, 0.1)
 
     def fwd(ws, w, lo=None, hi=None, shape=args):
-        return L.spa_attn_fwd_union(p, p, p, p, p, ws, *shape, w, lo, hi, None)
+        # the forward takes no workspace
+        return L.spa_attn_fwd_union(p, p, p, p, p, *shape, w, lo, hi, None)
 
     def bwd(ws, w, lo=None, hi=None, shape=args):
         return L.spa_attn_bwd_union(p, p, p, p, p, p, p, p, p, ws, *shape, w, lo, hi, None)
 
+    assert bwd(None, 8) == spa.SPA_ERR_INVAL                                # workspace
+    assert bwd(_fake((1 << 20) + 16), 8) == spa.SPA_ERR_UNSUPPORTED         # 32-byte aligned
     for call in (fwd, bwd):
         assert call(p, 0) == spa.SPA_ERR_INVAL            # window must be >= 1
         assert call(p, N + 1) == spa.SPA_ERR_INVAL        # and <= N
-        assert call(None, 8) == spa.SPA_ERR_INVAL         # workspace
-        assert call(_fake((1 << 20) + 16), 8) == spa.SPA_ERR_UNSUPPORTED  # 32-byte aligned
         assert call(p, 8, shape=(B, H, N, 96, 0.1)) == spa.SPA_ERR_UNSUPPORTED
         bad_lo = (ctypes.c_int32 * H)(0, 9, 5, 7)
         bad_hi = (ctypes.c_int32 * H)(4, 3, 6, 300)     # reversed and out-of-range bands
