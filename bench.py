@@ -52,6 +52,8 @@ from head_partitioned_distance_b200 import synth  # noqa: E402
 METRIC = "band-sparse attn fwd+bwd useful TFLOP/s and % of B200 bf16 tensor peak"
 UNIT = "TFLOP/s"
 DEFAULT_WORKLOAD = "b1_h32_n32768_d128"
+L2_BYTES = 126 * 2**20
+HOST_LEAD_CYCLES = 400_000  # about 0.2 ms at the B200's clocks
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # one step = the forward, the dQ pass (which also forms the row sums D) and the
 # dK/dV pass, in launch order
@@ -82,15 +84,33 @@ def union_pairs(N: int, window: int, bands) -> int:
 
 
 def kernel_work(w, pairs: int):
-    """Algorithmic work per launch of each kernel (FLOPs over permitted pairs,
-    or bytes for the row-sum kernel)."""
+    """Algorithmic work per launch of each kernel: (FLOPs over the permitted
+    pairs, bytes every launch must move at least).  T is one [B, H, N, d] bf16
+    tensor, R one [B, H, N] fp32 row vector (lse or D)."""
     d = w.d
     rows = w.B * w.H * w.N
+    T, R = rows * d * 2, rows * 4
     return {
-        "spa_fwd_kernel": ("tensor", 4 * d * pairs),            # S = QK^T, O += PV
-        "spa_bwd_dkdv_kernel": ("tensor", 8 * d * pairs),       # S^T, dP^T, dV, dK
-        "spa_bwd_dq_kernel": ("tensor", 6 * d * pairs),         # S, dP, dQ (and D = rowsum(dO * O))
+        "spa_fwd_kernel": (4 * d * pairs, 4 * T + R),           # S = QK^T, O += PV; q k v in, o lse out
+        "spa_bwd_dq_kernel": (6 * d * pairs, 6 * T + 2 * R),    # S, dP, dQ, D = rowsum(dO * O); q k v o dO lse in, dq D out
+        "spa_bwd_dkdv_kernel": (8 * d * pairs, 6 * T + 2 * R),  # S^T, dP^T, dV, dK; q k v dO lse D in, dk dv out
     }
+
+
+def step_work(w, pairs: int):
+    """(useful FLOPs, least bytes) of one forward + backward step: 14 d per
+    pair (the forward's two GEMMs, the backward's five), and q k v in, o lse
+    out, then q k v o dO lse in, dq dk dv out (12 T + 2 R).  The kernels
+    execute more FLOPs (S and dP in both backward passes) and move more bytes
+    (each backward pass reads q, k, v, dO); this is the method's floor."""
+    rows = w.B * w.H * w.N
+    return 14 * w.d * pairs, 12 * rows * w.d * 2 + 2 * rows * 4
+
+
+def roofline_bound(flops: float, nbytes: float, peaks) -> str:
+    """"tensor" when the FLOPs at the bf16 peak take longer than the bytes at
+    the HBM peak, else "hbm" (the attainable-performance roofline)."""
+    return "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >= nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
 
 
 def load_peaks():
@@ -551,7 +571,14 @@ def run_spa(args):
     torch.cuda.set_device(device)
     w = synth.WORKLOADS[args.workload]
     B, H, N, d = w.B, w.H, w.N, w.d
-    bands = spa.spa_band_bounds(N, H)
+    if args.full_bands:
+        # every head's band is [0, N): dense causal attention on every head,
+        # through the same kernels (the explicit-band entry points)
+        bands = ([0] * H, [N] * H)
+        lo_hi = {"lo": bands[0], "hi": bands[1]}
+    else:
+        bands = spa.spa_band_bounds(N, H)
+        lo_hi = {}
     pairs = B * workload_pairs(N, bands)
     useful = 14 * d * pairs
 
@@ -565,17 +592,22 @@ def run_spa(args):
     ws = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=device)
     stream = torch.cuda.current_stream(device)
     scale = w.scale
+    # inputs smaller than L2 are flushed out of it before every timed step (a
+    # write of a buffer twice its size, outside the timed spans)
+    flush = None
+    if B * H * N * d * 2 < L2_BYTES:
+        flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
 
     def step(ev=None):
-        spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, stream=stream)
-        if ev is not None:
-            ev[0].record(stream)
-        spa.spa_attn_bwd_dq_delta(qd, kd, vd, o, dod, lse, ws, dq, scale, stream=stream)
+        spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, stream=stream, **lo_hi)
         if ev is not None:
             ev[1].record(stream)
-        spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, ws, dk, dv, scale, stream=stream)
+        spa.spa_attn_bwd_dq_delta(qd, kd, vd, o, dod, lse, ws, dq, scale, stream=stream, **lo_hi)
         if ev is not None:
             ev[2].record(stream)
+        spa.spa_attn_bwd_dkdv(qd, kd, vd, dod, lse, ws, dk, dv, scale, stream=stream, **lo_hi)
+        if ev is not None:
+            ev[3].record(stream)
 
     for _ in range(args.warmup):
         step()
@@ -587,14 +619,20 @@ def run_spa(args):
     sampler = ClockSampler(visible.split(",")[local] if visible else local)
     sampler.start()
     K = args.steps
-    t_start = torch.cuda.Event(enable_timing=True)
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS))] for _ in range(K)]
+    # per step: its start, then the end of each kernel
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)] for _ in range(K)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize(device)
     sampler.mark_start()
-    t_start.record(stream)
     for s in range(K):
+        if flush is not None:
+            flush.fill_(float(s))
+            # a short device-side wait, untimed, lets the host queue the
+            # step's three calls before the GPU reaches them, so that the
+            # timed spans hold device time and not the host's call overhead
+            torch.cuda._sleep(HOST_LEAD_CYCLES)
+        evs[s][0].record(stream)
         step(evs[s])
     torch.cuda.synchronize(device)
     sampler.mark_end()
@@ -603,15 +641,14 @@ def run_spa(args):
     clocks = sampler.stop()
     if spa.spa_device_status(stream) != spa.SPA_OK:
         raise SystemExit("device status not OK after the timed region")
-    elapsed_ms = t_start.elapsed_time(evs[-1][-1])
+    if flush is None:
+        elapsed_ms = evs[0][0].elapsed_time(evs[-1][-1])
+    else:
+        elapsed_ms = sum(e[0].elapsed_time(e[-1]) for e in evs)
     per_kernel_ms = {name: 0.0 for name in KERNELS}
-    prev = t_start
-    for s in range(K):
-        e = evs[s]
-        per_kernel_ms["spa_fwd_kernel"] += prev.elapsed_time(e[0])
-        per_kernel_ms["spa_bwd_dq_kernel"] += e[0].elapsed_time(e[1])
-        per_kernel_ms["spa_bwd_dkdv_kernel"] += e[1].elapsed_time(e[2])
-        prev = e[2]
+    for e in evs:
+        for i, name in enumerate(KERNELS):
+            per_kernel_ms[name] += e[i].elapsed_time(e[i + 1])
     max_ms = reduce_max(elapsed_ms, device)
     value = aggregate(useful, K, world, max_ms)
 
@@ -620,9 +657,9 @@ def run_spa(args):
     dev0 = dict(q=qd, k=kd, v=vd, do=dod, o=o, lse=lse, dq=dq, dk=dk, dv=dv, ws=ws)
 
     def compute(S):
-        spa.spa_attn_fwd(S["q"], S["k"], S["v"], S["o"], S["lse"], scale, stream=stream)
+        spa.spa_attn_fwd(S["q"], S["k"], S["v"], S["o"], S["lse"], scale, stream=stream, **lo_hi)
         spa.spa_attn_bwd(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"],
-                         S["ws"], scale, stream=stream)
+                         S["ws"], scale, stream=stream, **lo_hi)
 
     e2e_ms, h2d, d2h = pipelined_e2e(device, stream, host, dev0, ("o", "lse", "dq", "dk", "dv"), compute, E,
                                      dist)
@@ -635,24 +672,42 @@ def run_spa(args):
         work = kernel_work(w, pairs)
         kern = {}
         for name in KERNELS:
-            bound, units = work[name]
+            flops, nbytes = work[name]
+            bound = roofline_bound(flops, nbytes, peaks)
             avg_ms = per_kernel_ms[name] / K
             if bound == "tensor":
-                achieved = units / (avg_ms * 1e-3) / 1e12
+                achieved = flops / (avg_ms * 1e-3) / 1e12
                 peak = peaks["bf16_tflops"]
                 unit = "TFLOP/s"
+                units = flops
             else:
-                achieved = units / (avg_ms * 1e-3) / 1e9
+                achieved = nbytes / (avg_ms * 1e-3) / 1e9
                 peak = peaks["hbm_gbs"]
                 unit = "GB/s"
+                units = nbytes
             kern[name] = {"bound": bound, "avg_ms": avg_ms, "share": per_kernel_ms[name] / elapsed_ms,
                           "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                          "algorithmic_per_launch": units}
+                          "algorithmic_per_launch": units, "flops_per_launch": flops,
+                          "bytes_per_launch": nbytes,
+                          "tflops": flops / (avg_ms * 1e-3) / 1e12,
+                          "gbs": nbytes / (avg_ms * 1e-3) / 1e9}
+        # the whole step against its attainable roofline: the slower of the
+        # useful FLOPs at the bf16 peak and the bytes any forward + backward
+        # must move at the HBM peak
+        step_flops, step_bytes = step_work(w, pairs)
+        t_flops = step_flops / (peaks["bf16_tflops"] * 1e12) * 1e3
+        t_bytes = step_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+        step_ms = max_ms / K
+        step_roofline = {"bound": "tensor" if t_flops >= t_bytes else "hbm",
+                         "flops": step_flops, "bytes": step_bytes,
+                         "t_flops_ms": t_flops, "t_bytes_ms": t_bytes, "t_measured_ms": step_ms,
+                         "frac": max(t_flops, t_bytes) / step_ms}
         dom = max(KERNELS, key=lambda n: per_kernel_ms[n])
         dk_ = kern[dom]
         roofline = {"bound": dk_["bound"], "achieved": dk_["achieved"], "peak": dk_["peak"],
                     "unit": dk_["unit"], "frac": dk_["frac"],
-                    "traffic": ncu_traffic(dom, w.name), "kernel": dom,
+                    "traffic": ncu_traffic(dom, w.name + ("/full-bands" if args.full_bands else "")),
+                    "kernel": dom,
                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if dk_['bound'] == 'tensor' else 'hbm_gbs'})"}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -671,12 +726,17 @@ def run_spa(args):
             "peaks": {**peaks, "source": peak_src},
             "tokens_per_s": world * B * N * K / (max_ms * 1e-3),
             "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d,
-                       "bands": "balanced distance partitioning", "pairs_per_rank": pairs,
+                       "bands": ("full: [0, N) on every head (dense causal per head)" if args.full_bands
+                                 else "balanced distance partitioning"),
+                       "pairs_per_rank": pairs,
                        "useful_flops_per_rank_step": useful,
-                       "l2": "no flush: q, k, v, dout are each larger than L2 "
-                             f"({B * H * N * d * 2 / 2**20:.0f} MiB bf16)",
+                       "l2": ("no flush: q, k, v, dout are each larger than L2 "
+                              f"({B * H * N * d * 2 / 2**20:.0f} MiB bf16)") if flush is None else
+                             (f"flushed before every step (a {2 * L2_BYTES / 2**20:.0f} MiB write, then a "
+                              f"{HOST_LEAD_CYCLES}-cycle device wait; neither timed)"),
                        "parallelism": f"{world} independent replicas (one batch each)"},
             "roofline": roofline,
+            "step_roofline": step_roofline,
             "kernels": kern,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
@@ -861,6 +921,9 @@ def main(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--union", type=int, default=0, metavar="W",
                     help="time band plus a local window [0, W) shared by every head instead")
+    ap.add_argument("--full-bands", action="store_true",
+                    help="run every head with the full band [0, N) (dense causal per head) through the same "
+                         "kernels, to show the work the bands save")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (one new token per sequence) instead of fwd+bwd")
     args = ap.parse_args(argv)

@@ -344,10 +344,6 @@ __global__ void __launch_bounds__(384, 1)
         else if (actv(1, it - 1)) prev = 1;
         else if (actv(0, it - 1)) prev = 0;
         else prev = last_owner;
-        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[t], (cs++) & 1, abort_flag));
-        if (ok && prev == 1 - t) ok = __all_sync(0xffffffffu, bar_wait(&bars->turn[t], (turns++) & 1, abort_flag));
-        if (!ok) break;
-        ptx::tc_fence_after();
         const int64_t j0 = (int64_t)it * C::BK;
         const bool interior = tile_is_interior(N, U.lo, U.hi, it0, C::BQ, j0, C::BK);
         // Edge tile: the permitted keys of this row are the columns c with
@@ -365,13 +361,34 @@ __global__ void __launch_bounds__(384, 1)
             span = (uint32_t)(c_last - c_first);
           }
         }
+        // owner of the next step in this CTA's order
+        int nxt = -1;
+        if (t == 0 && actv(1, it)) nxt = 1;
+        else if (actv(0, it + 1)) nxt = 0;
+        else if (actv(1, it + 1)) nxt = 1;
+        else if (u + (int)gridDim.x < num_units) {
+          const FwdUnit V = fwd_decode<D>(u + gridDim.x, p);
+          nxt = (V.act[0] && V.a[0] == V.u0) ? 0 : 1;
+        }
+        const bool pass_turn = nxt == 1 - t;
+        const bool fast = __all_sync(0xffffffffu, m_ref != -INFINITY);
+        ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[t], (cs++) & 1, abort_flag));
+        if (!ok) break;
+        if (prev == 1 - t) ok = __all_sync(0xffffffffu, bar_wait(&bars->turn[t], (turns++) & 1, abort_flag));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        // Hand the turn over as soon as this step's exponentials are done
+        // (before P is stored) if the next step belongs to the other tile.
+        auto hand_turn = [&]() {
+          if (pass_turn) ptx::mbar_arrive(&bars->turn[1 - t]);
+        };
         // Fast path, for every tile after a row's first: exponentiate against
         // the current reference max while tracking this tile's max, keeping P
         // packed in registers.  Only if some row's max rose past the reference
         // by more than 2^8 is the tile redone by the two-pass path below (S is
         // still intact then: nothing has been stored over it).
         bool done = false;
-        if (__all_sync(0xffffffffu, m_ref != -INFINITY)) {
+        if (fast) {
           const float2 c2v = make_float2(p.scale_log2, p.scale_log2);
           const float2 mnv = make_float2(-m_ref, -m_ref);
           float2 sa = make_float2(0.f, 0.f), sb = make_float2(0.f, 0.f);
@@ -422,6 +439,7 @@ __global__ void __launch_bounds__(384, 1)
           const float sm0 = sa.x, sm1 = sa.y, sm2 = sb.x, sm3 = sb.y;
           const bool over = fmaxf(mx0, mx1) * c2 > m_ref + 8.f;
           if (!__any_sync(0xffffffffu, over)) {
+            hand_turn();
             ptx::tmem_st32(tS, pk[0]);
             ptx::tmem_st32(tS + 32, pk[1]);
             l += (sm0 + sm1) + (sm2 + sm3);
@@ -531,20 +549,11 @@ __global__ void __launch_bounds__(384, 1)
             ptx::tmem_st16(tS + q * 16, pk);
           }
           l += (sm0 + sm1) + (sm2 + sm3);
+          hand_turn();
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full[t]);
-        // hand the turn over if the next step belongs to the other tile
-        int nxt = -1;
-        if (t == 0 && actv(1, it)) nxt = 1;
-        else if (actv(0, it + 1)) nxt = 0;
-        else if (actv(1, it + 1)) nxt = 1;
-        else if (u + (int)gridDim.x < num_units) {
-          const FwdUnit V = fwd_decode<D>(u + gridDim.x, p);
-          nxt = (V.act[0] && V.a[0] == V.u0) ? 0 : 1;
-        }
-        if (nxt == 1 - t) ptx::mbar_arrive(&bars->turn[1 - t]);
       }
       last_owner = U.act[1] ? 1 : 0;
       if (!ok) break;

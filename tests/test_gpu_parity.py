@@ -318,13 +318,17 @@ def test_tile_classes_on_device_bit_exact(spa, N, H, Bq, Bk):
 LARGE = ["b8_h16_n4096_d128", "b4_h32_n8192_d128", "b1_h32_n32768_d128", "b1_h32_n30001_d128"]
 
 
-def _sampled_check(spa, w, n_random, n_key_rows):
+def _sampled_check(spa, w, n_random, n_key_rows, full_bands=False):
     q, k, v, do = synth.workload_inputs(w)
-    got = _gpu_run(spa, q, k, v, do, w.scale)
+    B, H, N, d = w.B, w.H, w.N, w.d
+    if full_bands:  # [0, N) on every head: dense causal attention per head
+        lo, hi = np.zeros(H, dtype=np.int64), np.full(H, N, dtype=np.int64)
+        got = _gpu_run(spa, q, k, v, do, w.scale, [0] * H, [N] * H)
+    else:
+        lo, hi = oracle.bands(N, H)
+        got = _gpu_run(spa, q, k, v, do, w.scale)
     for name in ("o", "lse", "dq", "dk", "dv"):
         assert not np.isnan(got[name]).any(), name
-    B, H, N, d = w.B, w.H, w.N, w.d
-    lo, hi = oracle.bands(N, H)
     per_head = [[int(lo[h]) - 1, int(lo[h]), int(lo[h]) + 1, int(lo[h]) + 127, int(lo[h]) + 128]
                 for h in range(H)]
     rows = synth.sample_rows(B, H, N, n_random, seed=w.seed, per_head=per_head)
@@ -366,6 +370,11 @@ def _sampled_check(spa, w, n_random, n_key_rows):
 def test_full_size_workloads_sampled_rows(spa, name):
     w = synth.WORKLOADS[name]
     _sampled_check(spa, w, n_random=48, n_key_rows=12)
+
+
+def test_full_bands_full_size_sampled_rows(spa):
+    # the dense-causal-per-head run the benchmark times beside the bands
+    _sampled_check(spa, synth.WORKLOADS["b4_h32_n8192_d128"], n_random=24, n_key_rows=8, full_bands=True)
 
 
 def test_device_wait_timeout_reports_and_recovers(spa):

@@ -61,3 +61,25 @@ def test_band_pair_counting_matches_oracle():
         assert bench.workload_pairs(N, (lo.tolist(), hi.tolist())) == want == N * (N + 1) // 2
     # prefix counts used by the CPU-baseline sample
     assert bench.band_pairs_prefix(10, 0, 4) == sum(min(i + 1, 4) for i in range(10))
+
+
+def test_kernel_work_and_roofline_bound():
+    import bench
+    from head_partitioned_distance_b200 import synth
+    peaks = {"bf16_tflops": 1600.0, "hbm_gbs": 6400.0}  # ridge point 250 FLOP per byte
+    w = synth.WORKLOADS["b1_h32_n32768_d128"]
+    pairs = w.B * w.N * (w.N + 1) // 2  # the bands partition the causal distances
+    work = bench.kernel_work(w, pairs)
+    T, R = w.B * w.H * w.N * w.d * 2, w.B * w.H * w.N * 4
+    # S and dP run in both backward passes: 18 d per pair executed, 14 d useful
+    assert sum(f for f, _ in work.values()) == 18 * w.d * pairs
+    assert sum(b for _, b in work.values()) == 16 * T + 5 * R
+    assert bench.step_work(w, pairs) == (14 * w.d * pairs, 12 * T + 2 * R)
+    # width-1024 bands: about 4 d W FLOPs against 8 d bytes per row in the forward
+    assert all(bench.roofline_bound(f, b, peaks) == "tensor" for f, b in work.values())
+    # width-256 bands at d = 128 move more bytes than the tensor cores need time for
+    w = synth.WORKLOADS["b8_h16_n4096_d128"]
+    work = bench.kernel_work(w, w.B * w.N * (w.N + 1) // 2)
+    assert bench.roofline_bound(*work["spa_fwd_kernel"], peaks) == "hbm"
+    assert bench.roofline_bound(1000.0, 4.0, peaks) == "tensor"
+    assert bench.roofline_bound(1000.0, 4.1, peaks) == "hbm"
