@@ -113,7 +113,11 @@ __device__ __forceinline__ FwdUnit fwd_decode(int u, const AttnParams& p) {
 // disjoint from this kernel's bands (spa_attn_fwd_merge); each row is
 // combined with it through the two lse values, and rows this kernel's bands
 // do not reach are left as they are.
-template <int D, bool MERGE = false>
+// TURN: the two softmax warpgroups take turns (below).  That pays when the
+// key strips are long; with short strips (narrow bands) the turn order also
+// serialises the pipeline's refill at every unit boundary, and the two
+// warpgroups run freely instead.  The host picks from the band widths.
+template <int D, bool MERGE = false, bool TURN = true>
 __global__ void __launch_bounds__(384, 1)
     spa_fwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ AttnParams p) {
@@ -374,13 +378,14 @@ __global__ void __launch_bounds__(384, 1)
         const bool fast = __all_sync(0xffffffffu, m_ref != -INFINITY);
         ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[t], (cs++) & 1, abort_flag));
         if (!ok) break;
-        if (prev == 1 - t) ok = __all_sync(0xffffffffu, bar_wait(&bars->turn[t], (turns++) & 1, abort_flag));
+        if (TURN && prev == 1 - t)
+          ok = __all_sync(0xffffffffu, bar_wait(&bars->turn[t], (turns++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
         // Hand the turn over as soon as this step's exponentials are done
         // (before P is stored) if the next step belongs to the other tile.
         auto hand_turn = [&]() {
-          if (pass_turn) ptx::mbar_arrive(&bars->turn[1 - t]);
+          if (TURN && pass_turn) ptx::mbar_arrive(&bars->turn[1 - t]);
         };
         // Fast path, for every tile after a row's first: exponentiate against
         // the current reference max while tracking this tile's max, keeping P

@@ -155,22 +155,33 @@ int set_work_lists(AttnParams& p, Units units_of, Fills fills_of) {
   return SPA_OK;
 }
 
+// mean band width from which the forward's softmax warpgroups take turns
+constexpr int64_t kFwdTurnMinWidth = 768;
+
 template <int D>
 int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, AttnParams& p,
              cudaStream_t stream, bool merge) {
   using C = spa::FwdCfg<D>;
-  // one (prepared, register check) pair per kernel instantiation: [merging]
-  static std::atomic<uint64_t> prepared[2];
-  static std::atomic<int> regs_ok[2];
-  auto* kernel = merge ? spa::spa_fwd_kernel<D, true> : spa::spa_fwd_kernel<D, false>;
+  // one (prepared, register check) pair per kernel instantiation:
+  // [merging][turns]
+  static std::atomic<uint64_t> prepared[2][2];
+  static std::atomic<int> regs_ok[2][2];
+  // The softmax warpgroups take turns when the bands are wide on average:
+  // measured on B1 H32 N32768 d128, taking turns is 5 % slower at width
+  // 512, even at 768, 5 % faster at 1024 and 13 % at 2048.
+  int64_t width_sum = 0;
+  for (int h = 0; h < p.H; ++h) width_sum += (int64_t)(p.hi[h] - p.lo[h]);
+  const bool turn = width_sum >= kFwdTurnMinWidth * (int64_t)p.H;
+  auto* kernel = merge ? (turn ? spa::spa_fwd_kernel<D, true, true> : spa::spa_fwd_kernel<D, true, false>)
+                       : (turn ? spa::spa_fwd_kernel<D, false, true> : spa::spa_fwd_kernel<D, false, false>);
   const int64_t BH = (int64_t)p.B * p.H;
   CUtensorMap mq, mk, mv;
   int st;
   if ((st = make_map(&mq, q, p.N, BH, D, C::BQ)) || (st = make_map(&mk, k, p.N, BH, D, C::BK)) ||
       (st = make_map(&mv, v, p.N, BH, D, C::BK)))
     return st;
-  if ((st = prepare_kernel(kernel, C::SMEM_BYTES, prepared[merge]))) return st;
-  if ((st = check_regs(kernel, (int)C::LAUNCH_REGS, regs_ok[merge]))) return st;
+  if ((st = prepare_kernel(kernel, C::SMEM_BYTES, prepared[merge][turn]))) return st;
+  if ((st = check_regs(kernel, (int)C::LAUNCH_REGS, regs_ok[merge][turn]))) return st;
   // Work list of the persistent grid: per batch, every 256-row block of every
   // head from the one holding lo_h on (units), and the blocks before it (fills).
   const int64_t nblk = (p.N + C::BU - 1) / C::BU;
