@@ -115,6 +115,24 @@ def test_edge_shapes_every_element(spa, B, H, N, d):
     _full_check(spa, q, k, v, do, 1 / math.sqrt(d))
 
 
+# Mean band width of at least 768: the forward's two softmax warpgroups take
+# turns (the narrower shapes above run them freely), with ragged tails and both
+# head dims; the last two are dense causal attention on every head.
+WIDE_SHAPES = [(1, 1, 1000, 64), (2, 2, 1777, 128), (1, 3, 2500, 64), (1, 1, 3001, 128)]
+
+
+@pytest.mark.parametrize("B,H,N,d", WIDE_SHAPES)
+def test_wide_bands_every_element(spa, B, H, N, d):
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=11 + N + H)
+    _full_check(spa, q, k, v, do, 1 / math.sqrt(d))
+
+
+@pytest.mark.parametrize("B,H,N,d", [(1, 2, 1100, 64), (2, 3, 900, 128)])
+def test_full_bands_every_element(spa, B, H, N, d):
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=13 + N)
+    _full_check(spa, q, k, v, do, 1 / math.sqrt(d), [0] * H, [N] * H)
+
+
 @pytest.mark.parametrize("kind", ["full", "first_half", "shared_window", "odd"])
 def test_explicit_bands(spa, kind):
     B, H, N, d = 1, 4, 600, 64

@@ -54,6 +54,10 @@ CASES = [
     (1, 8, 1001, 64, 64),
     (1, 3, 129, 128, 5),
     (1, 32, 2048, 128, 256),
+    # both parts at least 768 wide on average: the merging forward in the
+    # form whose softmax warpgroups take turns
+    (1, 1, 2000, 64, 10),
+    (2, 2, 3200, 128, 700),
 ]
 
 
