@@ -1,0 +1,52 @@
+"""bench.py on CPU: the reference arm (the fp64 oracle, the only arm that runs
+without a GPU) prints one JSON line with the keys the benchmark contract
+names; the CUDA arm refuses to run without a device instead of falling back;
+fewer than three warm-up steps are rejected."""
+import json
+import os
+import subprocess
+import sys
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench(*args, timeout=300):
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    return subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), *args], cwd=ROOT, env=env,
+                          capture_output=True, text=True, timeout=timeout)
+
+
+def test_reference_arm_prints_the_contract_line():
+    r = _bench("--impl", "reference", "--workload", "b1_h4_n256_d64", "--steps", "1", "--warmup", "3")
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    for key in ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better",
+                "scaling", "vs_baseline", "dtype", "data", "config", "cpu_baseline", "e2e"):
+        assert key in line, key
+    assert line["impl"] == "reference"
+    assert line["value"] > 0 and line["ms_per_step"] > 0
+    assert line["steps"] == 1 and line["warmup"] == 3 and line["n_gpus"] == 1
+    assert line["higher_is_better"] is True and line["vs_baseline"] is None
+    assert line["config"]["workload"] == "b1_h4_n256_d64"
+    cpu = line["cpu_baseline"]
+    assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] == line["value"]
+    e2e = line["e2e"]
+    assert e2e["value"] == line["value"] and e2e["unit"] == line["unit"]
+    assert e2e["h2d_bytes_per_step"] == 0 and e2e["d2h_bytes_per_step"] == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the behaviour without a CUDA device")
+@pytest.mark.parametrize("extra", [[], ["--decode"], ["--union", "256"]])
+def test_cuda_arm_refuses_to_run_without_a_device(extra):
+    r = _bench("--steps", "1", "--warmup", "3", *extra)
+    assert r.returncode != 0
+    assert "needs a CUDA device" in (r.stdout + r.stderr)
+
+
+def test_fewer_than_three_warmup_steps_are_rejected():
+    r = _bench("--impl", "reference", "--workload", "b1_h4_n256_d64", "--steps", "1", "--warmup", "2")
+    assert r.returncode != 0
+    assert "--warmup must be >= 3" in r.stderr
