@@ -1,7 +1,8 @@
 """bench.py on CPU: the reference arm (the fp64 oracle, the only arm that runs
 without a GPU) prints one JSON line with the keys the benchmark contract
 names; the CUDA arm refuses to run without a device instead of falling back;
-fewer than three warm-up steps are rejected."""
+fewer than three warm-up steps are rejected; the DRAM traffic of a kernel is
+read from an ncu summary only when the summary names the current sources."""
 import json
 import os
 import subprocess
@@ -50,3 +51,22 @@ def test_fewer_than_three_warmup_steps_are_rejected():
     r = _bench("--impl", "reference", "--workload", "b1_h4_n256_d64", "--steps", "1", "--warmup", "2")
     assert r.returncode != 0
     assert "--warmup must be >= 3" in r.stderr
+
+
+def test_traffic_is_read_only_from_a_summary_of_the_current_sources(tmp_path, monkeypatch):
+    import bench
+    csrc = tmp_path / "head_partitioned_distance_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cuh").write_text("// kernel v1\n")
+    (tmp_path / "profiles").mkdir()
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    sha = bench.kernel_src_sha()
+    (tmp_path / "profiles" / "k_w.md").write_text(
+        "# summary\n\ntraffic: kernel=spa_k workload=w1 src_sha=%s dram_bytes_per_launch=12345\n" % sha)
+    assert bench.ncu_traffic("spa_k", "w1") == 12345.0
+    assert bench.ncu_traffic("spa_k", "w2") is None          # another workload
+    assert bench.ncu_traffic("spa_other", "w1") is None      # another kernel
+    (csrc / "k.cuh").write_text("// kernel v2\n")             # the kernel changed since the capture
+    assert bench.kernel_src_sha() != sha
+    assert bench.ncu_traffic("spa_k", "w1") is None
+
