@@ -72,6 +72,8 @@ def seq_to_heads(x: torch.Tensor, heads: Sequence[Sequence[int]], group=None) ->
     order), by one all-to-all.  ``heads[r]`` lists rank r's heads."""
     world = _group_size(group)
     B, H, n, d = x.shape
+    if len(heads) != world or any(len(hs) * world != H for hs in heads):
+        raise ValueError("heads must list H / world heads for each rank of the group")
     hl = H // world
     send = torch.stack([x[:, list(heads[r])] for r in range(world)]).contiguous()  # [world, B, hl, n, d]
     recv = torch.empty_like(send)
@@ -84,6 +86,10 @@ def heads_to_seq(y: torch.Tensor, heads: Sequence[Sequence[int]], group=None) ->
     """Inverse of seq_to_heads: [B, H / world, N, d] -> [B, H, N / world, d]."""
     world = _group_size(group)
     B, hl, N, d = y.shape
+    if N % world != 0:
+        raise ValueError(f"the sequence ({N} tokens) must split evenly over the {world} ranks")
+    if len(heads) != world or any(len(hs) != hl for hs in heads):
+        raise ValueError("heads must list H / world heads for each rank of the group")
     n = N // world
     send = y.reshape(B, hl, world, n, d).permute(2, 0, 1, 3, 4).contiguous()  # [world, B, hl, n, d]
     recv = torch.empty_like(send)

@@ -121,3 +121,15 @@ def test_sequence_parallel_attention_equals_unsharded(world):
     for _ in range(world):
         rank, errs = q.get(timeout=10)
         assert max(errs) < 1e-12, (rank, errs)
+
+
+def test_exchanges_reject_shapes_that_do_not_split_over_the_group(monkeypatch):
+    # checked before any collective, so no process group is needed
+    monkeypatch.setattr(sharding, "_group_size", lambda group: 2)
+    heads = sharding.paired_heads(4, 2)
+    with pytest.raises(ValueError):
+        sharding.heads_to_seq(torch.zeros(1, 2, 7, 4), heads)        # 7 tokens over 2 ranks
+    with pytest.raises(ValueError):
+        sharding.heads_to_seq(torch.zeros(1, 3, 8, 4), heads)        # 3 local heads, 2 listed per rank
+    with pytest.raises(ValueError):
+        sharding.seq_to_heads(torch.zeros(1, 4, 4, 4), heads[:1])    # one rank's heads for a group of 2
