@@ -83,34 +83,83 @@ def union_pairs(N: int, window: int, bands) -> int:
     return total
 
 
-def kernel_work(w, pairs: int):
-    """Algorithmic work per launch of each kernel: (FLOPs over the permitted
-    pairs, bytes every launch must move at least).  T is one [B, H, N, d] bf16
-    tensor, R one [B, H, N] fp32 row vector (lse or D)."""
+def active_rows(w, bands) -> int:
+    """act = sum over (b, h) of N - lo_h: the query rows whose band is not
+    empty, which equals the number of key rows some query reaches."""
+    return w.B * sum(w.N - int(lo) for lo in bands[0])
+
+
+def kernel_work(w, pairs: int, act: int):
+    """Algorithmic work per launch of each kernel, the accounting of the
+    scope table's measurement section: (useful FLOPs, executed FLOPs, least
+    bytes).  Inputs are counted over the active rows only (head h never reads
+    query rows i < lo_h nor key rows j > N - 1 - lo_h); outputs over every
+    row (every element is written).  T_act / T_all: one [B, H, N, d] bf16
+    tensor over the active / all rows; R_act / R_all: one fp32 row vector
+    (lse or D).  The dQ pass executes S, dP and dQ (6 d per pair) but only
+    dQ is work the dK/dV pass does not already do, so its useful FLOPs are
+    2 d per pair."""
     d = w.d
     rows = w.B * w.H * w.N
-    T, R = rows * d * 2, rows * 4
+    T_all, T_act, R_all, R_act = rows * d * 2, act * d * 2, rows * 4, act * 4
     return {
-        "spa_fwd_kernel": (4 * d * pairs, 4 * T + R),           # S = QK^T, O += PV; q k v in, o lse out
-        "spa_bwd_dq_kernel": (6 * d * pairs, 6 * T + 2 * R),    # S, dP, dQ, D = rowsum(dO * O); q k v o dO lse in, dq D out
-        "spa_bwd_dkdv_kernel": (8 * d * pairs, 6 * T + 2 * R),  # S^T, dP^T, dV, dK; q k v dO lse D in, dk dv out
+        # q k v in over active rows; o, lse out for every row
+        "spa_fwd_kernel": (4 * d * pairs, 4 * d * pairs, 3 * T_act + T_all + R_all),
+        # q k v o dO and lse in over active rows; dq out for every row, D out
+        "spa_bwd_dq_kernel": (2 * d * pairs, 6 * d * pairs, 5 * T_act + 2 * R_act + T_all),
+        # q k v dO, lse and D in over active rows; dk dv out for every row
+        "spa_bwd_dkdv_kernel": (8 * d * pairs, 8 * d * pairs, 4 * T_act + 2 * R_act + 2 * T_all),
     }
 
 
-def step_work(w, pairs: int):
+def step_work(w, pairs: int, act: int):
     """(useful FLOPs, least bytes) of one forward + backward step: 14 d per
-    pair (the forward's two GEMMs, the backward's five), and q k v in, o lse
-    out, then q k v o dO lse in, dq dk dv out (12 T + 2 R).  The kernels
-    execute more FLOPs (S and dP in both backward passes) and move more bytes
-    (each backward pass reads q, k, v, dO); this is the method's floor."""
+    pair (the forward's two GEMMs, the backward's five), and the scope
+    table's bytes -- forward: q k v over active rows in, o lse out for every
+    row; backward: q k v o dO over active rows in, lse and D over active rows,
+    dq dk dv out for every row."""
     rows = w.B * w.H * w.N
-    return 14 * w.d * pairs, 12 * rows * w.d * 2 + 2 * rows * 4
+    d = w.d
+    T_all, T_act, R_all, R_act = rows * d * 2, act * d * 2, rows * 4, act * 4
+    fwd = 3 * T_act + T_all + R_all
+    bwd = 5 * T_act + 2 * R_act + 3 * T_all
+    return 14 * d * pairs, fwd + bwd
 
 
 def roofline_bound(flops: float, nbytes: float, peaks) -> str:
     """"tensor" when the FLOPs at the bf16 peak take longer than the bytes at
     the HBM peak, else "hbm" (the attainable-performance roofline)."""
     return "tensor" if flops / (peaks["bf16_tflops"] * 1e12) >= nbytes / (peaks["hbm_gbs"] * 1e9) else "hbm"
+
+
+def kernel_report(useful: float, executed: float, nbytes: float, avg_ms: float, share: float, peaks):
+    """One kernel against its roofline.  The bound compares the kernel's
+    useful FLOPs at the bf16 peak with its least bytes at the HBM peak;
+    "achieved" is the algorithmic work of that bound (useful FLOPs or least
+    bytes) over the kernel's average launch time.  The executed FLOPs
+    (recomputation included) are reported beside it."""
+    bound = roofline_bound(useful, nbytes, peaks)
+    sec = avg_ms * 1e-3
+    if bound == "tensor":
+        achieved, peak, unit, units = useful / sec / 1e12, peaks["bf16_tflops"], "TFLOP/s", useful
+    else:
+        achieved, peak, unit, units = nbytes / sec / 1e9, peaks["hbm_gbs"], "GB/s", nbytes
+    return {"bound": bound, "avg_ms": avg_ms, "share": share, "achieved": achieved, "peak": peak, "unit": unit,
+            "frac": achieved / peak, "algorithmic_per_launch": units,
+            "useful_flops_per_launch": useful, "executed_flops_per_launch": executed,
+            "bytes_per_launch": nbytes,
+            "useful_tflops": useful / sec / 1e12, "executed_tflops": executed / sec / 1e12,
+            "frac_useful_of_bf16_peak": useful / sec / 1e12 / peaks["bf16_tflops"],
+            "frac_executed_of_bf16_peak": executed / sec / 1e12 / peaks["bf16_tflops"],
+            "gbs": nbytes / sec / 1e9, "frac_of_hbm_peak": nbytes / sec / 1e9 / peaks["hbm_gbs"]}
+
+
+def step_roofline_report(step_flops: float, step_bytes: float, step_ms: float, peaks):
+    t_flops = step_flops / (peaks["bf16_tflops"] * 1e12) * 1e3
+    t_bytes = step_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+    return {"bound": "tensor" if t_flops >= t_bytes else "hbm", "flops": step_flops, "bytes": step_bytes,
+            "t_flops_ms": t_flops, "t_bytes_ms": t_bytes, "t_measured_ms": step_ms,
+            "frac": max(t_flops, t_bytes) / step_ms}
 
 
 def load_peaks():
@@ -158,35 +207,109 @@ def ncu_traffic(kernel: str, workload: str):
 
 
 # --------------------------------------------------------------------- clocks
+# NVML clock-event reason bits (nvmlClocksEventReason*)
+_NVML_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+
 class ClockSampler:
+    """SM clock, power and clock-event reasons of one GPU, sampled every
+    `period_s` by a host thread through NVML (reading only) while the timed
+    region runs, so that even a region of a few tens of milliseconds holds
+    samples.  Falls back to `nvidia-smi -lms 100` when NVML is unavailable."""
+
     FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, torch_device=None, period_s: float = 0.002):
         self.gpu_index = gpu_index
+        self.torch_device = torch_device
+        self.period_s = period_s
         self.proc = None
+        self.thread = None
+        self.samples = []  # (perf_counter, sm_mhz, sm_max_mhz, power_w, reason bits)
         self.t0 = self.t1 = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        if self.torch_device is not None:
+            props = torch.cuda.get_device_properties(self.torch_device)
+            try:
+                return pynvml.nvmlDeviceGetHandleByUUID("GPU-" + str(props.uuid))
+            except Exception:
+                bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+                return pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+        return pynvml.nvmlDeviceGetHandleByIndex(int(self.gpu_index))
 
     def start(self):
+        import threading
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "100", "-i", str(self.gpu_index)],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            import pynvml
+            h = self._nvml_handle()
+            smax = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+            self._stop = threading.Event()
+
+            def loop():
+                while not self._stop.is_set():
+                    try:
+                        t = time.perf_counter()
+                        sm = pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM)
+                        pw = pynvml.nvmlDeviceGetPowerUsage(h) / 1000.0
+                        rs = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                        self.samples.append((t, float(sm), float(smax), pw, int(rs)))
+                    except Exception:
+                        pass
+                    self._stop.wait(self.period_s)
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            self.source = f"NVML, every {self.period_s * 1e3:.0f} ms"
         except Exception:
-            self.proc = None
-        time.sleep(0.3)
+            self.thread = None
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                     "-lms", "100", "-i", str(self.gpu_index)],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                self.source = "nvidia-smi -lms 100"
+            except Exception:
+                self.proc = None
+        time.sleep(0.05)
 
     def mark_start(self):
-        self.t0 = _dt.datetime.now()
+        self.t0 = time.perf_counter()
+        self.d0 = _dt.datetime.now()
 
     def mark_end(self):
-        self.t1 = _dt.datetime.now()
+        self.t1 = time.perf_counter()
+        self.d1 = _dt.datetime.now()
+
+    def _summary(self, rows, inside):
+        sm = [r[1] for r in rows]
+        reasons = set()
+        for r in rows:
+            for bit, name in _NVML_REASONS.items():
+                if r[4] & bit:
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max((r[2] for r in rows if r[2] is not None), default=None),
+                "reasons": sorted(reasons), "samples": len(rows),
+                "window": "timed region" if inside else "whole run (no sample fell inside the timed region)",
+                "power_w_max": max((r[3] for r in rows if r[3] is not None), default=None),
+                "source": self.source}
 
     def stop(self):
+        if self.thread is not None:
+            time.sleep(0.01)
+            self._stop.set()
+            self.thread.join(timeout=5)
+            inside = [r for r in self.samples if self.t0 is not None and self.t0 <= r[0] <= self.t1]
+            return self._summary(inside if inside else self.samples, bool(inside))
         if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"],
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"],
                     "samples": 0}
         time.sleep(0.25)
         self.proc.terminate()
@@ -200,23 +323,16 @@ class ClockSampler:
                 ts = _dt.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f")
             except ValueError:
                 continue
-            rows.append((ts, parts))
-        inside = [p for ts, p in rows if self.t0 and self.t1 and self.t0 <= ts <= self.t1]
-        sample = inside if inside else [p for _, p in rows]
-        sm = [float(p[2]) for p in sample if p[2].replace(".", "").isdigit()]
-        smax = [float(p[3]) for p in sample if p[3].replace(".", "").isdigit()]
-        reasons = set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for p in sample:
-            for n, val in zip(names, p[6:10]):
+            num = lambda x: float(x) if x.replace(".", "").isdigit() else None
+            bits = 0
+            for bit, val in zip((0x8, 0x40, 0x20, 0x4), parts[6:10]):
                 if val.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None,
-                "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sample),
-                "window": "timed region" if inside else "whole run (no sample fell inside the timed region)",
-                "power_w_max": max((float(p[4]) for p in sample
-                                    if p[4].replace(".", "").isdigit()), default=None)}
+                    bits |= bit
+            rows.append((ts, num(parts[2]), num(parts[3]), num(parts[4]), bits))
+        inside = [r for r in rows if self.t0 is not None and self.d0 <= r[0] <= self.d1]
+        sample = inside if inside else rows
+        sample = [r for r in sample if r[1] is not None]
+        return self._summary(sample, bool(inside))
 
 
 # --------------------------------------------------------------------- distributed
@@ -329,10 +445,10 @@ def run_reference(args):
         total_s += s
     value = total_flops / total_s / 1e12
     line = {
-        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total_s / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name, "B": w.B, "H": w.H, "N": w.N, "d": w.d},
+        "data": "synthetic", "config": spa_config(w, w.B * workload_pairs(w.N, bands), world, False),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": desc + " per step"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -390,7 +506,7 @@ def run_decode(args):
     if spa.spa_device_status(stream) != spa.SPA_OK:
         raise SystemExit("device status not OK after warm-up")
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
-    sampler = ClockSampler(visible.split(",")[local] if visible else local)
+    sampler = ClockSampler(visible.split(",")[local] if visible else local, device)
     sampler.start()
     K = args.steps
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -560,6 +676,26 @@ def pipelined_e2e(device, stream, host, dev0, out_names, compute, E, dist):
     return reduce_max(e0.elapsed_time(e1), device), h2d, d2h
 
 
+def flush_needed(w) -> bool:
+    """Inputs smaller than L2 are flushed out of it before every timed step."""
+    return w.B * w.H * w.N * w.d * 2 < L2_BYTES
+
+
+def spa_config(w, pairs: int, world: int, full_bands: bool):
+    """The "config" object of the training-step line (both arms print it)."""
+    B, H, N, d = w.B, w.H, w.N, w.d
+    return {"workload": w.name, "B": B, "H": H, "N": N, "d": d,
+            "bands": ("full: [0, N) on every head (dense causal per head)" if full_bands
+                      else "balanced distance partitioning"),
+            "pairs_per_rank": pairs,
+            "useful_flops_per_rank_step": 14 * d * pairs,
+            "l2": (f"flushed before every step (a {2 * L2_BYTES / 2**20:.0f} MiB write, then a "
+                   f"{HOST_LEAD_CYCLES}-cycle device wait; neither timed)") if flush_needed(w) else
+                  ("no flush: q, k, v, dout are each larger than L2 "
+                   f"({B * H * N * d * 2 / 2**20:.0f} MiB bf16)"),
+            "parallelism": f"{world} independent replicas (one batch each)"}
+
+
 def run_spa(args):
     from head_partitioned_distance_b200 import spa
 
@@ -595,7 +731,7 @@ def run_spa(args):
     # inputs smaller than L2 are flushed out of it before every timed step (a
     # write of a buffer twice its size, outside the timed spans)
     flush = None
-    if B * H * N * d * 2 < L2_BYTES:
+    if flush_needed(w):
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
 
     def step(ev=None):
@@ -616,7 +752,7 @@ def run_spa(args):
         raise SystemExit("device status not OK after warm-up")
 
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
-    sampler = ClockSampler(visible.split(",")[local] if visible else local)
+    sampler = ClockSampler(visible.split(",")[local] if visible else local, device)
     sampler.start()
     K = args.steps
     # per step: its start, then the end of each kernel
@@ -669,45 +805,22 @@ def run_spa(args):
 
     if rank == 0:
         peaks, peak_src = load_peaks()
-        work = kernel_work(w, pairs)
-        kern = {}
-        for name in KERNELS:
-            flops, nbytes = work[name]
-            bound = roofline_bound(flops, nbytes, peaks)
-            avg_ms = per_kernel_ms[name] / K
-            if bound == "tensor":
-                achieved = flops / (avg_ms * 1e-3) / 1e12
-                peak = peaks["bf16_tflops"]
-                unit = "TFLOP/s"
-                units = flops
-            else:
-                achieved = nbytes / (avg_ms * 1e-3) / 1e9
-                peak = peaks["hbm_gbs"]
-                unit = "GB/s"
-                units = nbytes
-            kern[name] = {"bound": bound, "avg_ms": avg_ms, "share": per_kernel_ms[name] / elapsed_ms,
-                          "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
-                          "algorithmic_per_launch": units, "flops_per_launch": flops,
-                          "bytes_per_launch": nbytes,
-                          "tflops": flops / (avg_ms * 1e-3) / 1e12,
-                          "gbs": nbytes / (avg_ms * 1e-3) / 1e9}
+        act = active_rows(w, bands)
+        work = kernel_work(w, pairs, act)
+        kern = {name: kernel_report(*work[name], per_kernel_ms[name] / K, per_kernel_ms[name] / elapsed_ms,
+                                    peaks) for name in KERNELS}
         # the whole step against its attainable roofline: the slower of the
         # useful FLOPs at the bf16 peak and the bytes any forward + backward
         # must move at the HBM peak
-        step_flops, step_bytes = step_work(w, pairs)
-        t_flops = step_flops / (peaks["bf16_tflops"] * 1e12) * 1e3
-        t_bytes = step_bytes / (peaks["hbm_gbs"] * 1e9) * 1e3
-        step_ms = max_ms / K
-        step_roofline = {"bound": "tensor" if t_flops >= t_bytes else "hbm",
-                         "flops": step_flops, "bytes": step_bytes,
-                         "t_flops_ms": t_flops, "t_bytes_ms": t_bytes, "t_measured_ms": step_ms,
-                         "frac": max(t_flops, t_bytes) / step_ms}
+        step_flops, step_bytes = step_work(w, pairs, act)
+        step_roofline = step_roofline_report(step_flops, step_bytes, max_ms / K, peaks)
         dom = max(KERNELS, key=lambda n: per_kernel_ms[n])
         dk_ = kern[dom]
         roofline = {"bound": dk_["bound"], "achieved": dk_["achieved"], "peak": dk_["peak"],
                     "unit": dk_["unit"], "frac": dk_["frac"],
                     "traffic": ncu_traffic(dom, w.name + ("/full-bands" if args.full_bands else "")),
                     "kernel": dom,
+                    "algorithmic_per_launch": dk_["algorithmic_per_launch"],
                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if dk_['bound'] == 'tensor' else 'hbm_gbs'})"}
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
@@ -720,21 +833,14 @@ def run_spa(args):
             "warmup": args.warmup, "ms_per_step": max_ms / K, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "pct_of_bf16_peak": 100.0 * per_gpu / peaks["bf16_tflops"],
-            # the metric's literal wording (10 d per pair over the fwd+bwd time)
+            # the metric's literal wording: 10 d per pair over the fwd+bwd time
+            # (the headline counts 14 d: the forward's 4 d and the backward's 10 d)
             "value_literal_10d": value * 10.0 / 14.0,
+            "pct_of_bf16_peak_literal_10d": 100.0 * per_gpu * 10.0 / 14.0 / peaks["bf16_tflops"],
             "pct_of_bf16_peak_sustained": 100.0 * per_gpu / peaks["bf16_tflops_sustained"],
             "peaks": {**peaks, "source": peak_src},
             "tokens_per_s": world * B * N * K / (max_ms * 1e-3),
-            "config": {"workload": w.name, "B": B, "H": H, "N": N, "d": d,
-                       "bands": ("full: [0, N) on every head (dense causal per head)" if args.full_bands
-                                 else "balanced distance partitioning"),
-                       "pairs_per_rank": pairs,
-                       "useful_flops_per_rank_step": useful,
-                       "l2": ("no flush: q, k, v, dout are each larger than L2 "
-                              f"({B * H * N * d * 2 / 2**20:.0f} MiB bf16)") if flush is None else
-                             (f"flushed before every step (a {2 * L2_BYTES / 2**20:.0f} MiB write, then a "
-                              f"{HOST_LEAD_CYCLES}-cycle device wait; neither timed)"),
-                       "parallelism": f"{world} independent replicas (one batch each)"},
+            "config": spa_config(w, pairs, world, args.full_bands),
             "roofline": roofline,
             "step_roofline": step_roofline,
             "kernels": kern,
@@ -807,7 +913,7 @@ def run_union(args):
         raise SystemExit("device status not OK after warm-up")
 
     visible = os.environ.get("CUDA_VISIBLE_DEVICES")
-    sampler = ClockSampler(visible.split(",")[local] if visible else local)
+    sampler = ClockSampler(visible.split(",")[local] if visible else local, device)
     sampler.start()
     K = args.steps
     t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -909,7 +1015,51 @@ def run_union(args):
     return 0
 
 
+def free_port() -> int:
+    import socket
+    s_ = socket.socket()
+    s_.bind(("127.0.0.1", 0))
+    port = s_.getsockname()[1]
+    s_.close()
+    return port
+
+
+def relaunch(nproc: int, argv) -> int:
+    """`--gpus N` without a torchrun world: start N ranks on this node with
+    torch.distributed.run (rendezvous on 127.0.0.1) running this same
+    command line, and return their exit status."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={nproc}",
+           "--master-addr", "127.0.0.1", f"--master-port={free_port()}", os.path.abspath(__file__), *argv]
+    return subprocess.call(cmd)
+
+
+def run_dry(args):
+    """The launch and reporting path without any GPU work: every rank joins a
+    gloo group, takes part in the barrier and the max over ranks of a
+    (host-timed, trivial) step time, and rank 0 prints the line.  Lets a CPU
+    machine check what --gpus N does."""
+    rank, local, world = dist_setup()
+    dist = dist_init("gloo", local) if world > 1 else None
+    t0 = time.perf_counter()
+    x = torch.ones(64)
+    for _ in range(args.steps):
+        x = x * 1.0
+    ms = (time.perf_counter() - t0) * 1e3
+    if dist:
+        dist.barrier()
+    max_ms = reduce_max(ms, torch.device("cpu"))
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "metric": METRIC, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+                          "warmup": args.warmup, "ms_per_step": max_ms / max(args.steps, 1),
+                          "ranks_reporting": world, "config": {"workload": args.workload}}), flush=True)
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
 def main(argv=None):
+    argv = list(sys.argv[1:] if argv is None else argv)
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=300)
@@ -926,9 +1076,20 @@ def main(argv=None):
                          "kernels, to show the work the bands save")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (one new token per sequence) instead of fwd+bwd")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="run the launch and reporting path (ranks, barrier, max over ranks) with no GPU work")
     args = ap.parse_args(argv)
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    world_env = os.environ.get("WORLD_SIZE")
+    if world_env is None and args.gpus > 1:
+        return relaunch(args.gpus, argv)  # one rank per GPU, this node
+    if world_env is not None and int(world_env) != args.gpus:
+        ap.error(f"--gpus {args.gpus} but this process is one of a world of {world_env} ranks")
+    if args.dry_run:
+        return run_dry(args)
     if args.impl == "reference":
         return run_reference(args)
     if args.decode:

@@ -399,7 +399,11 @@ int union_merge(void* o, float* lse, const void* o2, const float* lse2, int B, i
   if (!aligned(o, 16) || !aligned(o2, 16) || !aligned(lse, 4) || !aligned(lse2, 4)) return SPA_ERR_UNSUPPORTED;
   const int64_t rows = (int64_t)B * H * N;
   const int64_t threads = rows * (d / 8);
-  const unsigned blocks = (unsigned)((threads + 255) / 256);
+  // a grid-stride kernel: at most eight blocks per SM
+  int sms = 0;
+  if ((st = sm_count(&sms))) return st;
+  const int64_t want = (threads + 255) / 256;
+  const unsigned blocks = (unsigned)(want < (int64_t)sms * 8 ? want : (int64_t)sms * 8);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d == 64)
     spa::spa_union_merge_kernel<64><<<blocks, 256, 0, s>>>(static_cast<uint16_t*>(o), lse,
@@ -477,23 +481,61 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
+struct NoallocSlot {
+  unsigned long long ctx_id;  // unique id of the context the address belongs to
+  void* ptr;
+};
+NoallocSlot g_noalloc[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetCurrentFn)(CUcontext*);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long*);
+
+// Unique id of the context current on this thread (ids are never reused
+// within a process, unlike context handles); 0 when it cannot be had.
+unsigned long long current_ctx_id() {
+  static CtxGetCurrentFn get_cur = nullptr;
+  static CtxGetIdFn get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<CtxGetCurrentFn>(p);
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<CtxGetIdFn>(p);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (!get_cur || !get_id || get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr || get_id(ctx, &id) != CUDA_SUCCESS)
+    return 0;
+  return id;
+}
 
 // Device address of g_spa_noalloc_delta on the current device.  The first
-// call on a device resolves it with cudaGetSymbolAddress (that device being
-// current) and caches it; later calls only read the cache.
+// call on a device (with that device current) resolves it with
+// cudaGetSymbolAddress and caches it together with the id of the context it
+// belongs to; later calls in the same context only read the cache.  After a
+// device reset the primary context, and with it the module and its arrays, is
+// new: its id differs, so the address is resolved again.
 int noalloc_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return SPA_ERR_CUDA;
   if (dev < 0 || dev >= kMaxDevices) return SPA_ERR_UNSUPPORTED;
+  // make the device's primary context current on this thread (a thread that
+  // has made no runtime call yet has none)
+  if (cudaSetDevice(dev) != cudaSuccess) return SPA_ERR_CUDA;
+  const unsigned long long id = current_ctx_id();
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_ptr[dev] == nullptr) {
+  NoallocSlot& slot = g_noalloc[dev];
+  if (slot.ptr == nullptr || id == 0 || slot.ctx_id != id) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_spa_noalloc_delta) != cudaSuccess || p == nullptr)
-      return SPA_ERR_CUDA;
-    g_noalloc_ptr[dev] = p;
+    if (cudaGetSymbolAddress(&p, g_spa_noalloc_delta) != cudaSuccess || p == nullptr) return SPA_ERR_CUDA;
+    slot.ptr = p;
+    slot.ctx_id = id;
   }
-  *out = g_noalloc_ptr[dev];
+  *out = slot.ptr;
   return SPA_OK;
 }
 
@@ -646,8 +688,10 @@ int spa_attn_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if ((int64_t)B * H * N > (int64_t)SPA_NOALLOC_MAX_ROWS) return SPA_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   if ((st = noalloc_scratch(&scratch))) return st;
-  // The preprocess step overwrites D for every row before the two passes read
-  // it, so the scratch needs no clearing between calls.
+  // The dQ pass forms D and writes it for every row of the 128-row query
+  // blocks that some band reaches, before the dK/dV pass reads it; the dK/dV
+  // pass reads D only for those rows, so whatever an earlier call left in the
+  // scratch is never read and the array needs no clearing between calls.
   return bwd_entry(q, k, v, o, dout, lse, dq, dk, dv, scratch, B, H, N, d, scale, nullptr, nullptr,
                    stream, kStepAll);
 }

@@ -36,38 +36,45 @@ __device__ __forceinline__ uint4 pack8_bf16(const float (&f)[8]) {
 }
 
 // (o, lse) <- merge of (o, lse) and (o2, lse2), row by row; D / 8 threads per
-// row (16 bytes each), rows of a warp never split across warps.  A row with
-// both parts empty stays o = 0, lse = -inf.
+// row (16 bytes each), rows of a warp never split across warps; grid-stride
+// over the rows, every lane of a warp taking the same number of rounds.  A row
+// with both parts empty stays o = 0, lse = -inf.
 template <int D>
 __global__ void __launch_bounds__(256) spa_union_merge_kernel(uint16_t* __restrict__ o, float* __restrict__ lse,
                                                               const uint16_t* __restrict__ o2,
                                                               const float* __restrict__ lse2, int64_t rows) {
   constexpr int TPR = D / 8;
-  const int64_t t = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int64_t row = t / TPR;
-  const int c = (int)(t % TPR);
-  if (row >= rows) return;
-  const float l1 = lse[row], l2 = lse2[row];
-  const float m = fmaxf(l1, l2);
-  float L = -INFINITY, w1 = 0.f, w2 = 0.f;
-  if (m != -INFINITY) {
-    const float e1 = expf(l1 - m), e2 = expf(l2 - m);
-    const float s = e1 + e2;
-    L = m + logf(s);
-    w1 = e1 / s;
-    w2 = e2 / s;
-  }
-  uint4* po = reinterpret_cast<uint4*>(o + row * D) + c;
-  const uint4 a = *po;
-  const uint4 b = reinterpret_cast<const uint4*>(o2 + row * D)[c];
-  float fa[8], fb[8];
-  unpack8_bf16(a, fa);
-  unpack8_bf16(b, fb);
+  const int64_t total = rows * TPR;
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  for (int64_t base = (int64_t)blockIdx.x * blockDim.x; base < total; base += stride) {
+    const int64_t t = base + threadIdx.x;
+    const int64_t row = t / TPR;
+    const int c = (int)(t % TPR);
+    const bool valid = t < total;
+    const float l1 = valid ? lse[row] : -INFINITY, l2 = valid ? lse2[row] : -INFINITY;
+    // every lane of the row has read lse[row] before lane c = 0 rewrites it
+    __syncwarp();
+    if (!valid) continue;
+    const float m = fmaxf(l1, l2);
+    float L = -INFINITY, w1 = 0.f, w2 = 0.f;
+    if (m != -INFINITY) {
+      const float e1 = expf(l1 - m), e2 = expf(l2 - m);
+      const float s = e1 + e2;
+      L = m + logf(s);
+      w1 = e1 / s;
+      w2 = e2 / s;
+    }
+    uint4* po = reinterpret_cast<uint4*>(o + row * D) + c;
+    const uint4 a = *po;
+    const uint4 b = reinterpret_cast<const uint4*>(o2 + row * D)[c];
+    float fa[8], fb[8];
+    unpack8_bf16(a, fa);
+    unpack8_bf16(b, fb);
 #pragma unroll
-  for (int e = 0; e < 8; ++e) fa[e] = w1 * fa[e] + w2 * fb[e];
-  *po = pack8_bf16(fa);
-  // every lane of the row has read lse[row] (same warp, earlier instruction)
-  if (c == 0) lse[row] = L;
+    for (int e = 0; e < 8; ++e) fa[e] = w1 * fa[e] + w2 * fb[e];
+    *po = pack8_bf16(fa);
+    if (c == 0) lse[row] = L;
+  }
 }
 
 // dst_t += src_t (bf16, summed in fp32, rounded once) for three tensors of

@@ -27,11 +27,13 @@ import torch.distributed as dist
 
 # --------------------------------------------------------------------- assignment
 def band_bounds(N: int, H: int):
-    """Balanced Distance Partitioning bands, lo_h = floor(h N / H),
-    hi_h = floor((h + 1) N / H), as two lists (host integers)."""
+    """Balanced Distance Partitioning bands as two lists (host integers), from
+    the library's own host entry point spa_band_bounds, so the sharding and
+    the kernels can never disagree on them."""
     if H < 1 or N < H:
         raise ValueError("need 1 <= H <= N")
-    return [h * N // H for h in range(H)], [(h + 1) * N // H for h in range(H)]
+    from . import spa  # the C-ABI library; fails loudly when it is not built
+    return spa.spa_band_bounds(N, H)
 
 
 def paired_heads(H: int, world: int) -> List[List[int]]:

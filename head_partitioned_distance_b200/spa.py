@@ -168,9 +168,7 @@ def spa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, scale: float, lo=
                  (dv, "dv")):
         _need(t, (B, H, N, d), torch.bfloat16, n)
     _need(lse, (B, H, N), torch.float32, "lse")
-    if not workspace.is_cuda or workspace.numel() * workspace.element_size() < \
-            spa_attn_bwd_workspace_bytes(B, H, N):
-        raise ValueError("workspace: CUDA tensor of spa_attn_bwd_workspace_bytes(B, H, N) bytes")
+    _need_workspace(workspace, B, H, N)
     s = _stream_ptr(stream)
     ptrs = [t.data_ptr() for t in (q, k, v, o, dout, lse, dq, dk, dv, workspace)]
     if lo is None:
@@ -201,8 +199,27 @@ def spa_attn_bwd_noalloc(q, k, v, o, dout, lse, dq, dk, dv, scale: float, stream
     return dq, dk, dv
 
 
+def _need_workspace(workspace, B, H, N):
+    if not workspace.is_cuda or not workspace.is_contiguous() or \
+            workspace.numel() * workspace.element_size() < spa_attn_bwd_workspace_bytes(B, H, N):
+        raise ValueError("workspace: contiguous CUDA tensor of spa_attn_bwd_workspace_bytes(B, H, N) bytes")
+
+
+def _need_step(B, H, N, d, tensors, lse=None, workspace=None):
+    """The checks spa_attn_bwd makes, for the step entry points: every tensor
+    [B, H, N, d] bf16, contiguous, on the GPU; lse [B, H, N] fp32; the
+    workspace large enough for D."""
+    for t, n in tensors:
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    if lse is not None:
+        _need(lse, (B, H, N), torch.float32, "lse")
+    if workspace is not None:
+        _need_workspace(workspace, B, H, N)
+
+
 def spa_attn_bwd_preprocess(o, dout, workspace, stream=None):
     B, H, N, d = _dims(o)
+    _need_step(B, H, N, d, ((o, "o"), (dout, "dout")), workspace=workspace)
     _check(_lib.spa_attn_bwd_preprocess(o.data_ptr(), dout.data_ptr(), workspace.data_ptr(), B, H, N, d,
                                         _stream_ptr(stream)), "spa_attn_bwd_preprocess")
 
@@ -210,6 +227,8 @@ def spa_attn_bwd_preprocess(o, dout, workspace, stream=None):
 def spa_attn_bwd_dkdv(q, k, v, dout, lse, workspace, dk, dv, scale: float, lo=None, hi=None,
                       stream=None):
     B, H, N, d = _dims(q)
+    _need_step(B, H, N, d, ((q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (dk, "dk"), (dv, "dv")), lse,
+               workspace)
     lo_a = None if lo is None else _i32(lo)
     hi_a = None if hi is None else _i32(hi)
     _check(_lib.spa_attn_bwd_dkdv(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
@@ -220,6 +239,7 @@ def spa_attn_bwd_dkdv(q, k, v, dout, lse, workspace, dk, dv, scale: float, lo=No
 
 def spa_attn_bwd_dq(q, k, v, dout, lse, workspace, dq, scale: float, lo=None, hi=None, stream=None):
     B, H, N, d = _dims(q)
+    _need_step(B, H, N, d, ((q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (dq, "dq")), lse, workspace)
     lo_a = None if lo is None else _i32(lo)
     hi_a = None if hi is None else _i32(hi)
     _check(_lib.spa_attn_bwd_dq(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
@@ -231,6 +251,8 @@ def spa_attn_bwd_dkdv_add(q, k, v, dout, lse, workspace, dk, dv, scale: float, l
                           stream=None):
     """The dk/dv pass adding to dk, dv instead of overwriting them."""
     B, H, N, d = _dims(q)
+    _need_step(B, H, N, d, ((q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (dk, "dk"), (dv, "dv")), lse,
+               workspace)
     lo_a = None if lo is None else _i32(lo)
     hi_a = None if hi is None else _i32(hi)
     _check(_lib.spa_attn_bwd_dkdv_add(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
@@ -242,6 +264,7 @@ def spa_attn_bwd_dkdv_add(q, k, v, dout, lse, workspace, dk, dv, scale: float, l
 def spa_attn_bwd_dq_add(q, k, v, dout, lse, workspace, dq, scale: float, lo=None, hi=None, stream=None):
     """The dq pass adding to dq instead of overwriting it."""
     B, H, N, d = _dims(q)
+    _need_step(B, H, N, d, ((q, "q"), (k, "k"), (v, "v"), (dout, "dout"), (dq, "dq")), lse, workspace)
     lo_a = None if lo is None else _i32(lo)
     hi_a = None if hi is None else _i32(hi)
     _check(_lib.spa_attn_bwd_dq_add(q.data_ptr(), k.data_ptr(), v.data_ptr(), dout.data_ptr(),
@@ -252,6 +275,8 @@ def spa_attn_bwd_dq_add(q, k, v, dout, lse, workspace, dq, scale: float, lo=None
 def spa_attn_bwd_dq_delta(q, k, v, o, dout, lse, workspace, dq, scale: float, lo=None, hi=None,
                           stream=None):
     B, H, N, d = _dims(q)
+    _need_step(B, H, N, d, ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq")), lse,
+               workspace)
     lo_a = None if lo is None else _i32(lo)
     hi_a = None if hi is None else _i32(hi)
     _check(_lib.spa_attn_bwd_dq_delta(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(),
@@ -321,8 +346,15 @@ def spa_attn_decode(q, k, v, pos, o, lse, workspace, scale: float, lo=None, hi=N
     """One new token per sequence: q [B, H, d] at positions pos (int32 [B]) of
     the caches k, v [B, H, N, d]; writes o [B, H, d] and lse [B, H]."""
     B, H, N, d = _dims(k)
-    if q.shape != (B, H, d) or pos.dtype != torch.int32 or pos.numel() != B:
-        raise ValueError("q is [B, H, d] and pos int32 [B] for caches [B, H, N, d]")
+    _need(k, (B, H, N, d), torch.bfloat16, "k")
+    _need(v, (B, H, N, d), torch.bfloat16, "v")
+    _need(q, (B, H, d), torch.bfloat16, "q")
+    _need(o, (B, H, d), torch.bfloat16, "o")
+    _need(lse, (B, H), torch.float32, "lse")
+    _need(pos, (B,), torch.int32, "pos")
+    if not workspace.is_cuda or not workspace.is_contiguous() or \
+            workspace.numel() * workspace.element_size() < spa_attn_decode_workspace_bytes(B, H, N, d, lo, hi):
+        raise ValueError("workspace: contiguous CUDA tensor of spa_attn_decode_workspace_bytes(...) bytes")
     lo_a = None if lo is None else _i32(lo)
     hi_a = None if hi is None else _i32(hi)
     _check(_lib.spa_attn_decode(q.data_ptr(), k.data_ptr(), v.data_ptr(), pos.data_ptr(), o.data_ptr(),

@@ -203,8 +203,11 @@ SPA_API int spa_attn_bwd_dq_delta(const void* q, const void* k, const void* v, c
  *    library until the process exits.  B * H * N above SPA_NOALLOC_MAX_ROWS is
  *    rejected with SPA_ERR_UNSUPPORTED before anything is launched.
  *  - The first call on a device looks up the array's device address
- *    (cudaGetSymbolAddress, with that device current) and caches it; make that
- *    first call before any stream capture.
+ *    (cudaGetSymbolAddress, with that device current) and caches it with the
+ *    id of the context it belongs to; make that first call before any stream
+ *    capture.  A device reset (cudaDeviceReset) destroys the context and the
+ *    array with it: the first call in the new context looks the address up
+ *    again, and that call too belongs before any capture.
  *  - All calls share the one array and it keeps the last call's contents
  *    (nothing in it needs to start at zero: each call rewrites the rows it
  *    uses before reading them).  Calls whose work overlaps on the GPU -- two

@@ -7,6 +7,7 @@ import re
 
 import numpy as np
 import pytest
+import torch
 
 import oracle
 from head_partitioned_distance_b200 import spa
@@ -245,3 +246,34 @@ def test_union_parts_split_each_head_into_two_disjoint_intervals(N, H, w):
         assert p1 | p2 == want
     with pytest.raises(spa.SpaError):
         spa.spa_union_parts(16, 16, 1)  # head 0 is the single distance 0
+
+
+def test_step_wrappers_reject_bad_tensors_before_the_library():
+    # Every backward step wrapper, like spa_attn_bwd, checks shape, dtype,
+    # contiguity, device and the workspace size before it hands pointers to
+    # the library; on this CPU-only machine a check that passed would reach
+    # the library with host pointers, so each case must raise ValueError.
+    from head_partitioned_distance_b200 import spa
+    B, H, N, d = 1, 2, 64, 64
+    t = lambda *shape, dt=torch.bfloat16: torch.zeros(shape, dtype=dt)
+    q, k, v, o, do, dq, dk, dv = (t(B, H, N, d) for _ in range(8))
+    lse = t(B, H, N, dt=torch.float32)
+    ws = t(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dt=torch.float32)
+    short = t(B * H * N // 2, dt=torch.float32)
+    bad_do = t(B, H, N - 1, d)
+    bad_lse = t(B, H, N, dt=torch.float16)
+    calls = [
+        lambda: spa.spa_attn_bwd_preprocess(o, do, ws),
+        lambda: spa.spa_attn_bwd_preprocess(o, bad_do, ws),
+        lambda: spa.spa_attn_bwd_dkdv(q, k, v, do, lse, ws, dk, dv, 0.1),
+        lambda: spa.spa_attn_bwd_dkdv(q, k, v, bad_do, lse, ws, dk, dv, 0.1),
+        lambda: spa.spa_attn_bwd_dq(q, k, v, do, bad_lse, ws, dq, 0.1),
+        lambda: spa.spa_attn_bwd_dkdv_add(q, k, v, do, lse, short, dk, dv, 0.1),
+        lambda: spa.spa_attn_bwd_dq_add(q, k, v, do, lse, ws, dq.float(), 0.1),
+        lambda: spa.spa_attn_bwd_dq_delta(q, k, v, o, do, lse, ws, dq, 0.1),
+        lambda: spa.spa_attn_bwd_dq_delta(q, k, v, o.transpose(2, 3), do, lse, ws, dq, 0.1),
+    ]
+    for i, call in enumerate(calls):
+        with pytest.raises(ValueError):
+            call()
+            pytest.fail(f"call {i} was not rejected")

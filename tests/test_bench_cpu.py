@@ -32,6 +32,11 @@ def test_reference_arm_prints_the_contract_line():
     assert line["steps"] == 1 and line["warmup"] == 3 and line["n_gpus"] == 1
     assert line["higher_is_better"] is True and line["vs_baseline"] is None
     assert line["config"]["workload"] == "b1_h4_n256_d64"
+    # the same config keys the CUDA arm prints, so the two lines compare
+    import bench
+    from head_partitioned_distance_b200 import synth
+    w = synth.WORKLOADS["b1_h4_n256_d64"]
+    assert line["config"] == bench.spa_config(w, 256 * 257 // 2, 1, False)
     cpu = line["cpu_baseline"]
     assert cpu["kind"] == "oracle" and cpu["cores"] >= 1 and cpu["value"] == line["value"]
     e2e = line["e2e"]
@@ -70,3 +75,21 @@ def test_traffic_is_read_only_from_a_summary_of_the_current_sources(tmp_path, mo
     assert bench.kernel_src_sha() != sha
     assert bench.ncu_traffic("spa_k", "w1") is None
 
+
+def test_gpus_n_starts_n_ranks():
+    # --gpus 2 without a torchrun world starts two ranks itself; the dry run
+    # takes the launch and reporting path with no GPU work (gloo group,
+    # barrier, max over ranks), and rank 0 alone prints the line.
+    r = _bench("--gpus", "2", "--dry-run", "--steps", "3", "--warmup", "3", timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = [json.loads(x) for x in r.stdout.strip().splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    assert lines[0]["n_gpus"] == 2 and lines[0]["dry_run"] is True
+
+
+def test_gpus_must_match_the_world_it_runs_in():
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="", WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--dry-run"], cwd=ROOT,
+                       env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode != 0
+    assert "world of 1 ranks" in r.stderr

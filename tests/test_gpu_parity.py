@@ -115,6 +115,23 @@ def test_edge_shapes_every_element(spa, B, H, N, d):
     _full_check(spa, q, k, v, do, 1 / math.sqrt(d))
 
 
+# Plain bands at d = 128 where the dK/dV and dQ passes run more than one unit
+# per CTA (the persistent grid has at most 148 CTAs): unit boundaries, the
+# epilogue overlapping the next unit's first steps, TMEM reuse across units.
+# B1 H16 N4096: 272 key-tile units, 272 query-tile units; B2 H8 N3000: a
+# ragged tail and bands of width 375.
+MULTI_UNIT_SHAPES = [(1, 16, 4096, 128), (2, 8, 3000, 128)]
+
+
+@pytest.mark.parametrize("B,H,N,d", MULTI_UNIT_SHAPES)
+def test_multi_unit_per_cta_every_element(spa, B, H, N, d):
+    lo, _ = oracle.bands(N, H)
+    units = B * sum((N - 1 - int(l)) // 128 + 1 for l in lo)
+    assert units > 148  # more units than CTAs on a B200
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=17 + N + H)
+    _full_check(spa, q, k, v, do, 1 / math.sqrt(d))
+
+
 # Mean band width of at least 768: the forward's two softmax warpgroups take
 # turns (the narrower shapes above run them freely), with ragged tails and both
 # head dims; the last two are dense causal attention on every head.
@@ -336,6 +353,23 @@ def test_tile_classes_on_device_bit_exact(spa, N, H, Bq, Bk):
 LARGE = ["b8_h16_n4096_d128", "b4_h32_n8192_d128", "b1_h32_n32768_d128", "b1_h32_n30001_d128"]
 
 
+def _targeted_key_rows(B, H, N, lo):
+    """Key rows of every head (in batch h mod B) where the dK/dV pass changes
+    regime: the last key some query reaches (N - 1 - lo_h), the first that
+    none does (N - lo_h, whose dk and dv must be exactly 0), both sides of
+    the 128-key tile boundaries at the first tile, the middle of the head
+    and the last reached tile, and the last key of the sequence (the ragged
+    tail tile when N is not a multiple of 128)."""
+    out = []
+    for h in range(H):
+        last = N - 1 - int(lo[h])
+        tiles = {1, (N // 2) // 128, last // 128}
+        cand = {last, last + 1, N - 1} | {128 * t - 1 for t in tiles} | {128 * t for t in tiles}
+        base = ((h % B) * H + h) * N
+        out += [base + j for j in cand if 0 <= j < N]
+    return out
+
+
 def _sampled_check(spa, w, n_random, n_key_rows, full_bands=False):
     q, k, v, do = synth.workload_inputs(w)
     B, H, N, d = w.B, w.H, w.N, w.d
@@ -351,8 +385,8 @@ def _sampled_check(spa, w, n_random, n_key_rows, full_bands=False):
                 for h in range(H)]
     rows = synth.sample_rows(B, H, N, n_random, seed=w.seed, per_head=per_head)
     g = torch.Generator().manual_seed(w.seed + 1)
-    key_rows = sorted(set(torch.randint(0, B * H * N, (n_key_rows,), generator=g).tolist()
-                          + [N - 1, (H - 1) * N + N - 1 - int(lo[H - 1])]))
+    key_rows = sorted(set(torch.randint(0, B * H * N, (n_key_rows,), generator=g).tolist())
+                      | set(_targeted_key_rows(B, H, N, lo)))
     flat = lambda x: x.reshape(B * H * N, -1)
     ok = {"o": [], "dq": [], "dk": [], "dv": []}
     refs = {"o": [], "dq": [], "dk": [], "dv": []}
@@ -377,6 +411,10 @@ def _sampled_check(spa, w, n_random, n_key_rows, full_bands=False):
             idx = [bh * N + j for j in ks]
             ok["dk"].append(flat(got["dk"])[idx]); refs["dk"].append(dk_r)
             ok["dv"].append(flat(got["dv"])[idx]); refs["dv"].append(dv_r)
+    # keys that no query reaches (j > N - 1 - lo_h) get exactly zero
+    unreached = [r for r in key_rows if (r % N) > N - 1 - int(lo[(r // N) % H])]
+    for name in ("dk", "dv"):
+        assert not flat(got[name])[unreached].any(), name
     cat = lambda xs: np.concatenate(xs, axis=0)
     assert np.abs(cat(ok["o"]) - cat(refs["o"])).max() <= O_TOL
     _check_lse(np.concatenate(lse_got), np.concatenate(lse_ref))

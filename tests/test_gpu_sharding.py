@@ -1,14 +1,17 @@
 """Head sharding with the CUDA op inside: a one-rank NCCL group on cuda:0
 (the only multi-GPU form this suite can run) must give exactly the unsharded
 spattention output and gradients, since one rank holds every head in order
-and the all-to-alls are copies."""
+and the all-to-alls are copies, and both must match the fp64 oracle within
+the parity tolerances."""
 import os
 import socket
 
+import numpy as np
 import pytest
 import torch
 import torch.distributed as dist
 
+import oracle
 from head_partitioned_distance_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -43,5 +46,12 @@ def test_one_rank_sequence_parallel_attention_is_spattention():
         assert torch.equal(o, orf)
         for a, b in ((qs.grad, qr.grad), (ks.grad, kr.grad), (vs.grad, vr.grad)):
             assert torch.equal(a, b)
+        # the sharded run against the oracle (the gradient of sum(o * do))
+        f64 = lambda t: t.detach().to("cpu", torch.float64).numpy()
+        qf, kf, vf, dof = (f64(t) for t in (q, k, v, do))
+        o_ref, _ = oracle.spa_fwd(qf, kf, vf, 0.125)
+        assert np.abs(f64(o) - o_ref).max() <= 2e-2
+        for g, ref in zip((qs.grad, ks.grad, vs.grad), oracle.spa_bwd(qf, kf, vf, dof, 0.125)):
+            assert np.abs(f64(g) - ref).max() / np.abs(ref).max() <= 5e-2
     finally:
         dist.destroy_process_group()

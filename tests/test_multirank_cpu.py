@@ -67,19 +67,52 @@ def test_kernel_work_and_roofline_bound():
     import bench
     from head_partitioned_distance_b200 import synth
     peaks = {"bf16_tflops": 1600.0, "hbm_gbs": 6400.0}  # ridge point 250 FLOP per byte
+    # B4 H32 N8192 d128 by hand: lo_h = 256 h, so the active rows (query rows
+    # with a non-empty band, = key rows some query reaches) are
+    # 4 * sum_h (8192 - 256 h) = 4 * (32 * 8192 - 256 * 496) = 540672.
+    w = synth.WORKLOADS["b4_h32_n8192_d128"]
+    bands = ([256 * h for h in range(32)], [256 * (h + 1) for h in range(32)])
+    act = bench.active_rows(w, bands)
+    assert act == 540672
+    pairs = 4 * 8192 * 8193 // 2
+    T_act, T_all = 540672 * 128 * 2, 4 * 32 * 8192 * 128 * 2  # bf16 tensors: active rows / every row
+    R_act, R_all = 540672 * 4, 4 * 32 * 8192 * 4              # fp32 row vectors
+    work = bench.kernel_work(w, pairs, act)
+    assert work["spa_fwd_kernel"] == (4 * 128 * pairs, 4 * 128 * pairs, 3 * T_act + T_all + R_all)
+    assert work["spa_bwd_dq_kernel"] == (2 * 128 * pairs, 6 * 128 * pairs, 5 * T_act + 2 * R_act + T_all)
+    assert work["spa_bwd_dkdv_kernel"] == (8 * 128 * pairs, 8 * 128 * pairs, 4 * T_act + 2 * R_act + 2 * T_all)
+    flops, nbytes = bench.step_work(w, pairs, act)
+    assert flops == 14 * 128 * pairs
+    # the measurement section's figures for this workload: 0.69 GB forward,
+    # 1.50 GB backward
+    assert round((3 * T_act + T_all + R_all) / 1e9, 2) == 0.69
+    assert round((5 * T_act + 2 * R_act + 3 * T_all) / 1e9, 2) == 1.50
+    assert nbytes == 8 * T_act + 4 * T_all + R_all + 2 * R_act
+    # useful FLOPs over the three kernels: 4 + 2 + 8 = 14 d per pair; executed 18 d
+    assert sum(u for u, _, _ in work.values()) == 14 * 128 * pairs
+    assert sum(e for _, e, _ in work.values()) == 18 * 128 * pairs
+    # at width 256 every kernel moves more bytes than its useful FLOPs need time
+    assert all(bench.roofline_bound(u, b, peaks) == "hbm" for u, _, b in work.values())
+    # width-1024 bands (B1 H32 N32768): the forward and dK/dV are tensor-bound,
+    # the dQ pass's 2 d useful FLOPs per pair are not
     w = synth.WORKLOADS["b1_h32_n32768_d128"]
-    pairs = w.B * w.N * (w.N + 1) // 2  # the bands partition the causal distances
-    work = bench.kernel_work(w, pairs)
-    T, R = w.B * w.H * w.N * w.d * 2, w.B * w.H * w.N * 4
-    # S and dP run in both backward passes: 18 d per pair executed, 14 d useful
-    assert sum(f for f, _ in work.values()) == 18 * w.d * pairs
-    assert sum(b for _, b in work.values()) == 16 * T + 5 * R
-    assert bench.step_work(w, pairs) == (14 * w.d * pairs, 12 * T + 2 * R)
-    # width-1024 bands: about 4 d W FLOPs against 8 d bytes per row in the forward
-    assert all(bench.roofline_bound(f, b, peaks) == "tensor" for f, b in work.values())
-    # width-256 bands at d = 128 move more bytes than the tensor cores need time for
-    w = synth.WORKLOADS["b8_h16_n4096_d128"]
-    work = bench.kernel_work(w, w.B * w.N * (w.N + 1) // 2)
-    assert bench.roofline_bound(*work["spa_fwd_kernel"], peaks) == "hbm"
+    bands = ([1024 * h for h in range(32)], [1024 * (h + 1) for h in range(32)])
+    pairs = 32768 * 32769 // 2
+    work = bench.kernel_work(w, pairs, bench.active_rows(w, bands))
+    assert bench.roofline_bound(work["spa_fwd_kernel"][0], work["spa_fwd_kernel"][2], peaks) == "tensor"
+    assert bench.roofline_bound(work["spa_bwd_dkdv_kernel"][0], work["spa_bwd_dkdv_kernel"][2], peaks) == "tensor"
+    assert bench.roofline_bound(work["spa_bwd_dq_kernel"][0], work["spa_bwd_dq_kernel"][2], peaks) == "hbm"
     assert bench.roofline_bound(1000.0, 4.0, peaks) == "tensor"
     assert bench.roofline_bound(1000.0, 4.1, peaks) == "hbm"
+
+
+def test_kernel_report_uses_the_bound_s_algorithmic_work():
+    import bench
+    peaks = {"bf16_tflops": 1600.0, "hbm_gbs": 6400.0}
+    r = bench.kernel_report(1.6e12, 3.2e12, 1e6, 2.0, 0.5, peaks)  # 1.6 TFLOP in 2 ms: tensor-bound
+    assert r["bound"] == "tensor" and r["unit"] == "TFLOP/s"
+    assert r["achieved"] == pytest.approx(800.0) and r["frac"] == pytest.approx(0.5)
+    assert r["executed_tflops"] == pytest.approx(1600.0)
+    r = bench.kernel_report(1e9, 1e9, 6.4e9, 2.0, 0.5, peaks)  # 6.4 GB in 2 ms: HBM-bound
+    assert r["bound"] == "hbm" and r["unit"] == "GB/s"
+    assert r["achieved"] == pytest.approx(3200.0) and r["frac"] == pytest.approx(0.5)

@@ -1,10 +1,11 @@
 """Head sharding (head_partitioned_distance_b200/sharding.py) on CPU: the pair
 assignment and its balance, and -- with 2 and 4 gloo ranks -- the
 sequence <-> head all-to-all and sequence-parallel attention, whose output and
-gradients must equal the same attention run unsharded.  The attention inside
-is injected: a differentiable fp64 CPU band attention written here (the
-CUDA op needs a GPU), identical in the sharded and unsharded runs, so these
-tests check the sharding and the exchange, not the kernel."""
+gradients must equal the oracle's on the unsharded tensors.  The attention
+inside each rank is the fp64 oracle (spa_fwd / spa_bwd with the rank's heads
+and their global bands) wrapped as an autograd function, since the CUDA op
+needs a GPU: these tests check the sharding and the exchange against the
+oracle's whole-batch result, not the kernel."""
 import os
 import socket
 
@@ -25,23 +26,30 @@ def _free_port():
     return port
 
 
-def band_attention_cpu(q, k, v, scale=None, lo=None, hi=None):
-    """Band-sparse attention on [B, Hl, N, d] fp64 CPU tensors, head i with
-    band [lo[i], hi[i]); rows with no permitted key give 0."""
-    B, Hl, N, d = q.shape
-    scale = d ** -0.5 if scale is None else scale
-    i = torch.arange(N)[:, None]
-    j = torch.arange(N)[None, :]
-    outs = []
-    for h in range(Hl):
-        mask = (j <= i) & (i - j >= lo[h]) & (i - j < hi[h])
-        s = scale * q[:, h] @ k[:, h].transpose(-1, -2)
-        s = s.masked_fill(~mask, float("-inf"))
-        m = s.amax(-1, keepdim=True).clamp(min=-1e300).detach()
-        e = torch.exp(s - m) * mask
-        p = e / e.sum(-1, keepdim=True).clamp(min=1e-300)
-        outs.append(p @ v[:, h])
-    return torch.stack(outs, 1)
+class _OracleAttention(torch.autograd.Function):
+    """The oracle's band attention on [B, Hl, N, d] fp64 CPU tensors, head i
+    with band [lo[i], hi[i]); the backward is the oracle's gradient of
+    sum(o * dout)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, scale, lo, hi):
+        ctx.save_for_backward(q, k, v)
+        ctx.scale, ctx.lo, ctx.hi = scale, lo, hi
+        o, _ = oracle.spa_fwd(q.numpy(), k.numpy(), v.numpy(), scale, lo, hi)
+        return torch.from_numpy(o)
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v = ctx.saved_tensors
+        grads = oracle.spa_bwd(q.numpy(), k.numpy(), v.numpy(), dout.contiguous().numpy(), ctx.scale,
+                               ctx.lo, ctx.hi)
+        return tuple(torch.from_numpy(g) for g in grads) + (None, None, None)
+
+
+def oracle_attention(q, k, v, scale=None, lo=None, hi=None):
+    scale = q.shape[-1] ** -0.5 if scale is None else scale
+    return _OracleAttention.apply(q.contiguous(), k.contiguous(), v.contiguous(), scale,
+                                  [int(x) for x in lo], [int(x) for x in hi])
 
 
 # ------------------------------------------------------------------ assignment
@@ -90,25 +98,24 @@ def _worker(rank, world, port, q):
         xh = sharding.seq_to_heads(chunk(full[0]), heads)
         assert torch.equal(xh, full[0][:, heads[rank]])
         assert torch.equal(sharding.heads_to_seq(xh, heads), chunk(full[0]))
-        # sequence-parallel attention against the unsharded run
+        # sequence-parallel attention against the oracle on the whole batch
         ql, kl, vl = (chunk(t).requires_grad_(True) for t in full[:3])
-        o = sharding.sequence_parallel_attention(ql, kl, vl, H, scale=0.3, attn_fn=band_attention_cpu)
+        o = sharding.sequence_parallel_attention(ql, kl, vl, H, scale=0.3, attn_fn=oracle_attention)
         (o * chunk(full[3])).sum().backward()
-        lo, hi = sharding.band_bounds(N, H)
-        qf, kf, vf = (t.clone().requires_grad_(True) for t in full[:3])
-        of = band_attention_cpu(qf, kf, vf, scale=0.3, lo=lo, hi=hi)
-        (of * full[3]).sum().backward()
-        errs = [(o - chunk(of)).abs().max().item()]
+        qn, kn, vn, dn = (t.numpy() for t in full)
+        of, _ = oracle.spa_fwd(qn, kn, vn, 0.3)
+        gq, gk, gv = oracle.spa_bwd(qn, kn, vn, dn, 0.3)
+        errs = [(o - chunk(torch.from_numpy(of))).abs().max().item()]
         # each token's gradient comes back to the rank that holds the token
-        for gl, gf in ((ql.grad, qf.grad), (kl.grad, kf.grad), (vl.grad, vf.grad)):
-            errs.append((gl - chunk(gf)).abs().max().item())
+        for gl, gf in ((ql.grad, gq), (kl.grad, gk), (vl.grad, gv)):
+            errs.append((gl - chunk(torch.from_numpy(gf))).abs().max().item())
         q.put((rank, errs))
     finally:
         dist.destroy_process_group()
 
 
 @pytest.mark.parametrize("world", [2, 4])
-def test_sequence_parallel_attention_equals_unsharded(world):
+def test_sequence_parallel_attention_equals_the_oracle(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()

@@ -20,9 +20,6 @@ from head_partitioned_distance_b200 import synth
 
 pytestmark = pytest.mark.gpu
 
-# the tolerance the parity tests use for gradients: max|g - g_ref| / max|g_ref|
-GRAD_TOL = 5e-2
-
 
 @pytest.fixture(scope="module")
 def spa():
@@ -40,29 +37,31 @@ def _noalloc(spa, q, k, v, o, do, lse, dq, dk, dv, scale):
     return spa._lib.spa_attn_bwd_noalloc(*ptrs, B, H, N, d, ctypes.c_float(scale), stream)
 
 
-def _rel(a, b):
-    a, b = a.double(), b.double()
-    denom = b.abs().max().item()
-    err = (a - b).abs().max().item()
-    return err if denom == 0 else err / denom
+def _case(spa, B, H, N, d, seed):
+    dev = torch.device("cuda:0")
+    q, k, v, do = (t.to(dev) for t in synth.make_inputs(B, H, N, d, seed=seed))
+    scale = 1 / math.sqrt(d)
+    o, lse = spa.attention_forward(q, k, v, scale)
+    return q, k, v, o, do, lse, scale
 
 
 @pytest.mark.parametrize("B,H,N,d", [(1, 8, 1001, 64), (2, 4, 777, 128), (1, 32, 32768, 128)])
 def test_noalloc_backward_matches_workspace_backward_twice(spa, B, H, N, d):
-    dev = torch.device("cuda:0")
-    q, k, v, do = (t.to(dev) for t in synth.make_inputs(B, H, N, d, seed=31 + N))
-    scale = 1 / math.sqrt(d)
-    o, lse = spa.attention_forward(q, k, v, scale)
-    ref = spa.attention_backward(q, k, v, o, do, lse, scale)
-    torch.cuda.synchronize()
-    for call in range(2):  # two calls in a row share (and reuse) the scratch array
+    # Both entry points run the same two kernels on the same D, so the
+    # gradients must be bit-identical.  The first no-allocation call runs on
+    # other inputs of the same shape, so the scratch array holds a different D
+    # when the second call starts: the second call is right only if it writes
+    # every D value it reads.
+    first = _case(spa, B, H, N, d, seed=97 + N)
+    second = _case(spa, B, H, N, d, seed=31 + N)
+    for call, (q, k, v, o, do, lse, scale) in enumerate((first, second)):
+        ref = spa.attention_backward(q, k, v, o, do, lse, scale)
         dq, dk, dv = (torch.full_like(q, float("nan")) for _ in range(3))
         assert _noalloc(spa, q, k, v, o, do, lse, dq, dk, dv, scale) == spa.SPA_OK
         torch.cuda.synchronize()
         assert spa.spa_device_status() == spa.SPA_OK
         for got, want, name in zip((dq, dk, dv), ref, ("dq", "dk", "dv")):
-            assert not torch.isnan(got).any(), (call, name)
-            assert _rel(got, want) <= GRAD_TOL, (call, name)
+            assert torch.equal(got, want), (call, name)
 
 
 def test_noalloc_rejects_sizes_beyond_its_scratch(spa):
