@@ -55,9 +55,13 @@ DEFAULT_WORKLOAD = "b1_h32_n32768_d128"
 L2_BYTES = 126 * 2**20
 HOST_LEAD_CYCLES = 400_000  # about 0.2 ms at the B200's clocks
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-# one step = the forward, the dQ pass (which also forms the row sums D) and the
-# dK/dV pass, in launch order
-KERNELS = ("spa_fwd_kernel", "spa_bwd_dq_kernel", "spa_bwd_dkdv_kernel")
+# one step = the forward, then the backward, in launch order.  Two-pass
+# backward: the dQ pass (which also forms the row sums D) and the dK/dV pass.
+# One-pass backward: D and the zeroed fp32 dq sums, the pass over key tiles,
+# and dq from the sums.
+KERNELS_TWO_PASS = ("spa_fwd_kernel", "spa_bwd_dq_kernel", "spa_bwd_dkdv_kernel")
+KERNELS_FUSED = ("spa_fwd_kernel", "spa_bwd_fused_prep_kernel", "spa_bwd_fused_kernel", "spa_bwd_dq_convert_kernel")
+KERNELS = KERNELS_TWO_PASS
 
 
 # --------------------------------------------------------------------- counting
@@ -102,9 +106,18 @@ def kernel_work(w, pairs: int, act: int):
     d = w.d
     rows = w.B * w.H * w.N
     T_all, T_act, R_all, R_act = rows * d * 2, act * d * 2, rows * 4, act * 4
+    F_act = act * d * 4  # one fp32 [B, H, N, d] buffer over the active rows
     return {
         # q k v in over active rows; o, lse out for every row
         "spa_fwd_kernel": (4 * d * pairs, 4 * d * pairs, 3 * T_act + T_all + R_all),
+        # one-pass backward: o dO in, D out, fp32 dq sums zeroed over the
+        # active rows; dq zeroed on the others
+        "spa_bwd_fused_prep_kernel": (0, 0, 2 * T_act + R_act + F_act + (T_all - T_act)),
+        # S^T, dP^T, dV, dK, dQ: q k v dO lse D in over active rows, dk dv out
+        # for every row, the fp32 dq sums read and written once
+        "spa_bwd_fused_kernel": (10 * d * pairs, 10 * d * pairs, 4 * T_act + 2 * R_act + 2 * T_all + 2 * F_act),
+        # dq from the sums over the active rows
+        "spa_bwd_dq_convert_kernel": (0, 0, F_act + T_act),
         # q k v o dO and lse in over active rows; dq out for every row, D out
         "spa_bwd_dq_kernel": (2 * d * pairs, 6 * d * pairs, 5 * T_act + 2 * R_act + T_all),
         # q k v dO, lse and D in over active rows; dk dv out for every row
@@ -204,6 +217,66 @@ def ncu_traffic(kernel: str, workload: str):
                             and fields.get("src_sha") == sha):
                         return float(fields["dram_bytes_per_launch"])
     return None
+
+
+# --------------------------------------------------------------------- ncu summaries
+_NCU_UNITS = {"byte": 1.0, "Kbyte": 1e3, "Mbyte": 1e6, "Gbyte": 1e9, "Tbyte": 1e12}
+_NCU_ROWS = [
+    ("gpu__time_duration.sum", "duration (serialised, under ncu)"),
+    ("sm__cycles_elapsed.avg.per_second", "SM clock under ncu"),
+    ("dram__bytes_read.sum", "DRAM bytes read"),
+    ("dram__bytes_write.sum", "DRAM bytes written"),
+    ("gpu__dram_throughput.avg.pct_of_peak_sustained_elapsed", "DRAM throughput, % of peak"),
+    ("sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active", "tensor pipe active, % of active cycles"),
+    ("sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_elapsed", "tensor pipe active, % of elapsed cycles"),
+    ("smsp__issue_active.avg.pct_of_peak_sustained_active", "issue active, % of peak"),
+    ("lts__throughput.avg.pct_of_peak_sustained_elapsed", "L2 throughput, % of peak"),
+    ("sm__warps_active.avg.pct_of_peak_sustained_active", "warps active, % of peak"),
+    ("launch__registers_per_thread", "registers per thread at launch"),
+]
+
+
+def ncu_summary(csv_path: str, kernel: str, workload: str, command: str, src_sha: str, note: str = "") -> str:
+    """Markdown summary of one captured launch from `ncu -i REP --page raw
+    --csv` output: the metrics the roofline uses (DRAM bytes, tensor-pipe and
+    issue activity, L2 and DRAM throughput), the three largest warp stall
+    reasons, and the `traffic:` line that bench.py reads back (DRAM bytes
+    read + written by the launch, tagged with the kernel sources' hash)."""
+    import csv
+    rows = list(csv.reader(open(csv_path)))
+    start = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
+    hdr, units = rows[start], rows[start + 1]
+    data = [r for r in rows[start + 2:] if len(r) == len(hdr) and kernel in r[hdr.index("Kernel Name")]]
+    if len(data) != 1:
+        raise SystemExit(f"{csv_path}: expected one launch of {kernel}, found {len(data)}")
+    rec = dict(zip(hdr, data[0]))
+    unit = dict(zip(hdr, units))
+
+    def val(name):
+        return float(rec[name].replace(",", ""))
+
+    dram = {}
+    for name in ("dram__bytes_read.sum", "dram__bytes_write.sum"):
+        dram[name] = val(name) * _NCU_UNITS.get(unit[name], 1.0)
+    lines = [f"# ncu --set full -- {rec['Kernel Name'].split('(')[0]}, workload {workload}", "",
+             "Command (after the same command exited 0 without ncu; one kernel, one launch):", "",
+             f"    {command}", ""]
+    if note:
+        lines += [note, ""]
+    lines += ["| metric | value |", "|---|---|"]
+    for name, desc in _NCU_ROWS:
+        if name in rec and rec[name] != "":
+            lines.append(f"| {desc} (`{name}`) | {rec[name]} {unit[name]} |")
+    stalls = sorted(((val(h), h) for h in hdr if h.startswith("smsp__average_warps_issue_stalled_")
+                     and h.endswith("_per_issue_active.ratio") and rec.get(h, "") != ""
+                     and "selected" not in h), reverse=True)[:3]
+    lines.append("| top stalls per issued instruction | " + ", ".join(
+        f"{h[len('smsp__average_warps_issue_stalled_'):-len('_per_issue_active.ratio')]} {v:.2f}" for v, h in stalls)
+        + " |")
+    total = dram["dram__bytes_read.sum"] + dram["dram__bytes_write.sum"]
+    lines += ["", f"DRAM bytes per launch (read + written): {total / 1e9:.4f} GB.", "",
+              f"traffic: kernel={kernel} workload={workload} src_sha={src_sha} dram_bytes_per_launch={int(total)}"]
+    return "\n".join(lines) + "\n"
 
 
 # --------------------------------------------------------------------- clocks
@@ -734,10 +807,24 @@ def run_spa(args):
     if flush_needed(w):
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
 
+    fused = args.bwd == "fused"
+    kernels = KERNELS_FUSED if fused else KERNELS_TWO_PASS
+    if fused:
+        ws = torch.empty(spa.spa_attn_bwd_fused_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32,
+                         device=device)
+
     def step(ev=None):
         spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, stream=stream, **lo_hi)
         if ev is not None:
             ev[1].record(stream)
+        if fused:
+            # the three launches of spa_attn_bwd_fused, an event after each
+            for i, st in enumerate((1, 2, 4)):
+                spa.spa_attn_bwd_fused(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, scale, stream=stream, steps=st,
+                                       **lo_hi)
+                if ev is not None:
+                    ev[2 + i].record(stream)
+            return
         spa.spa_attn_bwd_dq_delta(qd, kd, vd, o, dod, lse, ws, dq, scale, stream=stream, **lo_hi)
         if ev is not None:
             ev[2].record(stream)
@@ -756,7 +843,7 @@ def run_spa(args):
     sampler.start()
     K = args.steps
     # per step: its start, then the end of each kernel
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)] for _ in range(K)]
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(len(kernels) + 1)] for _ in range(K)]
     if dist:
         dist.barrier()
     torch.cuda.synchronize(device)
@@ -781,9 +868,9 @@ def run_spa(args):
         elapsed_ms = evs[0][0].elapsed_time(evs[-1][-1])
     else:
         elapsed_ms = sum(e[0].elapsed_time(e[-1]) for e in evs)
-    per_kernel_ms = {name: 0.0 for name in KERNELS}
+    per_kernel_ms = {name: 0.0 for name in kernels}
     for e in evs:
-        for i, name in enumerate(KERNELS):
+        for i, name in enumerate(kernels):
             per_kernel_ms[name] += e[i].elapsed_time(e[i + 1])
     max_ms = reduce_max(elapsed_ms, device)
     value = aggregate(useful, K, world, max_ms)
@@ -794,8 +881,9 @@ def run_spa(args):
 
     def compute(S):
         spa.spa_attn_fwd(S["q"], S["k"], S["v"], S["o"], S["lse"], scale, stream=stream, **lo_hi)
-        spa.spa_attn_bwd(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"],
-                         S["ws"], scale, stream=stream, **lo_hi)
+        bwd = spa.spa_attn_bwd_fused if fused else spa.spa_attn_bwd
+        bwd(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"], S["ws"], scale,
+            stream=stream, **lo_hi)
 
     e2e_ms, h2d, d2h = pipelined_e2e(device, stream, host, dev0, ("o", "lse", "dq", "dk", "dv"), compute, E,
                                      dist)
@@ -808,13 +896,13 @@ def run_spa(args):
         act = active_rows(w, bands)
         work = kernel_work(w, pairs, act)
         kern = {name: kernel_report(*work[name], per_kernel_ms[name] / K, per_kernel_ms[name] / elapsed_ms,
-                                    peaks) for name in KERNELS}
+                                    peaks) for name in kernels}
         # the whole step against its attainable roofline: the slower of the
         # useful FLOPs at the bf16 peak and the bytes any forward + backward
         # must move at the HBM peak
         step_flops, step_bytes = step_work(w, pairs, act)
         step_roofline = step_roofline_report(step_flops, step_bytes, max_ms / K, peaks)
-        dom = max(KERNELS, key=lambda n: per_kernel_ms[n])
+        dom = max(kernels, key=lambda n: per_kernel_ms[n])
         dk_ = kern[dom]
         roofline = {"bound": dk_["bound"], "achieved": dk_["achieved"], "peak": dk_["peak"],
                     "unit": dk_["unit"], "frac": dk_["frac"],
@@ -848,7 +936,9 @@ def run_spa(args):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": e2e_ms / E,
                     "schedule": E2E_SCHEDULE},
-            "gpu_launches": len(KERNELS) * K,
+            "gpu_launches": len(kernels) * K,
+            "backward": ("one pass over key tiles (spa_attn_bwd_fused: prep, pass, dq convert)" if fused
+                         else "two passes (spa_attn_bwd: dQ pass forming D, dK/dV pass)"),
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -1074,11 +1164,25 @@ def main(argv=None):
     ap.add_argument("--full-bands", action="store_true",
                     help="run every head with the full band [0, N) (dense causal per head) through the same "
                          "kernels, to show the work the bands save")
+    ap.add_argument("--bwd", choices=["fused", "two-pass"], default="two-pass",
+                    help="backward of the timed step: the one-pass backward (spa_attn_bwd_fused) or the "
+                         "deterministic two-pass one (spa_attn_bwd)")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (one new token per sequence) instead of fwd+bwd")
+    ap.add_argument("--ncu-summary", metavar="CSV",
+                    help="print the markdown summary of one launch from `ncu -i REP --page raw --csv` output "
+                         "(with --ncu-kernel, --ncu-command; --workload names the workload captured)")
+    ap.add_argument("--ncu-kernel", default="")
+    ap.add_argument("--ncu-command", default="")
+    ap.add_argument("--ncu-note", default="")
+    ap.add_argument("--src-sha", default="", help="kernel sources the capture ran on (default: the current ones)")
     ap.add_argument("--dry-run", action="store_true",
                     help="run the launch and reporting path (ranks, barrier, max over ranks) with no GPU work")
     args = ap.parse_args(argv)
+    if args.ncu_summary:
+        print(ncu_summary(args.ncu_summary, args.ncu_kernel, args.workload, args.ncu_command,
+                          args.src_sha or kernel_src_sha(), args.ncu_note), end="")
+        return 0
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
     if args.gpus < 1:

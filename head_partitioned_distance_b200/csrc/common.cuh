@@ -47,6 +47,7 @@ struct AttnParams {
   void* dv;
   const void* o_in;
   const void* dout;
+  float* dq_acc;      // fused backward: fp32 dQ sums, [B, H, N, d]
   int32_t lo[kMaxHeads];
   int32_t hi[kMaxHeads];
   int32_t unit_start[kMaxHeads + 1];

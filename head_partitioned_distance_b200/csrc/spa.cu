@@ -13,6 +13,7 @@
 #include "spa.h"
 
 #include "bwd.cuh"
+#include "bwd_fused.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "fwd.cuh"
@@ -291,6 +292,67 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     const int64_t units = (int64_t)p.B * upb;
     const unsigned grid = (unsigned)(units < sms ? units : sms);
     kernel_kv<<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
+    if ((st = launch_status())) return st;
+  }
+  return SPA_OK;
+}
+
+// Bytes of the fused backward's workspace: D (fp32 [B H N], padded to 256
+// bytes) then the fp32 dQ sums [B H N d].
+size_t fused_delta_bytes(int64_t rows) { return (size_t)((rows * 4 + 255) & ~int64_t(255)); }
+
+// The fused backward: D and the zeroed dQ sums (prep kernel), the one pass
+// over key tiles (dK, dV and the dQ sums), dq from the sums (convert kernel).
+enum FusedStep { kFusedPrep = 1, kFusedPass = 2, kFusedConvert = 4, kFusedAll = 7 };
+
+template <int D>
+int fused_impl(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, void* workspace, AttnParams& p, cudaStream_t stream, int steps) {
+  using C = spa::FusedCfg<D>;
+  static std::atomic<uint64_t> prepared;
+  static std::atomic<int> regs_ok;
+  const int64_t BH = (int64_t)p.B * p.H;
+  const int64_t rows = BH * p.N;
+  int st;
+  p.lse = const_cast<float*>(lse);
+  p.delta = static_cast<float*>(workspace);
+  p.dq_acc = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + fused_delta_bytes(rows));
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.o_in = o;
+  p.dout = dout;
+  int sms = 0;
+  if ((st = sm_count(&sms))) return st;
+  const int64_t cap = (int64_t)sms * 8;
+  const int64_t want = (rows * (D / 8) + 255) / 256;
+  const unsigned eblocks = (unsigned)(want < cap ? want : cap);
+  if (steps & kFusedPrep) {
+    spa::spa_bwd_fused_prep_kernel<D><<<eblocks, 256, 0, stream>>>(p);
+    if ((st = launch_status())) return st;
+  }
+  if (steps & kFusedPass) {
+  CUtensorMap kq, kk, kv, kdo, kdk, kdv;
+  if ((st = make_map(&kq, q, p.N, BH, D, C::BQ)) || (st = make_map(&kk, k, p.N, BH, D, C::BK)) ||
+      (st = make_map(&kv, v, p.N, BH, D, C::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, C::BQ)) ||
+      (st = make_map(&kdk, dk, p.N, BH, D, 32)) || (st = make_map(&kdv, dv, p.N, BH, D, 32)))
+    return st;
+  auto* kernel = spa::spa_bwd_fused_kernel<D>;
+  if ((st = prepare_kernel(kernel, C::SMEM_BYTES, prepared))) return st;
+  if ((st = check_regs(kernel, (int)C::LAUNCH_REGS, regs_ok))) return st;
+  const int64_t nkt = (p.N + 127) / 128;
+  if (BH * nkt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+  if ((st = set_work_lists(
+           p, [&](int h) { return (p.N - 1 - p.lo[h]) / 128 + 1; },
+           [&](int h) { return nkt - ((p.N - 1 - p.lo[h]) / 128 + 1); })))
+    return st;
+  const int64_t units = (int64_t)p.B * p.units_per_batch;
+  const unsigned grid = (unsigned)(units < sms ? units : sms);
+  kernel<<<grid, C::NTHREADS, C::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
+  if ((st = launch_status())) return st;
+  }
+  if (steps & kFusedConvert) {
+    spa::spa_bwd_dq_convert_kernel<D><<<eblocks, 256, 0, stream>>>(p);
     if ((st = launch_status())) return st;
   }
   return SPA_OK;
@@ -633,6 +695,46 @@ int spa_attn_bwd_dq_delta(const void* q, const void* k, const void* v, const voi
                           float scale, const int32_t* lo, const int32_t* hi, void* stream) {
   return bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, workspace, B, H, N, d, scale, lo, hi, stream,
                    kStepDqDelta);
+}
+
+size_t spa_attn_bwd_fused_workspace_bytes(int B, int H, int64_t N, int d) {
+  if (check_shape(B, H, N, d)) return 0;
+  const int64_t rows = (int64_t)B * H * N;
+  return fused_delta_bytes(rows) + (size_t)rows * (size_t)d * sizeof(float);
+}
+
+int spa_attn_bwd_fused(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                       const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int H, int64_t N,
+                       int d, float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+  return spa_attn_bwd_fused_steps(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, d, scale, lo, hi, stream,
+                                  kFusedAll);
+}
+
+int spa_attn_bwd_fused_steps(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                             const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int H,
+                             int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi, void* stream,
+                             int steps) {
+  if (steps < 1 || steps > kFusedAll) return SPA_ERR_INVAL;
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return SPA_ERR_INVAL;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return SPA_ERR_INVAL;
+  for (const void* t : {q, k, v, o, dout, (const void*)dq})
+    if (!aligned(t, 16)) return SPA_ERR_UNSUPPORTED;
+  // dk and dv leave in 32-byte stores, the workspace in 16-byte reductions
+  if (!aligned(dk, 32) || !aligned(dv, 32) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return SPA_ERR_UNSUPPORTED;
+  static AttnParams zero{};
+  AttnParams p = zero;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.scale = scale;
+  p.scale_log2 = scale * spa::kLog2e;
+  if ((st = fill_bands(p, H, N, lo, hi))) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return d == 64 ? fused_impl<64>(q, k, v, o, dout, lse, dq, dk, dv, workspace, p, s, steps)
+                 : fused_impl<128>(q, k, v, o, dout, lse, dq, dk, dv, workspace, p, s, steps);
 }
 
 int spa_tile_schedule(int64_t N, int H, const int32_t* lo, const int32_t* hi, int Bq, int Bk,

@@ -51,6 +51,9 @@ EXPORTS = {
     "spa_attn_decode_workspace_bytes": ([_int, _int, _i64, _int, _i32p, _i32p], ctypes.c_size_t),
     "spa_attn_decode": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_noalloc": ([_vp] * 9 + [_int, _int, _i64, _int, _f32, _vp], _int),
+    "spa_attn_bwd_fused_workspace_bytes": ([_int, _int, _i64, _int], ctypes.c_size_t),
+    "spa_attn_bwd_fused": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
+    "spa_attn_bwd_fused_steps": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp, _int], _int),
     "spa_attn_union_workspace_bytes": ([_int, _int, _i64, _int], ctypes.c_size_t),
     "spa_union_parts": ([_i64, _int, _i64, _i32p, _i32p, _i32p, _i32p, _i32p, _i32p], _int),
     "spa_attn_union_merge": ([_vp] * 4 + [_int, _int, _i64, _int, _vp], _int),
@@ -177,6 +180,45 @@ def spa_attn_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, scale: float, lo=
         _check(_lib.spa_attn_bwd_ex(*ptrs, B, H, N, d, scale, _i32(lo), _i32(hi), s),
                "spa_attn_bwd_ex")
     return dq, dk, dv
+
+
+def spa_attn_bwd_fused_workspace_bytes(B: int, H: int, N: int, d: int) -> int:
+    return int(_lib.spa_attn_bwd_fused_workspace_bytes(B, H, N, d))
+
+
+def spa_attn_bwd_fused(q, k, v, o, dout, lse, dq, dk, dv, workspace, scale: float, lo=None, hi=None,
+                       stream=None, steps: int = 7):
+    """The backward in one pass over the key tiles (spa_attn_bwd_fused in
+    spa.h): same gradients as spa_attn_bwd, dq summed in fp32 by reductions
+    (not bit-reproducible from call to call).  workspace: CUDA tensor of at
+    least spa_attn_bwd_fused_workspace_bytes(B, H, N, d) bytes."""
+    B, H, N, d = _dims(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    _need(lse, (B, H, N), torch.float32, "lse")
+    if not workspace.is_cuda or not workspace.is_contiguous() or \
+            workspace.numel() * workspace.element_size() < spa_attn_bwd_fused_workspace_bytes(B, H, N, d):
+        raise ValueError("workspace: contiguous CUDA tensor of spa_attn_bwd_fused_workspace_bytes(B, H, N, d) bytes")
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    ptrs = [t.data_ptr() for t in (q, k, v, o, dout, lse, dq, dk, dv, workspace)]
+    if steps == 7:
+        _check(_lib.spa_attn_bwd_fused(*ptrs, B, H, N, d, scale, lo_a, hi_a, _stream_ptr(stream)),
+               "spa_attn_bwd_fused")
+    else:  # one or two of its launches (spa_attn_bwd_fused_steps)
+        _check(_lib.spa_attn_bwd_fused_steps(*ptrs, B, H, N, d, scale, lo_a, hi_a, _stream_ptr(stream), steps),
+               "spa_attn_bwd_fused_steps")
+    return dq, dk, dv
+
+
+def attention_backward_fused(q, k, v, o, dout, lse, scale=None, lo=None, hi=None):
+    """Allocate dq / dk / dv / workspace and run spa_attn_bwd_fused."""
+    B, H, N, d = _dims(q)
+    scale = d ** -0.5 if scale is None else scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(spa_attn_bwd_fused_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32, device=q.device)
+    return spa_attn_bwd_fused(q, k, v, o, dout, lse, dq, dk, dv, ws, scale, lo, hi)
 
 
 SPA_NOALLOC_MAX_ROWS = 1 << 20

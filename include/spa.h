@@ -138,6 +138,47 @@ SPA_API int spa_attn_bwd_ex(const void* q, const void* k, const void* v, const v
                     const int32_t* lo, const int32_t* hi, void* stream);
 
 /*
+ * Backward in one pass over the key tiles: the same gradients as
+ * spa_attn_bwd (the derivative written above), with S and dP computed once
+ * per tile pair instead of once in each of two passes.  dk and dv are
+ * accumulated per key tile as in spa_attn_bwd; dq is produced per (key tile,
+ * query tile) pair and summed over the key tiles in an fp32 buffer by
+ * reduction operations, then rounded to bf16 once.  Because those sums
+ * arrive in no fixed order, dq may differ in its last bits from one call to
+ * the next (dk and dv are bit-reproducible); spa_attn_bwd is the
+ * deterministic backward.
+ *   workspace: DEVICE buffer of spa_attn_bwd_fused_workspace_bytes(B, H, N, d)
+ *              bytes, 256-byte aligned, caller-owned, contents overwritten
+ *              (D and the fp32 sums; nothing in it needs to be initialised)
+ *   lo, hi:    HOST band arrays (rules of spa_attn_fwd_ex) or both NULL for
+ *              the Balanced Distance Partitioning bands
+ * Other arguments, layouts and errors as spa_attn_bwd; dk and dv must be
+ * 32-byte aligned and dq 16-byte aligned.
+ */
+SPA_API size_t spa_attn_bwd_fused_workspace_bytes(int B, int H, int64_t N, int d);
+SPA_API int spa_attn_bwd_fused(const void* q, const void* k, const void* v, const void* o,
+                               const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                               void* workspace, int B, int H, int64_t N, int d, float scale,
+                               const int32_t* lo, const int32_t* hi, void* stream);
+
+/*
+ * The three launches of spa_attn_bwd_fused, callable one at a time (to time
+ * each, or to let other work run between them); `steps` is a bit mask, and
+ * the three bits together are spa_attn_bwd_fused:
+ *   1  D_i = sum_c dout_ic o_ic into the workspace and the fp32 dq sums set
+ *      to zero, for every row of the query tiles some band reaches; dq = 0 on
+ *      the rows before them;
+ *   2  the pass over the key tiles: dk and dv written, dq sums added to;
+ *   4  dq = bf16(scale * sums) on the rows of the reached query tiles.
+ * Each step needs the ones before it to have run on the same workspace.  A
+ * mask outside [1, 7] is SPA_ERR_INVAL.
+ */
+SPA_API int spa_attn_bwd_fused_steps(const void* q, const void* k, const void* v, const void* o,
+                                     const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                     void* workspace, int B, int H, int64_t N, int d, float scale,
+                                     const int32_t* lo, const int32_t* hi, void* stream, int steps);
+
+/*
  * The three steps spa_attn_bwd runs, callable one by one (for example to run
  * the dk/dv and dq passes on two streams once the first step is done).  Same
  * tensors and rules as spa_attn_bwd; lo/hi are HOST band arrays or both NULL

@@ -156,6 +156,37 @@ def test_entry_points_reject_bad_arguments_before_any_launch():
     assert L.spa_attn_bwd(p, p, p, p, p, p, p, p, p, None, 1, 4, 256, 64, 0.1, None) == spa.SPA_ERR_INVAL
 
 
+def test_fused_backward_rejects_bad_arguments_before_any_launch():
+    L = spa._lib
+    p = _fake(1 << 20)
+    f = lambda *a, steps=7: L.spa_attn_bwd_fused_steps(*a, 1, 4, 256, 64, 0.1, None, None, None, steps)
+    ten = [p] * 10
+    assert f(*ten, steps=0) == spa.SPA_ERR_INVAL
+    assert f(*ten, steps=8) == spa.SPA_ERR_INVAL
+    for i in range(10):  # every pointer is required
+        args = list(ten)
+        args[i] = None
+        assert f(*args) == spa.SPA_ERR_INVAL
+        assert L.spa_attn_bwd_fused(*args, 1, 4, 256, 64, 0.1, None, None, None) == spa.SPA_ERR_INVAL
+    half = _fake((1 << 20) + 16)
+    for i in (7, 8):  # dk, dv leave in 32-byte stores
+        args = list(ten)
+        args[i] = half
+        assert f(*args) == spa.SPA_ERR_UNSUPPORTED
+    args = list(ten)
+    args[9] = _fake((1 << 20) + 128)  # workspace must be 256-byte aligned
+    assert f(*args) == spa.SPA_ERR_UNSUPPORTED
+    assert L.spa_attn_bwd_fused(*ten, 1, 4, 256, 96, 0.1, None, None, None) == spa.SPA_ERR_UNSUPPORTED
+    assert L.spa_attn_bwd_fused(*ten, 1, 8, 4, 64, 0.1, None, None, None) == spa.SPA_ERR_INVAL
+
+
+def test_fused_workspace_size():
+    # D (fp32 per row, padded to 256 bytes), then the fp32 dq sums
+    assert spa.spa_attn_bwd_fused_workspace_bytes(1, 32, 32768, 128) == 4 * 32 * 32768 * (1 + 128)
+    assert spa.spa_attn_bwd_fused_workspace_bytes(1, 1, 3, 64) == 256 + 4 * 3 * 64
+    assert spa.spa_attn_bwd_fused_workspace_bytes(1, 1, 3, 96) == 0
+
+
 def test_workspace_size():
     assert spa.spa_attn_bwd_workspace_bytes(4, 32, 8192) == 4 * 32 * 8192 * 4
     assert spa.spa_attn_bwd_workspace_bytes(0, 1, 1) == 0

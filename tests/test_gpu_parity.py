@@ -37,13 +37,14 @@ def _f64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def _gpu_run(spa, q, k, v, do, scale, lo=None, hi=None, backward=True):
+def _gpu_run(spa, q, k, v, do, scale, lo=None, hi=None, backward=True, fused=False):
     dev = torch.device("cuda:0")
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     o, lse = spa.attention_forward(qd, kd, vd, scale, lo, hi)
     out = {"o": o, "lse": lse}
     if backward:
-        dq, dk, dv = spa.attention_backward(qd, kd, vd, o, dod, lse, scale, lo, hi)
+        bwd = spa.attention_backward_fused if fused else spa.attention_backward
+        dq, dk, dv = bwd(qd, kd, vd, o, dod, lse, scale, lo, hi)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     assert spa.spa_device_status() == spa.SPA_OK
@@ -73,8 +74,8 @@ def _check_grad(g, ref, name):
         assert err / denom <= GRAD_TOL, (name, err, denom)
 
 
-def _full_check(spa, q, k, v, do, scale, lo=None, hi=None):
-    got = _gpu_run(spa, q, k, v, do, scale, lo, hi)
+def _full_check(spa, q, k, v, do, scale, lo=None, hi=None, fused=False):
+    got = _gpu_run(spa, q, k, v, do, scale, lo, hi, fused=fused)
     qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
     lo_o = None if lo is None else np.array(lo)
     hi_o = None if hi is None else np.array(hi)
@@ -370,15 +371,15 @@ def _targeted_key_rows(B, H, N, lo):
     return out
 
 
-def _sampled_check(spa, w, n_random, n_key_rows, full_bands=False):
+def _sampled_check(spa, w, n_random, n_key_rows, full_bands=False, fused=False):
     q, k, v, do = synth.workload_inputs(w)
     B, H, N, d = w.B, w.H, w.N, w.d
     if full_bands:  # [0, N) on every head: dense causal attention per head
         lo, hi = np.zeros(H, dtype=np.int64), np.full(H, N, dtype=np.int64)
-        got = _gpu_run(spa, q, k, v, do, w.scale, [0] * H, [N] * H)
+        got = _gpu_run(spa, q, k, v, do, w.scale, [0] * H, [N] * H, fused=fused)
     else:
         lo, hi = oracle.bands(N, H)
-        got = _gpu_run(spa, q, k, v, do, w.scale)
+        got = _gpu_run(spa, q, k, v, do, w.scale, fused=fused)
     for name in ("o", "lse", "dq", "dk", "dv"):
         assert not np.isnan(got[name]).any(), name
     per_head = [[int(lo[h]) - 1, int(lo[h]), int(lo[h]) + 1, int(lo[h]) + 127, int(lo[h]) + 128]
@@ -443,3 +444,58 @@ def test_device_wait_timeout_reports_and_recovers(spa):
     w = synth.WORKLOADS["b1_h4_n256_d64"]
     q, k, v, do = synth.workload_inputs(w)
     _full_check(spa, q, k, v, do, w.scale)
+
+
+# ---------------------------------------------------------------------------
+# the one-pass backward (spa_attn_bwd_fused): the same gradients, dq summed
+# over key tiles in fp32 by reductions; every element on small shapes, sampled
+# rows at full size, the same tolerances
+# ---------------------------------------------------------------------------
+FUSED_SHAPES = EDGE_SHAPES + MULTI_UNIT_SHAPES + WIDE_SHAPES
+
+
+@pytest.mark.parametrize("B,H,N,d", FUSED_SHAPES)
+def test_fused_backward_every_element(spa, B, H, N, d):
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=23 + N + H + d)
+    _full_check(spa, q, k, v, do, 1 / math.sqrt(d), fused=True)
+
+
+@pytest.mark.parametrize("kind", ["full", "first_half", "odd"])
+def test_fused_backward_explicit_bands(spa, kind):
+    B, H, N, d = 1, 4, 600, 128
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=101)
+    lo, hi = oracle.bands(N, H)
+    if kind == "full":
+        lo, hi = [0] * H, [N] * H
+    elif kind == "first_half":
+        hi = [int(a + max((b - a) // 2, 1)) for a, b in zip(lo, hi)]
+        lo = [int(a) for a in lo]
+    else:
+        lo, hi = [0, 3, 257, 599], [1, 400, 300, 600]
+    _full_check(spa, q, k, v, do, 0.125, [int(x) for x in lo], [int(x) for x in hi], fused=True)
+
+
+@pytest.mark.parametrize("name", SMALL_WORKLOADS)
+def test_fused_backward_small_workloads(spa, name):
+    w = synth.WORKLOADS[name]
+    q, k, v, do = synth.workload_inputs(w)
+    _full_check(spa, q, k, v, do, w.scale, fused=True)
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_fused_backward_full_size_sampled_rows(spa, name):
+    _sampled_check(spa, synth.WORKLOADS[name], n_random=32, n_key_rows=8, fused=True)
+
+
+def test_fused_backward_dk_dv_match_the_two_pass_backward(spa):
+    # dk and dv come from the same products in the same order as the dK/dV
+    # pass; only D is summed in another order (one row sum per thread group
+    # instead of inside the dQ pass), so they agree to a few bf16 ulps, and
+    # dq agrees within the fp32 reassociation of its sums
+    B, H, N, d = 1, 8, 2048, 128
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=5)
+    a = _gpu_run(spa, q, k, v, do, 1 / math.sqrt(d))
+    b = _gpu_run(spa, q, k, v, do, 1 / math.sqrt(d), fused=True)
+    for name in ("dq", "dk", "dv"):
+        scale = np.abs(a[name]).max()
+        assert np.abs(a[name] - b[name]).max() <= 2e-2 * scale, name

@@ -88,9 +88,16 @@ def test_kernel_work_and_roofline_bound():
     assert round((3 * T_act + T_all + R_all) / 1e9, 2) == 0.69
     assert round((5 * T_act + 2 * R_act + 3 * T_all) / 1e9, 2) == 1.50
     assert nbytes == 8 * T_act + 4 * T_all + R_all + 2 * R_act
-    # useful FLOPs over the three kernels: 4 + 2 + 8 = 14 d per pair; executed 18 d
-    assert sum(u for u, _, _ in work.values()) == 14 * 128 * pairs
-    assert sum(e for _, e, _ in work.values()) == 18 * 128 * pairs
+    # useful FLOPs over the three kernels of the two-pass step: 4 + 2 + 8 = 14 d
+    # per pair; executed 18 d.  The one-pass step executes 14 d.
+    two = [work[k] for k in bench.KERNELS_TWO_PASS]
+    one = [work[k] for k in bench.KERNELS_FUSED]
+    assert sum(u for u, _, _ in two) == sum(u for u, _, _ in one) == 14 * 128 * pairs
+    assert sum(e for _, e, _ in two) == 18 * 128 * pairs
+    assert sum(e for _, e, _ in one) == 14 * 128 * pairs
+    F_act = 540672 * 128 * 4  # the fp32 dq sums over the active rows
+    assert work["spa_bwd_fused_kernel"][2] == 4 * T_act + 2 * R_act + 2 * T_all + 2 * F_act
+    assert work["spa_bwd_dq_convert_kernel"][2] == F_act + T_act
     # at width 256 every kernel moves more bytes than its useful FLOPs need time
     assert all(bench.roofline_bound(u, b, peaks) == "hbm" for u, _, b in work.values())
     # width-1024 bands (B1 H32 N32768): the forward and dK/dV are tensor-bound,
