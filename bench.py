@@ -279,6 +279,43 @@ def ncu_summary(csv_path: str, kernel: str, workload: str, command: str, src_sha
     return "\n".join(lines) + "\n"
 
 
+def ncu_launch_list(csv_path: str, workload: str, command: str, bench_json: str = "", note: str = "") -> str:
+    """Markdown launch list from `ncu --metrics gpu__time_duration.sum --csv`
+    output: per kernel its launches, total time and share under ncu (cold
+    cache, serialised), beside the shares of the same kernels in a bench line
+    (CUDA events), which are what the ncu shares should agree with."""
+    import csv
+    rows = [r for r in csv.reader(l for l in open(csv_path) if l.startswith('"'))]
+    hdr = rows[0]
+    ki, mi, vi = hdr.index("Kernel Name"), hdr.index("Metric Name"), hdr.index("Metric Value")
+    tot = {}
+    for r in rows[1:]:
+        if r[mi] != "gpu__time_duration.sum":
+            continue
+        name = r[ki].split("(")[0].replace("void ", "")
+        n, t = tot.get(name, (0, 0.0))
+        tot[name] = (n + 1, t + float(r[vi].replace(",", "")) * 1e-3)  # ns -> us
+    all_us = sum(t for _, t in tot.values())
+    bench = {}
+    if bench_json:
+        line = json.loads(open(bench_json).read().strip().splitlines()[-1])
+        bench = line.get("kernels", {})
+    lines = [f"# ncu launch list -- bench step, workload {workload}", "",
+             "Command (after the same command exited 0 without ncu):", "", f"    {command}", ""]
+    if note:
+        lines += [note, ""]
+    lines += ["| kernel | launches | total us (ncu) | share (ncu) | bench avg ms (events) | share (bench events) |",
+              "|---|---|---|---|---|---|"]
+    for name, (n, t) in tot.items():
+        base = name.split("<")[0]
+        b = bench.get(base, {})
+        bms = f"{b['avg_ms']:.4f}" if b else "-"
+        bsh = f"{100 * b['share']:.1f} %" if b else "-"
+        lines.append(f"| {name} | {n} | {t:.1f} | {100 * t / all_us:.1f} % | {bms} | {bsh} |")
+    lines += ["", f"Kernel sources: src_sha={kernel_src_sha()}."]
+    return "\n".join(lines) + "\n"
+
+
 # --------------------------------------------------------------------- clocks
 # NVML clock-event reason bits (nvmlClocksEventReason*)
 _NVML_REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
@@ -1172,6 +1209,10 @@ def main(argv=None):
     ap.add_argument("--ncu-summary", metavar="CSV",
                     help="print the markdown summary of one launch from `ncu -i REP --page raw --csv` output "
                          "(with --ncu-kernel, --ncu-command; --workload names the workload captured)")
+    ap.add_argument("--ncu-launch-list", metavar="CSV",
+                    help="print the markdown launch list from `ncu --metrics gpu__time_duration.sum --csv` output "
+                         "(with --ncu-command; --bench-json adds the bench line's event shares)")
+    ap.add_argument("--bench-json", default="")
     ap.add_argument("--ncu-kernel", default="")
     ap.add_argument("--ncu-command", default="")
     ap.add_argument("--ncu-note", default="")
@@ -1179,6 +1220,10 @@ def main(argv=None):
     ap.add_argument("--dry-run", action="store_true",
                     help="run the launch and reporting path (ranks, barrier, max over ranks) with no GPU work")
     args = ap.parse_args(argv)
+    if args.ncu_launch_list:
+        print(ncu_launch_list(args.ncu_launch_list, args.workload, args.ncu_command, args.bench_json, args.ncu_note),
+              end="")
+        return 0
     if args.ncu_summary:
         print(ncu_summary(args.ncu_summary, args.ncu_kernel, args.workload, args.ncu_command,
                           args.src_sha or kernel_src_sha(), args.ncu_note), end="")

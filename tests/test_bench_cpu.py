@@ -93,3 +93,28 @@ def test_gpus_must_match_the_world_it_runs_in():
                        env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode != 0
     assert "world of 1 ranks" in r.stderr
+
+
+def test_ncu_summaries_from_csv(tmp_path):
+    # the summaries under profiles/ are written by these two functions from
+    # ncu's CSV output; check them on a tiny hand-made CSV of each kind
+    import bench
+    raw = tmp_path / "raw.csv"
+    hdr = ["ID", "Kernel Name", "gpu__time_duration.sum", "dram__bytes_read.sum", "dram__bytes_write.sum",
+           "sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active",
+           "smsp__average_warps_issue_stalled_wait_per_issue_active.ratio",
+           "smsp__average_warps_issue_stalled_long_scoreboard_per_issue_active.ratio"]
+    units = ["", "", "us", "Mbyte", "Gbyte", "%", "inst", "inst"]
+    vals = ["0", "void spa_k<128>(CUtensorMap_st)", "12.5", "500", "0.25", "51.5", "1.5", "2.5"]
+    raw.write_text("\n".join(",".join(f'"{x}"' for x in r) for r in (hdr, units, vals)) + "\n")
+    md = bench.ncu_summary(str(raw), "spa_k", "w1", "ncu ...", "abc123")
+    assert "traffic: kernel=spa_k workload=w1 src_sha=abc123 dram_bytes_per_launch=750000000" in md
+    assert "51.5 %" in md and "long_scoreboard 2.50, wait 1.50" in md
+    ll = tmp_path / "ll.csv"
+    rows = [["ID", "Kernel Name", "Metric Name", "Metric Value"]]
+    for i, (k, ns) in enumerate([("a", 300), ("b", 100), ("a", 300), ("b", 300)]):
+        rows.append([str(i), f"void spa_{k}_kernel<128>(x)", "gpu__time_duration.sum", str(ns)])
+    ll.write_text("==PROF== noise\n" + "\n".join(",".join(f'"{x}"' for x in r) for r in rows) + "\n")
+    md = bench.ncu_launch_list(str(ll), "w1", "ncu ...")
+    assert "| spa_a_kernel<128> | 2 | 0.6 | 60.0 % |" in md
+    assert "| spa_b_kernel<128> | 2 | 0.4 | 40.0 % |" in md
