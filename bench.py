@@ -14,9 +14,19 @@ step (forward 4 d, backward 10 d per pair -- the two GEMMs of the forward and
 the five of the backward, over the band's pairs only, never the tile padding),
 over the device time of the K timed steps, max over ranks.
 
+After the headline measurement, a one-GPU run also times every other
+workload of the scope table and the same kernels with full bands (dense causal
+attention on every head), a few steps each, and adds them to the line as
+"per_workload" (ms per step, useful TFLOP/s, % of the bf16 peak, tokens/s,
+fraction of the step roofline); --no-sweep skips it.
+
 N > 1 (torchrun, one process per GPU): every rank runs its own independent
 batch of the same workload (weak scaling); the only collectives are the
-barrier and the max of the timings.
+barrier and the max of the timings.  --gpus N without torchrun starts the N
+ranks itself.
+
+--bwd fused times the one-pass backward (spa_attn_bwd_fused) instead of the
+two-pass one.
 
 --impl reference times the fp64 CPU oracle (the slow, plain implementation the
 tests check against) on a bounded sample of the same workload and prints the
@@ -806,6 +816,72 @@ def spa_config(w, pairs: int, world: int, full_bands: bool):
             "parallelism": f"{world} independent replicas (one batch each)"}
 
 
+SWEEP = [("b1_h4_n256_d64", 50, False), ("b1_h8_n1024_d64", 50, False), ("b1_h8_n1000_d64", 50, False),
+         ("b1_h8_n1001_d64", 50, False), ("b8_h16_n4096_d128", 20, False), ("b4_h32_n8192_d128", 20, False),
+         ("b1_h32_n32768_d128", 10, False), ("b1_h32_n30001_d128", 10, False), ("b4_h32_n8192_d128", 3, True),
+         ("b1_h32_n32768_d128", 3, True)]
+
+
+def sweep_workloads(spa, device, stream, peaks, fused: bool, warmup: int = 3):
+    """Every workload of the scope table, a few steps each, after the headline
+    measurement: ms per step, useful TFLOP/s, % of the bf16 peak, tokens/s and
+    the step's roofline fraction, plus the same kernels with full bands (dense
+    causal attention on every head) at two sizes.  Inputs are drawn on the
+    device with each workload's recipe; workloads smaller than L2 are flushed
+    out of it before every step (untimed); each step is timed with CUDA events
+    on the launching stream and the steps' times are summed."""
+    out = {}
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    for name, K, full in SWEEP:
+        w = synth.WORKLOADS[name]
+        B, H, N, d = w.B, w.H, w.N, w.d
+        bands = ([0] * H, [N] * H) if full else spa.spa_band_bounds(N, H)
+        lo_hi = {"lo": bands[0], "hi": bands[1]} if full else {}
+        q, k, v, do = synth.make_inputs(B, H, N, d, w.seed, w.qkv_mult, w.rms_qk, w.do_mult, device=device)
+        o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
+        lse = torch.empty((B, H, N), dtype=torch.float32, device=device)
+        if fused:
+            ws = torch.empty(spa.spa_attn_bwd_fused_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32,
+                             device=device)
+        else:
+            ws = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=device)
+        bwd = spa.spa_attn_bwd_fused if fused else spa.spa_attn_bwd
+
+        def step():
+            spa.spa_attn_fwd(q, k, v, o, lse, w.scale, stream=stream, **lo_hi)
+            bwd(q, k, v, o, do, lse, dq, dk, dv, ws, w.scale, stream=stream, **lo_hi)
+
+        for _ in range(warmup):
+            step()
+        small = flush_needed(w)
+        ms = 0.0
+        for _ in range(K):
+            if small:
+                flush.fill_(1.0)
+                torch.cuda._sleep(HOST_LEAD_CYCLES)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            e1.synchronize()
+            ms += e0.elapsed_time(e1)
+        if spa.spa_device_status(stream) != spa.SPA_OK:
+            raise SystemExit(f"device status not OK in the sweep ({name})")
+        pairs = B * workload_pairs(N, bands)
+        flops, nbytes = step_work(w, pairs, active_rows(w, bands))
+        step_ms = ms / K
+        sr = step_roofline_report(flops, nbytes, step_ms, peaks)
+        out[name + ("/full-bands" if full else "")] = {
+            "steps": K, "ms_per_step": step_ms, "useful_tflops": flops / (step_ms * 1e-3) / 1e12,
+            "pct_of_bf16_peak": 100.0 * flops / (step_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
+            "tokens_per_s": B * N / (step_ms * 1e-3), "step_bound": sr["bound"],
+            "pct_of_step_roofline": 100.0 * sr["frac"], "pairs": pairs,
+            "l2": "flushed before every step" if small else "inputs larger than L2"}
+        del q, k, v, do, o, dq, dk, dv, lse, ws
+        torch.cuda.empty_cache()
+    return out
+
+
 def run_spa(args):
     from head_partitioned_distance_b200 import spa
 
@@ -947,6 +1023,9 @@ def run_spa(args):
                     "kernel": dom,
                     "algorithmic_per_launch": dk_["algorithmic_per_launch"],
                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if dk_['bound'] == 'tensor' else 'hbm_gbs'})"}
+        per_workload = None
+        if world == 1 and not args.no_sweep:
+            per_workload = sweep_workloads(spa, device, stream, peaks, fused)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             P, fl, secs, cores, desc = calibrate_prefix(w, bands, args.cpu_seconds, start=512)
@@ -973,6 +1052,7 @@ def run_spa(args):
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h, "steps": E, "ms_per_step": e2e_ms / E,
                     "schedule": E2E_SCHEDULE},
+            "per_workload": per_workload,
             "gpu_launches": len(kernels) * K,
             "backward": ("one pass over key tiles (spa_attn_bwd_fused: prep, pass, dq convert)" if fused
                          else "two passes (spa_attn_bwd: dQ pass forming D, dK/dV pass)"),
@@ -1196,6 +1276,8 @@ def main(argv=None):
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true",
+                    help="skip the short run of every other workload (and of the full bands) after the headline")
     ap.add_argument("--union", type=int, default=0, metavar="W",
                     help="time band plus a local window [0, W) shared by every head instead")
     ap.add_argument("--full-bands", action="store_true",

@@ -71,14 +71,17 @@ def _rms_rows(x: torch.Tensor) -> torch.Tensor:
 
 
 def make_inputs(B: int, H: int, N: int, d: int, seed: int, qkv_mult: float = 1.0,
-                rms_qk: bool = False, do_mult: float = 1.0):
-    """Return bf16 CPU tensors (q, k, v, dout), each [B, H, N, d]."""
-    g = torch.Generator().manual_seed(seed)
+                rms_qk: bool = False, do_mult: float = 1.0, device=None):
+    """Return bf16 tensors (q, k, v, dout), each [B, H, N, d], on the CPU (the
+    values the oracle and the parity tests use) or, with ``device``, drawn by
+    that device's generator with the same recipe (other values, same
+    distribution; for timing runs)."""
+    g = torch.Generator(device=device or "cpu").manual_seed(seed)
     shape = (B, H, N, d)
-    q = torch.randn(shape, generator=g, dtype=torch.float32)
-    k = torch.randn(shape, generator=g, dtype=torch.float32)
-    v = torch.randn(shape, generator=g, dtype=torch.float32)
-    dout = torch.randn(shape, generator=g, dtype=torch.float32)
+    q = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    k = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    v = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
+    dout = torch.randn(shape, generator=g, dtype=torch.float32, device=device)
     if rms_qk:
         q = _rms_rows(q)
         k = _rms_rows(k)
