@@ -195,13 +195,24 @@ def load_peaks():
         return dict(FALLBACK_PEAKS), "fallback"
 
 
+def _code_only(src: str) -> str:
+    """Source text with comments and blank lines removed and each line's
+    surrounding whitespace stripped: what the compiler sees of it, so that an
+    edit of a comment does not count as a change of the kernels."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    lines = (re.sub(r"//.*$", "", line).strip() for line in src.splitlines())
+    return "\n".join(line for line in lines if line)
+
+
 def kernel_src_sha() -> str:
+    """Hash of the kernel sources' code (comments and layout ignored)."""
     csrc = os.path.join(ROOT, "head_partitioned_distance_b200", "csrc")
     h = hashlib.sha256()
     for name in sorted(os.listdir(csrc)):
         if name.endswith((".cu", ".cuh")):
-            with open(os.path.join(csrc, name), "rb") as f:
-                h.update(name.encode() + b"\0" + f.read())
+            with open(os.path.join(csrc, name), encoding="utf-8") as f:
+                h.update(name.encode() + b"\0" + _code_only(f.read()).encode())
     return h.hexdigest()[:16]
 
 

@@ -27,10 +27,17 @@
 //                     (warp 9), drained by the warpgroups into the buffer
 //   dV  += P^T dO     TS MMA (A = P^T from TMEM)  -> TMEM [256, 384)  (warp 11)
 //   dK  += dS^T Q     SS MMA (A = dS^T from smem) -> TMEM [384, 512)  (warp 9)
-// Warp 9 issues, per tile: dQ_0, then (once dQ_0 is drained) dQ_1 (d = 128)
-// and dK, then -- once dV has read P^T and the last dQ piece is drained --
-// dP^T of the next tile.  The epilogue writes dK and dV exactly as the dK/dV
-// pass does, staged in the same shared tile that carries dS^T.
+// Warp 9 issues, per tile: dQ_0 and dK (for d = 64, whose dQ is one piece,
+// dK before dQ_0's commit, so that the piece's completion covers every read
+// of dS^T), then -- once the warpgroups hold dQ_0 -- dQ_1 (d = 128), then --
+// once dV has read P^T and the last piece is drained -- dP^T of the next
+// tile.  The epilogue writes dK and dV exactly as the dK/dV pass does, staged
+// in the same shared tile that carries dS^T.
+//
+// Measured on B200 this pass is slower than the two-pass backward it
+// replaces: the reductions of the dQ pieces (per thread, 32 rows x 16 bytes
+// per warp instruction) occupy the SM's memory-instruction path long enough
+// to delay the barrier arrivals and MMA issues queued behind them.
 #pragma once
 
 #include "bwd.cuh"

@@ -62,7 +62,7 @@ def test_traffic_is_read_only_from_a_summary_of_the_current_sources(tmp_path, mo
     import bench
     csrc = tmp_path / "head_partitioned_distance_b200" / "csrc"
     csrc.mkdir(parents=True)
-    (csrc / "k.cuh").write_text("// kernel v1\n")
+    (csrc / "k.cuh").write_text("int k_v1;  // kernel v1\n")
     (tmp_path / "profiles").mkdir()
     monkeypatch.setattr(bench, "ROOT", str(tmp_path))
     sha = bench.kernel_src_sha()
@@ -71,7 +71,11 @@ def test_traffic_is_read_only_from_a_summary_of_the_current_sources(tmp_path, mo
     assert bench.ncu_traffic("spa_k", "w1") == 12345.0
     assert bench.ncu_traffic("spa_k", "w2") is None          # another workload
     assert bench.ncu_traffic("spa_other", "w1") is None      # another kernel
-    (csrc / "k.cuh").write_text("// kernel v2\n")             # the kernel changed since the capture
+    # a comment or layout edit is not a change of the kernel
+    (csrc / "k.cuh").write_text("/* the kernel */\n\n   int k_v1;   // first version, reworded\n")
+    assert bench.kernel_src_sha() == sha
+    assert bench.ncu_traffic("spa_k", "w1") == 12345.0
+    (csrc / "k.cuh").write_text("int k_v2;  // kernel v2\n")   # the kernel changed since the capture
     assert bench.kernel_src_sha() != sha
     assert bench.ncu_traffic("spa_k", "w1") is None
 
