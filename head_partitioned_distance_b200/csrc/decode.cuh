@@ -10,7 +10,9 @@
 // scores, then each lane accumulates d/32 output columns over the warp's
 // keys with an online max and sum.  The warps' partials merge in shared
 // memory into one (m, l, o[d]) per chunk; spa_decode_merge_kernel merges the
-// chunks of each (b, h) into o (bf16) and lse (natural log).
+// chunks of each (b, h) into o (bf16) and lse (natural log); it is launched
+// as a programmatic dependent of the chunk kernel, so its launch overlaps the
+// chunk kernel's last CTAs and it waits for that grid before reading.
 #pragma once
 
 #include "common.cuh"
@@ -165,6 +167,9 @@ __global__ void __launch_bounds__(128) spa_decode_chunk_kernel(const __grid_cons
       }
     }
   }
+  // the merge kernel (launched as this grid's programmatic dependent) may
+  // start its launch now; it reads nothing before this grid has completed
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   // merge the four warps
   if (lane == 0) {
     s_m[warp] = m;
@@ -198,6 +203,9 @@ __global__ void __launch_bounds__(128) spa_decode_chunk_kernel(const __grid_cons
 // Merge the chunks of each (b, h): o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
 template <int D>
 __global__ void __launch_bounds__(128) spa_decode_merge_kernel(const __grid_constant__ DecodeParams p) {
+  // launched as the chunk kernel's programmatic dependent: wait until that
+  // grid has completed and its partials are visible
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   const int h = blockIdx.x, b = blockIdx.y;
   const int64_t bh = (int64_t)b * p.H + h;
   int64_t jlo, jhi;

@@ -853,14 +853,27 @@ int spa_attn_decode(const void* q, const void* k, const void* v, const int32_t* 
   std::memcpy(p.hi, bands.hi, sizeof(p.hi));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const dim3 grid_c((unsigned)nchunk, (unsigned)H, (unsigned)B), grid_m((unsigned)H, (unsigned)B);
+  // the merge kernel is the chunk kernel's programmatic dependent: its launch
+  // may begin once every chunk CTA has finished its keys, and it waits for
+  // the chunk grid (griddepcontrol.wait) before reading the partials
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid_m;
+  cfg.blockDim = dim3(128, 1, 1);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (d == 64) {
     spa::spa_decode_chunk_kernel<64><<<grid_c, 128, 0, s>>>(p);
     if ((st = launch_status())) return st;
-    spa::spa_decode_merge_kernel<64><<<grid_m, 128, 0, s>>>(p);
+    if (cudaLaunchKernelEx(&cfg, spa::spa_decode_merge_kernel<64>, p) != cudaSuccess) return SPA_ERR_CUDA;
   } else {
     spa::spa_decode_chunk_kernel<128><<<grid_c, 128, 0, s>>>(p);
     if ((st = launch_status())) return st;
-    spa::spa_decode_merge_kernel<128><<<grid_m, 128, 0, s>>>(p);
+    if (cudaLaunchKernelEx(&cfg, spa::spa_decode_merge_kernel<128>, p) != cudaSuccess) return SPA_ERR_CUDA;
   }
   return launch_status();
 }

@@ -429,25 +429,30 @@ class SPAttentionFunction(torch.autograd.Function):
     """Band-sparse attention as an autograd function (bf16 [B, H, N, d])."""
 
     @staticmethod
-    def forward(ctx, q, k, v, scale, lo, hi):
+    def forward(ctx, q, k, v, scale, lo, hi, fused=False):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         o, lse = attention_forward(q, k, v, scale, lo, hi)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.scale, ctx.lo, ctx.hi = scale, lo, hi
+        ctx.scale, ctx.lo, ctx.hi, ctx.fused = scale, lo, hi, fused
         return o
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = attention_backward(q, k, v, o, dout.contiguous(), lse, ctx.scale, ctx.lo, ctx.hi)
-        return dq, dk, dv, None, None, None
+        bwd = attention_backward_fused if ctx.fused else attention_backward
+        dq, dk, dv = bwd(q, k, v, o, dout.contiguous(), lse, ctx.scale, ctx.lo, ctx.hi)
+        return dq, dk, dv, None, None, None, None
 
 
-def spattention(q, k, v, scale=None, lo=None, hi=None):
+def spattention(q, k, v, scale=None, lo=None, hi=None, backward: str = "two-pass"):
     """SPAttention: head h of H attends to causal distances in its Balanced
-    Distance Partitioning band (or the explicit bands lo/hi)."""
+    Distance Partitioning band (or the explicit bands lo/hi).  backward:
+    "two-pass" (spa_attn_bwd, deterministic) or "fused" (spa_attn_bwd_fused,
+    dq summed by fp32 reductions)."""
+    if backward not in ("two-pass", "fused"):
+        raise ValueError("backward is 'two-pass' or 'fused'")
     scale = q.shape[-1] ** -0.5 if scale is None else scale
-    return SPAttentionFunction.apply(q, k, v, scale, lo, hi)
+    return SPAttentionFunction.apply(q, k, v, scale, lo, hi, backward == "fused")
 
 
 # ------------------------------------------------------------- band + shared window
@@ -524,6 +529,32 @@ def attention_backward_union(q, k, v, o, dout, lse, window: int, scale=None, lo=
     scale = d ** -0.5 if scale is None else scale
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     return spa_attn_bwd_union(q, k, v, o, dout, lse, dq, dk, dv, _union_workspace(q), scale, window, lo, hi)
+
+
+class SPAttentionUnionFunction(torch.autograd.Function):
+    """Band plus a local window shared by every head, as an autograd function."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, window, scale, lo, hi):
+        q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
+        o, lse = attention_forward_union(q, k, v, window, scale, lo, hi)
+        ctx.save_for_backward(q, k, v, o, lse)
+        ctx.window, ctx.scale, ctx.lo, ctx.hi = window, scale, lo, hi
+        return o
+
+    @staticmethod
+    def backward(ctx, dout):
+        q, k, v, o, lse = ctx.saved_tensors
+        dq, dk, dv = attention_backward_union(q, k, v, o, dout.contiguous(), lse, ctx.window, ctx.scale, ctx.lo,
+                                              ctx.hi)
+        return dq, dk, dv, None, None, None, None
+
+
+def spattention_union(q, k, v, window: int, scale=None, lo=None, hi=None):
+    """Each head attends to its band and to the distances [0, window) that
+    every head shares (spa_attn_fwd_union / spa_attn_bwd_union); differentiable."""
+    scale = q.shape[-1] ** -0.5 if scale is None else scale
+    return SPAttentionUnionFunction.apply(q, k, v, int(window), scale, lo, hi)
 
 
 def spa_attn_union_merge(o, lse, o2, lse2, stream=None):

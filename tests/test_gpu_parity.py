@@ -247,6 +247,22 @@ def test_autograd_function(spa):
         _check_grad(_f64(g), ref, n)
 
 
+def test_autograd_function_with_the_one_pass_backward(spa):
+    B, H, N, d = 2, 4, 700, 128
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=19)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (t.to(dev).requires_grad_() for t in (q, k, v))
+    o = spa.spattention(qd, kd, vd, backward="fused")
+    o.backward(do.to(dev))
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    o_ref, _ = oracle.spa_fwd(qf, kf, vf, d ** -0.5)
+    assert np.abs(_f64(o) - o_ref).max() <= O_TOL
+    for g, ref, n in zip((qd.grad, kd.grad, vd.grad), oracle.spa_bwd(qf, kf, vf, dof, d ** -0.5), "qkv"):
+        _check_grad(_f64(g), ref, n)
+    with pytest.raises(ValueError):
+        spa.spattention(qd, kd, vd, backward="other")
+
+
 @pytest.mark.parametrize("B,H,N,d,explicit", [(3, 4, 1000, 64, False), (2, 8, 4096, 128, False),
                                              (2, 3, 700, 128, True), (1, 32, 2048, 128, False)])
 def test_decode_matches_the_forward_row(spa, B, H, N, d, explicit):

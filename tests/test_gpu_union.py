@@ -75,6 +75,21 @@ def test_union_every_element(spa, B, H, N, d, w):
         _check_grad(got[name], ref, name)
 
 
+def test_union_autograd_function(spa):
+    B, H, N, d, w = 1, 8, 1001, 64, 64
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=211)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (t.to(dev).requires_grad_() for t in (q, k, v))
+    o = spa.spattention_union(qd, kd, vd, w)
+    o.backward(do.to(dev))
+    scale = d ** -0.5
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    o_ref, _ = oracle.union_fwd(qf, kf, vf, scale, w)
+    assert np.abs(_f64(o) - o_ref).max() <= O_TOL
+    for g, ref, name in zip((qd.grad, kd.grad, vd.grad), oracle.union_bwd(qf, kf, vf, dof, scale, w), "qkv"):
+        _check_grad(_f64(g), ref, name)
+
+
 def test_union_with_explicit_bands(spa):
     B, H, N, d, w = 1, 4, 600, 64, 50
     lo, hi = [0, 3, 257, 40], [1, 400, 300, 600]
