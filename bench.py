@@ -5,8 +5,9 @@
                     [--decode | --union W]
 
 One step = one pass of the whole hot path over one batch of synthetic input:
-spa_attn_fwd (1 kernel) then the backward as two passes (the dQ pass, which
-also forms the row sums D, and the dK/dV pass).  Inputs are resident in HBM
+spa_attn_fwd (1 kernel) then the backward (by default spa_attn_bwd_stored: the
+row sums D, the dK/dV pass, which also stores each tile pair's dS^T, and the dQ
+pass from the stored tiles; see --bwd).  Inputs are resident in HBM
 when the timed region starts;
 each of q, k, v, dout is larger than the 126 MB L2, so no flush is needed
 between steps.  The metric is useful TFLOP/s: 14 * d * (permitted pairs) per
@@ -25,8 +26,11 @@ batch of the same workload (weak scaling); the only collectives are the
 barrier and the max of the timings.  --gpus N without torchrun starts the N
 ranks itself.
 
---bwd fused times the one-pass backward (spa_attn_bwd_fused) instead of the
-two-pass one.
+The step's backward is the one that stores dS (spa_attn_bwd_stored: D, the
+dK/dV pass writing each tile pair's dS^T, the dQ pass contracting it with k);
+--bwd two-pass times the two-pass backward (spa_attn_bwd: the dQ pass
+computing S and dP again) and --bwd fused the one-pass backward
+(spa_attn_bwd_fused) instead.
 
 --impl reference times the fp64 CPU oracle (the slow, plain implementation the
 tests check against) on a bounded sample of the same workload and prints the
@@ -71,7 +75,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # and dq from the sums.
 KERNELS_TWO_PASS = ("spa_fwd_kernel", "spa_bwd_dq_kernel", "spa_bwd_dkdv_kernel")
 KERNELS_FUSED = ("spa_fwd_kernel", "spa_bwd_fused_prep_kernel", "spa_bwd_fused_kernel", "spa_bwd_dq_convert_kernel")
+# Backward that stores dS: D over the reached query tiles, the dK/dV pass that
+# also writes each tile pair's dS^T (the DS instantiation of
+# spa_bwd_dkdv_kernel, named spa_bwd_dkdv_kernel_ds here), and the dQ pass
+# from the stored tiles.
+KERNELS_STORED = ("spa_fwd_kernel", "spa_bwd_delta_band_kernel", "spa_bwd_dkdv_kernel_ds", "spa_bwd_dq_stored_kernel")
 KERNELS = KERNELS_TWO_PASS
+KERNELS_OF = {"two-pass": KERNELS_TWO_PASS, "fused": KERNELS_FUSED, "stored": KERNELS_STORED}
+STORED_TILE_BYTES = 128 * 128 * 2
 
 
 # --------------------------------------------------------------------- counting
@@ -103,7 +114,7 @@ def active_rows(w, bands) -> int:
     return w.B * sum(w.N - int(lo) for lo in bands[0])
 
 
-def kernel_work(w, pairs: int, act: int):
+def kernel_work(w, pairs: int, act: int, tiles: int = 0):
     """Algorithmic work per launch of each kernel, the accounting of the
     scope table's measurement section: (useful FLOPs, executed FLOPs, least
     bytes).  Inputs are counted over the active rows only (head h never reads
@@ -112,7 +123,10 @@ def kernel_work(w, pairs: int, act: int):
     tensor over the active / all rows; R_act / R_all: one fp32 row vector
     (lse or D).  The dQ pass executes S, dP and dQ (6 d per pair) but only
     dQ is work the dK/dV pass does not already do, so its useful FLOPs are
-    2 d per pair."""
+    2 d per pair.  `tiles` is the number of 128 x 128 tile pairs the dK/dV
+    pass walks (stored_tiles): the stored-dS backward writes and reads one
+    bf16 dS^T tile for each, and its dQ pass executes 2 d per element of
+    those tiles."""
     d = w.d
     rows = w.B * w.H * w.N
     T_all, T_act, R_all, R_act = rows * d * 2, act * d * 2, rows * 4, act * 4
@@ -132,7 +146,23 @@ def kernel_work(w, pairs: int, act: int):
         "spa_bwd_dq_kernel": (2 * d * pairs, 6 * d * pairs, 5 * T_act + 2 * R_act + T_all),
         # q k v dO, lse and D in over active rows; dk dv out for every row
         "spa_bwd_dkdv_kernel": (8 * d * pairs, 8 * d * pairs, 4 * T_act + 2 * R_act + 2 * T_all),
+        # stored-dS backward: o dO in and D out over the active rows
+        "spa_bwd_delta_band_kernel": (0, 0, 2 * T_act + R_act),
+        # the dK/dV pass, plus every tile pair's dS^T out
+        "spa_bwd_dkdv_kernel_ds": (8 * d * pairs, 8 * d * pairs,
+                                   4 * T_act + 2 * R_act + 2 * T_all + tiles * STORED_TILE_BYTES),
+        # dS^T tiles and k over active rows in, dq out for every row
+        "spa_bwd_dq_stored_kernel": (2 * d * pairs, 2 * d * tiles * 128 * 128,
+                                     tiles * STORED_TILE_BYTES + T_act + T_all),
     }
+
+
+def stored_tiles(spa, w, bands) -> int:
+    """Tile pairs (key tile, query tile) the dK/dV pass walks over the whole
+    workload: the lengths of its query strips, from the library's schedule."""
+    sch = spa.spa_tile_schedule(w.N, w.H, 128, 128, bands[0], bands[1])
+    lens = sch["qt_end"] - sch["qt_begin"] + 1
+    return w.B * int(lens[lens > 0].sum())
 
 
 def step_work(w, pairs: int, act: int):
@@ -833,17 +863,41 @@ SWEEP = [("b1_h4_n256_d64", 50, False), ("b1_h8_n1024_d64", 50, False), ("b1_h8_
          ("b1_h32_n32768_d128", 3, True)]
 
 
-def sweep_workloads(spa, device, stream, peaks, fused: bool, warmup: int = 3):
+def backward_call(spa, mode: str, B: int, H: int, N: int, d: int, device, bands=None):
+    """(the public backward entry of a mode, a workspace for it)."""
+    lo, hi = (None, None) if bands is None else bands
+    if mode == "fused":
+        return spa.spa_attn_bwd_fused, torch.empty(spa.spa_attn_bwd_fused_workspace_bytes(B, H, N, d) // 4,
+                                                   dtype=torch.float32, device=device)
+    if mode == "stored":
+        return spa.spa_attn_bwd_stored, torch.empty(spa.spa_attn_bwd_stored_workspace_bytes(B, H, N, d, lo, hi),
+                                                    dtype=torch.uint8, device=device)
+    return spa.spa_attn_bwd, torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32,
+                                         device=device)
+
+
+def sweep_workloads(spa, device, stream, peaks, mode: str, warmup: int = 3):
     """Every workload of the scope table, a few steps each, after the headline
     measurement: ms per step, useful TFLOP/s, % of the bf16 peak, tokens/s and
     the step's roofline fraction, plus the same kernels with full bands (dense
-    causal attention on every head) at two sizes.  Inputs are drawn on the
-    device with each workload's recipe; workloads smaller than L2 are flushed
-    out of it before every step (untimed); each step is timed with CUDA events
-    on the launching stream and the steps' times are summed."""
+    causal attention on every head) at two sizes.  The band workloads run with
+    the headline's backward and, when that is not the two-pass one, with the
+    two-pass backward too (key "<workload>/two-pass"); the full-band runs use
+    the two-pass backward.  Inputs are drawn on the device with each
+    workload's recipe; workloads smaller than L2 are flushed out of it before
+    every step (untimed); each step is timed with CUDA events on the launching
+    stream and the steps' times are summed."""
     out = {}
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
+    runs = []
     for name, K, full in SWEEP:
+        if full:
+            runs.append((name, K, full, "two-pass"))
+        else:
+            runs.append((name, K, full, mode))
+            if mode != "two-pass":
+                runs.append((name, K, full, "two-pass"))
+    for name, K, full, bmode in runs:
         w = synth.WORKLOADS[name]
         B, H, N, d = w.B, w.H, w.N, w.d
         bands = ([0] * H, [N] * H) if full else spa.spa_band_bounds(N, H)
@@ -851,12 +905,7 @@ def sweep_workloads(spa, device, stream, peaks, fused: bool, warmup: int = 3):
         q, k, v, do = synth.make_inputs(B, H, N, d, w.seed, w.qkv_mult, w.rms_qk, w.do_mult, device=device)
         o, dq, dk, dv = (torch.empty_like(q) for _ in range(4))
         lse = torch.empty((B, H, N), dtype=torch.float32, device=device)
-        if fused:
-            ws = torch.empty(spa.spa_attn_bwd_fused_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32,
-                             device=device)
-        else:
-            ws = torch.empty(spa.spa_attn_bwd_workspace_bytes(B, H, N) // 4, dtype=torch.float32, device=device)
-        bwd = spa.spa_attn_bwd_fused if fused else spa.spa_attn_bwd
+        bwd, ws = backward_call(spa, bmode, B, H, N, d, device, bands if full else None)
 
         def step():
             spa.spa_attn_fwd(q, k, v, o, lse, w.scale, stream=stream, **lo_hi)
@@ -882,8 +931,9 @@ def sweep_workloads(spa, device, stream, peaks, fused: bool, warmup: int = 3):
         flops, nbytes = step_work(w, pairs, active_rows(w, bands))
         step_ms = ms / K
         sr = step_roofline_report(flops, nbytes, step_ms, peaks)
-        out[name + ("/full-bands" if full else "")] = {
-            "steps": K, "ms_per_step": step_ms, "useful_tflops": flops / (step_ms * 1e-3) / 1e12,
+        key = name + ("/full-bands" if full else "") + ("/two-pass" if bmode != mode and not full else "")
+        out[key] = {
+            "backward": bmode, "steps": K, "ms_per_step": step_ms, "useful_tflops": flops / (step_ms * 1e-3) / 1e12,
             "pct_of_bf16_peak": 100.0 * flops / (step_ms * 1e-3) / 1e12 / peaks["bf16_tflops"],
             "tokens_per_s": B * N / (step_ms * 1e-3), "step_bound": sr["bound"],
             "pct_of_step_roofline": 100.0 * sr["frac"], "pairs": pairs,
@@ -891,6 +941,13 @@ def sweep_workloads(spa, device, stream, peaks, fused: bool, warmup: int = 3):
         del q, k, v, do, o, dq, dk, dv, lse, ws
         torch.cuda.empty_cache()
     return out
+
+
+BACKWARD_DESCRIPTION = {
+    "two-pass": "two passes (spa_attn_bwd: dQ pass forming D, dK/dV pass)",
+    "fused": "one pass over key tiles (spa_attn_bwd_fused: prep, pass, dq convert)",
+    "stored": "dS stored (spa_attn_bwd_stored: D, dK/dV pass writing each tile pair's dS^T, dQ from the tiles)",
+}
 
 
 def run_spa(args):
@@ -931,21 +988,18 @@ def run_spa(args):
     if flush_needed(w):
         flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=device)
 
-    fused = args.bwd == "fused"
-    kernels = KERNELS_FUSED if fused else KERNELS_TWO_PASS
-    if fused:
-        ws = torch.empty(spa.spa_attn_bwd_fused_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32,
-                         device=device)
+    mode = args.bwd
+    kernels = KERNELS_OF[mode]
+    bwd_call, ws = backward_call(spa, mode, B, H, N, d, device, bands if args.full_bands else None)
 
     def step(ev=None):
         spa.spa_attn_fwd(qd, kd, vd, o, lse, scale, stream=stream, **lo_hi)
         if ev is not None:
             ev[1].record(stream)
-        if fused:
-            # the three launches of spa_attn_bwd_fused, an event after each
+        if mode in ("fused", "stored"):
+            # the three launches of the backward, an event after each
             for i, st in enumerate((1, 2, 4)):
-                spa.spa_attn_bwd_fused(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, scale, stream=stream, steps=st,
-                                       **lo_hi)
+                bwd_call(qd, kd, vd, o, dod, lse, dq, dk, dv, ws, scale, stream=stream, steps=st, **lo_hi)
                 if ev is not None:
                     ev[2 + i].record(stream)
             return
@@ -1005,9 +1059,8 @@ def run_spa(args):
 
     def compute(S):
         spa.spa_attn_fwd(S["q"], S["k"], S["v"], S["o"], S["lse"], scale, stream=stream, **lo_hi)
-        bwd = spa.spa_attn_bwd_fused if fused else spa.spa_attn_bwd
-        bwd(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"], S["ws"], scale,
-            stream=stream, **lo_hi)
+        bwd_call(S["q"], S["k"], S["v"], S["o"], S["do"], S["lse"], S["dq"], S["dk"], S["dv"], S["ws"], scale,
+                 stream=stream, **lo_hi)
 
     e2e_ms, h2d, d2h = pipelined_e2e(device, stream, host, dev0, ("o", "lse", "dq", "dk", "dv"), compute, E,
                                      dist)
@@ -1018,7 +1071,7 @@ def run_spa(args):
     if rank == 0:
         peaks, peak_src = load_peaks()
         act = active_rows(w, bands)
-        work = kernel_work(w, pairs, act)
+        work = kernel_work(w, pairs, act, stored_tiles(spa, w, bands) if mode == "stored" else 0)
         kern = {name: kernel_report(*work[name], per_kernel_ms[name] / K, per_kernel_ms[name] / elapsed_ms,
                                     peaks) for name in kernels}
         # the whole step against its attainable roofline: the slower of the
@@ -1036,7 +1089,7 @@ def run_spa(args):
                     "peak_source": f"{peak_src} ({'bf16_tflops burst' if dk_['bound'] == 'tensor' else 'hbm_gbs'})"}
         per_workload = None
         if world == 1 and not args.no_sweep:
-            per_workload = sweep_workloads(spa, device, stream, peaks, fused)
+            per_workload = sweep_workloads(spa, device, stream, peaks, mode)
         cpu = None
         if world == 1 and not args.no_cpu_baseline:
             P, fl, secs, cores, desc = calibrate_prefix(w, bands, args.cpu_seconds, start=512)
@@ -1065,8 +1118,7 @@ def run_spa(args):
                     "schedule": E2E_SCHEDULE},
             "per_workload": per_workload,
             "gpu_launches": len(kernels) * K,
-            "backward": ("one pass over key tiles (spa_attn_bwd_fused: prep, pass, dq convert)" if fused
-                         else "two passes (spa_attn_bwd: dQ pass forming D, dK/dV pass)"),
+            "backward": BACKWARD_DESCRIPTION[mode],
             "clocks": clocks,
         }
         print(json.dumps(line), flush=True)
@@ -1294,9 +1346,10 @@ def main(argv=None):
     ap.add_argument("--full-bands", action="store_true",
                     help="run every head with the full band [0, N) (dense causal per head) through the same "
                          "kernels, to show the work the bands save")
-    ap.add_argument("--bwd", choices=["fused", "two-pass"], default="two-pass",
-                    help="backward of the timed step: the one-pass backward (spa_attn_bwd_fused) or the "
-                         "deterministic two-pass one (spa_attn_bwd)")
+    ap.add_argument("--bwd", choices=["stored", "two-pass", "fused"], default="stored",
+                    help="backward of the timed step: the one that stores dS (spa_attn_bwd_stored, "
+                         "deterministic; the default), the two-pass one (spa_attn_bwd, deterministic) or the "
+                         "one-pass one (spa_attn_bwd_fused)")
     ap.add_argument("--decode", action="store_true",
                     help="time the decode step (one new token per sequence) instead of fwd+bwd")
     ap.add_argument("--ncu-summary", metavar="CSV",

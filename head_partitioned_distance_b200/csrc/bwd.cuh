@@ -50,6 +50,44 @@ __global__ void __launch_bounds__(256) spa_bwd_delta_kernel(const uint16_t* __re
   if (row < rows && part == 0) delta[row] = acc;
 }
 
+// The same row sums for the rows the dK/dV pass reads only: rows i >= 128
+// floor(lo_h / 128) of every (b, h), the 128-row query tiles its bands reach.
+// blockIdx.y walks the (b, h) pairs and blockIdx.x the rows of one, 256 / (D / 8)
+// rows per block and round; a round's rows are the same for every lane of a
+// warp, so every lane takes part in the row's shuffle.  Rows before the first
+// reached tile are neither read nor written.
+template <int D>
+__global__ void __launch_bounds__(256) spa_bwd_delta_band_kernel(const uint16_t* __restrict__ o,
+                                                                 const uint16_t* __restrict__ dout,
+                                                                 const __grid_constant__ AttnParams p) {
+  constexpr int TPR = D / 8;
+  constexpr int RPB = 256 / TPR;  // rows per block and round
+  const int part = threadIdx.x % TPR;
+  const int BH = p.B * p.H;
+  const int64_t N = p.N;
+  for (int bh = blockIdx.y; bh < BH; bh += gridDim.y) {
+    const int64_t r0 = (int64_t)(p.lo[bh % p.H] / 128) * 128;
+    const uint16_t* ob = o + (int64_t)bh * N * D;
+    const uint16_t* gb = dout + (int64_t)bh * N * D;
+    float* db = p.delta + (int64_t)bh * N;
+    for (int64_t base = r0 + (int64_t)blockIdx.x * RPB; base < N; base += (int64_t)gridDim.x * RPB) {
+      const int64_t i = base + threadIdx.x / TPR;
+      const bool live = i < N;
+      float acc = 0.f;
+      if (live) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(ob + i * D) + part);
+        const uint4 g = __ldg(reinterpret_cast<const uint4*>(gb + i * D) + part);
+        acc = bf16lo(a.x) * bf16lo(g.x) + bf16hi(a.x) * bf16hi(g.x) + bf16lo(a.y) * bf16lo(g.y) +
+              bf16hi(a.y) * bf16hi(g.y) + bf16lo(a.z) * bf16lo(g.z) + bf16hi(a.z) * bf16hi(g.z) +
+              bf16lo(a.w) * bf16lo(g.w) + bf16hi(a.w) * bf16hi(g.w);
+      }
+#pragma unroll
+      for (int off = TPR / 2; off > 0; off /= 2) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (live && part == 0) db[i] = acc;
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------
 // dK, dV: persistent grid; a unit is (b, h, key tile of 128 keys), walking
 // the 128-query tiles its band reaches.  Per query tile:
@@ -150,12 +188,17 @@ __device__ __forceinline__ DkvUnit dkv_decode(int u, const AttnParams& p) {
 
 // ACC: add dk, dv to what the outputs hold (spa_attn_bwd_dkdv_add) and leave
 // the keys no query reaches untouched.
-template <int D, bool ACC = false>
+// DS: each tile pair's dS^T (bf16, the A operand of dK) also leaves for the
+// stored-dS backward's dQ pass, through tm_ds ([slots][128 keys][128
+// queries]): once the dK product may read it from TMEM, every warp stages
+// its 32 x 64 box in its slice of the epilogue staging tile and sends it by
+// a bulk tensor store (the staging tile is idle between epilogues).
+template <int D, bool ACC = false, bool DS = false>
 __global__ void __launch_bounds__(384, 1)
     spa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                        const __grid_constant__ AttnParams p) {
+                        const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ AttnParams p) {
   using C = DkvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -494,6 +537,7 @@ __global__ void __launch_bounds__(384, 1)
           }
         }
         // ---- dP^T into registers; its columns take P^T (A of dV), then dS^T
+        uint32_t dsk[32];  // dS^T of this key row, bf16 pairs over the warpgroup's 64 queries
         ok = __all_sync(0xffffffffu, bar_wait(&bars->dp_full, (cdp++) & 1, abort_flag));
         if (!ok) break;
         ptx::tc_fence_after();
@@ -518,7 +562,6 @@ __global__ void __launch_bounds__(384, 1)
           ptx::reg_fence(dr[1]);
           // ---- dS^T = P^T (dP^T - D); vd holds -D of the 64 queries, in pairs
           const float4* nd4 = reinterpret_cast<const float4*>(vd);
-          uint32_t pk[32];
 #pragma unroll
           for (int q4 = 0; q4 < 16; ++q4) {
             const float4 nd = nd4[q4];
@@ -531,15 +574,34 @@ __global__ void __launch_bounds__(384, 1)
                                          __fadd2_rn(make_float2(__uint_as_float(dr[q / 32][q % 32 + 2]),
                                                                 __uint_as_float(dr[q / 32][q % 32 + 3])),
                                                     make_float2(nd.z, nd.w)));
-            pk[2 * q4] = ptx::pack_bf16x2(da.x, da.y);
-            pk[2 * q4 + 1] = ptx::pack_bf16x2(db.x, db.y);
+            dsk[2 * q4] = ptx::pack_bf16x2(da.x, da.y);
+            dsk[2 * q4 + 1] = ptx::pack_bf16x2(db.x, db.y);
           }
-          ptx::tmem_st32(tDST, pk);
+          ptx::tmem_st32(tDST, dsk);
           ptx::tmem_wait_st();
         }
         ptx::tc_fence_before();
         ptx::mbar_arrive(&bars->ds_full);
         ptx::mbar_arrive(&bars->vec_empty[gq % C::NS]);  // last read of this vector stage
+        if constexpr (DS) {
+          // this warp's 32 key rows x 64 queries of dS^T, through its slice
+          const int wq = warp % 4;
+          const uint32_t srow = sP + (uint32_t)w * (C::BK * 128) + (uint32_t)r * 128;
+          if (lane == 0) ptx::bulk_wait_group_read_all();  // the slice's previous store has read it
+          __syncwarp();
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            ptx::st_shared_v4(srow + ((k ^ (r & 7)) << 4), dsk[4 * k], dsk[4 * k + 1], dsk[4 * k + 2],
+                              dsk[4 * k + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int64_t slot = stored_slot(p, U.bh / p.H, U.bh % p.H, (int)(U.j0 / 128), qt, U.qa);
+            ptx::tma_store_3d(&tm_ds, smem + C::OFF_P + (uint32_t)w * (C::BK * 128) + (uint32_t)wq * (32 * 128),
+                              64 * w, 32 * wq, (int)slot);
+            ptx::bulk_commit_group();
+          }
+        }
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue

@@ -48,11 +48,26 @@ struct AttnParams {
   const void* o_in;
   const void* dout;
   float* dq_acc;      // fused backward: fp32 dQ sums, [B, H, N, d]
+  // stored-dS backward: the dS^T buffer's tiles of head h start at tile
+  // ds_base[h]; each of its B x (key tiles some query reaches) key tiles owns
+  // ds_len[h] consecutive tiles (stored_slot)
+  int64_t ds_base[kMaxHeads];
+  int32_t ds_len[kMaxHeads];
+  void* ds;  // the dS^T tiles
   int32_t lo[kMaxHeads];
   int32_t hi[kMaxHeads];
   int32_t unit_start[kMaxHeads + 1];
   int32_t fill_start[kMaxHeads + 1];
 };
+
+// Index of the 128 x 128 dS^T tile of (b, h, key tile u, query tile t) in
+// the stored-dS backward's buffer.  Head h's key tiles 0 .. reached - 1 of
+// batch b own ds_len[h] consecutive tiles each, one per query tile of the
+// key tile's strip from its first, qa.
+__host__ __device__ __forceinline__ int64_t stored_slot(const AttnParams& p, int b, int h, int u, int t, int qa) {
+  const int64_t reached = (p.N - 1 - p.lo[h]) / 128 + 1;
+  return p.ds_base[h] + ((int64_t)b * reached + u) * p.ds_len[h] + (t - qa);
+}
 
 // Head whose range [start[h], start[h + 1]) holds r, for 0 <= r < start[H]:
 // the number of k in [1, H] with start[k] <= r (start is non-decreasing).

@@ -14,6 +14,7 @@
 
 #include "bwd.cuh"
 #include "bwd_fused.cuh"
+#include "bwd_stored.cuh"
 #include "common.cuh"
 #include "decode.cuh"
 #include "fwd.cuh"
@@ -206,29 +207,60 @@ int fwd_impl(const void* q, const void* k, const void* v, void* o, float* lse, A
 // serves the three-step entry points.  kStepAccumulate makes the dQ and dK/dV
 // passes add to their outputs (the second part of the band-plus-window
 // backward).
+// The stored-dS backward runs D, then the dK/dV pass writing every tile
+// pair's dS^T to `ds` (the layout of stored_layout), then kStepDqStored.
 enum BwdStep {
   kStepDelta = 1,
   kStepDkDv = 2,
   kStepDq = 4,
   kStepDqDelta = 8,
   kStepAccumulate = 16,
-  kStepAll = kStepDqDelta | kStepDkDv
+  kStepDqStored = 32,
+  kStepDeltaBand = 64,  // D of the rows the dK/dV pass reads only
+  kStepAll = kStepDqDelta | kStepDkDv,
+  kStepStored = kStepDeltaBand | kStepDkDv | kStepDqStored
 };
+
+// The stored-dS backward's workspace: D (fp32 [B H N], padded to 1024
+// bytes), then the dS^T tiles, 128 x 128 bf16 each.  Head h owns, for each
+// batch and each key tile some query reaches, ds_len[h] consecutive tiles:
+// a key tile's query strip starts at tile u + lo / 128 and ends at most at
+// u + (hi + 126) / 128, so it has at most (hi + 126) / 128 - lo / 128 + 1
+// tiles.  Fills p.ds_base / p.ds_len (bands already in p) and returns the
+// number of tiles, or -1 when it does not fit the kernels' 32-bit tile index.
+constexpr size_t kStoredTileBytes = 128 * 128 * 2;
+size_t stored_delta_bytes(int64_t rows) { return (size_t)((rows * 4 + 1023) & ~int64_t(1023)); }
+int64_t stored_layout(AttnParams& p) {
+  int64_t n = 0;
+  for (int h = 0; h < p.H; ++h) {
+    p.ds_base[h] = n;
+    p.ds_len[h] = (int32_t)((p.hi[h] + 126LL) / 128 - p.lo[h] / 128 + 1);
+    n += (int64_t)p.B * ((p.N - 1 - p.lo[h]) / 128 + 1) * p.ds_len[h];
+    if (n > 2147483647LL) return -1;
+  }
+  return n;
+}
+int64_t stored_tiles(const AttnParams& p) {
+  const int h = p.H - 1;
+  return p.ds_base[h] + (int64_t)p.B * ((p.N - 1 - p.lo[h]) / 128 + 1) * p.ds_len[h];
+}
 
 template <int D>
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
              const float* lse, void* dq, void* dk, void* dv, float* delta, AttnParams& p,
-             cudaStream_t stream, int steps) {
+             cudaStream_t stream, int steps, void* ds = nullptr) {
   using KC = spa::DkvCfg<D>;
   using QC = spa::DqCfg<D>;
-  // one (prepared, register check) pair per kernel instantiation: [adding]
-  static std::atomic<uint64_t> prepared_kv[2], prepared_q[2];
-  static std::atomic<int> regs_kv[2], regs_q[2];
+  // one (prepared, register check) pair per kernel instantiation: [adding],
+  // and the dK/dV pass that also stores dS^T
+  static std::atomic<uint64_t> prepared_kv[2], prepared_q[2], prepared_kvs, prepared_qs;
+  static std::atomic<int> regs_kv[2], regs_q[2], regs_kvs;
   const bool acc = (steps & kStepAccumulate) != 0;
   const int64_t BH = (int64_t)p.B * p.H;
   int st;
   p.lse = const_cast<float*>(lse);
   p.delta = delta;
+  p.ds = ds;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
@@ -239,6 +271,19 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if (blocks > 2147483647LL) return SPA_ERR_UNSUPPORTED;
     spa::spa_bwd_delta_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(
         static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), delta, rows);
+    if ((st = launch_status())) return st;
+  }
+  if (steps & kStepDeltaBand) {
+    // about eight blocks per SM: the (b, h) pairs on y, each pair's rows on x
+    int sms = 0;
+    if ((st = sm_count(&sms))) return st;
+    const int64_t target = (int64_t)sms * 8;
+    const unsigned gy = (unsigned)(BH < 65535 ? BH : 65535);
+    const int64_t rows_blocks = (p.N + (256 / (D / 8)) - 1) / (256 / (D / 8));
+    int64_t gx = (target + gy - 1) / gy;
+    gx = gx < rows_blocks ? gx : rows_blocks;
+    spa::spa_bwd_delta_band_kernel<D><<<dim3((unsigned)gx, gy), 256, 0, stream>>>(
+        static_cast<const uint16_t*>(o), static_cast<const uint16_t*>(dout), p);
     if ((st = launch_status())) return st;
   }
   if (steps & (kStepDq | kStepDqDelta)) {
@@ -272,15 +317,19 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     // persistent grid over key tiles of 128 that some query reaches; the
     // other key tiles only get zero rows
     // dk and dv leave through bulk tensor stores of 32-row boxes
-    CUtensorMap kq, kk, kv, kdo, kdk, kdv;
+    CUtensorMap kq, kk, kv, kdo, kdk, kdv, kds;
     if ((st = make_map(&kq, q, p.N, BH, D, KC::BQ)) || (st = make_map(&kk, k, p.N, BH, D, KC::BK)) ||
         (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)) ||
         (st = make_map(&kdk, dk, p.N, BH, D, 32)) || (st = make_map(&kdv, dv, p.N, BH, D, 32)))
       return st;
-    auto* kernel_kv = acc ? spa::spa_bwd_dkdv_kernel<D, true> : spa::spa_bwd_dkdv_kernel<D, false>;
-    if ((st = prepare_kernel(kernel_kv, KC::SMEM_BYTES, prepared_kv[acc]))) return st;
-    if ((st = check_regs(kernel_kv, (int)KC::LAUNCH_REGS, regs_kv[acc]))) return st;
     const int64_t nkt = (p.N + 127) / 128;
+    // the dS^T buffer: [tiles][128 keys][128 queries] bf16, stored in 32 x 64 boxes
+    if (ds && (st = make_map(&kds, ds, 128, stored_tiles(p), 128, 32))) return st;
+    if (!ds) kds = kdk;  // not read
+    auto* kernel_kv = ds ? spa::spa_bwd_dkdv_kernel<D, false, true>
+                         : (acc ? spa::spa_bwd_dkdv_kernel<D, true> : spa::spa_bwd_dkdv_kernel<D, false>);
+    if ((st = prepare_kernel(kernel_kv, KC::SMEM_BYTES, ds ? prepared_kvs : prepared_kv[acc]))) return st;
+    if ((st = check_regs(kernel_kv, (int)KC::LAUNCH_REGS, ds ? regs_kvs : regs_kv[acc]))) return st;
     if ((int64_t)p.B * p.H * nkt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
     if ((st = set_work_lists(
              p, [&](int h) { return (p.N - 1 - p.lo[h]) / 128 + 1; },
@@ -291,11 +340,37 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if ((st = sm_count(&sms))) return st;
     const int64_t units = (int64_t)p.B * upb;
     const unsigned grid = (unsigned)(units < sms ? units : sms);
-    kernel_kv<<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
+    kernel_kv<<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, kds, p);
+    if ((st = launch_status())) return st;
+  }
+  if (steps & kStepDqStored) {
+    // persistent grid over query tiles of 128 with a row inside its band,
+    // contracting the stored dS tiles with K; whole tiles before the band
+    // only get zero rows
+    using SC = spa::DqStoredCfg<D>;
+    if (!ds) return SPA_ERR_INVAL;
+    const int64_t nqt = (p.N + 127) / 128;
+    CUtensorMap mds, mk;
+    if ((st = make_map(&mds, ds, 128, stored_tiles(p), 128, 128)) ||
+        (st = make_map(&mk, k, p.N, BH, D, SC::BK)))
+      return st;
+    auto* kernel_qs = spa::spa_bwd_dq_stored_kernel<D>;
+    if ((st = prepare_kernel(kernel_qs, SC::SMEM_BYTES, prepared_qs))) return st;
+    if ((int64_t)p.B * p.H * nqt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
+    if ((st = set_work_lists(
+             p, [&](int h) { return nqt - p.lo[h] / 128; }, [&](int h) { return (int64_t)(p.lo[h] / 128); })))
+      return st;
+    int sms = 0;
+    if ((st = sm_count(&sms))) return st;
+    const int64_t units = (int64_t)p.B * p.units_per_batch;
+    const unsigned grid = (unsigned)(units < sms ? units : sms);
+    kernel_qs<<<grid, SC::NTHREADS, SC::SMEM_BYTES, stream>>>(mds, mk, p);
     if ((st = launch_status())) return st;
   }
   return SPA_OK;
 }
+
+
 
 // Bytes of the fused backward's workspace: D (fp32 [B H N], padded to 256
 // bytes) then the fp32 dQ sums [B H N d].
@@ -695,6 +770,58 @@ int spa_attn_bwd_dq_delta(const void* q, const void* k, const void* v, const voi
                           float scale, const int32_t* lo, const int32_t* hi, void* stream) {
   return bwd_entry(q, k, v, o, dout, lse, dq, nullptr, nullptr, workspace, B, H, N, d, scale, lo, hi, stream,
                    kStepDqDelta);
+}
+
+size_t spa_attn_bwd_stored_workspace_bytes(int B, int H, int64_t N, int d, const int32_t* lo,
+                                           const int32_t* hi) {
+  if (check_shape(B, H, N, d)) return 0;
+  static AttnParams zero{};
+  AttnParams p = zero;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  if (fill_bands(p, H, N, lo, hi)) return 0;
+  const int64_t tiles = stored_layout(p);
+  if (tiles < 0) return 0;
+  return stored_delta_bytes((int64_t)B * H * N) + (size_t)tiles * kStoredTileBytes;
+}
+
+int spa_attn_bwd_stored(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                        const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int H, int64_t N,
+                        int d, float scale, const int32_t* lo, const int32_t* hi, void* stream) {
+  return spa_attn_bwd_stored_steps(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, N, d, scale, lo, hi, stream,
+                                   7);
+}
+
+int spa_attn_bwd_stored_steps(const void* q, const void* k, const void* v, const void* o, const void* dout,
+                              const float* lse, void* dq, void* dk, void* dv, void* workspace, int B, int H,
+                              int64_t N, int d, float scale, const int32_t* lo, const int32_t* hi, void* stream,
+                              int steps) {
+  if (steps < 1 || steps > 7) return SPA_ERR_INVAL;
+  int st = check_shape(B, H, N, d);
+  if (st) return st;
+  if (!q || !k || !v || !o || !dout || !lse || !dq || !dk || !dv || !workspace) return SPA_ERR_INVAL;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return SPA_ERR_INVAL;
+  for (const void* t : {q, k, v, o, dout})
+    if (!aligned(t, 16)) return SPA_ERR_UNSUPPORTED;
+  // the gradients leave in 32-byte stores; the dS^T tiles are copied by TMA
+  if (!aligned(dq, 32) || !aligned(dk, 32) || !aligned(dv, 32) || !aligned(lse, 4) || !aligned(workspace, 256))
+    return SPA_ERR_UNSUPPORTED;
+  static AttnParams zero{};
+  AttnParams p = zero;
+  p.B = B;
+  p.H = H;
+  p.N = N;
+  p.scale = scale;
+  p.scale_log2 = scale * spa::kLog2e;
+  if ((st = fill_bands(p, H, N, lo, hi))) return st;
+  if (stored_layout(p) < 0) return SPA_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* delta = static_cast<float*>(workspace);
+  void* ds = static_cast<uint8_t*>(workspace) + stored_delta_bytes((int64_t)B * H * N);
+  const int bits = ((steps & 1) ? kStepDeltaBand : 0) | ((steps & 2) ? kStepDkDv : 0) | ((steps & 4) ? kStepDqStored : 0);
+  return d == 64 ? bwd_impl<64>(q, k, v, o, dout, lse, dq, dk, dv, delta, p, s, bits, ds)
+                 : bwd_impl<128>(q, k, v, o, dout, lse, dq, dk, dv, delta, p, s, bits, ds);
 }
 
 size_t spa_attn_bwd_fused_workspace_bytes(int B, int H, int64_t N, int d) {

@@ -52,6 +52,9 @@ EXPORTS = {
     "spa_attn_decode": ([_vp] * 7 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_noalloc": ([_vp] * 9 + [_int, _int, _i64, _int, _f32, _vp], _int),
     "spa_attn_bwd_fused_workspace_bytes": ([_int, _int, _i64, _int], ctypes.c_size_t),
+    "spa_attn_bwd_stored_workspace_bytes": ([_int, _int, _i64, _int, _i32p, _i32p], ctypes.c_size_t),
+    "spa_attn_bwd_stored": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
+    "spa_attn_bwd_stored_steps": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp, _int], _int),
     "spa_attn_bwd_fused": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp], _int),
     "spa_attn_bwd_fused_steps": ([_vp] * 10 + [_int, _int, _i64, _int, _f32, _i32p, _i32p, _vp, _int], _int),
     "spa_attn_union_workspace_bytes": ([_int, _int, _i64, _int], ctypes.c_size_t),
@@ -219,6 +222,50 @@ def attention_backward_fused(q, k, v, o, dout, lse, scale=None, lo=None, hi=None
     dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
     ws = torch.empty(spa_attn_bwd_fused_workspace_bytes(B, H, N, d) // 4, dtype=torch.float32, device=q.device)
     return spa_attn_bwd_fused(q, k, v, o, dout, lse, dq, dk, dv, ws, scale, lo, hi)
+
+
+def spa_attn_bwd_stored_workspace_bytes(B: int, H: int, N: int, d: int, lo=None, hi=None) -> int:
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    return int(_lib.spa_attn_bwd_stored_workspace_bytes(B, H, N, d, lo_a, hi_a))
+
+
+def spa_attn_bwd_stored(q, k, v, o, dout, lse, dq, dk, dv, workspace, scale: float, lo=None, hi=None,
+                        stream=None, steps: int = 7):
+    """The backward that stores dS (spa_attn_bwd_stored in spa.h): same
+    gradients as spa_attn_bwd, bit-reproducible; the dK/dV pass writes every
+    tile pair's dS^T to the workspace and the dQ pass contracts it with k.
+    workspace: CUDA tensor of at least
+    spa_attn_bwd_stored_workspace_bytes(B, H, N, d, lo, hi) bytes."""
+    B, H, N, d = _dims(q)
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (dout, "dout"), (dq, "dq"), (dk, "dk"),
+                 (dv, "dv")):
+        _need(t, (B, H, N, d), torch.bfloat16, n)
+    _need(lse, (B, H, N), torch.float32, "lse")
+    need = spa_attn_bwd_stored_workspace_bytes(B, H, N, d, lo, hi)
+    if need == 0 or not workspace.is_cuda or not workspace.is_contiguous() or \
+            workspace.numel() * workspace.element_size() < need:
+        raise ValueError("workspace: contiguous CUDA tensor of spa_attn_bwd_stored_workspace_bytes(B, H, N, d, "
+                         "lo, hi) bytes")
+    lo_a = None if lo is None else _i32(lo)
+    hi_a = None if hi is None else _i32(hi)
+    ptrs = [t.data_ptr() for t in (q, k, v, o, dout, lse, dq, dk, dv, workspace)]
+    if steps == 7:
+        _check(_lib.spa_attn_bwd_stored(*ptrs, B, H, N, d, scale, lo_a, hi_a, _stream_ptr(stream)),
+               "spa_attn_bwd_stored")
+    else:  # one or two of its launches (spa_attn_bwd_stored_steps)
+        _check(_lib.spa_attn_bwd_stored_steps(*ptrs, B, H, N, d, scale, lo_a, hi_a, _stream_ptr(stream), steps),
+               "spa_attn_bwd_stored_steps")
+    return dq, dk, dv
+
+
+def attention_backward_stored(q, k, v, o, dout, lse, scale=None, lo=None, hi=None):
+    """Allocate dq / dk / dv / workspace and run spa_attn_bwd_stored."""
+    B, H, N, d = _dims(q)
+    scale = d ** -0.5 if scale is None else scale
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(q), torch.empty_like(q)
+    ws = torch.empty(spa_attn_bwd_stored_workspace_bytes(B, H, N, d, lo, hi), dtype=torch.uint8, device=q.device)
+    return spa_attn_bwd_stored(q, k, v, o, dout, lse, dq, dk, dv, ws, scale, lo, hi)
 
 
 SPA_NOALLOC_MAX_ROWS = 1 << 20
@@ -429,30 +476,35 @@ class SPAttentionFunction(torch.autograd.Function):
     """Band-sparse attention as an autograd function (bf16 [B, H, N, d])."""
 
     @staticmethod
-    def forward(ctx, q, k, v, scale, lo, hi, fused=False):
+    def forward(ctx, q, k, v, scale, lo, hi, backward="two-pass"):
         q, k, v = q.contiguous(), k.contiguous(), v.contiguous()
         o, lse = attention_forward(q, k, v, scale, lo, hi)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.scale, ctx.lo, ctx.hi, ctx.fused = scale, lo, hi, fused
+        ctx.scale, ctx.lo, ctx.hi, ctx.backward = scale, lo, hi, backward
         return o
 
     @staticmethod
     def backward(ctx, dout):
         q, k, v, o, lse = ctx.saved_tensors
-        bwd = attention_backward_fused if ctx.fused else attention_backward
+        bwd = BACKWARDS[ctx.backward]
         dq, dk, dv = bwd(q, k, v, o, dout.contiguous(), lse, ctx.scale, ctx.lo, ctx.hi)
         return dq, dk, dv, None, None, None, None
+
+
+BACKWARDS = {"two-pass": attention_backward, "fused": attention_backward_fused,
+             "stored": attention_backward_stored}
 
 
 def spattention(q, k, v, scale=None, lo=None, hi=None, backward: str = "two-pass"):
     """SPAttention: head h of H attends to causal distances in its Balanced
     Distance Partitioning band (or the explicit bands lo/hi).  backward:
-    "two-pass" (spa_attn_bwd, deterministic) or "fused" (spa_attn_bwd_fused,
-    dq summed by fp32 reductions)."""
-    if backward not in ("two-pass", "fused"):
-        raise ValueError("backward is 'two-pass' or 'fused'")
+    "two-pass" (spa_attn_bwd, deterministic), "fused" (spa_attn_bwd_fused,
+    dq summed by fp32 reductions) or "stored" (spa_attn_bwd_stored,
+    deterministic, dS kept in a workspace of about 2 bytes per causal pair)."""
+    if backward not in BACKWARDS:
+        raise ValueError("backward is 'two-pass', 'fused' or 'stored'")
     scale = q.shape[-1] ** -0.5 if scale is None else scale
-    return SPAttentionFunction.apply(q, k, v, scale, lo, hi, backward == "fused")
+    return SPAttentionFunction.apply(q, k, v, scale, lo, hi, backward)
 
 
 # ------------------------------------------------------------- band + shared window

@@ -179,6 +179,42 @@ SPA_API int spa_attn_bwd_fused_steps(const void* q, const void* k, const void* v
                                      const int32_t* lo, const int32_t* hi, void* stream, int steps);
 
 /*
+ * Backward that stores dS: the same gradients as spa_attn_bwd (the
+ * derivative written above), bit-reproducible, with S and dP computed once per
+ * tile pair.  The dK/dV pass, which forms each 128 x 128 tile pair's dS^T in
+ * bf16 for its dK product, also writes it to the workspace.  The dQ pass then
+ * computes dq_i = scale sum_j dS_ij k_j from the stored tiles and k alone,
+ * instead of computing S and dP again.  It runs three kernels: D (for the
+ * 128-row query tiles the bands reach), dK/dV, dQ.
+ *   workspace: DEVICE buffer of spa_attn_bwd_stored_workspace_bytes(B, H, N,
+ *              d, lo, hi) bytes, 256-byte aligned, caller-owned, contents
+ *              overwritten (D, then the dS^T tiles; nothing in it needs to
+ *              be initialised).  Its size is about 2 bytes per causal pair
+ *              of every (b, h), plus padding: 2.7 GB for B1 H32 N32768.
+ *   dq, dk, dv: 32-byte aligned.  lo/hi: HOST band arrays, or both NULL for
+ *              the Balanced Distance Partitioning bands.
+ * Other tensors and rules as spa_attn_bwd.  A tile count past 2^31 - 1 is
+ * SPA_ERR_UNSUPPORTED.
+ */
+SPA_API size_t spa_attn_bwd_stored_workspace_bytes(int B, int H, int64_t N, int d, const int32_t* lo,
+                                                   const int32_t* hi);
+SPA_API int spa_attn_bwd_stored(const void* q, const void* k, const void* v, const void* o,
+                                const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                void* workspace, int B, int H, int64_t N, int d, float scale,
+                                const int32_t* lo, const int32_t* hi, void* stream);
+/*
+ * The same backward one launch at a time, for timing each kernel: `steps` is
+ * a bitmask, 1 = D, 2 = the dK/dV pass (dk, dv and the dS^T tiles), 4 = the
+ * dQ pass from the stored tiles; spa_attn_bwd_stored runs 7.  Each step needs
+ * the ones before it to have run on the same workspace.  A mask outside
+ * [1, 7] is SPA_ERR_INVAL.
+ */
+SPA_API int spa_attn_bwd_stored_steps(const void* q, const void* k, const void* v, const void* o,
+                                      const void* dout, const float* lse, void* dq, void* dk, void* dv,
+                                      void* workspace, int B, int H, int64_t N, int d, float scale,
+                                      const int32_t* lo, const int32_t* hi, void* stream, int steps);
+
+/*
  * The three steps spa_attn_bwd runs, callable one by one (for example to run
  * the dk/dv and dq passes on two streams once the first step is done).  Same
  * tensors and rules as spa_attn_bwd; lo/hi are HOST band arrays or both NULL

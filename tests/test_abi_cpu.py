@@ -180,6 +180,62 @@ def test_fused_backward_rejects_bad_arguments_before_any_launch():
     assert L.spa_attn_bwd_fused(*ten, 1, 8, 4, 64, 0.1, None, None, None) == spa.SPA_ERR_INVAL
 
 
+def test_stored_backward_rejects_bad_arguments_before_any_launch():
+    L = spa._lib
+    p = _fake(1 << 20)
+    f = lambda *a, B=1, H=4, N=256, d=64: L.spa_attn_bwd_stored(*a, B, H, N, d, 0.1, None, None, None)
+    ten = [p] * 10
+    for i in range(10):  # every pointer is required
+        args = list(ten)
+        args[i] = None
+        assert f(*args) == spa.SPA_ERR_INVAL
+    half = _fake((1 << 20) + 16)
+    for i in (6, 7, 8):  # dq, dk, dv leave in 32-byte stores
+        args = list(ten)
+        args[i] = half
+        assert f(*args) == spa.SPA_ERR_UNSUPPORTED
+    args = list(ten)
+    args[9] = _fake((1 << 20) + 128)  # workspace must be 256-byte aligned
+    assert f(*args) == spa.SPA_ERR_UNSUPPORTED
+    assert f(*ten, d=96) == spa.SPA_ERR_UNSUPPORTED
+    assert f(*ten, H=8, N=4) == spa.SPA_ERR_INVAL
+    # more dS^T tiles than a 32-bit index holds
+    assert f(*ten, B=65535, H=256, N=2 ** 20) == spa.SPA_ERR_UNSUPPORTED
+    assert spa.spa_attn_bwd_stored_workspace_bytes(65535, 256, 2 ** 20, 64) == 0
+    st = lambda steps: L.spa_attn_bwd_stored_steps(*ten, 1, 4, 256, 64, 0.1, None, None, None, steps)
+    assert st(0) == spa.SPA_ERR_INVAL and st(8) == spa.SPA_ERR_INVAL
+
+
+@pytest.mark.parametrize("N,H,lo,hi", [(32768, 32, None, None), (30001, 32, None, None), (8192, 32, None, None),
+                                       (1001, 8, None, None), (129, 3, None, None),
+                                       (500, 5, [0, 0, 37, 100, 499], [500, 1, 250, 101, 500])])
+def test_stored_workspace_holds_every_tile_pair(N, H, lo, hi):
+    # D, padded to 1024 bytes, then the dS^T tiles (128 x 128 bf16): head h
+    # owns, per batch and per key tile some query reaches, L_h tiles, where
+    # L_h = (hi + 126) // 128 - lo // 128 + 1 must cover the dK/dV strip of
+    # every such key tile (the schedule's qt_begin..qt_end, itself checked
+    # against the oracle's brute-force tile classes above).  A Balanced
+    # Distance Partitioning band that ends well before N reaches the bound; a
+    # band that N clips may need a tile less.
+    B, d = 2, 128
+    got = spa.spa_attn_bwd_stored_workspace_bytes(B, H, N, d, lo, hi)
+    sch = spa.spa_tile_schedule(N, H, 128, 128, lo, hi)
+    if lo is None:
+        lo, hi = oracle.bands(N, H)
+    tiles = 0
+    for h in range(H):
+        reached = (N - 1 - int(lo[h])) // 128 + 1
+        L = (int(hi[h]) + 126) // 128 - int(lo[h]) // 128 + 1
+        strips = sch["qt_end"][h] - sch["qt_begin"][h] + 1
+        assert (strips[:reached] >= 1).all() and (strips[reached:] <= 0).all()
+        assert strips.max() <= L
+        tiles += B * reached * L
+    if N in (32768, 30001, 8192):
+        assert all((hh + 126) // 128 - ll // 128 + 1 == (sch["qt_end"][h] - sch["qt_begin"][h] + 1).max()
+                   for h, (ll, hh) in enumerate(zip(lo, hi)) if hh <= N - 256)
+    assert got == -(-4 * B * H * N // 1024) * 1024 + tiles * 32768
+
+
 def test_fused_workspace_size():
     # D (fp32 per row, padded to 256 bytes), then the fp32 dq sums
     assert spa.spa_attn_bwd_fused_workspace_bytes(1, 32, 32768, 128) == 4 * 32 * 32768 * (1 + 128)

@@ -37,14 +37,13 @@ def _f64(t):
     return t.detach().to("cpu", torch.float64).numpy()
 
 
-def _gpu_run(spa, q, k, v, do, scale, lo=None, hi=None, backward=True, fused=False):
+def _gpu_run(spa, q, k, v, do, scale, lo=None, hi=None, backward=True, bwd="two-pass"):
     dev = torch.device("cuda:0")
     qd, kd, vd, dod = (t.to(dev) for t in (q, k, v, do))
     o, lse = spa.attention_forward(qd, kd, vd, scale, lo, hi)
     out = {"o": o, "lse": lse}
     if backward:
-        bwd = spa.attention_backward_fused if fused else spa.attention_backward
-        dq, dk, dv = bwd(qd, kd, vd, o, dod, lse, scale, lo, hi)
+        dq, dk, dv = spa.BACKWARDS[bwd](qd, kd, vd, o, dod, lse, scale, lo, hi)
         out.update(dq=dq, dk=dk, dv=dv)
     torch.cuda.synchronize()
     assert spa.spa_device_status() == spa.SPA_OK
@@ -74,8 +73,8 @@ def _check_grad(g, ref, name):
         assert err / denom <= GRAD_TOL, (name, err, denom)
 
 
-def _full_check(spa, q, k, v, do, scale, lo=None, hi=None, fused=False):
-    got = _gpu_run(spa, q, k, v, do, scale, lo, hi, fused=fused)
+def _full_check(spa, q, k, v, do, scale, lo=None, hi=None, bwd="two-pass"):
+    got = _gpu_run(spa, q, k, v, do, scale, lo, hi, bwd=bwd)
     qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
     lo_o = None if lo is None else np.array(lo)
     hi_o = None if hi is None else np.array(hi)
@@ -387,15 +386,15 @@ def _targeted_key_rows(B, H, N, lo):
     return out
 
 
-def _sampled_check(spa, w, n_random, n_key_rows, full_bands=False, fused=False):
+def _sampled_check(spa, w, n_random, n_key_rows, full_bands=False, bwd="two-pass"):
     q, k, v, do = synth.workload_inputs(w)
     B, H, N, d = w.B, w.H, w.N, w.d
     if full_bands:  # [0, N) on every head: dense causal attention per head
         lo, hi = np.zeros(H, dtype=np.int64), np.full(H, N, dtype=np.int64)
-        got = _gpu_run(spa, q, k, v, do, w.scale, [0] * H, [N] * H, fused=fused)
+        got = _gpu_run(spa, q, k, v, do, w.scale, [0] * H, [N] * H, bwd=bwd)
     else:
         lo, hi = oracle.bands(N, H)
-        got = _gpu_run(spa, q, k, v, do, w.scale, fused=fused)
+        got = _gpu_run(spa, q, k, v, do, w.scale, bwd=bwd)
     for name in ("o", "lse", "dq", "dk", "dv"):
         assert not np.isnan(got[name]).any(), name
     per_head = [[int(lo[h]) - 1, int(lo[h]), int(lo[h]) + 1, int(lo[h]) + 127, int(lo[h]) + 128]
@@ -473,7 +472,7 @@ FUSED_SHAPES = EDGE_SHAPES + MULTI_UNIT_SHAPES + WIDE_SHAPES
 @pytest.mark.parametrize("B,H,N,d", FUSED_SHAPES)
 def test_fused_backward_every_element(spa, B, H, N, d):
     q, k, v, do = synth.make_inputs(B, H, N, d, seed=23 + N + H + d)
-    _full_check(spa, q, k, v, do, 1 / math.sqrt(d), fused=True)
+    _full_check(spa, q, k, v, do, 1 / math.sqrt(d), bwd="fused")
 
 
 @pytest.mark.parametrize("kind", ["full", "first_half", "odd"])
@@ -488,19 +487,19 @@ def test_fused_backward_explicit_bands(spa, kind):
         lo = [int(a) for a in lo]
     else:
         lo, hi = [0, 3, 257, 599], [1, 400, 300, 600]
-    _full_check(spa, q, k, v, do, 0.125, [int(x) for x in lo], [int(x) for x in hi], fused=True)
+    _full_check(spa, q, k, v, do, 0.125, [int(x) for x in lo], [int(x) for x in hi], bwd="fused")
 
 
 @pytest.mark.parametrize("name", SMALL_WORKLOADS)
 def test_fused_backward_small_workloads(spa, name):
     w = synth.WORKLOADS[name]
     q, k, v, do = synth.workload_inputs(w)
-    _full_check(spa, q, k, v, do, w.scale, fused=True)
+    _full_check(spa, q, k, v, do, w.scale, bwd="fused")
 
 
 @pytest.mark.parametrize("name", LARGE)
 def test_fused_backward_full_size_sampled_rows(spa, name):
-    _sampled_check(spa, synth.WORKLOADS[name], n_random=32, n_key_rows=8, fused=True)
+    _sampled_check(spa, synth.WORKLOADS[name], n_random=32, n_key_rows=8, bwd="fused")
 
 
 def test_fused_backward_dk_dv_match_the_two_pass_backward(spa):
@@ -511,7 +510,74 @@ def test_fused_backward_dk_dv_match_the_two_pass_backward(spa):
     B, H, N, d = 1, 8, 2048, 128
     q, k, v, do = synth.make_inputs(B, H, N, d, seed=5)
     a = _gpu_run(spa, q, k, v, do, 1 / math.sqrt(d))
-    b = _gpu_run(spa, q, k, v, do, 1 / math.sqrt(d), fused=True)
+    b = _gpu_run(spa, q, k, v, do, 1 / math.sqrt(d), bwd="fused")
     for name in ("dq", "dk", "dv"):
         scale = np.abs(a[name]).max()
         assert np.abs(a[name] - b[name]).max() <= 2e-2 * scale, name
+
+
+# ---------------------------------------------------------------------------
+# the backward that stores dS (spa_attn_bwd_stored): the dK/dV pass writes
+# every tile pair's dS^T, the dQ pass contracts it with k; every element on
+# small shapes, sampled rows at full size, the same tolerances
+# ---------------------------------------------------------------------------
+@pytest.mark.parametrize("B,H,N,d", FUSED_SHAPES)
+def test_stored_backward_every_element(spa, B, H, N, d):
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=29 + N + H + d)
+    _full_check(spa, q, k, v, do, 1 / math.sqrt(d), bwd="stored")
+
+
+@pytest.mark.parametrize("kind", ["full", "first_half", "odd"])
+def test_stored_backward_explicit_bands(spa, kind):
+    B, H, N, d = 1, 4, 600, 128
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=103)
+    lo, hi = oracle.bands(N, H)
+    if kind == "full":
+        lo, hi = [0] * H, [N] * H
+    elif kind == "first_half":
+        hi = [int(a + max((b - a) // 2, 1)) for a, b in zip(lo, hi)]
+        lo = [int(a) for a in lo]
+    else:
+        lo, hi = [0, 3, 257, 599], [1, 400, 300, 600]
+    _full_check(spa, q, k, v, do, 0.125, [int(x) for x in lo], [int(x) for x in hi], bwd="stored")
+
+
+@pytest.mark.parametrize("name", SMALL_WORKLOADS)
+def test_stored_backward_small_workloads(spa, name):
+    w = synth.WORKLOADS[name]
+    q, k, v, do = synth.workload_inputs(w)
+    _full_check(spa, q, k, v, do, w.scale, bwd="stored")
+
+
+@pytest.mark.parametrize("name", LARGE)
+def test_stored_backward_full_size_sampled_rows(spa, name):
+    _sampled_check(spa, synth.WORKLOADS[name], n_random=32, n_key_rows=8, bwd="stored")
+
+
+def test_stored_backward_is_bit_reproducible_and_matches_the_two_pass_backward(spa):
+    # no reductions in any order: two calls agree bit for bit.  Against the
+    # two-pass backward: dk and dv come from the same dK/dV products (only D
+    # is summed in another order), dq from the dS^T the dK/dV pass formed
+    # (S^T = K Q^T) instead of the dQ pass's own S = Q K^T
+    B, H, N, d = 1, 8, 2048, 128
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=7)
+    a = _gpu_run(spa, q, k, v, do, 1 / math.sqrt(d), bwd="stored")
+    b = _gpu_run(spa, q, k, v, do, 1 / math.sqrt(d), bwd="stored")
+    for name in a:
+        assert np.array_equal(a[name], b[name]), name
+    c = _gpu_run(spa, q, k, v, do, 1 / math.sqrt(d))
+    for name in ("dq", "dk", "dv"):
+        scale = np.abs(c[name]).max()
+        assert np.abs(a[name] - c[name]).max() <= 2e-2 * scale, name
+
+
+def test_autograd_function_with_the_stored_backward(spa):
+    B, H, N, d = 2, 4, 700, 128
+    q, k, v, do = synth.make_inputs(B, H, N, d, seed=31)
+    dev = torch.device("cuda:0")
+    qd, kd, vd = (t.to(dev).requires_grad_() for t in (q, k, v))
+    o = spa.spattention(qd, kd, vd, backward="stored")
+    o.backward(do.to(dev))
+    qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
+    for g, ref, n in zip((qd.grad, kd.grad, vd.grad), oracle.spa_bwd(qf, kf, vf, dof, d ** -0.5), "qkv"):
+        _check_grad(_f64(g), ref, n)

@@ -123,3 +123,32 @@ def test_kernel_report_uses_the_bound_s_algorithmic_work():
     r = bench.kernel_report(1e9, 1e9, 6.4e9, 2.0, 0.5, peaks)  # 6.4 GB in 2 ms: HBM-bound
     assert r["bound"] == "hbm" and r["unit"] == "GB/s"
     assert r["achieved"] == pytest.approx(3200.0) and r["frac"] == pytest.approx(0.5)
+
+
+def test_stored_backward_work_counts_every_tile_pair_once():
+    # the stored-dS backward writes and reads one bf16 128 x 128 dS^T tile
+    # per tile pair the dK/dV pass walks: the pairs holding a permitted
+    # element, counted here by the oracle's brute-force tile classes
+    import numpy as np
+
+    import bench
+    import oracle
+    from head_partitioned_distance_b200 import spa, synth
+    w = synth.WORKLOADS["b8_h16_n4096_d128"]
+    bands = spa.spa_band_bounds(w.N, w.H)
+    lo, hi = oracle.bands(w.N, w.H)
+    tiles = w.B * int(np.count_nonzero(oracle.tile_classes(w.N, lo, hi, 128, 128)))
+    assert bench.stored_tiles(spa, w, bands) == tiles
+    pairs = w.B * bench.workload_pairs(w.N, bands)
+    act = bench.active_rows(w, bands)
+    d = w.d
+    T_act, T_all = act * d * 2, w.B * w.H * w.N * d * 2
+    work = bench.kernel_work(w, pairs, act, tiles)
+    assert work["spa_bwd_dkdv_kernel_ds"][:2] == work["spa_bwd_dkdv_kernel"][:2]
+    assert work["spa_bwd_dkdv_kernel_ds"][2] == work["spa_bwd_dkdv_kernel"][2] + tiles * 32768
+    assert work["spa_bwd_dq_stored_kernel"] == (2 * d * pairs, 2 * d * tiles * 16384, tiles * 32768 + T_act + T_all)
+    assert work["spa_bwd_delta_band_kernel"] == (0, 0, 2 * T_act + act * 4)
+    # the three backwards' useful FLOPs agree: 10 d per pair
+    useful = lambda ks: sum(work[k][0] for k in ks if k != "spa_fwd_kernel")
+    assert useful(bench.KERNELS_STORED) == useful(bench.KERNELS_TWO_PASS) == useful(bench.KERNELS_FUSED) \
+        == 10 * d * pairs
