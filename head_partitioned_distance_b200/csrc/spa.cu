@@ -260,7 +260,6 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   int st;
   p.lse = const_cast<float*>(lse);
   p.delta = delta;
-  p.ds = ds;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
