@@ -297,7 +297,9 @@ def ncu_summary(csv_path: str, kernel: str, workload: str, command: str, src_sha
     rows = list(csv.reader(open(csv_path)))
     start = next(i for i, r in enumerate(rows) if "Kernel Name" in r)
     hdr, units = rows[start], rows[start + 1]
-    data = [r for r in rows[start + 2:] if len(r) == len(hdr) and kernel in r[hdr.index("Kernel Name")]]
+    ki = hdr.index("Kernel Name")
+    data = [r for r in rows[start + 2:]
+            if len(r) == len(hdr) and bench_kernel_key(r[ki].split("(")[0].replace("void ", "")) == kernel]
     if len(data) != 1:
         raise SystemExit(f"{csv_path}: expected one launch of {kernel}, found {len(data)}")
     rec = dict(zip(hdr, data[0]))
@@ -330,6 +332,17 @@ def ncu_summary(csv_path: str, kernel: str, workload: str, command: str, src_sha
     return "\n".join(lines) + "\n"
 
 
+def bench_kernel_key(ncu_name: str) -> str:
+    """The bench line's key of a kernel that ncu names with its template
+    arguments: the base name, except the dK/dV pass that stores dS (third
+    template argument 1) is spa_bwd_dkdv_kernel_ds."""
+    base = ncu_name.split("<")[0].strip()
+    args = ncu_name[len(base):].strip("<> ").split(",")
+    if base == "spa_bwd_dkdv_kernel" and len(args) == 3 and args[2].strip() in ("1", "true"):
+        return "spa_bwd_dkdv_kernel_ds"
+    return base
+
+
 def ncu_launch_list(csv_path: str, workload: str, command: str, bench_json: str = "", note: str = "") -> str:
     """Markdown launch list from `ncu --metrics gpu__time_duration.sum --csv`
     output: per kernel its launches, total time and share under ncu (cold
@@ -358,8 +371,7 @@ def ncu_launch_list(csv_path: str, workload: str, command: str, bench_json: str 
     lines += ["| kernel | launches | total us (ncu) | share (ncu) | bench avg ms (events) | share (bench events) |",
               "|---|---|---|---|---|---|"]
     for name, (n, t) in tot.items():
-        base = name.split("<")[0]
-        b = bench.get(base, {})
+        b = bench.get(bench_kernel_key(name), {})
         bms = f"{b['avg_ms']:.4f}" if b else "-"
         bsh = f"{100 * b['share']:.1f} %" if b else "-"
         lines.append(f"| {name} | {n} | {t:.1f} | {100 * t / all_us:.1f} % | {bms} | {bsh} |")

@@ -122,3 +122,7 @@ def test_ncu_summaries_from_csv(tmp_path):
     md = bench.ncu_launch_list(str(ll), "w1", "ncu ...")
     assert "| spa_a_kernel<128> | 2 | 0.6 | 60.0 % |" in md
     assert "| spa_b_kernel<128> | 2 | 0.4 | 40.0 % |" in md
+    # the dK/dV pass that stores dS has its own key in the bench line
+    assert bench.bench_kernel_key("spa_bwd_dkdv_kernel<128, 0, 1>") == "spa_bwd_dkdv_kernel_ds"
+    assert bench.bench_kernel_key("spa_bwd_dkdv_kernel<128, 0, 0>") == "spa_bwd_dkdv_kernel"
+    assert bench.bench_kernel_key("spa_fwd_kernel<128, 0, 1>") == "spa_fwd_kernel"
