@@ -581,3 +581,23 @@ def test_autograd_function_with_the_stored_backward(spa):
     qf, kf, vf, dof = (_f64(t) for t in (q, k, v, do))
     for g, ref, n in zip((qd.grad, kd.grad, vd.grad), oracle.spa_bwd(qf, kf, vf, dof, d ** -0.5), "qkv"):
         _check_grad(_f64(g), ref, n)
+
+
+def test_stored_backward_step_by_step_equals_the_whole_call(spa):
+    # the benchmark times spa_attn_bwd_stored_steps launch by launch (D, then
+    # dK/dV storing dS^T, then dQ from the tiles); that composition is the call
+    B, H, N, d = 2, 6, 1500, 128
+    q, k, v, do = (t.to("cuda") for t in synth.make_inputs(B, H, N, d, seed=37))
+    scale = 1 / math.sqrt(d)
+    o, lse = spa.attention_forward(q, k, v, scale)
+    ws = torch.empty(spa.spa_attn_bwd_stored_workspace_bytes(B, H, N, d), dtype=torch.uint8, device="cuda")
+    whole = [torch.empty_like(q) for _ in range(3)]
+    spa.spa_attn_bwd_stored(q, k, v, o, do, lse, *whole, ws, scale)
+    parts = [torch.empty_like(q) for _ in range(3)]
+    ws.fill_(0xFF)  # nothing of the first call may be left for the second
+    for st in (1, 2, 4):
+        spa.spa_attn_bwd_stored(q, k, v, o, do, lse, *parts, ws, scale, steps=st)
+    torch.cuda.synchronize()
+    assert spa.spa_device_status() == spa.SPA_OK
+    for a, b, n in zip(whole, parts, ("dq", "dk", "dv")):
+        assert torch.equal(a, b), n
