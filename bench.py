@@ -47,7 +47,6 @@ import argparse
 import datetime as _dt
 import hashlib
 import json
-import math
 import os
 import statistics
 import subprocess
@@ -80,7 +79,6 @@ KERNELS_FUSED = ("spa_fwd_kernel", "spa_bwd_fused_prep_kernel", "spa_bwd_fused_k
 # spa_bwd_dkdv_kernel, named spa_bwd_dkdv_kernel_ds here), and the dQ pass
 # from the stored tiles.
 KERNELS_STORED = ("spa_fwd_kernel", "spa_bwd_delta_band_kernel", "spa_bwd_dkdv_kernel_ds", "spa_bwd_dq_stored_kernel")
-KERNELS = KERNELS_TWO_PASS
 KERNELS_OF = {"two-pass": KERNELS_TWO_PASS, "fused": KERNELS_FUSED, "stored": KERNELS_STORED}
 STORED_TILE_BYTES = 128 * 128 * 2
 
