@@ -190,7 +190,9 @@ SPA_API int spa_attn_bwd_fused_steps(const void* q, const void* k, const void* v
  *              d, lo, hi) bytes, 256-byte aligned, caller-owned, contents
  *              overwritten (D, then the dS^T tiles; nothing in it needs to
  *              be initialised).  Its size is about 2 bytes per causal pair
- *              of every (b, h), plus padding: 2.7 GB for B1 H32 N32768.
+ *              of every (b, h), plus padding: 1.25 GB for B1 H32 N32768 with
+ *              the Balanced Distance Partitioning bands.  The size function
+ *              returns 0 on bad sizes or bands, or past the tile limit below.
  *   dq, dk, dv: 32-byte aligned.  lo/hi: HOST band arrays, or both NULL for
  *              the Balanced Distance Partitioning bands.
  * Other tensors and rules as spa_attn_bwd.  A tile count past 2^31 - 1 is
