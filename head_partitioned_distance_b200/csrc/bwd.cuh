@@ -189,16 +189,17 @@ __device__ __forceinline__ DkvUnit dkv_decode(int u, const AttnParams& p) {
 // ACC: add dk, dv to what the outputs hold (spa_attn_bwd_dkdv_add) and leave
 // the keys no query reaches untouched.
 // DS: each tile pair's dS^T (bf16, the A operand of dK) also leaves for the
-// stored-dS backward's dQ pass, through tm_ds ([slots][128 keys][128
-// queries]): once the dK product may read it from TMEM, every warp stages
-// its 32 x 64 box in its slice of the epilogue staging tile and sends it by
-// a bulk tensor store (the staging tile is idle between epilogues).
+// stored-dS backward's dQ pass, to its tile in p.ds (the layout of
+// bwd_stored.cuh: 8 x 8 core matrices).  Once the dK product may read dS^T
+// from TMEM, every thread writes its key row's 64 queries as eight 16-byte
+// pieces; the 32 rows of a warp make each store instruction 512 contiguous
+// bytes.
 template <int D, bool ACC = false, bool DS = false>
 __global__ void __launch_bounds__(384, 1)
     spa_bwd_dkdv_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                         const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                         const __grid_constant__ CUtensorMap tm_dk, const __grid_constant__ CUtensorMap tm_dv,
-                        const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ AttnParams p) {
+                        const __grid_constant__ AttnParams p) {
   using C = DkvCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -460,6 +461,11 @@ __global__ void __launch_bounds__(384, 1)
     for (int u = blockIdx.x; ok && u < num_units; u += gridDim.x) {
       const DkvUnit U = dkv_decode(u, p);
       const int64_t j = U.j0 + r;
+      // the unit's dS^T tiles are consecutive, from its first query tile's
+      uint8_t* const utile =
+          DS ? static_cast<uint8_t*>(p.ds) + stored_slot(p, U.bh / p.H, U.bh % p.H, (int)(U.j0 / 128), U.qa, U.qa) *
+                                                 (128 * 128 * 2)
+             : nullptr;
       for (int qt = U.qa; qt <= U.qb; ++qt, ++gq) {
         const int64_t i0 = (int64_t)qt * C::BQ;
         const bool interior = tile_is_interior(N, U.lo, U.hi, i0, C::BQ, U.j0, C::BK);
@@ -584,23 +590,13 @@ __global__ void __launch_bounds__(384, 1)
         ptx::mbar_arrive(&bars->ds_full);
         ptx::mbar_arrive(&bars->vec_empty[gq % C::NS]);  // last read of this vector stage
         if constexpr (DS) {
-          // this warp's 32 key rows x 64 queries of dS^T, through its slice
-          const int wq = warp % 4;
-          const uint32_t srow = sP + (uint32_t)w * (C::BK * 128) + (uint32_t)r * 128;
-          if (lane == 0) ptx::bulk_wait_group_read_all();  // the slice's previous store has read it
-          __syncwarp();
+          // this key row's 64 queries of dS^T as eight 8-query pieces: piece
+          // c of key r at byte (c * 128 + r) * 16 of the tile
+          uint8_t* tile = utile + (qt - U.qa) * (128 * 128 * 2);
 #pragma unroll
           for (int k = 0; k < 8; ++k)
-            ptx::st_shared_v4(srow + ((k ^ (r & 7)) << 4), dsk[4 * k], dsk[4 * k + 1], dsk[4 * k + 2],
+            ptx::st_global_v4(tile + ((8 * w + k) * 128 + r) * 16, dsk[4 * k], dsk[4 * k + 1], dsk[4 * k + 2],
                               dsk[4 * k + 3]);
-          ptx::fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            const int64_t slot = stored_slot(p, U.bh / p.H, U.bh % p.H, (int)(U.j0 / 128), qt, U.qa);
-            ptx::tma_store_3d(&tm_ds, smem + C::OFF_P + (uint32_t)w * (C::BK * 128) + (uint32_t)wq * (32 * 128),
-                              64 * w, 32 * wq, (int)slot);
-            ptx::bulk_commit_group();
-          }
         }
       }
       if (!ok) break;

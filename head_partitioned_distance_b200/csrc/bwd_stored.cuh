@@ -8,14 +8,18 @@
 // (spa_bwd_dkdv_kernel with DS).  This pass then only contracts the stored
 // tiles with K:
 //   dQ(t) = scale sum_{u in key strip of t} dS(t, u) K(u)
+// A stored tile is 32 KB of 8 x 8 core matrices: the 8 queries [8c, 8c + 8)
+// of key k are the 16 bytes at (c * 128 + k) * 16, so a tile is, unchanged,
+// the A operand dS (queries x keys) in MN-major form without swizzle: core
+// matrices 128 bytes apart along the keys (K) and 2048 along the queries
+// (M).  The dK/dV pass writes it that way with coalesced stores, and this
+// pass copies it whole.
 // Persistent grid (one CTA per SM); a unit is (b, h, query tile of 128 rows)
 // walking the same key strip as the forward.  Per key tile the copy engine
-// brings the 128 x 128 dS^T tile (keys x queries, queries contiguous) and the
-// K tile into a 3-stage ring.  dS^T read with the queries as the contiguous
-// dimension is the A operand dS (queries x keys) in MN-major form, K along d
-// the B operand in MN-major form.  8 SS MMAs of 16 keys add into a TMEM
-// accumulator; the accumulator is double-buffered, so one unit's epilogue
-// overlaps the next unit's products.
+// brings the stored tile (one 32 KB bulk copy) and the K tile (TMA, the B
+// operand, MN-major along d) into a 3-stage ring.  8 SS MMAs of 16 keys add
+// into a TMEM accumulator; the accumulator is double-buffered, so one unit's
+// epilogue overlaps the next unit's products.
 //
 // Warp roles (192 threads): warps 0-3 epilogue (thread r = row r = TMEM lane
 // r: scale * dQ as bf16 straight to global), warp 4 TMA producer, warp 5 MMA
@@ -55,8 +59,7 @@ struct DqStoredBars {
 
 template <int D>
 __global__ void __launch_bounds__(192, 1)
-    spa_bwd_dq_stored_kernel(const __grid_constant__ CUtensorMap tm_ds, const __grid_constant__ CUtensorMap tm_k,
-                             const __grid_constant__ AttnParams p) {
+    spa_bwd_dq_stored_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ AttnParams p) {
   using C = DqStoredCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = align1024(smem_raw);
@@ -83,10 +86,7 @@ __global__ void __launch_bounds__(192, 1)
     ptx::tmem_alloc(&bars->tmem_base, C::TMEM_COLS);
     ptx::tmem_relinquish();
   }
-  if (warp == 4 && lane == 0) {
-    ptx::prefetch_tmap(&tm_ds);
-    ptx::prefetch_tmap(&tm_k);
-  }
+  if (warp == 4 && lane == 0) ptx::prefetch_tmap(&tm_k);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -124,9 +124,9 @@ __global__ void __launch_bounds__(192, 1)
           const int qa = query_strip(N, lo, hi, (int64_t)kt * 128, 128, 128).begin;
           const int slot = (int)stored_slot(p, bh / p.H, bh % p.H, kt, t, qa);
           ptx::mbar_arrive_expect_tx(&bars->full[st], C::DS_BYTES + C::KT_BYTES);
-          for (int c = 0; c < 2; ++c)  // queries [64c, 64c + 64) of all 128 keys
-            ptx::tma_load_3d(smem + C::OFF_DS + st * C::DS_BYTES + c * (C::BK * 128), &tm_ds, &bars->full[st],
-                             c * 64, 0, slot);
+          ptx::bulk_load_1d(smem + C::OFF_DS + st * C::DS_BYTES,
+                            static_cast<const uint8_t*>(p.ds) + (int64_t)slot * C::DS_BYTES, C::DS_BYTES,
+                            &bars->full[st]);
           for (int c = 0; c < C::DB; ++c)
             ptx::tma_load_3d(smem + C::OFF_K + st * C::KT_BYTES + c * (C::BK * 128), &tm_k, &bars->full[st],
                              c * 64, kt * 128, bh);
@@ -141,8 +141,8 @@ __global__ void __launch_bounds__(192, 1)
   } else if (warp == 5) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      // dQ (queries x d) += dS (queries x keys, MN-major: query runs of 64 at
-      // 16 KB) x K (keys x d, MN-major: head-dim runs of 64 at 16 KB)
+      // dQ (queries x d) += dS (queries x keys, MN-major core matrices) x K
+      // (keys x d, MN-major: head-dim runs of 64 at 16 KB)
       constexpr uint32_t idesc = ptx::idesc_bf16_f32(128, D, true, true);
       const uint32_t sDS = ptx::smem_u32(smem + C::OFF_DS), sK = ptx::smem_u32(smem + C::OFF_K);
       int g = 0, n = 0;
@@ -161,11 +161,11 @@ __global__ void __launch_bounds__(192, 1)
           ok = bar_wait(&bars->full[st], (g / C::NS) & 1, abort_flag);
           if (!ok) break;
           ptx::tc_fence_after();
-          const uint64_t da = ptx::sdesc_sw128(sDS + st * C::DS_BYTES, C::BK * 128, 1024);
+          const uint64_t da = ptx::sdesc_noswz(sDS + st * C::DS_BYTES, 128, 2048);
           const uint64_t db = ptx::sdesc_sw128(sK + st * C::KT_BYTES, C::BK * 128, 1024);
 #pragma unroll
           for (int kk = 0; kk < C::BK / 16; ++kk)
-            ptx::mma_bf16(tmem + (uint32_t)b * D, ptx::sdesc_advance(da, kk * (16 * 128)),
+            ptx::mma_bf16(tmem + (uint32_t)b * D, ptx::sdesc_advance(da, kk * 256),  // 16 keys: 2 core matrices
                           ptx::sdesc_advance(db, kk * (16 * 128)), idesc, (kt > s.begin || kk > 0) ? 1 : 0);
           ptx::mma_commit(&bars->empty[st]);
         }

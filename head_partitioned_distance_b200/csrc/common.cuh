@@ -53,6 +53,7 @@ struct AttnParams {
   // ds_len[h] consecutive tiles (stored_slot)
   int64_t ds_base[kMaxHeads];
   int32_t ds_len[kMaxHeads];
+  void* ds;  // the dS^T tiles (layout in bwd_stored.cuh)
   int32_t lo[kMaxHeads];
   int32_t hi[kMaxHeads];
   int32_t unit_start[kMaxHeads + 1];

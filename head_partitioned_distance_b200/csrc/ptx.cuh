@@ -74,6 +74,15 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Contiguous copy of `bytes` (a multiple of 16, both ends 16-byte aligned)
+// from global into shared memory, completion counted on `bar` (bytes).
+__device__ __forceinline__ void bulk_load_1d(void* smem_dst, const void* gsrc, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(smem_dst)),
+               "l"(gsrc), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
 // 3-D tiled store from shared memory (rows past the tensor's extent are clipped).
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* m, const void* smem_src, int c0,
                                              int c1, int c2) {
@@ -203,6 +212,19 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   d |= (uint64_t)1 << 46;  // descriptor version for sm_100
   d |= (uint64_t)2 << 61;  // swizzle: 128 B
   return d;
+}
+
+// Shared-memory matrix descriptor of an operand without swizzle, made of
+// core matrices of 8 rows x 16 bytes (128 contiguous bytes each).  For an
+// MN-major operand (16 bytes = 8 elements along M/N per row, the rows along
+// K): core matrices `lbo` bytes apart along K and `sbo` bytes apart along M/N.
+__device__ __forceinline__ uint64_t sdesc_noswz(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+  return d;                // swizzle field 0: none
 }
 
 // Descriptor `d` with its start address advanced by `bytes`.  Operand tiles

@@ -240,10 +240,6 @@ int64_t stored_layout(AttnParams& p) {
   }
   return n;
 }
-int64_t stored_tiles(const AttnParams& p) {
-  const int h = p.H - 1;
-  return p.ds_base[h] + (int64_t)p.B * ((p.N - 1 - p.lo[h]) / 128 + 1) * p.ds_len[h];
-}
 
 template <int D>
 int bwd_impl(const void* q, const void* k, const void* v, const void* o, const void* dout,
@@ -260,6 +256,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
   int st;
   p.lse = const_cast<float*>(lse);
   p.delta = delta;
+  p.ds = ds;
   p.dq = dq;
   p.dk = dk;
   p.dv = dv;
@@ -316,15 +313,12 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     // persistent grid over key tiles of 128 that some query reaches; the
     // other key tiles only get zero rows
     // dk and dv leave through bulk tensor stores of 32-row boxes
-    CUtensorMap kq, kk, kv, kdo, kdk, kdv, kds;
+    CUtensorMap kq, kk, kv, kdo, kdk, kdv;
     if ((st = make_map(&kq, q, p.N, BH, D, KC::BQ)) || (st = make_map(&kk, k, p.N, BH, D, KC::BK)) ||
         (st = make_map(&kv, v, p.N, BH, D, KC::BK)) || (st = make_map(&kdo, dout, p.N, BH, D, KC::BQ)) ||
         (st = make_map(&kdk, dk, p.N, BH, D, 32)) || (st = make_map(&kdv, dv, p.N, BH, D, 32)))
       return st;
     const int64_t nkt = (p.N + 127) / 128;
-    // the dS^T buffer: [tiles][128 keys][128 queries] bf16, stored in 32 x 64 boxes
-    if (ds && (st = make_map(&kds, ds, 128, stored_tiles(p), 128, 32))) return st;
-    if (!ds) kds = kdk;  // not read
     auto* kernel_kv = ds ? spa::spa_bwd_dkdv_kernel<D, false, true>
                          : (acc ? spa::spa_bwd_dkdv_kernel<D, true> : spa::spa_bwd_dkdv_kernel<D, false>);
     if ((st = prepare_kernel(kernel_kv, KC::SMEM_BYTES, ds ? prepared_kvs : prepared_kv[acc]))) return st;
@@ -339,7 +333,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if ((st = sm_count(&sms))) return st;
     const int64_t units = (int64_t)p.B * upb;
     const unsigned grid = (unsigned)(units < sms ? units : sms);
-    kernel_kv<<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, kds, p);
+    kernel_kv<<<grid, KC::NTHREADS, KC::SMEM_BYTES, stream>>>(kq, kk, kv, kdo, kdk, kdv, p);
     if ((st = launch_status())) return st;
   }
   if (steps & kStepDqStored) {
@@ -349,10 +343,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     using SC = spa::DqStoredCfg<D>;
     if (!ds) return SPA_ERR_INVAL;
     const int64_t nqt = (p.N + 127) / 128;
-    CUtensorMap mds, mk;
-    if ((st = make_map(&mds, ds, 128, stored_tiles(p), 128, 128)) ||
-        (st = make_map(&mk, k, p.N, BH, D, SC::BK)))
-      return st;
+    CUtensorMap mk;
+    if ((st = make_map(&mk, k, p.N, BH, D, SC::BK))) return st;
     auto* kernel_qs = spa::spa_bwd_dq_stored_kernel<D>;
     if ((st = prepare_kernel(kernel_qs, SC::SMEM_BYTES, prepared_qs))) return st;
     if ((int64_t)p.B * p.H * nqt > 2147483647LL) return SPA_ERR_UNSUPPORTED;
@@ -363,7 +355,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const void* o, const v
     if ((st = sm_count(&sms))) return st;
     const int64_t units = (int64_t)p.B * p.units_per_batch;
     const unsigned grid = (unsigned)(units < sms ? units : sms);
-    kernel_qs<<<grid, SC::NTHREADS, SC::SMEM_BYTES, stream>>>(mds, mk, p);
+    kernel_qs<<<grid, SC::NTHREADS, SC::SMEM_BYTES, stream>>>(mk, p);
     if ((st = launch_status())) return st;
   }
   return SPA_OK;
