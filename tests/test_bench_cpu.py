@@ -126,3 +126,18 @@ def test_ncu_summaries_from_csv(tmp_path):
     assert bench.bench_kernel_key("spa_bwd_dkdv_kernel<128, 0, 1>") == "spa_bwd_dkdv_kernel_ds"
     assert bench.bench_kernel_key("spa_bwd_dkdv_kernel<128, 0, 0>") == "spa_bwd_dkdv_kernel"
     assert bench.bench_kernel_key("spa_fwd_kernel<128, 0, 1>") == "spa_fwd_kernel"
+
+
+def test_backward_modes_are_consistent():
+    # every backward the bench can time has a kernel list, a description and
+    # a work entry for each kernel it launches (the line's per-kernel roofline)
+    import bench
+    from head_partitioned_distance_b200 import synth
+    modes = {"two-pass", "stored", "fused"}
+    assert set(bench.KERNELS_OF) == set(bench.BACKWARD_DESCRIPTION) == modes
+    w = synth.WORKLOADS["b1_h8_n1001_d64"]
+    work = bench.kernel_work(w, 1000, 500, 10)
+    for mode, kernels in bench.KERNELS_OF.items():
+        assert kernels[0] == "spa_fwd_kernel", mode
+        for k in kernels:
+            assert k in work, (mode, k)
